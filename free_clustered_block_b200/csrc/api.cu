@@ -1,0 +1,318 @@
+// libca C ABI: validation, workspace layout, and launch sequencing.
+// Every check runs on the host before the first launch, so a call that
+// returns an error has launched nothing.
+#include <cstring>
+#include <cstdio>
+
+#include "ca_internal.cuh"
+
+namespace ca {
+size_t route_smem_bytes(int C, int D);
+cudaError_t device_error_read_clear(unsigned* out, cudaStream_t st);
+void set_wait_limit(uint64_t spins);
+}  // namespace ca
+
+using namespace ca;
+
+namespace {
+
+constexpr int kMaxRouteC = 8192;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ca_status check_shape(const ca_shape* s) {
+  if (!s) return CA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->n_valid < 1 || s->N_alloc < s->n_valid) return CA_ERR_INVALID_ARG;
+  if (s->dtype != CA_BF16 && s->dtype != CA_FP32) return CA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return CA_ERR_UNSUPPORTED;
+  if (s->c != 64 && s->c != 128 && s->c != 256) return CA_ERR_UNSUPPORTED;
+  // every per-head index fits in int32; whole tensors fit in size_t
+  const long long C = ((long long)s->n_valid + s->c - 1) / s->c;
+  if ((long long)s->N_alloc > (1ll << 30) || C * s->c > (1ll << 30)) return CA_ERR_UNSUPPORTED;
+  if ((long long)s->B * s->H > 65535) return CA_ERR_UNSUPPORTED;   // grid.y
+  return CA_OK;
+}
+
+bool plan_for(const ca_shape* s, TreePlan* plan) { return host_plan(s->n_valid, s->c, plan); }
+
+size_t dir_smem(int d, int a) {
+  const size_t m_cap = (size_t)a * d;
+  return (size_t)d * d * 8 + 256 * 8 + m_cap * 16 + (size_t)d * 32 + 16 + m_cap * (d + 1) * 4;
+}
+
+ca_status check_params(const ca_shape* s, const ca_cluster_params* p) {
+  if (!p) return CA_OK;
+  if (p->power_iters < 0 || p->power_iters > 1000 || p->sample_factor < 0) return CA_ERR_INVALID_ARG;
+  const int a = p->sample_factor > 0 ? p->sample_factor : 1;
+  if (dir_smem(s->d, a) > 227 * 1024) return CA_ERR_UNSUPPORTED;
+  if (p->transform != 0 && p->transform != 1) return CA_ERR_INVALID_ARG;
+  return CA_OK;
+}
+
+ca_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return CA_OK;
+  fprintf(stderr, "libca: CUDA error %s\n", cudaGetErrorString(e));
+  return CA_ERR_CUDA;
+}
+
+// Layout of ca_forward's workspace: clusters, routes, then the cluster and
+// attention workspaces (which are used one after the other and may overlap).
+struct ForwardWs {
+  size_t perm_q, perm_k, count_q, count_k, qbar, kbar, kept_idx, kept_bits, scratch, total;
+  size_t cluster_bytes, attend_bytes;
+};
+
+bool forward_layout(const ca_shape* s, int k, ForwardWs* f) {
+  TreePlan plan;
+  if (!plan_for(s, &plan)) return false;
+  ClusterWs cw;
+  AttendWs aw;
+  cluster_ws_layout(s, plan, &cw);
+  attend_ws_layout(s, &aw);
+  const size_t BH = (size_t)s->B * s->H, C = plan.C, c = s->c, d = s->d;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+  f->perm_q = take(BH * C * c * 4);
+  f->perm_k = take(BH * C * c * 4);
+  f->count_q = take(BH * C * 4);
+  f->count_k = take(BH * C * 4);
+  f->qbar = take(BH * C * d * 8);
+  f->kbar = take(BH * C * d * 8);
+  f->kept_idx = take(BH * C * (size_t)k * 4);
+  f->kept_bits = take(BH * C * ((C + 31) / 32) * 4);
+  f->cluster_bytes = cw.total;
+  f->attend_bytes = aw.total;
+  f->scratch = take(cw.total > aw.total ? cw.total : aw.total);
+  f->total = o;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ca_num_clusters(const ca_shape* s) {
+  if (check_shape(s) != CA_OK) return -1;
+  return (s->n_valid + s->c - 1) / s->c;
+}
+
+ca_status ca_check_shape(const ca_shape* s) { return check_shape(s); }
+
+size_t ca_cluster_workspace_bytes(const ca_shape* s) {
+  if (check_shape(s) != CA_OK) return 0;
+  TreePlan plan;
+  if (!plan_for(s, &plan)) return 0;
+  ClusterWs w;
+  cluster_ws_layout(s, plan, &w);
+  return w.total;
+}
+
+size_t ca_attend_workspace_bytes(const ca_shape* s) {
+  if (check_shape(s) != CA_OK) return 0;
+  AttendWs w;
+  attend_ws_layout(s, &w);
+  return w.total;
+}
+
+size_t ca_dense_workspace_bytes(const ca_shape* s) {
+  (void)s;
+  return 0;
+}
+
+size_t ca_forward_workspace_bytes(const ca_shape* s, int k) {
+  if (check_shape(s) != CA_OK) return 0;
+  const int C = (s->n_valid + s->c - 1) / s->c;
+  if (k < 1 || k > C) return 0;
+  ForwardWs f;
+  if (!forward_layout(s, k, &f)) return 0;
+  return f.total;
+}
+
+ca_status ca_cluster(const void* Q, const void* K, const ca_shape* s, const ca_cluster_params* params,
+                     const ca_clusters* out, void* workspace, size_t workspace_bytes, void* stream) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!Q || !K || !out || !out->perm_q || !out->perm_k || !out->count_q || !out->count_k || !out->qbar ||
+      !out->kbar)
+    return CA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K)) return CA_ERR_INVALID_ARG;
+  if ((st = check_params(s, params)) != CA_OK) return st;
+  TreePlan plan;
+  if (!plan_for(s, &plan)) return CA_ERR_UNSUPPORTED;
+  ClusterWs L;
+  cluster_ws_layout(s, plan, &L);
+  if (workspace_bytes < L.total) return CA_ERR_WORKSPACE;
+  if (!workspace) return CA_ERR_INVALID_ARG;
+  ca_cluster_params p = {8, 1, 1, 0, 0ull};
+  if (params) p = *params;
+  return cuda_status(launch_cluster(Q, K, s, &p, out, plan, L, static_cast<char*>(workspace),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+ca_status ca_route(const ca_shape* s, const ca_clusters* cen, const ca_routes* out, void* stream) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!cen || !cen->qbar || !cen->kbar || !out || !out->kept_idx || !out->kept_bits) return CA_ERR_INVALID_ARG;
+  const int C = (s->n_valid + s->c - 1) / s->c;
+  if (out->k < 1 || out->k > C) return CA_ERR_INVALID_ARG;
+  if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
+  return cuda_status(launch_route(s, C, cen->qbar, cen->kbar, out->k, out->kept_idx, out->kept_bits,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* s, const ca_clusters* cl,
+                    const ca_routes* rt, int compensate, void* O, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!Q || !K || !V || !O || !cl || !rt || !cl->perm_q || !cl->perm_k || !cl->count_k || !cl->kbar ||
+      !rt->kept_idx || !rt->kept_bits)
+    return CA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return CA_ERR_INVALID_ARG;
+  const int C = (s->n_valid + s->c - 1) / s->c;
+  if (rt->k < 1 || rt->k > C) return CA_ERR_INVALID_ARG;
+  AttendWs L;
+  attend_ws_layout(s, &L);
+  if (workspace_bytes < L.total) return CA_ERR_WORKSPACE;
+  if (!workspace) return CA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  cudaError_t e = launch_attend_prep(Q, K, V, s, cl, L, ws, cs);
+  if (e == cudaSuccess) {
+    e = launch_attend_simt(Q, K, V, s, cl, rt, compensate, O, L, ws, cs);
+  }
+  if (e == cudaSuccess) e = launch_zero_pad_rows(O, s, cs);
+  return cuda_status(e);
+}
+
+ca_status ca_dense_attend(const void* Q, const void* K, const void* V, const ca_shape* s, void* O,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace; (void)workspace_bytes;
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!Q || !K || !V || !O) return CA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return CA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (s->dtype == CA_BF16) ? launch_dense_tc(Q, K, V, s, O, cs)
+                                        : launch_dense_simt(Q, K, V, s, O, cs);
+  if (e == cudaSuccess) e = launch_zero_pad_rows(O, s, cs);
+  return cuda_status(e);
+}
+
+ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape* s,
+                     const ca_cluster_params* params, int k, int compensate, void* O, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!Q || !K || !V || !O) return CA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return CA_ERR_INVALID_ARG;
+  if ((st = check_params(s, params)) != CA_OK) return st;
+  const int C = (s->n_valid + s->c - 1) / s->c;
+  if (k < 1 || k > C) return CA_ERR_INVALID_ARG;
+  if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
+  ForwardWs f;
+  if (!forward_layout(s, k, &f)) return CA_ERR_UNSUPPORTED;
+  if (workspace_bytes < f.total) return CA_ERR_WORKSPACE;
+  if (!workspace) return CA_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  ca_clusters cl;
+  cl.perm_q = reinterpret_cast<int32_t*>(ws + f.perm_q);
+  cl.perm_k = reinterpret_cast<int32_t*>(ws + f.perm_k);
+  cl.count_q = reinterpret_cast<int32_t*>(ws + f.count_q);
+  cl.count_k = reinterpret_cast<int32_t*>(ws + f.count_k);
+  cl.qbar = reinterpret_cast<double*>(ws + f.qbar);
+  cl.kbar = reinterpret_cast<double*>(ws + f.kbar);
+  ca_routes rt;
+  rt.k = k;
+  rt.kept_idx = reinterpret_cast<int32_t*>(ws + f.kept_idx);
+  rt.kept_bits = reinterpret_cast<uint32_t*>(ws + f.kept_bits);
+  st = ca_cluster(Q, K, s, params, &cl, ws + f.scratch, f.cluster_bytes, stream);
+  if (st != CA_OK) return st;
+  st = ca_route(s, &cl, &rt, stream);
+  if (st != CA_OK) return st;
+  return ca_attend(Q, K, V, s, &cl, &rt, compensate, O, ws + f.scratch, f.attend_bytes, stream);
+}
+
+size_t ca_forward_host_workspace_bytes(const ca_shape* s, int k) {
+  const size_t base = ca_forward_workspace_bytes(s, k);
+  if (!base) return 0;
+  const size_t esz = s->dtype == CA_BF16 ? 2 : 4;
+  const size_t t = (size_t)s->B * s->H * s->N_alloc * s->d * esz;
+  return base + 4 * align_up(t);
+}
+
+ca_status ca_forward_host(const void* Qh, const void* Kh, const void* Vh, const ca_shape* s,
+                          const ca_cluster_params* params, int k, int compensate, void* Oh, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!Qh || !Kh || !Vh || !Oh) return CA_ERR_INVALID_ARG;
+  const size_t need = ca_forward_host_workspace_bytes(s, k);
+  if (!need) return CA_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return CA_ERR_WORKSPACE;
+  if (!workspace) return CA_ERR_INVALID_ARG;
+  const size_t esz = s->dtype == CA_BF16 ? 2 : 4;
+  const size_t t = (size_t)s->B * s->H * s->N_alloc * s->d * esz;
+  char* ws = static_cast<char*>(workspace);
+  const size_t base = ca_forward_workspace_bytes(s, k);
+  char* dQ = ws + base;
+  char* dK = dQ + align_up(t);
+  char* dV = dK + align_up(t);
+  char* dO = dV + align_up(t);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(dQ, Qh, t, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dK, Kh, t, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dV, Vh, t, cudaMemcpyHostToDevice, cs);
+  if (e != cudaSuccess) return cuda_status(e);
+  st = ca_forward(dQ, dK, dV, s, params, k, compensate, dO, ws, base, stream);
+  if (st != CA_OK) return st;
+  e = cudaMemcpyAsync(Oh, dO, t, cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  return cuda_status(e);
+}
+
+ca_status ca_get_device_error(void* stream) {
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_status(e);
+  unsigned word = 0;
+  e = device_error_read_clear(&word, cs);
+  if (e != cudaSuccess) return cuda_status(e);
+  return word ? static_cast<ca_status>(word) : CA_OK;
+}
+
+void ca_set_wait_limit(uint64_t spins) { set_wait_limit(spins); }
+
+int ca_launch_count(const ca_shape* s, int stage) {
+  if (check_shape(s) != CA_OK) return -1;
+  const int pad = s->N_alloc > s->n_valid ? 1 : 0;
+  switch (stage) {
+    case 0: {
+      TreePlan plan;
+      if (!plan_for(s, &plan)) return -1;
+      // plan, colsum, syrk, metric reduce, query norms; per level: direction,
+      // projection, select, partition count, partition scatter; centroids.
+      return plan.levels > 0 ? 5 + 5 * plan.levels + 1 : 1;
+    }
+    case 1: return 1;
+    case 2: return (s->dtype == CA_BF16 ? 2 : 1) + 1 + pad;   // prep (+ permute), attention, pad rows
+    case 3: return 1 + pad;
+  }
+  return -1;
+}
+
+const char* ca_status_string(ca_status s) {
+  switch (s) {
+    case CA_OK: return "CA_OK";
+    case CA_ERR_INVALID_ARG: return "CA_ERR_INVALID_ARG";
+    case CA_ERR_UNSUPPORTED: return "CA_ERR_UNSUPPORTED";
+    case CA_ERR_WORKSPACE: return "CA_ERR_WORKSPACE";
+    case CA_ERR_CUDA: return "CA_ERR_CUDA";
+    case CA_ERR_TIMEOUT: return "CA_ERR_TIMEOUT";
+  }
+  return "CA_ERR_UNKNOWN";
+}
+
+const char* ca_version(void) { return "libca 0.1 (sm_100a)"; }
+
+}  // extern "C"

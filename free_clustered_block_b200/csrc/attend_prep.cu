@@ -1,0 +1,183 @@
+// Attention preparation: value centroids, compensation terms, and the
+// cluster-ordered copies of Q, K and V that the tensor-core kernel tiles.
+//
+// ClusterAttention paper, Appendix A, eq. 21-22: every excluded key cluster b
+// enters a query's softmax as one term with logit q . kbar_b / sqrt(d) + ln|b|
+// and value vbar_b, the mean value of its |b| real members.
+//
+// Centroids are fp64 from clustering. For the bf16 tensor-core path each
+// fp64 centroid is split into bf16 hi + lo parts (x ~ hi + lo, ~16 significant
+// bits) so that two bf16 products carry it into the fp32 accumulator.
+#include "ca_internal.cuh"
+
+namespace ca {
+namespace {
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// One block per key cluster: vbar (fp64 mean of the members' values), and the
+// fp32 / bf16 hi-lo forms of kbar and vbar; log count.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) centroid_prep_kernel(
+    const T* __restrict__ V, int N_alloc, int c, int C, int Cpad, const int32_t* __restrict__ perm_k,
+    const int32_t* __restrict__ count_k, const double* __restrict__ kbar, float* __restrict__ kbar32,
+    float* __restrict__ vbar32, __nv_bfloat16* __restrict__ kbar_hi, __nv_bfloat16* __restrict__ kbar_lo,
+    __nv_bfloat16* __restrict__ vbar_hi, __nv_bfloat16* __restrict__ vbar_lo, float* __restrict__ logcnt) {
+  constexpr int RG = 256 / D;
+  const int b = blockIdx.x, bh = blockIdx.y;
+  const int col = threadIdx.x % D, rg = threadIdx.x / D;
+  const size_t o_pad = ((size_t)bh * Cpad + b) * D + col;
+  if (b >= C) {   // padding centroids of the tensor-core tiles
+    if (rg == 0) {
+      const __nv_bfloat16 z = __float2bfloat16(0.f);
+      kbar_hi[o_pad] = z; kbar_lo[o_pad] = z; vbar_hi[o_pad] = z; vbar_lo[o_pad] = z;
+      if (col == 0) logcnt[(size_t)bh * Cpad + b] = -INFINITY;
+    }
+    return;
+  }
+  const int cnt = count_k[(size_t)bh * C + b];
+  const int32_t* mem = perm_k + (size_t)bh * C * c + (size_t)b * c;
+  const T* Vh = V + (size_t)bh * N_alloc * D;
+  double s = 0.0;
+  for (int j = rg; j < cnt; j += RG) s += (double)to_f(Vh[(size_t)mem[j] * D + col]);
+  __shared__ double red[256];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  if (rg == 0) {
+    double t = 0.0;
+    for (int g = 0; g < RG; ++g) t += red[g * D + col];
+    const double vb = t / (double)cnt;
+    const double kb = kbar[((size_t)bh * C + b) * D + col];
+    const size_t o32 = ((size_t)bh * C + b) * D + col;
+    vbar32[o32] = (float)vb;
+    kbar32[o32] = (float)kb;
+    const __nv_bfloat16 khi = __double2bfloat16(kb);
+    const __nv_bfloat16 vhi = __double2bfloat16(vb);
+    kbar_hi[o_pad] = khi; kbar_lo[o_pad] = __double2bfloat16(kb - (double)__bfloat162float(khi));
+    vbar_hi[o_pad] = vhi; vbar_lo[o_pad] = __double2bfloat16(vb - (double)__bfloat162float(vhi));
+    if (col == 0) logcnt[(size_t)bh * Cpad + b] = logf((float)cnt);
+  }
+}
+
+// Cluster-ordered copy: dst[bh][slot] = src[bh][perm[slot]] (zero for pad
+// slots). One 16-byte vector per thread; blockIdx.z selects Q / K / V.
+template <int D>
+__global__ void __launch_bounds__(256) permute_rows_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+    const __nv_bfloat16* __restrict__ V, int N_alloc, int slots, const int32_t* __restrict__ perm_q,
+    const int32_t* __restrict__ perm_k, __nv_bfloat16* __restrict__ Qp, __nv_bfloat16* __restrict__ Kp,
+    __nv_bfloat16* __restrict__ Vp) {
+  constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
+  const int bh = blockIdx.y, z = blockIdx.z;
+  const __nv_bfloat16* src = (z == 0 ? Q : (z == 1 ? K : V)) + (size_t)bh * N_alloc * D;
+  __nv_bfloat16* dst = (z == 0 ? Qp : (z == 1 ? Kp : Vp)) + (size_t)bh * slots * D;
+  const int32_t* perm = (z == 0 ? perm_q : perm_k) + (size_t)bh * slots;
+  const size_t e = (size_t)blockIdx.x * 256 + threadIdx.x;
+  const int slot = (int)(e / VPR), v = (int)(e % VPR);
+  if (slot >= slots) return;
+  const int row = perm[slot];
+  uint4 val = make_uint4(0, 0, 0, 0);
+  if (row >= 0) val = *reinterpret_cast<const uint4*>(src + (size_t)row * D + v * 8);
+  *reinterpret_cast<uint4*>(dst + (size_t)slot * D + v * 8) = val;
+}
+
+__global__ void zero_rows_kernel(uint4* __restrict__ O, size_t row_vecs, size_t rows_per_head,
+                                 size_t first_row, size_t pad_rows, size_t BH) {
+  const size_t per_head = pad_rows * row_vecs;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < per_head * BH;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const size_t bh = e / per_head, r = e % per_head;
+    O[(bh * rows_per_head + first_row) * row_vecs + r] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+}  // namespace
+
+bool attend_ws_layout(const ca_shape* s, AttendWs* w) {
+  const size_t BH = (size_t)s->B * s->H, d = s->d, c = s->c;
+  const size_t C = (s->n_valid + c - 1) / c;
+  const size_t Cpad = (C + 127) / 128 * 128;
+  w->C = (int)C; w->Cpad = (int)Cpad;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+  const bool tc = (s->dtype == CA_BF16);
+  const size_t rows = BH * C * c * d * 2;
+  w->qp = take(tc ? rows : 0);
+  w->kp = take(tc ? rows : 0);
+  w->vp = take(tc ? rows : 0);
+  w->kbar_hi = take(BH * Cpad * d * 2);
+  w->kbar_lo = take(BH * Cpad * d * 2);
+  w->vbar_hi = take(BH * Cpad * d * 2);
+  w->vbar_lo = take(BH * Cpad * d * 2);
+  w->vbar32 = take(BH * C * d * 4);
+  w->kbar32 = take(BH * C * d * 4);
+  w->logcnt = take(BH * Cpad * 4);
+  w->total = o;
+  return true;
+}
+
+cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, const ca_shape* s,
+                               const ca_clusters* cl, const AttendWs& L, char* ws, cudaStream_t st) {
+  const int BH = s->B * s->H, C = L.C, Cpad = L.Cpad, c = s->c;
+  float* kbar32 = reinterpret_cast<float*>(ws + L.kbar32);
+  float* vbar32 = reinterpret_cast<float*>(ws + L.vbar32);
+  __nv_bfloat16* khi = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_hi);
+  __nv_bfloat16* klo = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_lo);
+  __nv_bfloat16* vhi = reinterpret_cast<__nv_bfloat16*>(ws + L.vbar_hi);
+  __nv_bfloat16* vlo = reinterpret_cast<__nv_bfloat16*>(ws + L.vbar_lo);
+  float* logcnt = reinterpret_cast<float*>(ws + L.logcnt);
+  const dim3 g(Cpad, BH);
+  if (s->dtype == CA_BF16) {
+    using T = __nv_bfloat16;
+    if (s->d == 64)
+      centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+                                                     cl->count_k, cl->kbar, kbar32, vbar32, khi, klo, vhi,
+                                                     vlo, logcnt);
+    else
+      centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+                                                      cl->count_k, cl->kbar, kbar32, vbar32, khi, klo,
+                                                      vhi, vlo, logcnt);
+    const int slots = C * c;
+    const size_t vecs = (size_t)slots * (s->d * 2 / 16);
+    const dim3 gp((unsigned)((vecs + 255) / 256), BH, 3);
+    T* Qp = reinterpret_cast<T*>(ws + L.qp);
+    T* Kp = reinterpret_cast<T*>(ws + L.kp);
+    T* Vp = reinterpret_cast<T*>(ws + L.vp);
+    if (s->d == 64)
+      permute_rows_kernel<64><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc, slots,
+                                                  cl->perm_q, cl->perm_k, Qp, Kp, Vp);
+    else
+      permute_rows_kernel<128><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc,
+                                                   slots, cl->perm_q, cl->perm_k, Qp, Kp, Vp);
+  } else {
+    using T = float;
+    if (s->d == 64)
+      centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+                                                     cl->count_k, cl->kbar, kbar32, vbar32, khi, klo, vhi,
+                                                     vlo, logcnt);
+    else
+      centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+                                                      cl->count_k, cl->kbar, kbar32, vbar32, khi, klo,
+                                                      vhi, vlo, logcnt);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_pad_rows(void* O, const ca_shape* s, cudaStream_t st) {
+  if (s->N_alloc <= s->n_valid) return cudaSuccess;
+  const size_t esz = (s->dtype == CA_BF16) ? 2 : 4;
+  const size_t row_vecs = (size_t)s->d * esz / 16;
+  const size_t BH = (size_t)s->B * s->H;
+  const size_t pad = (size_t)(s->N_alloc - s->n_valid);
+  const size_t total = pad * row_vecs * BH;
+  const unsigned blocks = (unsigned)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
+  zero_rows_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<uint4*>(O), row_vecs, (size_t)s->N_alloc,
+                                           (size_t)s->n_valid, pad, BH);
+  return cudaGetLastError();
+}
+
+}  // namespace ca

@@ -1,0 +1,776 @@
+// Clustering kernels: metric matrices, per-node principal direction by power
+// iteration, projection, radix select of the split threshold, stable
+// partition, centroids.
+//
+// ClusterAttention paper, Section 3.2 "Clustering" (3.2.1 basic recursive
+// splitting, 3.2.2 transforms) and Section 6.1 (the metric matrix injected
+// into the power iteration instead of an eigendecomposition).
+//
+// Arithmetic that decides the partition is fp64 throughout: inputs (bf16 or
+// fp32) widen exactly to fp64, metric matrices, query norms, directions and
+// projections are fp64, and the split is an exact order statistic of the
+// fp64 projections, equal values ordered by row index.
+#include "ca_internal.cuh"
+
+namespace ca {
+
+namespace {
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// Warp sum of a double, fixed butterfly order (deterministic).
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Tree tables on the device (one thread; the host runs the same function).
+// ---------------------------------------------------------------------------
+__global__ void plan_kernel(int n, int c, TreeNode* nodes, int* level_begin) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) plan_tree(n, c, nodes, level_begin, kMaxLevels);
+}
+
+// ---------------------------------------------------------------------------
+// S1: column sums of K (for the key mean), per row chunk.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, int N_alloc, int n,
+                                                     double* __restrict__ part) {
+  constexpr int RG = 256 / D;
+  const int bh = blockIdx.y, ch = blockIdx.x, nch = gridDim.x;
+  const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
+  const int col = threadIdx.x % D, rg = threadIdx.x / D;
+  const T* base = K + (size_t)bh * N_alloc * D;
+  double acc = 0.0;
+  for (int r = r0 + rg; r < r1; r += RG) acc += (double)to_f(base[(size_t)r * D + col]);
+  __shared__ double red[256];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  if (rg == 0) {
+    double s = 0.0;
+    for (int g = 0; g < RG; ++g) s += red[g * D + col];
+    part[((size_t)bh * nch + ch) * D + col] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// S1: partial second-moment matrices over a row chunk.
+// z = 0: Q^T Q (uncentred); z = 1: (K - kmean)^T (K - kmean).
+// Thread (ty, tx) owns entries (ty + 16 i, tx + 16 j).
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) syrk_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                                                   int N_alloc, int n, int nch,
+                                                   const double* __restrict__ colpart,
+                                                   double* __restrict__ part) {
+  constexpr int TR = 32;
+  constexpr int B = D / 16;
+  __shared__ double xs[TR][D];
+  __shared__ double mean[D];
+  const int bh = blockIdx.y, z = blockIdx.z, ch = blockIdx.x;
+  const T* X = (z == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  if (threadIdx.x < D) {
+    double m = 0.0;
+    if (z == 1) {
+      for (int i = 0; i < nch; ++i) m += colpart[((size_t)bh * nch + i) * D + threadIdx.x];
+      m /= (double)n;
+    }
+    mean[threadIdx.x] = m;
+  }
+  __syncthreads();
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  double acc[B][B];
+#pragma unroll
+  for (int i = 0; i < B; ++i)
+#pragma unroll
+    for (int j = 0; j < B; ++j) acc[i][j] = 0.0;
+  const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
+  for (int rt = r0; rt < r1; rt += TR) {
+    for (int e = threadIdx.x; e < TR * D; e += 256) {
+      const int rr = e / D, cc = e % D, r = rt + rr;
+      xs[rr][cc] = (r < r1) ? (double)to_f(X[(size_t)r * D + cc]) - mean[cc] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rr = 0; rr < TR; ++rr) {
+      double a[B], b[B];
+#pragma unroll
+      for (int i = 0; i < B; ++i) a[i] = xs[rr][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < B; ++j) b[j] = xs[rr][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < B; ++i)
+#pragma unroll
+        for (int j = 0; j < B; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  double* out = part + (((size_t)bh * 2 + z) * nch + ch) * D * D;
+#pragma unroll
+  for (int i = 0; i < B; ++i)
+#pragma unroll
+    for (int j = 0; j < B; ++j) out[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+}
+
+// M[th] for tensor-head th = 2 bh + tensor: queries (tensor 0) are split in
+// the key metric M_k, keys (tensor 1) in the query metric M_q.
+template <int D>
+__global__ void __launch_bounds__(256) metric_reduce_kernel(const double* __restrict__ part, int nch,
+                                                            int n, int transform,
+                                                            double* __restrict__ M) {
+  const int th = blockIdx.x, bh = th >> 1, tensor = th & 1;
+  const int src = 1 - tensor;  // z index: 0 = Q^T Q, 1 = K_c^T K_c
+  const double* p = part + ((size_t)bh * 2 + src) * nch * D * D;
+  for (int e = threadIdx.x; e < D * D; e += 256) {
+    double v;
+    if (transform) {
+      v = 0.0;
+      for (int ch = 0; ch < nch; ++ch) v += p[(size_t)ch * D * D + e];
+      v /= (double)n;
+    } else {
+      v = (e / D == e % D) ? 1.0 : 0.0;
+    }
+    M[(size_t)th * D * D + e] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Query scale 1/|R_k q| = 1/sqrt(q^T M_k q) (eq. 16), 0 when q^T M_k q <= 0.
+// 128 rows per block; thread (ty,tx) computes T = X M for rows ty+16i, cols
+// tx+16j, then the row dot with X.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int N_alloc, int n,
+                                                    const double* __restrict__ M, int transform,
+                                                    double* __restrict__ inv_s) {
+  constexpr int R = 128, B = D / 16, RS = D + 1;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* Ms = reinterpret_cast<double*>(smem_raw);           // [D][D]
+  float* xs = reinterpret_cast<float*>(Ms + D * D);           // [R][D+1]
+  const int bh = blockIdx.y, r0 = blockIdx.x * R;
+  const int th = bh * 2;  // queries use M_k, stored at the queries' tensor-head
+  if (!transform) {
+    for (int r = threadIdx.x; r < R; r += 256)
+      if (r0 + r < n) inv_s[(size_t)bh * n + r0 + r] = 1.0;
+    return;
+  }
+  for (int e = threadIdx.x; e < D * D; e += 256) Ms[e] = M[(size_t)th * D * D + e];
+  const T* X = Q + (size_t)bh * N_alloc * D;
+  for (int e = threadIdx.x; e < R * D; e += 256) {
+    const int rr = e / D, cc = e % D, r = r0 + rr;
+    xs[rr * RS + cc] = (r < n) ? to_f(X[(size_t)r * D + cc]) : 0.f;
+  }
+  __syncthreads();
+  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  constexpr int RI = R / 16;  // 8 rows per thread
+  double acc[RI][B];
+#pragma unroll
+  for (int i = 0; i < RI; ++i)
+#pragma unroll
+    for (int j = 0; j < B; ++j) acc[i][j] = 0.0;
+#pragma unroll 2
+  for (int k = 0; k < D; ++k) {
+    double a[RI], b[B];
+#pragma unroll
+    for (int i = 0; i < RI; ++i) a[i] = (double)xs[(ty + 16 * i) * RS + k];
+#pragma unroll
+    for (int j = 0; j < B; ++j) b[j] = Ms[k * D + tx + 16 * j];
+#pragma unroll
+    for (int i = 0; i < RI; ++i)
+#pragma unroll
+      for (int j = 0; j < B; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < RI; ++i) {
+    double s = 0.0;
+#pragma unroll
+    for (int j = 0; j < B; ++j) s = fma(acc[i][j], (double)xs[(ty + 16 * i) * RS + tx + 16 * j], s);
+    // reduce over the 16 lanes sharing ty (lanes 0-15 / 16-31 of the warp)
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const int r = r0 + ty + 16 * i;
+    if (tx == 0 && r < n) inv_s[(size_t)bh * n + r] = (s > 0.0) ? 1.0 / sqrt(s) : 0.0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K1: per-node principal direction by power iteration, metric injected.
+//
+// With the transformed vectors y = R x (R = sqrt(M)), the sample covariance
+// is C_y = R C_x R. Writing the iterate as u = R z, u <- C_y u becomes
+// z <- C_x M z and |u|^2 = z^T M z; the projection y . u = x^T (M z). So the
+// node's direction for projection is w = M z, with no root or eigenproblem.
+// Queries use x = q / |R_k q| (eq. 16).
+// Warm start (Section 3.2.1): mean of the parent's (unit) estimate and a
+// random normal vector of unit norm; g is drawn in the untransformed
+// coordinates and mapped through R: g_hat = R g / |R g|, i.e. z_g = g / sqrt(g^T M g).
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ void block_matvec_sym(const double* Ms, const double* x, double* y, double* red) {
+  // y = M x with M symmetric: y_a = sum_b M[b][a] x_b, column access.
+  constexpr int G = 256 / D;
+  const int a = threadIdx.x % D, p = threadIdx.x / D;
+  double s = 0.0;
+  for (int b = p; b < D; b += G) s = fma(Ms[b * D + a], x[b], s);
+  red[p * D + a] = s;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    double t = 0.0;
+    for (int q = 0; q < G; ++q) t += red[q * D + threadIdx.x];
+    y[threadIdx.x] = t;
+  }
+  __syncthreads();
+}
+
+template <int D>
+__device__ double block_dot(const double* x, const double* y, double* bc) {
+  // Warp 0 sums; result broadcast through bc[0].
+  if (threadIdx.x < 32) {
+    double s = 0.0;
+    for (int i = threadIdx.x; i < D; i += 32) s = fma(x[i], y[i], s);
+    s = warp_sum(s);
+    if (threadIdx.x == 0) bc[0] = s;
+  }
+  __syncthreads();
+  double r = bc[0];
+  __syncthreads();
+  return r;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) dir_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                                                  int N_alloc, int n, const TreeNode* __restrict__ nodes,
+                                                  int lvl_begin, const double* __restrict__ M,
+                                                  const double* __restrict__ inv_s,
+                                                  const int* __restrict__ idx, int NI,
+                                                  double* __restrict__ zvec, double* __restrict__ wvec,
+                                                  uint64_t seed, int power_iters, int sample_factor) {
+  constexpr int XS = D + 1;            // padded fp32 row stride of the sample
+  const int node_id = lvl_begin + blockIdx.x;
+  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const TreeNode nd = nodes[node_id];
+  const int m_cap = sample_factor * D;
+  const int m = min(m_cap, nd.size);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* Ms = reinterpret_cast<double*>(smem_raw);   // D*D
+  double* red = Ms + D * D;                           // 256
+  double* scale = red + 256;                          // m_cap
+  double* xbar = scale + m_cap;                       // D
+  double* z = xbar + D;                               // D
+  double* w = z + D;                                  // D
+  double* g = w + D;                                  // D
+  double* v = g + D;                                  // m_cap
+  double* bc = v + m_cap;                             // 2
+  float* Xs = reinterpret_cast<float*>(bc + 2);       // m_cap * XS
+
+  for (int e = threadIdx.x; e < D * D; e += 256) Ms[e] = M[(size_t)th * D * D + e];
+  const uint64_t key = node_stream(seed, (uint64_t)bh, (uint64_t)tensor, nd.heap);
+  const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
+  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const int* idx_th = idx ? idx + (size_t)th * n : nullptr;
+  for (int e = threadIdx.x; e < m * D; e += 256) {
+    const int j = e / D, col = e % D;
+    const int pos = (nd.size > m) ? (int)(((uint64_t)j * (uint64_t)nd.size + r) / (uint64_t)m) : j;
+    const int row = idx_th ? idx_th[nd.off + pos] : nd.off + pos;
+    Xs[j * XS + col] = to_f(X[(size_t)row * D + col]);
+    if (col == 0) scale[j] = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
+  }
+  if (threadIdx.x < D) {
+    // Box-Muller on two SplitMix64 draws per coordinate.
+    const uint64_t ua = splitmix64(key + 2ull * threadIdx.x + 1ull);
+    const uint64_t ub = splitmix64(key + 2ull * threadIdx.x + 2ull);
+    const double u1 = (double)((ua >> 11) + 1ull) * 0x1.0p-53;
+    const double u2 = (double)(ub >> 11) * 0x1.0p-53;
+    g[threadIdx.x] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    double s = 0.0;
+    for (int j = 0; j < m; ++j) s = fma(scale[j], (double)Xs[j * XS + threadIdx.x], s);
+    xbar[threadIdx.x] = s / (double)m;
+  }
+  // z0 = (z_parent + g / sqrt(g^T M g)) / 2, or g / sqrt(g^T M g) at the root.
+  block_matvec_sym<D>(Ms, g, w, red);
+  {
+    const double gq = block_dot<D>(g, w, bc);
+    const double gi = (gq > 0.0) ? 1.0 / sqrt(gq) : 0.0;
+    if (threadIdx.x < D) {
+      const double gh = g[threadIdx.x] * gi;
+      z[threadIdx.x] = (nd.parent < 0)
+                           ? gh
+                           : 0.5 * (zvec[((size_t)th * NI + nd.parent) * D + threadIdx.x] + gh);
+    }
+    __syncthreads();
+  }
+  for (int it = 0; it < power_iters; ++it) {
+    block_matvec_sym<D>(Ms, z, w, red);       // w = M z
+    if (it > 0) {                              // normalise: |u|^2 = z^T M z
+      const double q = block_dot<D>(z, w, bc);
+      const double qi = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
+      if (threadIdx.x < D) { z[threadIdx.x] *= qi; w[threadIdx.x] *= qi; }
+      __syncthreads();
+    }
+    const double xw = block_dot<D>(xbar, w, bc);
+    // v_j = (x_j - xbar) . w over the sample
+    for (int j = threadIdx.x; j < m; j += 256) {
+      double s = 0.0;
+      for (int col = 0; col < D; ++col) s = fma((double)Xs[j * XS + col], w[col], s);
+      v[j] = fma(scale[j], s, -xw);
+    }
+    __syncthreads();
+    // z' = sum_j v_j (x_j - xbar) / m
+    if (threadIdx.x < D) {
+      double s = 0.0, sv = 0.0;
+      for (int j = 0; j < m; ++j) {
+        s = fma(v[j] * scale[j], (double)Xs[j * XS + threadIdx.x], s);
+        sv += v[j];
+      }
+      z[threadIdx.x] = (s - xbar[threadIdx.x] * sv) / (double)m;
+    }
+    __syncthreads();
+  }
+  block_matvec_sym<D>(Ms, z, w, red);
+  const double q = block_dot<D>(z, w, bc);
+  const double qi = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
+  if (threadIdx.x < D) {
+    const size_t o = ((size_t)th * NI + node_id) * D + threadIdx.x;
+    zvec[o] = z[threadIdx.x] * qi;
+    wvec[o] = w[threadIdx.x] * qi;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K2a: projection key_i = x_i . w_node for every position of the level's
+// internal nodes, stored as order-preserving uint64. One group of G lanes
+// reads one row (16 bytes per lane, coalesced).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int find_node(const TreeNode* nodes, int lb, int le, int pos) {
+  // last node in [lb, le) with off <= pos; -1 if none covers pos
+  int lo = lb, hi = le - 1, ans = -1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    if (nodes[mid].off <= pos) { ans = mid; lo = mid + 1; } else hi = mid - 1;
+  }
+  if (ans >= 0 && pos >= nodes[ans].off + nodes[ans].size) ans = -1;
+  return ans;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                                                      int N_alloc, int n, const TreeNode* __restrict__ nodes,
+                                                      int lb, int le, const double* __restrict__ inv_s,
+                                                      const int* __restrict__ idx, int NI,
+                                                      const double* __restrict__ wvec,
+                                                      uint64_t* __restrict__ keys) {
+  constexpr int EPL = 16 / sizeof(T);        // elements per lane (16 bytes)
+  constexpr int G = D / EPL;                 // lanes per row
+  constexpr int RPW = 32 / G;                // rows per warp step
+  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / G, gl = lane % G;
+  const int base = blockIdx.x * 256;
+  for (int rr = warp * RPW + sub; rr < 256; rr += 8 * RPW) {
+    const int pos = base + rr;
+    int node = -1;
+    if (pos < n) node = find_node(nodes, lb, le, pos);
+    double s = 0.0;
+    int row = 0;
+    if (node >= 0) {
+      row = idx ? idx[(size_t)th * n + pos] : pos;
+      const uint4 raw = *reinterpret_cast<const uint4*>(X + (size_t)row * D + gl * EPL);
+      const T* e = reinterpret_cast<const T*>(&raw);
+      const double* wn = wvec + ((size_t)th * NI + node) * D + gl * EPL;
+#pragma unroll
+      for (int q = 0; q < EPL; ++q) s = fma((double)to_f(e[q]), wn[q], s);
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (node >= 0 && gl == 0) {
+      const double sc = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
+      keys[(size_t)th * n + pos] = ordered_key(s * sc);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K2b: the t-th smallest key of a node (MSD radix select, 8-bit digits).
+// Candidates move to shared memory once they fit. Output: the threshold key T
+// and eq_left = how many keys equal to T go below the split (the first ones
+// in row order, so equal projections are ordered by row index).
+// ---------------------------------------------------------------------------
+struct SelectResult { uint64_t T; int eq_left; int pad; };
+constexpr int kSelCap = 8192;
+
+__global__ void __launch_bounds__(1024) select_kernel(const TreeNode* __restrict__ nodes, int lb,
+                                                      int nodes_in_level, int n,
+                                                      const uint64_t* __restrict__ keys,
+                                                      SelectResult* __restrict__ sel) {
+  __shared__ unsigned int hist[256];
+  __shared__ int s_digit, s_rank, s_cnt, s_ncand;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem_raw);   // kSelCap keys
+  const int th = blockIdx.y;
+  const TreeNode nd = nodes[lb + blockIdx.x];
+  const uint64_t* base = keys + (size_t)th * n + nd.off;
+  const int size = nd.size;
+  int rank = nd.t - 1;
+  uint64_t prefix = 0, mask = 0;
+  bool global_mode = true;
+  int ncand = 0;
+  const int lane = threadIdx.x & 31;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int cnt_total = global_mode ? size : ncand;
+    for (int i0 = 0; i0 < cnt_total; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      bool ok = false;
+      unsigned dg = 0;
+      if (i < cnt_total) {
+        const uint64_t k = global_mode ? base[i] : cand[i];
+        ok = (k & mask) == prefix;
+        dg = (unsigned)((k >> shift) & 0xFF);
+      }
+      // warp-aggregated histogram increment
+      const unsigned act = __ballot_sync(0xffffffffu, ok);
+      if (ok) {
+        const unsigned peers = __match_any_sync(act, dg);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[dg], (unsigned)__popc(peers));
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned cum = 0;
+      int dsel = 255, rsel = rank;
+      unsigned csel = 0;
+      for (int dgt = 0; dgt < 256; ++dgt) {
+        const unsigned h = hist[dgt];
+        if ((unsigned)rank < cum + h) { dsel = dgt; rsel = rank - (int)cum; csel = h; break; }
+        cum += h;
+      }
+      s_digit = dsel; s_rank = rsel; s_cnt = (int)csel;
+    }
+    __syncthreads();
+    rank = s_rank;
+    prefix |= (uint64_t)s_digit << shift;
+    mask |= (uint64_t)0xFF << shift;
+    const int cnt = s_cnt;
+    __syncthreads();
+    if (global_mode && cnt <= kSelCap && shift > 0) {
+      if (threadIdx.x == 0) s_ncand = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < size; i += blockDim.x) {
+        const uint64_t k = base[i];
+        if ((k & mask) == prefix) cand[atomicAdd(&s_ncand, 1)] = k;
+      }
+      __syncthreads();
+      ncand = s_ncand;
+      global_mode = false;
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x == 0) {
+    SelectResult r;
+    r.T = prefix; r.eq_left = rank + 1; r.pad = 0;
+    sel[(size_t)th * nodes_in_level + blockIdx.x] = r;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K2c: stable partition, two passes over node-aligned chunks.
+// Pass A counts keys below / equal to T per chunk; pass B scans and scatters
+// row indices to the children (a child that is a leaf writes straight into
+// the cluster permutation).
+// ---------------------------------------------------------------------------
+constexpr int kPartThreads = 256;
+constexpr int kPartPer = kPartChunk / kPartThreads;   // 8 positions per thread
+
+__global__ void __launch_bounds__(kPartThreads) part_count_kernel(
+    const TreeNode* __restrict__ nodes, int lb, int nodes_in_level, int n, int pch,
+    const uint64_t* __restrict__ keys, const SelectResult* __restrict__ sel, int2* __restrict__ cnt) {
+  const int th = blockIdx.z, nl = blockIdx.y, ch = blockIdx.x;
+  const TreeNode nd = nodes[lb + nl];
+  const SelectResult sr = sel[(size_t)th * nodes_in_level + nl];
+  const int p0 = ch * kPartChunk, p1 = min(nd.size, p0 + kPartChunk);
+  int less = 0, eq = 0;
+  for (int p = p0 + threadIdx.x; p < p1; p += kPartThreads) {
+    const uint64_t k = keys[(size_t)th * n + nd.off + p];
+    less += (k < sr.T);
+    eq += (k == sr.T);
+  }
+  __shared__ int rl[kPartThreads / 32], re[kPartThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    less += __shfl_xor_sync(0xffffffffu, less, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+  if ((threadIdx.x & 31) == 0) { rl[threadIdx.x >> 5] = less; re[threadIdx.x >> 5] = eq; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0, b = 0;
+    for (int i = 0; i < kPartThreads / 32; ++i) { a += rl[i]; b += re[i]; }
+    cnt[((size_t)th * nodes_in_level + nl) * pch + ch] = make_int2(a, b);
+  }
+}
+
+// Block-wide exclusive scan of one int per thread (256 threads).
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int i = 0; i < kPartThreads / 32; ++i) { const int t = warp_tot[i]; warp_tot[i] = s; s += t; }
+    *total = s;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + x - v;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kPartThreads) part_scatter_kernel(
+    const TreeNode* __restrict__ nodes, int lb, int nodes_in_level, int n, int c, int pch,
+    const uint64_t* __restrict__ keys, const SelectResult* __restrict__ sel,
+    const int2* __restrict__ cnt, const int* __restrict__ idx_in, int* __restrict__ idx_out,
+    int32_t* __restrict__ perm_q, int32_t* __restrict__ perm_k, int Cc) {
+  __shared__ int warp_tot[kPartThreads / 32];
+  __shared__ int total;
+  const int th = blockIdx.z, nl = blockIdx.y, ch = blockIdx.x;
+  const int bh = th >> 1, tensor = th & 1;
+  const TreeNode nd = nodes[lb + nl];
+  const int p0 = ch * kPartChunk;
+  if (p0 >= nd.size) return;
+  const SelectResult sr = sel[(size_t)th * nodes_in_level + nl];
+  const int2* cn = cnt + ((size_t)th * nodes_in_level + nl) * pch;
+  int less_before = 0, eq_before = 0;
+  for (int i = 0; i < ch; ++i) { less_before += cn[i].x; eq_before += cn[i].y; }
+  const int left_before = less_before + min(eq_before, sr.eq_left);
+  // this thread's positions: p0 + threadIdx.x * kPartPer + q
+  uint64_t kv[kPartPer];
+  int eq_local = 0;
+#pragma unroll
+  for (int q = 0; q < kPartPer; ++q) {
+    const int p = p0 + threadIdx.x * kPartPer + q;
+    kv[q] = (p < nd.size) ? keys[(size_t)th * n + nd.off + p] : ~0ull;
+    eq_local += (p < nd.size) && (kv[q] == sr.T);
+  }
+  const int eq_excl = block_excl_scan(eq_local, warp_tot, &total);
+  bool goes_left[kPartPer];
+  int left_local = 0;
+  {
+    int er = eq_before + eq_excl;
+#pragma unroll
+    for (int q = 0; q < kPartPer; ++q) {
+      const int p = p0 + threadIdx.x * kPartPer + q;
+      bool gl = false;
+      if (p < nd.size) {
+        if (kv[q] < sr.T) gl = true;
+        else if (kv[q] == sr.T) { gl = (er < sr.eq_left); ++er; }
+      }
+      goes_left[q] = gl;
+      left_local += gl;
+    }
+  }
+  const int left_excl = block_excl_scan(left_local, warp_tot, &total);
+  const int t = nd.t;
+  const bool left_leaf = (t <= c), right_leaf = (nd.size - t <= c);
+  int32_t* perm = (tensor == 0 ? perm_q : perm_k) + (size_t)bh * Cc;
+  int lrank = left_before + left_excl;
+#pragma unroll
+  for (int q = 0; q < kPartPer; ++q) {
+    const int p = p0 + threadIdx.x * kPartPer + q;
+    if (p >= nd.size) break;
+    const int row = idx_in ? idx_in[(size_t)th * n + nd.off + p] : nd.off + p;
+    if (goes_left[q]) {
+      const int dst = nd.off + lrank;
+      if (left_leaf) perm[dst] = row; else idx_out[(size_t)th * n + dst] = row;
+      ++lrank;
+    } else {
+      const int dst = nd.off + t + (p - lrank);
+      if (right_leaf) perm[dst] = row; else idx_out[(size_t)th * n + dst] = row;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// S5: counts, pad slots and centroids (fp64 means of the members' original
+// vectors, eq. 18). levels == 0 means the single cluster holds every token.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) centroid_kernel(const T* __restrict__ Q, const T* __restrict__ K,
+                                                       int N_alloc, int n, int c, int C, int levels,
+                                                       int32_t* __restrict__ perm_q, int32_t* __restrict__ perm_k,
+                                                       int32_t* __restrict__ count_q, int32_t* __restrict__ count_k,
+                                                       double* __restrict__ qbar, double* __restrict__ kbar) {
+  constexpr int RG = 256 / D;
+  const int a = blockIdx.x, th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int cnt = (a < C - 1) ? c : n - (C - 1) * c;
+  int32_t* perm = (tensor == 0 ? perm_q : perm_k) + (size_t)bh * C * c + (size_t)a * c;
+  if (levels == 0) {
+    for (int j = threadIdx.x; j < cnt; j += 256) perm[j] = j;
+    __syncthreads();
+  }
+  for (int j = cnt + threadIdx.x; j < c; j += 256) perm[j] = -1;
+  if (threadIdx.x == 0) ((tensor == 0) ? count_q : count_k)[(size_t)bh * C + a] = cnt;
+  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const int col = threadIdx.x % D, rg = threadIdx.x / D;
+  double s = 0.0;
+  for (int j = rg; j < cnt; j += RG) {
+    const int row = (levels == 0) ? j : perm[j];
+    s += (double)to_f(X[(size_t)row * D + col]);
+  }
+  __shared__ double red[256];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  if (rg == 0) {
+    double t = 0.0;
+    for (int g = 0; g < RG; ++g) t += red[g * D + col];
+    ((tensor == 0) ? qbar : kbar)[((size_t)bh * C + a) * D + col] = t / (double)cnt;
+  }
+}
+
+template <typename T, int D>
+cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_cluster_params* p,
+                        const ca_clusters* out, const TreePlan& plan, const ClusterWs& L, char* ws,
+                        cudaStream_t st) {
+  const int n = s->n_valid, N_alloc = s->N_alloc, c = s->c, C = plan.C;
+  const int BH = L.BH, TH = L.TH, NI = plan.internal;
+  const int nch = L.nch;
+  TreeNode* nodes = reinterpret_cast<TreeNode*>(ws + L.nodes);
+  int* level_begin = reinterpret_cast<int*>(ws + L.level_begin);
+  double* M = reinterpret_cast<double*>(ws + L.M);
+  double* colpart = reinterpret_cast<double*>(ws + L.colsum_part);
+  double* metpart = reinterpret_cast<double*>(ws + L.met_part);
+  double* inv_s = reinterpret_cast<double*>(ws + L.inv_s);
+  int* idxbuf[2] = {reinterpret_cast<int*>(ws + L.idx0), reinterpret_cast<int*>(ws + L.idx1)};
+  uint64_t* keys = reinterpret_cast<uint64_t*>(ws + L.keys);
+  double* zvec = reinterpret_cast<double*>(ws + L.zvec);
+  double* wvec = reinterpret_cast<double*>(ws + L.wvec);
+  SelectResult* sel = reinterpret_cast<SelectResult*>(ws + L.sel);
+  int2* ccnt = reinterpret_cast<int2*>(ws + L.chunk_cnt);
+  const int power_iters = p->power_iters > 0 ? p->power_iters : 8;
+  const int sample_factor = p->sample_factor > 0 ? p->sample_factor : 1;
+  const int transform = p->transform;
+
+  if (plan.levels > 0) {
+    plan_kernel<<<1, 1, 0, st>>>(n, c, nodes, level_begin);
+    colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
+    syrk_kernel<T, D><<<dim3(nch, BH, 2), 256, 0, st>>>(Q, K, N_alloc, n, nch, colpart, metpart);
+    metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
+    const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
+    cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
+    qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, transform, inv_s);
+    const int m_cap = sample_factor * D;
+    const size_t dir_smem = (size_t)D * D * 8 + 256 * 8 + (size_t)m_cap * 8 * 2 + (size_t)D * 8 * 4 + 16 +
+                            (size_t)m_cap * (D + 1) * 4;
+    cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
+    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
+    for (int l = 0; l < plan.levels; ++l) {
+      const int lb = plan.level_begin[l], le = plan.level_begin[l + 1], nl = le - lb;
+      const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
+      int* idx_out = idxbuf[(l + 1) & 1];
+      dir_kernel<T, D><<<dim3(nl, TH), 256, dir_smem, st>>>(Q, K, N_alloc, n, nodes, lb, M, inv_s, idx_in,
+                                                            NI, zvec, wvec, p->seed, power_iters,
+                                                            sample_factor);
+      project_kernel<T, D><<<dim3((n + 255) / 256, TH), 256, 0, st>>>(Q, K, N_alloc, n, nodes, lb, le,
+                                                                      inv_s, idx_in, NI, wvec, keys);
+      select_kernel<<<dim3(nl, TH), 1024, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
+      const int pch = (plan.level_max_size[l] + kPartChunk - 1) / kPartChunk;
+      part_count_kernel<<<dim3(pch, nl, TH), kPartThreads, 0, st>>>(nodes, lb, nl, n, pch, keys, sel, ccnt);
+      part_scatter_kernel<<<dim3(pch, nl, TH), kPartThreads, 0, st>>>(nodes, lb, nl, n, c, pch, keys, sel,
+                                                                      ccnt, idx_in, idx_out, out->perm_q,
+                                                                      out->perm_k, C * c);
+    }
+  }
+  centroid_kernel<T, D><<<dim3(C, TH), 256, 0, st>>>(Q, K, N_alloc, n, c, C, plan.levels, out->perm_q,
+                                                     out->perm_k, out->count_q, out->count_k, out->qbar,
+                                                     out->kbar);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool host_plan(int n, int c, TreePlan* plan) {
+  plan->n = n; plan->c = c; plan->C = (n + c - 1) / c;
+  plan->internal = plan->C - 1;
+  TreeNode* nodes = new TreeNode[plan->internal > 0 ? plan->internal : 1];
+  int lb[kMaxLevels + 1];
+  const int L = plan_tree(n, c, nodes, lb, kMaxLevels);
+  bool ok = true;
+  if (L >= kMaxLevels) ok = false;
+  plan->levels = L;
+  for (int l = 0; l <= L && l <= kMaxLevels; ++l) plan->level_begin[l] = lb[l];
+  for (int l = 0; l < L && l < kMaxLevels; ++l) {
+    int mx = 0;
+    for (int i = lb[l]; i < lb[l + 1]; ++i) mx = nodes[i].size > mx ? nodes[i].size : mx;
+    plan->level_max_size[l] = mx;
+  }
+  if (L > 0 && lb[L] != plan->internal) ok = false;
+  delete[] nodes;
+  return ok;
+}
+
+bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, ClusterWs* w) {
+  const size_t n = s->n_valid, d = s->d;
+  const size_t BH = (size_t)s->B * s->H, TH = 2 * BH;
+  const size_t NI = plan.internal > 0 ? plan.internal : 1;
+  w->BH = (int)BH; w->TH = (int)TH;
+  w->nch = (int)((n + kMetricChunk - 1) / kMetricChunk);
+  int pmax = 1;
+  size_t chunk_cnt = 1;
+  for (int l = 0; l < plan.levels; ++l) {
+    const int pch = (plan.level_max_size[l] + kPartChunk - 1) / kPartChunk;
+    const int nl = plan.level_begin[l + 1] - plan.level_begin[l];
+    pmax = pch > pmax ? pch : pmax;
+    const size_t need = (size_t)nl * pch;
+    chunk_cnt = need > chunk_cnt ? need : chunk_cnt;
+  }
+  w->pch_max = pmax;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+  w->nodes = take(NI * sizeof(TreeNode));
+  w->level_begin = take((kMaxLevels + 1) * sizeof(int));
+  w->M = take(TH * d * d * 8);
+  w->kmean = take(BH * d * 8);
+  w->colsum_part = take(BH * w->nch * d * 8);
+  w->met_part = take(BH * 2 * w->nch * d * d * 8);
+  w->inv_s = take(BH * n * 8);
+  w->idx0 = take(TH * n * 4);
+  w->idx1 = take(TH * n * 4);
+  w->keys = take(TH * n * 8);
+  w->zvec = take(TH * NI * d * 8);
+  w->wvec = take(TH * NI * d * 8);
+  w->sel = take(TH * NI * 16);
+  w->chunk_cnt = take(TH * chunk_cnt * 8);
+  w->total = o;
+  return true;
+}
+
+cudaError_t launch_cluster(const void* Q, const void* K, const ca_shape* s, const ca_cluster_params* p,
+                           const ca_clusters* out, const TreePlan& plan, const ClusterWs& L, char* ws,
+                           cudaStream_t st) {
+  if (s->dtype == CA_BF16) {
+    using T = __nv_bfloat16;
+    if (s->d == 64) return run_cluster<T, 64>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
+    return run_cluster<T, 128>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
+  }
+  using T = float;
+  if (s->d == 64) return run_cluster<T, 64>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
+  return run_cluster<T, 128>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
+}
+
+}  // namespace ca

@@ -1,0 +1,224 @@
+/*
+ * ca.h -- C ABI of libca, the B200 (sm_100a) ClusterAttention forward path.
+ *
+ * The operation is the forward pass of one bidirectional attention layer as
+ * described in "ClusterAttention: A training-free speedup of bidirectional
+ * attention" (arXiv 2608.26965), Section 1.1 (the four steps: cluster keys
+ * and queries, score and select key clusters per query cluster, attend over
+ * the selected clusters, compensate the unselected ones) and Section 3.1
+ * ("Overview": clustering, assignment, attention, per attention head).
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, except where a
+ *    name ends in _host. Nothing here allocates or frees device memory; work
+ *    that needs scratch takes a caller-provided workspace whose size is given
+ *    by the matching *_workspace_bytes() query.
+ *  - Q, K, V and O are head-major [B][H][N_alloc][d], rows contiguous, and
+ *    16-byte aligned. Rows n_valid..N_alloc-1 are padding: never read as
+ *    tokens; O's padding rows are written as 0.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Calls are asynchronous on it and never synchronise the host,
+ *    except ca_get_device_error() and the _host variant.
+ *  - Arguments are validated on the host before any launch; a call that
+ *    returns an error status has launched nothing and written nothing.
+ *  - Clustering, routing and the centroid-score arithmetic are fp64; the
+ *    attention computes in fp32 (fp32 inputs) or bf16 tensor-core products
+ *    with fp32 accumulation (bf16 inputs).
+ */
+#ifndef CA_H
+#define CA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CA_OK = 0,
+  CA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, k out of range, misaligned base */
+  CA_ERR_UNSUPPORTED = 2,   /* valid but not built: d not in {64,128}, c not in {64,128,256} ... */
+  CA_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_bytes() query */
+  CA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  CA_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (see ca_get_device_error) */
+} ca_status;
+
+typedef enum { CA_BF16 = 0, CA_FP32 = 1 } ca_dtype;
+
+/* Problem shape. C = ceil(n_valid / c) clusters for queries and for keys.
+ * Supported: d in {64, 128}; c in {64, 128, 256}; 1 <= n_valid <= N_alloc;
+ * dtype CA_BF16 or CA_FP32. */
+typedef struct {
+  int B, H;          /* batch, heads */
+  int N_alloc;       /* rows allocated per head */
+  int n_valid;       /* tokens per head (rows 0..n_valid-1) */
+  int d;             /* head dimension */
+  int c;             /* cluster size (queries and keys) */
+  int dtype;         /* ca_dtype of Q, K, V and O */
+} ca_shape;
+
+/* Clustering knobs (paper Section 3.2.1 "Basic recursive splitting"):
+ *  power_iters   p, power-iteration steps per split (0 -> default 8);
+ *  sample_factor a, sample size min(a d, |S|) per split (0 -> default 1);
+ *  transform     1 = interaction-aware transforms (Section 3.2.2), the default;
+ *                0 = split the raw vectors (the paper's ablation);
+ *  seed          counter-based generator seed for samples and warm starts. */
+typedef struct {
+  int power_iters;
+  int sample_factor;
+  int transform;
+  int reserved;
+  uint64_t seed;
+} ca_cluster_params;
+
+/* Clustering result, one entry per (b, h), C = ca_num_clusters(shape):
+ *  perm_q, perm_k  int32 [B][H][C*c]: slot a*c+j holds the original row of the
+ *                  j-th member of cluster a (ascending rows); -1 in pad slots.
+ *                  Every cluster holds c members except possibly the last,
+ *                  which holds n_valid - (C-1)*c (Section 3.1).
+ *  count_q, count_k int32 [B][H][C]: members per cluster.
+ *  qbar, kbar      fp64 [B][H][C][d]: centroids in the original, untransformed
+ *                  space (Section 3.3.1, eq. 18). */
+typedef struct {
+  int32_t* perm_q;
+  int32_t* perm_k;
+  int32_t* count_q;
+  int32_t* count_k;
+  double* qbar;
+  double* kbar;
+} ca_clusters;
+
+/* Routing result:
+ *  kept_idx  int32 [B][H][C][k]: the k key clusters kept by each query
+ *            cluster, ascending;
+ *  kept_bits uint32 [B][H][C][ceil(C/32)]: the same set as a bitmask
+ *            (bit b%32 of word b/32). */
+typedef struct {
+  int k;
+  int32_t* kept_idx;
+  uint32_t* kept_bits;
+} ca_routes;
+
+/* Number of clusters C = ceil(n_valid / c); -1 if the shape is invalid. Host only. */
+int ca_num_clusters(const ca_shape* shape);
+
+/* Validate a shape without launching anything. Host only. */
+ca_status ca_check_shape(const ca_shape* shape);
+
+/* Workspace sizes in bytes (0 if the shape is invalid). Host only, pure. */
+size_t ca_cluster_workspace_bytes(const ca_shape* shape);
+size_t ca_attend_workspace_bytes(const ca_shape* shape);
+size_t ca_dense_workspace_bytes(const ca_shape* shape);
+size_t ca_forward_workspace_bytes(const ca_shape* shape, int k);
+
+/*
+ * ca_cluster -- cluster the queries and the keys of every head.
+ * Paper Section 3.2 "Clustering": per head and separately for Q and K,
+ * the metric matrices M_q = Q^T Q / n (eq. 10-12) and M_k = K_c^T K_c / n
+ * (eq. 15, centred keys); keys are split in the space R_q k (eq. 14), queries
+ * in R_k q / |R_k q| (eq. 16); basic recursive splitting (PDDP): per set S,
+ * sample min(a d, |S|) vectors, estimate the first principal component by
+ * power iteration (warm-started from the mean of the parent's estimate and a
+ * random normal vector), project S, put the multiple of c closest to |S|/2
+ * below the split, recurse until every set but at most one holds c vectors.
+ * The metric is injected into the power iteration (Section 6.1), so no
+ * eigendecomposition is run. Ties between equal projections go by row index.
+ * Q, K: device [B][H][N_alloc][d] of shape->dtype. out: device buffers, see
+ * ca_clusters. workspace: device, >= ca_cluster_workspace_bytes(shape).
+ * Errors: CA_ERR_INVALID_ARG / CA_ERR_UNSUPPORTED / CA_ERR_WORKSPACE before
+ * any launch; CA_ERR_CUDA if a launch fails.
+ */
+ca_status ca_cluster(const void* Q, const void* K, const ca_shape* shape,
+                     const ca_cluster_params* params, const ca_clusters* out,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ca_route -- centroid scores and top-k selection.
+ * Paper Section 3.3.1 (score s_ab = qbar_a . kbar_b, eq. 18, computed in fp64)
+ * and Section 3.3.2 (keep the k best-scoring key clusters per query cluster).
+ * Exact top-k; equal scores go to the lower key-cluster index.
+ * centroids: device qbar/kbar (fp64) as produced by ca_cluster or supplied by
+ * the caller; only qbar and kbar are read. out: device kept_idx and kept_bits;
+ * out->k is k. 1 <= k <= C, C <= 8192.
+ */
+ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
+                   const ca_routes* out, void* stream);
+
+/*
+ * ca_attend -- block-sparse attention over the kept clusters with striped
+ * mean-compensation (SMC) of the excluded ones.
+ * Paper Section 1.2 (eq. 5-6) and Appendix A (eq. 21-22): for query i of
+ * cluster a,
+ *   o_i = ( sum_{b kept} sum_{j in b} e^{q_i.k_j/sqrt(d)} v_j
+ *         + sum_{b excluded} |b| e^{q_i.kbar_b/sqrt(d)} vbar_b ) / (same weights)
+ * with |b| the member count of key cluster b and vbar_b its mean value.
+ * compensate = 0 drops the second sum (plain block-sparse attention).
+ * Reads clusters->perm_q/perm_k/count_k/kbar and routes->kept_idx/kept_bits;
+ * vbar is computed here. O: device [B][H][N_alloc][d], written in original
+ * row order (padding rows 0). workspace >= ca_attend_workspace_bytes(shape).
+ */
+ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* shape,
+                    const ca_clusters* clusters, const ca_routes* routes, int compensate,
+                    void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ca_dense_attend -- plain softmax(Q K^T / sqrt(d)) V over the n_valid keys
+ * (paper eq. 1): the dense baseline the sparse path is measured against.
+ * Same layouts as ca_attend. workspace >= ca_dense_workspace_bytes(shape)
+ * (may be 0 bytes for shapes that need none).
+ */
+ca_status ca_dense_attend(const void* Q, const void* K, const void* V, const ca_shape* shape,
+                          void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ca_forward -- ca_cluster, ca_route and ca_attend in one call (compensation
+ * on when compensate != 0), with every intermediate carved from one
+ * workspace of ca_forward_workspace_bytes(shape, k) bytes. `clusters_out` and
+ * `routes_out` may be NULL; when given, their buffers receive the
+ * intermediates (otherwise they live in the workspace).
+ */
+ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape* shape,
+                     const ca_cluster_params* params, int k, int compensate, void* O,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ca_forward_host -- ca_forward on HOST buffers: copies Q, K, V (host, ideally
+ * pinned) into device staging carved from the workspace, runs the forward,
+ * copies O back to host, all on `stream`, and synchronises the stream before
+ * returning. workspace >= ca_forward_host_workspace_bytes(shape, k).
+ */
+size_t ca_forward_host_workspace_bytes(const ca_shape* shape, int k);
+ca_status ca_forward_host(const void* Q_host, const void* K_host, const void* V_host,
+                          const ca_shape* shape, const ca_cluster_params* params, int k,
+                          int compensate, void* O_host, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
+ * ca_get_device_error -- synchronise `stream` and report (then clear) the
+ * device-side error word of the current device: CA_ERR_TIMEOUT if a bounded
+ * wait inside a kernel gave up, CA_ERR_CUDA if the stream holds a CUDA error,
+ * CA_OK otherwise.
+ */
+ca_status ca_get_device_error(void* stream);
+
+/* Test hook: the iteration limit of every bounded device-side wait
+ * (mbarrier/TMA/TMEM). 0 restores the default. Host only; affects later launches. */
+void ca_set_wait_limit(uint64_t spins);
+
+/* Number of kernel launches one call makes for this shape (host only):
+ * stage 0 = ca_cluster, 1 = ca_route, 2 = ca_attend, 3 = ca_dense_attend;
+ * -1 for an invalid shape or stage. */
+int ca_launch_count(const ca_shape* shape, int stage);
+
+/* Human-readable name of a status. */
+const char* ca_status_string(ca_status status);
+
+/* Library version string. */
+const char* ca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CA_H */

@@ -1,0 +1,106 @@
+"""The C-ABI library loads, exports every entry point include/ca.h declares,
+and validates arguments on the host (no GPU needed: every call below is
+rejected before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import free_clustered_block_b200 as ca
+from oracle import ca_oracle as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from free_clustered_block_b200 import build
+    build.build()   # incremental: rebuilds only what changed
+    return ca.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "ca.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ca_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 15
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(ca.EXPORTED)
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in ca.version()
+    assert ca.status_string(ca.CA_ERR_WORKSPACE) == "CA_ERR_WORKSPACE"
+
+
+@pytest.mark.parametrize("n,c", [(1024, 64), (75600, 128), (65536, 128), (262144, 256), (100, 128), (1000, 64)])
+def test_num_clusters_matches_tree_rule(lib, n, c):
+    s = ca.make_shape(1, 2, n, n, 64, c, ca.CA_BF16)
+    assert ca.num_clusters(s) == orc.num_clusters(n, c)
+    assert ca.cluster_workspace_bytes(s) > 0
+    assert ca.attend_workspace_bytes(s) > 0
+
+
+def test_shape_validation(lib):
+    ok = ca.make_shape(1, 1, 1024, 1024, 64, 64, ca.CA_FP32)
+    assert lib.ca_check_shape(ctypes.byref(ok)) == ca.CA_OK
+    bad = [
+        (ca.make_shape(1, 1, 1024, 1024, 96, 64, ca.CA_FP32), ca.CA_ERR_UNSUPPORTED),   # d
+        (ca.make_shape(1, 1, 1024, 1024, 64, 100, ca.CA_FP32), ca.CA_ERR_UNSUPPORTED),  # c
+        (ca.make_shape(1, 1, 1000, 1024, 64, 64, ca.CA_FP32), ca.CA_ERR_INVALID_ARG),   # n > N_alloc
+        (ca.make_shape(0, 1, 1024, 1024, 64, 64, ca.CA_FP32), ca.CA_ERR_INVALID_ARG),   # B
+        (ca.make_shape(1, 1, 1024, 0, 64, 64, ca.CA_FP32), ca.CA_ERR_INVALID_ARG),      # empty
+        (ca.make_shape(1, 1, 1024, 1024, 64, 64, 7), ca.CA_ERR_INVALID_ARG),            # dtype
+    ]
+    for s, want in bad:
+        assert lib.ca_check_shape(ctypes.byref(s)) == want
+        assert lib.ca_num_clusters(ctypes.byref(s)) == -1
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_calls_are_rejected_before_launch(lib):
+    s = ca.make_shape(1, 1, 1024, 1024, 64, 64, ca.CA_FP32)
+    A = 0x10000
+    cl = ca.ca_clusters(A, A, A, A, A, A)
+    rt = ca.ca_routes(4, A, A)
+    need = ca.cluster_workspace_bytes(s)
+    # workspace too small
+    assert lib.ca_cluster(_fake(A), _fake(A), ctypes.byref(s), None, ctypes.byref(cl), _fake(A), need - 1,
+                          None) == ca.CA_ERR_WORKSPACE
+    # null input
+    assert lib.ca_cluster(None, _fake(A), ctypes.byref(s), None, ctypes.byref(cl), _fake(A), need,
+                          None) == ca.CA_ERR_INVALID_ARG
+    # misaligned input
+    assert lib.ca_cluster(_fake(A + 4), _fake(A), ctypes.byref(s), None, ctypes.byref(cl), _fake(A), need,
+                          None) == ca.CA_ERR_INVALID_ARG
+    # bad params
+    p = ca.make_params(power_iters=-1)
+    assert lib.ca_cluster(_fake(A), _fake(A), ctypes.byref(s), ctypes.byref(p), ctypes.byref(cl), _fake(A),
+                          need, None) == ca.CA_ERR_INVALID_ARG
+    # k out of range
+    for k in (0, 17):
+        r = ca.ca_routes(k, A, A)
+        assert lib.ca_route(ctypes.byref(s), ctypes.byref(cl), ctypes.byref(r), None) == ca.CA_ERR_INVALID_ARG
+    # attend: workspace too small, null O
+    aneed = ca.attend_workspace_bytes(s)
+    assert lib.ca_attend(_fake(A), _fake(A), _fake(A), ctypes.byref(s), ctypes.byref(cl), ctypes.byref(rt), 1,
+                         _fake(A), _fake(A), aneed - 1, None) == ca.CA_ERR_WORKSPACE
+    assert lib.ca_attend(_fake(A), _fake(A), _fake(A), ctypes.byref(s), ctypes.byref(cl), ctypes.byref(rt), 1,
+                         None, _fake(A), aneed, None) == ca.CA_ERR_INVALID_ARG
+    # forward: k out of range -> no workspace size
+    assert ca.forward_workspace_bytes(s, 0) == 0
+    assert ca.forward_workspace_bytes(s, 17) == 0
+    assert ca.forward_workspace_bytes(s, 4) > 0
+    # unsupported head dim anywhere
+    s96 = ca.make_shape(1, 1, 1024, 1024, 96, 64, ca.CA_FP32)
+    assert lib.ca_dense_attend(_fake(A), _fake(A), _fake(A), ctypes.byref(s96), _fake(A), None, 0,
+                               None) == ca.CA_ERR_UNSUPPORTED
