@@ -179,7 +179,8 @@ ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape*
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = launch_attend_prep(Q, K, V, s, cl, L, ws, cs);
   if (e == cudaSuccess) {
-    e = launch_attend_simt(Q, K, V, s, cl, rt, compensate, O, L, ws, cs);
+    if (s->dtype == CA_BF16) e = launch_attend_tc(s, cl, rt, compensate, O, L, ws, cs);
+    else e = launch_attend_simt(Q, K, V, s, cl, rt, compensate, O, L, ws, cs);
   }
   if (e == cudaSuccess) e = launch_zero_pad_rows(O, s, cs);
   return cuda_status(e);

@@ -1,12 +1,39 @@
-// Tensor-core (tcgen05) block-sparse attention: placeholder that routes to
-// the CUDA-core kernel until the sm_100a kernel lands.
+// Block-sparse attention with striped mean-compensation on the sm_100a
+// tensor cores (tcgen05, TMEM accumulators, TMA tiles).
+//
+// ClusterAttention paper, Section 3.1 (attention over the kept key clusters
+// of each query cluster, blocks of the permuted tokens) and Appendix A,
+// eq. 21-22 (every excluded key cluster b enters the softmax with logit
+// q . kbar_b / sqrt(d) + ln|b| and value vbar_b). The dense form (eq. 1) is
+// the same kernel with every key block kept and no compensation.
+//
+// One CTA handles one 128-row query tile of one head:
+//   warp 0      TMA producer: Q tile once, then a ring of stages holding
+//               (K, V) of a kept key block, (kbar_hi, kbar_lo) or
+//               (vbar_hi, vbar_lo) of a centroid block;
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
+//               S buffers; O += P_j V_j with P_j read from TMEM;
+//   warps 2..5  softmax: one thread per query row reads S_j from TMEM,
+//               applies the key mask / compensation bias, keeps a running
+//               max (rescaling O only when the max grows by more than 2^8),
+//               writes P_j as bf16 over S_j, and finally writes O / l to the
+//               query's original row.
+// Centroids are split into bf16 hi + lo parts and enter as two MMAs each.
+// Every wait is bounded: on a timeout the CTA sets the library's device error
+// word (CA_ERR_TIMEOUT), drains what it issued, frees TMEM and returns.
+#include <cuda.h>
+
 #include "ca_internal.cuh"
 
 namespace ca {
 
 __device__ unsigned int g_device_error = 0;
 static uint64_t g_wait_limit = 0;
-constexpr uint64_t kDefaultWaitLimit = 1ull << 26;
+// Bounded waits are timed with the global nanosecond timer.
+constexpr uint64_t kDefaultWaitLimit = 1000000000ull;   // 1 s
+// Drains (letting copies and MMAs already issued finish before the CTA
+// leaves) use their own bound, independent of the adjustable wait limit.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 uint64_t wait_limit() { return g_wait_limit ? g_wait_limit : kDefaultWaitLimit; }
 void set_wait_limit(uint64_t spins) { g_wait_limit = spins; }
@@ -23,14 +50,621 @@ cudaError_t device_error_read_clear(unsigned* out, cudaStream_t st) {
   return cudaStreamSynchronize(st);
 }
 
+namespace {
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* b) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+               : "memory");
+}
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u)
+      : "memory");
+}
+
+#define CA_TMEM_LD32(taddr, r)                                                                              \
+  asm volatile(                                                                                             \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                    \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),      \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),            \
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),          \
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),          \
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                               \
+      : "r"(taddr))
+
+#define CA_TMEM_ST32(taddr, r)                                                                              \
+  asm volatile(                                                                                             \
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16," \
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),                     \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),     \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),         \
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),        \
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                     \
+      : "memory")
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// AND of a predicate over the 128 softmax threads (named barrier 1); every
+// softmax thread executes the same sequence of these, so none can be left
+// waiting at the barrier.
+__device__ __forceinline__ bool group_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (canonical layouts of the
+// tcgen05 matrix descriptor: start >> 4 in bits 0-13, leading byte offset >> 4
+// in 16-29, stride byte offset >> 4 in 32-45, descriptor version 1 in 46-47,
+// swizzle mode 2 (128B) in 61-63).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, A K-major,
+// B K-major (b_mn = 0) or MN-major (b_mn = 1), N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void raise_timeout(volatile int* abort_flag) {
+  atomicCAS(&g_device_error, 0u, (unsigned)CA_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+// Bounded wait (limit in ns); false on timeout or when another role aborted.
+__device__ __noinline__ bool wait_bar(uint64_t* b, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(b, parity)) return true;
+    if ((i & 31) == 0) {
+      if (*abort_flag) return false;
+      if (now_ns() - t0 > limit_ns) { raise_timeout(abort_flag); return false; }
+    }
+  }
+}
+// Bounded wait used while draining: ignores the abort flag, fixed limit.
+__device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try(b, parity)) return;
+    if ((i & 31) == 31 && now_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel parameters
+// ---------------------------------------------------------------------------
+struct TcParams {
+  int C, c, k, Cpad, n_valid, N_alloc;
+  int tiles_per_cluster;      // c / 128 (>= 1)
+  int rows_per_tile;          // min(c, 128)
+  int compensate;
+  int dense;                  // 1: identity order, every key block kept
+  int dense_key_blocks;       // ceil(n_valid / KB) in dense mode
+  float scale_log2;           // log2(e) / sqrt(d)
+  const int32_t* perm_q;      // [BH][C*c]
+  const int32_t* count_k;     // [BH][C]
+  const int32_t* kept_idx;    // [BH][C][k]
+  const uint32_t* kept_bits;  // [BH][C][W]
+  const float* logcnt;        // [BH][Cpad] natural log of counts
+  __nv_bfloat16* O;           // [BH][N_alloc][D]
+  uint64_t wait_limit;
+};
+
+template <int D, int KB>
+struct TcCfg {
+  static constexpr int kStages = (D == 128 && KB == 128) ? 3 : 4;
+  static constexpr int kSub = D / 64;                                  // 64-column sub-tiles per row
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kBarOff = kQBytes + kStages * kStageBytes;
+  // + barriers, bias, alignment slack; at least 120 KB so that one CTA (and
+  // its 512 TMEM columns) occupies an SM.
+  static constexpr int kSmemCalc = kBarOff + 256 + KB * 4 + 1024;
+  static constexpr int kSmem = kSmemCalc > 120 * 1024 ? kSmemCalc : 120 * 1024;
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kOCol = 256;
+};
+
+// Items in load order: kept key sub-blocks (K,V), then per centroid block
+// (kbar hi, lo) and (vbar hi, vbar lo).
+struct Item { int kind; int row; };   // kind 0 KV, 1 KBAR, 2 VBAR
+
+template <int D, int KB>
+__global__ void __launch_bounds__(192, 1)
+tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khi,
+                 const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_vhi,
+                 const __grid_constant__ CUtensorMap tm_vlo, const TcParams p) {
+  using Cfg = TcCfg<D, KB>;
+  constexpr int NS = Cfg::kStages;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                         ~static_cast<uintptr_t>(1023));
+  unsigned char* sQ = smem;
+  unsigned char* sStage = smem + Cfg::kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
+  uint64_t* full = bars;              // [NS]
+  uint64_t* empty = bars + NS;        // [NS]
+  uint64_t* q_full = bars + 2 * NS;
+  uint64_t* s_full = q_full + 1;      // [2]
+  uint64_t* p_full = s_full + 2;      // [2]
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* drain = pv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* bias = reinterpret_cast<float*>(smem + Cfg::kBarOff + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int tile = blockIdx.x;
+  const int a = p.dense ? 0 : tile / p.tiles_per_cluster;          // query cluster
+  const int sub_tile = p.dense ? 0 : tile % p.tiles_per_cluster;
+  const int nsb = p.dense ? 1 : (p.c + KB - 1) / KB;               // key sub-blocks per cluster
+  const int J_kept = p.dense ? p.dense_key_blocks : p.k * nsb;
+  const int J_cent = (p.compensate && !p.dense) ? p.Cpad / KB : 0;
+  const int J = J_kept + J_cent;
+  const int n_items = J_kept + 2 * J_cent;
+  const int32_t* kept = p.dense ? nullptr : p.kept_idx + ((size_t)bh * p.C + a) * p.k;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(q_full, 1);
+    mbar_init(&s_full[0], 1); mbar_init(&s_full[1], 1);
+    mbar_init(&p_full[0], 128); mbar_init(&p_full[1], 128);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"(Cfg::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t limit = p.wait_limit;
+
+  auto item_of = [&](int i) -> Item {
+    Item it;
+    if (i < J_kept) {
+      it.kind = 0;
+      if (p.dense) it.row = i * KB;
+      else {
+        const int b = kept[i / nsb];
+        it.row = (bh * p.C + b) * p.c + (i % nsb) * KB;
+      }
+    } else {
+      const int t = i - J_kept;
+      it.kind = 1 + (t & 1);
+      it.row = bh * p.Cpad + (t >> 1) * KB;
+    }
+    return it;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      // Q tile
+      mbar_expect_tx(q_full, Cfg::kQBytes);
+      for (int s = 0; s < Cfg::kSub; ++s) {
+        if (p.dense) tma_3d(sQ + s * 128 * 128, &tm_q, q_full, s * 64, tile * 128, bh);
+        else tma_2d(sQ + s * 128 * 128, &tm_q, q_full, s * 64, (bh * p.C + a) * p.c + sub_tile * 128);
+      }
+      for (int i = 0; i < n_items && ok; ++i) {
+        const int s = i % NS, r = i / NS;
+        if (!wait_bar(&empty[s], (r & 1) ^ 1, limit, abort_flag)) { ok = false; break; }
+        const Item it = item_of(i);
+        unsigned char* dst = sStage + s * Cfg::kStageBytes;
+        mbar_expect_tx(&full[s], Cfg::kStageBytes);
+        const CUtensorMap* m0 = it.kind == 0 ? &tm_k : (it.kind == 1 ? &tm_khi : &tm_vhi);
+        const CUtensorMap* m1 = it.kind == 0 ? &tm_v : (it.kind == 1 ? &tm_klo : &tm_vlo);
+        for (int sb = 0; sb < Cfg::kSub; ++sb) {
+          if (p.dense) {
+            tma_3d(dst + sb * KB * 128, m0, &full[s], sb * 64, it.row, bh);
+            tma_3d(dst + Cfg::kTileBytes + sb * KB * 128, m1, &full[s], sb * 64, it.row, bh);
+          } else {
+            tma_2d(dst + sb * KB * 128, m0, &full[s], sb * 64, it.row);
+            tma_2d(dst + Cfg::kTileBytes + sb * KB * 128, m1, &full[s], sb * 64, it.row);
+          }
+        }
+        issued = i + 1;
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA leaves.
+        drain_bar(q_full, 0);
+        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) drain_bar(&full[i % NS], (i / NS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
+      constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
+      const uint32_t q_base = su32(sQ);
+      bool ok = wait_bar(q_full, 0, limit, abort_flag);
+      // consumption bookkeeping: item index of block j's QK and PV operands
+      auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
+      auto pv_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept) + 1; };
+      auto issue_qk = [&](int j) -> bool {
+        const int i = qk_item(j);
+        const int s = i % NS, r = i / NS;
+        if (!wait_bar(&full[s], r & 1, limit, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
+        const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 128);
+        const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
+        for (int mtx = 0; mtx < nmat; ++mtx) {
+          const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)((kk & 3) * 32);   // 16 bf16 along K inside the 128B row
+            const uint64_t ad = sdesc(q_base + (kk >> 2) * 128 * 128 + off, 16, 1024);
+            const uint64_t bd = sdesc(bbase + (kk >> 2) * KB * 128 + off, 16, 1024);
+            mma_ss(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(&s_full[j & 1]);
+        if (j >= J_kept) tc_commit(&empty[s]);   // kbar stage is free once S is computed
+        return true;
+      };
+      if (ok && J > 0) ok = issue_qk(0);
+      if (ok && J > 1) ok = issue_qk(1);
+      for (int j = 0; j < J && ok; ++j) {
+        if (!wait_bar(&p_full[j & 1], (j >> 1) & 1, limit, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const int i = pv_item(j);
+        const int s = i % NS, r = i / NS;
+        if (j >= J_kept) {
+          if (!wait_bar(&full[s], r & 1, limit, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+        }
+        const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
+        const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 128);
+        const int nmat = (j < J_kept) ? 1 : 2;
+        for (int mtx = 0; mtx < nmat; ++mtx) {
+          const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < KB / 16; ++kk) {
+            const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
+            mma_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(pv_done);
+        tc_commit(&empty[s]);
+        if (j + 2 < J) ok = issue_qk(j + 2);
+      }
+      // Drain: every MMA issued so far has completed once `drain` flips.
+      tc_commit(drain);
+      drain_bar(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int q4 = warp & 3;                  // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;           // row of the query tile
+    const int st = threadIdx.x - 64;          // 0..127 within the softmax group
+    const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    const uint32_t* kb_row = p.dense ? nullptr : p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
+    const float log2e = 1.4426950408889634f;
+    for (int j = 0; j < J; ++j) {
+      const bool cent = j >= J_kept;
+      if (cent) {
+        // per-column compensation bias of this centroid block (log2 units)
+        named_sync(1, 128);
+        if (st < KB) {
+          const int e = (j - J_kept) * KB + st;
+          float bv = -INFINITY;
+          if (e < p.C && !((kb_row[e >> 5] >> (e & 31)) & 1u)) bv = p.logcnt[(size_t)bh * p.Cpad + e] * log2e;
+          bias[st] = bv;
+        }
+        named_sync(1, 128);
+      }
+      int valid = KB;   // real keys in a kept block
+      if (!cent) {
+        if (p.dense) valid = min(KB, p.n_valid - j * KB);
+        else {
+          const int b = kept[j / nsb];
+          valid = min(KB, p.count_k[(size_t)bh * p.C + b] - (j % nsb) * KB);
+        }
+      }
+      ok = group_all(wait_bar(&s_full[j & 1], (j >> 1) & 1, limit, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[KB];
+#pragma unroll
+      for (int c0 = 0; c0 < KB; c0 += 32) CA_TMEM_LD32(lane_addr + (uint32_t)((j & 1) * 128 + c0), (&sv[c0]));
+      tmem_wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < KB; ++cc) {
+        float x = __uint_as_float(sv[cc]) * p.scale_log2;
+        if (cent) x += bias[cc];
+        else if (cc >= valid) x = -INFINITY;
+        sv[cc] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      // lazy rescale: move the reference max only when it grows by > 8 (x 256)
+      bool need = false;
+      float factor = 1.f;
+      if (mx > m_used + 8.f) {
+        factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - mx);
+        need = (j > 0);
+        m_used = mx;
+        l *= factor;
+      }
+      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
+      float rs = 0.f;
+      uint32_t pk[KB / 2];
+#pragma unroll
+      for (int cc = 0; cc < KB; cc += 2) {
+        const float p0 = ex2(__uint_as_float(sv[cc]) - mref);
+        const float p1 = ex2(__uint_as_float(sv[cc + 1]) - mref);
+        rs += p0 + p1;
+        pk[cc / 2] = pack_bf16(p0, p1);
+      }
+      l += rs;
+      // O correction (whole warp if any row needs it) once PV_{j-1} has finished.
+      bool wok = true;
+      if (__any_sync(0xffffffffu, need)) {
+        wok = __all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, limit, abort_flag));
+        if (wok) {
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
+            CA_TMEM_ST32(lane_addr + Cfg::kOCol + c0, ov);
+          }
+        }
+      }
+      ok = group_all(wok);
+      if (!ok) break;
+#pragma unroll
+      for (int c0 = 0; c0 < KB / 2; c0 += 32) CA_TMEM_ST32(lane_addr + (uint32_t)((j & 1) * 128 + c0), (&pk[c0]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[j & 1]);
+    }
+    // epilogue: O / l to the query's original row
+    if (ok && J > 0) ok = group_all(wait_bar(pv_done, (J - 1) & 1, limit, abort_flag));
+    if (ok && J > 0) {
+      tc_fence_after();
+      int orow;
+      if (p.dense) orow = tile * 128 + row < p.n_valid ? tile * 128 + row : -1;
+      else orow = row < p.rows_per_tile ? p.perm_q[(size_t)bh * p.C * p.c + (size_t)a * p.c + sub_tile * 128 + row]
+                                        : -1;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t ov[32];
+        CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);
+        tmem_wait_ld();
+        if (orow >= 0) {
+          uint4 w[4];
+          uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            wp[q] = pack_bf16(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
+          uint4* g = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) g[q] = w[q];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows][D], box {64, box_rows}, 128-byte swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, int D, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3-D bf16 map over [BH][N_alloc][D] exposing only rows < n_valid of each head.
+bool make_map_3d(CUtensorMap* m, const void* base, int BH, int N_alloc, int n_valid, int D, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n_valid, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N_alloc * D * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int KB>
+cudaError_t launch_tc(const CUtensorMap maps[7], const TcParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = TcCfg<D, KB>;
+  cudaError_t e = cudaFuncSetAttribute(tc_attend_kernel<D, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  tc_attend_kernel<D, KB><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                   maps[5], maps[6], p);
+  return cudaGetLastError();
+}
+
+cudaError_t dispatch(int D, int KB, const CUtensorMap maps[7], const TcParams& p, dim3 grid, cudaStream_t st) {
+  if (D == 64 && KB == 128) return launch_tc<64, 128>(maps, p, grid, st);
+  if (D == 64 && KB == 64) return launch_tc<64, 64>(maps, p, grid, st);
+  if (D == 128 && KB == 128) return launch_tc<128, 128>(maps, p, grid, st);
+  return launch_tc<128, 64>(maps, p, grid, st);
+}
+
+}  // namespace
+
 cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_routes* rt, int compensate,
                              void* O, const AttendWs& L, char* ws, cudaStream_t st) {
-  return cudaErrorNotSupported;
+  const int BH = s->B * s->H, D = s->d, c = s->c, C = L.C;
+  const int KB = c >= 128 ? 128 : 64;
+  const uint64_t slots = (uint64_t)BH * C * c;
+  CUtensorMap maps[7];
+  bool ok = make_map_2d(&maps[0], ws + L.qp, slots, D, 128) && make_map_2d(&maps[1], ws + L.kp, slots, D, KB) &&
+            make_map_2d(&maps[2], ws + L.vp, slots, D, KB) &&
+            make_map_2d(&maps[3], ws + L.kbar_hi, (uint64_t)BH * L.Cpad, D, KB) &&
+            make_map_2d(&maps[4], ws + L.kbar_lo, (uint64_t)BH * L.Cpad, D, KB) &&
+            make_map_2d(&maps[5], ws + L.vbar_hi, (uint64_t)BH * L.Cpad, D, KB) &&
+            make_map_2d(&maps[6], ws + L.vbar_lo, (uint64_t)BH * L.Cpad, D, KB);
+  if (!ok) return cudaErrorInvalidValue;
+  TcParams p;
+  p.C = C; p.c = c; p.k = rt->k; p.Cpad = L.Cpad; p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
+  p.tiles_per_cluster = c >= 128 ? c / 128 : 1;
+  p.rows_per_tile = c >= 128 ? 128 : c;
+  p.compensate = compensate;
+  p.dense = 0;
+  p.dense_key_blocks = 0;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  p.perm_q = cl->perm_q; p.count_k = cl->count_k; p.kept_idx = rt->kept_idx; p.kept_bits = rt->kept_bits;
+  p.logcnt = reinterpret_cast<const float*>(ws + L.logcnt);
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.wait_limit = wait_limit();
+  const dim3 grid(C * p.tiles_per_cluster, BH);
+  return dispatch(D, KB, maps, p, grid, st);
 }
 
 cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const ca_shape* s, void* O,
                             cudaStream_t st) {
-  return launch_dense_simt(Q, K, V, s, O, st);
+  const int BH = s->B * s->H, D = s->d;
+  constexpr int KB = 128;
+  CUtensorMap maps[7];
+  bool ok = make_map_3d(&maps[0], Q, BH, s->N_alloc, s->n_valid, D, 128) &&
+            make_map_3d(&maps[1], K, BH, s->N_alloc, s->n_valid, D, KB) &&
+            make_map_3d(&maps[2], V, BH, s->N_alloc, s->n_valid, D, KB);
+  if (!ok) return cudaErrorInvalidValue;
+  maps[3] = maps[1]; maps[4] = maps[1]; maps[5] = maps[2]; maps[6] = maps[2];
+  TcParams p{};
+  p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
+  p.tiles_per_cluster = 1; p.rows_per_tile = 128;
+  p.compensate = 0; p.dense = 1;
+  p.dense_key_blocks = (s->n_valid + KB - 1) / KB;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.wait_limit = wait_limit();
+  const dim3 grid((s->n_valid + 127) / 128, BH);
+  return dispatch(D, KB, maps, p, grid, st);
 }
 
 }  // namespace ca

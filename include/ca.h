@@ -202,9 +202,10 @@ ca_status ca_forward_host(const void* Q_host, const void* K_host, const void* V_
  */
 ca_status ca_get_device_error(void* stream);
 
-/* Test hook: the iteration limit of every bounded device-side wait
- * (mbarrier/TMA/TMEM). 0 restores the default. Host only; affects later launches. */
-void ca_set_wait_limit(uint64_t spins);
+/* Test hook: the time limit, in nanoseconds, of every bounded device-side
+ * wait (mbarrier waits on TMA copies and tensor-core work); 0 restores the
+ * default of 1 s. Host only; affects later launches. */
+void ca_set_wait_limit(uint64_t limit_ns);
 
 /* Number of kernel launches one call makes for this shape (host only):
  * stage 0 = ca_cluster, 1 = ca_route, 2 = ca_attend, 3 = ca_dense_attend;
