@@ -132,6 +132,13 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, 
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                     \
       : "memory")
 
+#define CA_TMEM_ST16(taddr, r)                                                                              \
+  asm volatile(                                                                                             \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" \
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),  \
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])           \
+      : "memory")
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ float ex2(float x) {
@@ -231,19 +238,22 @@ struct TcParams {
 
 template <int D, int KB>
 struct TcCfg {
-  static constexpr int kStages = (D == 128 && KB == 128) ? 3 : 4;
   static constexpr int kSub = D / 64;                                  // 64-column sub-tiles per row
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
   static constexpr int kStageBytes = 2 * kTileBytes;
+  // as many stages as fit in ~100 KB, so that two CTAs share an SM
+  static constexpr int kStagesFit = (100 * 1024 - kQBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 4 ? 4 : (kStagesFit < 2 ? 2 : kStagesFit);
   static constexpr int kBarOff = kQBytes + kStages * kStageBytes;
-  // + barriers, bias, alignment slack; at least 120 KB so that one CTA (and
-  // its 512 TMEM columns) occupies an SM.
-  static constexpr int kSmemCalc = kBarOff + 256 + KB * 4 + 1024;
-  static constexpr int kSmem = kSmemCalc > 120 * 1024 ? kSmemCalc : 120 * 1024;
-  static constexpr int kThreads = 192;
-  static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kOCol = 256;
+  static constexpr int kSmem = kBarOff + 256 + KB * 4 + 1024;          // + barriers, bias, alignment slack
+  static constexpr int kThreads = 160;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kSCol = 0;
+  static constexpr uint32_t kPCol = KB;                                // bf16 pairs: KB/2 columns
+  static constexpr uint32_t kOCol = (KB + KB / 2 + 31) / 32 * 32;
+  static_assert(kOCol + D <= kTmemCols, "S, P and O must fit in 256 TMEM columns");
+  static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
 };
 
 // Items in load order: kept key sub-blocks (K,V), then per centroid block
@@ -251,7 +261,7 @@ struct TcCfg {
 struct Item { int kind; int row; };   // kind 0 KV, 1 KBAR, 2 VBAR
 
 template <int D, int KB>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(160, 2)
 tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khi,
                  const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_vhi,
@@ -264,12 +274,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   unsigned char* sQ = smem;
   unsigned char* sStage = smem + Cfg::kQBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-  uint64_t* full = bars;              // [NS]
-  uint64_t* empty = bars + NS;        // [NS]
-  uint64_t* q_full = bars + 2 * NS;
-  uint64_t* s_full = q_full + 1;      // [2]
-  uint64_t* p_full = s_full + 2;      // [2]
-  uint64_t* pv_done = p_full + 2;
+  uint64_t* full = bars;              // [NS] stage loaded
+  uint64_t* empty = bars + NS;        // [NS] stage released
+  uint64_t* q_full = bars + 2 * NS;   // Q tile loaded
+  uint64_t* s_full = q_full + 1;      // S_j computed
+  uint64_t* s_free = s_full + 1;      // S_j read by every softmax thread
+  uint64_t* p_full = s_free + 1;      // P_j written
+  uint64_t* pv_done = p_full + 1;     // O += P_j V_j completed
   uint64_t* drain = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -290,8 +301,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1); mbar_init(&s_full[1], 1);
-    mbar_init(&p_full[0], 128); mbar_init(&p_full[1], 128);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -330,7 +342,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       int issued = 0;
       bool ok = true;
-      // Q tile
       mbar_expect_tx(q_full, Cfg::kQBytes);
       for (int s = 0; s < Cfg::kSub; ++s) {
         if (p.dense) tma_3d(sQ + s * 128 * 128, &tm_q, q_full, s * 64, tile * 128, bh);
@@ -361,14 +372,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) drain_bar(&full[i % NS], (i / NS) & 1);
       }
     }
-  } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 1) {
       constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
       const uint32_t q_base = su32(sQ);
       bool ok = wait_bar(q_full, 0, limit, abort_flag);
-      // consumption bookkeeping: item index of block j's QK and PV operands
+      // item index of block j's QK and PV operands
       auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
       auto pv_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept) + 1; };
       auto issue_qk = [&](int j) -> bool {
@@ -377,7 +387,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_bar(&full[s], r & 1, limit, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
-        const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 128);
         const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
         for (int mtx = 0; mtx < nmat; ++mtx) {
           const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
@@ -386,17 +395,23 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t off = (uint32_t)((kk & 3) * 32);   // 16 bf16 along K inside the 128B row
             const uint64_t ad = sdesc(q_base + (kk >> 2) * 128 * 128 + off, 16, 1024);
             const uint64_t bd = sdesc(bbase + (kk >> 2) * KB * 128 + off, 16, 1024);
-            mma_ss(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tmem + Cfg::kSCol, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc_commit(&s_full[j & 1]);
+        tc_commit(s_full);
         if (j >= J_kept) tc_commit(&empty[s]);   // kbar stage is free once S is computed
         return true;
       };
       if (ok && J > 0) ok = issue_qk(0);
-      if (ok && J > 1) ok = issue_qk(1);
       for (int j = 0; j < J && ok; ++j) {
-        if (!wait_bar(&p_full[j & 1], (j >> 1) & 1, limit, abort_flag)) { ok = false; break; }
+        if (j + 1 < J) {
+          // S_{j+1} may overwrite S_j once every softmax thread has read it.
+          if (!wait_bar(s_free, j & 1, limit, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          ok = issue_qk(j + 1);
+          if (!ok) break;
+        }
+        if (!wait_bar(p_full, j & 1, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int i = pv_item(j);
         const int s = i % NS, r = i / NS;
@@ -405,19 +420,18 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_fence_after();
         }
         const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
-        const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 128);
         const int nmat = (j < J_kept) ? 1 : 2;
         for (int mtx = 0; mtx < nmat; ++mtx) {
           const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < KB / 16; ++kk) {
             const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
-            mma_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + Cfg::kOCol, tmem + Cfg::kPCol + kk * 8, bd, id_pv,
+                   (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
         tc_commit(pv_done);
         tc_commit(&empty[s]);
-        if (j + 2 < J) ok = issue_qk(j + 2);
       }
       // Drain: every MMA issued so far has completed once `drain` flips.
       tc_commit(drain);
@@ -427,12 +441,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ------------------------------------------------------------- softmax
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;           // row of the query tile
-    const int st = threadIdx.x - 64;          // 0..127 within the softmax group
+    const int st = threadIdx.x - 32;          // 0..127 within the softmax group
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     const uint32_t* kb_row = p.dense ? nullptr : p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
     const float log2e = 1.4426950408889634f;
+    const float sc = p.scale_log2;
     for (int j = 0; j < J; ++j) {
       const bool cent = j >= J_kept;
       if (cent) {
@@ -454,22 +469,27 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           valid = min(KB, p.count_k[(size_t)bh * p.C + b] - (j % nsb) * KB);
         }
       }
-      ok = group_all(wait_bar(&s_full[j & 1], (j >> 1) & 1, limit, abort_flag));
+      ok = group_all(wait_bar(s_full, j & 1, limit, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[KB];
+      // pass 1: row max of the logits (log2 units), 32 columns at a time
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c0 = 0; c0 < KB; c0 += 32) CA_TMEM_LD32(lane_addr + (uint32_t)((j & 1) * 128 + c0), (&sv[c0]));
-      tmem_wait_ld();
-      float mx = -INFINITY;
+      for (int c0 = 0; c0 < KB; c0 += 32) {
+        float sv[32];
+        uint32_t* r = reinterpret_cast<uint32_t*>(sv);
+        CA_TMEM_LD32(lane_addr + Cfg::kSCol + (uint32_t)c0, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < KB; ++cc) {
-        float x = __uint_as_float(sv[cc]) * p.scale_log2;
-        if (cent) x += bias[cc];
-        else if (cc >= valid) x = -INFINITY;
-        sv[cc] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int q = 0; q < 32; ++q) {
+          float x = sv[q];
+          if (cent) x = fmaf(x, sc, bias[c0 + q]);
+          else if (c0 + q >= valid) x = -INFINITY;
+          m4[q & 3] = fmaxf(m4[q & 3], x);
+        }
       }
+      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      if (!cent) mx *= sc;
       // lazy rescale: move the reference max only when it grows by > 8 (x 256)
       bool need = false;
       float factor = 1.f;
@@ -480,40 +500,55 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         l *= factor;
       }
       const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
-      uint32_t pk[KB / 2];
-#pragma unroll
-      for (int cc = 0; cc < KB; cc += 2) {
-        const float p0 = ex2(__uint_as_float(sv[cc]) - mref);
-        const float p1 = ex2(__uint_as_float(sv[cc + 1]) - mref);
-        rs += p0 + p1;
-        pk[cc / 2] = pack_bf16(p0, p1);
-      }
-      l += rs;
-      // O correction (whole warp if any row needs it) once PV_{j-1} has finished.
+      // P_{j-1} and O are free once PV_{j-1} has completed.
       bool wok = true;
-      if (__any_sync(0xffffffffu, need)) {
-        wok = __all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, limit, abort_flag));
-        if (wok) {
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
-            CA_TMEM_ST32(lane_addr + Cfg::kOCol + c0, ov);
-          }
-        }
-      }
+      if (j > 0) wok = wait_bar(pv_done, (j - 1) & 1, limit, abort_flag);
       ok = group_all(wok);
       if (!ok) break;
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-      for (int c0 = 0; c0 < KB / 2; c0 += 32) CA_TMEM_ST32(lane_addr + (uint32_t)((j & 1) * 128 + c0), (&pk[c0]));
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t ov[32];
+          CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
+          CA_TMEM_ST32(lane_addr + Cfg::kOCol + c0, ov);
+        }
+      }
+      // pass 2: P = 2^(x - mref) as bf16 pairs, row sum in fp32
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float nb = -mref;
+#pragma unroll
+      for (int c0 = 0; c0 < KB; c0 += 32) {
+        float sv[32];
+        uint32_t* r = reinterpret_cast<uint32_t*>(sv);
+        CA_TMEM_LD32(lane_addr + Cfg::kSCol + (uint32_t)c0, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float x0 = sv[2 * q], x1 = sv[2 * q + 1];
+          float p0, p1;
+          if (cent) {
+            p0 = ex2(fmaf(x0, sc, bias[c0 + 2 * q]) + nb);
+            p1 = ex2(fmaf(x1, sc, bias[c0 + 2 * q + 1]) + nb);
+          } else {
+            p0 = (c0 + 2 * q < valid) ? ex2(fmaf(x0, sc, nb)) : 0.f;
+            p1 = (c0 + 2 * q + 1 < valid) ? ex2(fmaf(x1, sc, nb)) : 0.f;
+          }
+          rs4[q & 3] += p0 + p1;
+          pk[q] = pack_bf16(p0, p1);
+        }
+        CA_TMEM_ST16(lane_addr + Cfg::kPCol + (uint32_t)(c0 / 2), pk);
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);                   // S_j fully read: the MMA may compute S_{j+1}
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(p_full);
     }
     // epilogue: O / l to the query's original row
     if (ok && J > 0) ok = group_all(wait_bar(pv_done, (J - 1) & 1, limit, abort_flag));
@@ -607,10 +642,13 @@ cudaError_t launch_tc(const CUtensorMap maps[7], const TcParams& p, dim3 grid, c
   return cudaGetLastError();
 }
 
+// Key-block width: 128 keys for d = 64; 64 keys for d = 128 (and for c = 64),
+// so that S, P and O fit in 256 TMEM columns.
+int key_block(int D, int c) { return (D == 64 && c >= 128) ? 128 : 64; }
+
 cudaError_t dispatch(int D, int KB, const CUtensorMap maps[7], const TcParams& p, dim3 grid, cudaStream_t st) {
   if (D == 64 && KB == 128) return launch_tc<64, 128>(maps, p, grid, st);
-  if (D == 64 && KB == 64) return launch_tc<64, 64>(maps, p, grid, st);
-  if (D == 128 && KB == 128) return launch_tc<128, 128>(maps, p, grid, st);
+  if (D == 64) return launch_tc<64, 64>(maps, p, grid, st);
   return launch_tc<128, 64>(maps, p, grid, st);
 }
 
@@ -619,7 +657,7 @@ cudaError_t dispatch(int D, int KB, const CUtensorMap maps[7], const TcParams& p
 cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_routes* rt, int compensate,
                              void* O, const AttendWs& L, char* ws, cudaStream_t st) {
   const int BH = s->B * s->H, D = s->d, c = s->c, C = L.C;
-  const int KB = c >= 128 ? 128 : 64;
+  const int KB = key_block(D, c);
   const uint64_t slots = (uint64_t)BH * C * c;
   CUtensorMap maps[7];
   bool ok = make_map_2d(&maps[0], ws + L.qp, slots, D, 128) && make_map_2d(&maps[1], ws + L.kp, slots, D, KB) &&
@@ -648,7 +686,7 @@ cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_
 cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const ca_shape* s, void* O,
                             cudaStream_t st) {
   const int BH = s->B * s->H, D = s->d;
-  constexpr int KB = 128;
+  const int KB = key_block(D, 128);
   CUtensorMap maps[7];
   bool ok = make_map_3d(&maps[0], Q, BH, s->N_alloc, s->n_valid, D, 128) &&
             make_map_3d(&maps[1], K, BH, s->N_alloc, s->n_valid, D, KB) &&
@@ -660,6 +698,7 @@ cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const c
   p.tiles_per_cluster = 1; p.rows_per_tile = 128;
   p.compensate = 0; p.dense = 1;
   p.dense_key_blocks = (s->n_valid + KB - 1) / KB;
+  p.c = KB;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.wait_limit = wait_limit();
