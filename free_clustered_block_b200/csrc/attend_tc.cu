@@ -242,17 +242,19 @@ struct TcCfg {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
   static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kOnesBytes = 16 * KB * 2;                       // B operand of the row sums
   // as many stages as fit in ~100 KB, so that two CTAs share an SM
-  static constexpr int kStagesFit = (100 * 1024 - kQBytes) / kStageBytes;
+  static constexpr int kStagesFit = (100 * 1024 - kQBytes - kOnesBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 4 ? 4 : (kStagesFit < 2 ? 2 : kStagesFit);
-  static constexpr int kBarOff = kQBytes + kStages * kStageBytes;
+  static constexpr int kOnesOff = kQBytes + kStages * kStageBytes;
+  static constexpr int kBarOff = kOnesOff + kOnesBytes;
   static constexpr int kSmem = kBarOff + 256 + KB * 4 + 1024;          // + barriers, bias, alignment slack
   static constexpr int kThreads = 160;
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kSCol = 0;
-  static constexpr uint32_t kPCol = KB;                                // bf16 pairs: KB/2 columns
-  static constexpr uint32_t kOCol = (KB + KB / 2 + 31) / 32 * 32;
-  static_assert(kOCol + D <= kTmemCols, "S, P and O must fit in 256 TMEM columns");
+  static constexpr uint32_t kSCol = 0;       // S_j (fp32, KB columns); P_j (bf16 pairs) overwrites its front half
+  static constexpr uint32_t kOCol = KB;      // O (fp32, D columns)
+  static constexpr uint32_t kLCol = KB + D;  // row sums of P (fp32, 16 columns, column 0 used)
+  static_assert(kLCol + 16 <= kTmemCols, "S/P, O and the row sums must fit in 256 TMEM columns");
   static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
 };
 
@@ -273,13 +275,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                          ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = smem;
   unsigned char* sStage = smem + Cfg::kQBytes;
+  unsigned char* sOnes = smem + Cfg::kOnesOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* full = bars;              // [NS] stage loaded
   uint64_t* empty = bars + NS;        // [NS] stage released
   uint64_t* q_full = bars + 2 * NS;   // Q tile loaded
-  uint64_t* s_full = q_full + 1;      // S_j computed
-  uint64_t* s_free = s_full + 1;      // S_j read by every softmax thread
-  uint64_t* p_full = s_free + 1;      // P_j written
+  uint64_t* s_full = q_full + 1;      // S_j computed (and every earlier MMA finished)
+  uint64_t* p_full = s_full + 1;      // P_j written
   uint64_t* pv_done = p_full + 1;     // O += P_j V_j completed
   uint64_t* drain = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -298,11 +300,15 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int n_items = J_kept + 2 * J_cent;
   const int32_t* kept = p.dense ? nullptr : p.kept_idx + ((size_t)bh * p.C + a) * p.k;
 
+  // bf16 ones (0x3F80): the B operand that turns P into its row sums. Every
+  // element is equal, so the swizzled layout needs no address arithmetic.
+  for (int i = threadIdx.x; i < Cfg::kOnesBytes / 4; i += Cfg::kThreads)
+    reinterpret_cast<uint32_t*>(sOnes)[i] = 0x3F803F80u;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> tensor-core reads
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
@@ -376,7 +382,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 1) {
       constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
+      constexpr uint32_t id_l = idesc_bf16(128, 16, 0);
       const uint32_t q_base = su32(sQ);
+      const uint32_t ones = su32(sOnes);
       bool ok = wait_bar(q_full, 0, limit, abort_flag);
       // item index of block j's QK and PV operands
       auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
@@ -398,19 +406,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_ss(tmem + Cfg::kSCol, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
+        // Commits track every earlier MMA of this thread too: when s_full
+        // flips, PV_{j-1} (and its reads of P_{j-1}) has completed as well.
         tc_commit(s_full);
         if (j >= J_kept) tc_commit(&empty[s]);   // kbar stage is free once S is computed
         return true;
       };
       if (ok && J > 0) ok = issue_qk(0);
       for (int j = 0; j < J && ok; ++j) {
-        if (j + 1 < J) {
-          // S_{j+1} may overwrite S_j once every softmax thread has read it.
-          if (!wait_bar(s_free, j & 1, limit, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          ok = issue_qk(j + 1);
-          if (!ok) break;
-        }
         if (!wait_bar(p_full, j & 1, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int i = pv_item(j);
@@ -426,12 +429,23 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
           for (int kk = 0; kk < KB / 16; ++kk) {
             const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
-            mma_ts(tmem + Cfg::kOCol, tmem + Cfg::kPCol + kk * 8, bd, id_pv,
+            mma_ts(tmem + Cfg::kOCol, tmem + Cfg::kSCol + kk * 8, bd, id_pv,
                    (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
+        // row sums: L += P_j 1 (the bf16 P the numerator used)
+#pragma unroll
+        for (int kk = 0; kk < KB / 16; ++kk) {
+          const uint64_t bd = sdesc(ones + (kk >> 2) * 16 * 128 + (kk & 3) * 32, 16, 1024);
+          mma_ts(tmem + Cfg::kLCol, tmem + Cfg::kSCol + kk * 8, bd, id_l, (j > 0 || kk > 0) ? 1u : 0u);
+        }
         tc_commit(pv_done);
         tc_commit(&empty[s]);
+        // S_{j+1} overwrites P_j: ordered after PV_j in this thread's MMA stream.
+        if (j + 1 < J) {
+          ok = issue_qk(j + 1);
+          if (!ok) break;
+        }
       }
       // Drain: every MMA issued so far has completed once `drain` flips.
       tc_commit(drain);
@@ -443,7 +457,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int row = q4 * 32 + lane;           // row of the query tile
     const int st = threadIdx.x - 32;          // 0..127 within the softmax group
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY;
     bool ok = true;
     const uint32_t* kb_row = p.dense ? nullptr : p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
     const float log2e = 1.4426950408889634f;
@@ -472,7 +486,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       ok = group_all(wait_bar(s_full, j & 1, limit, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: row max of the logits (log2 units), 32 columns at a time
+      const int mode = cent ? 2 : (valid < KB ? 1 : 0);   // 0 full block, 1 partial block, 2 centroids
+      // pass 1: row max of the logits, 32 columns at a time
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c0 = 0; c0 < KB; c0 += 32) {
@@ -480,16 +495,19 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t* r = reinterpret_cast<uint32_t*>(sv);
         CA_TMEM_LD32(lane_addr + Cfg::kSCol + (uint32_t)c0, r);
         tmem_wait_ld();
+        if (mode == 0) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          float x = sv[q];
-          if (cent) x = fmaf(x, sc, bias[c0 + q]);
-          else if (c0 + q >= valid) x = -INFINITY;
-          m4[q & 3] = fmaxf(m4[q & 3], x);
+          for (int q = 0; q < 32; ++q) m4[q & 3] = fmaxf(m4[q & 3], sv[q]);
+        } else if (mode == 1) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) if (c0 + q < valid) m4[q & 3] = fmaxf(m4[q & 3], sv[q]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) m4[q & 3] = fmaxf(m4[q & 3], fmaf(sv[q], sc, bias[c0 + q]));
         }
       }
       float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      if (!cent) mx *= sc;
+      if (mode != 2) mx *= sc;             // log2 units
       // lazy rescale: move the reference max only when it grows by > 8 (x 256)
       bool need = false;
       float factor = 1.f;
@@ -497,29 +515,21 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - mx);
         need = (j > 0);
         m_used = mx;
-        l *= factor;
       }
-      const float mref = (m_used == -INFINITY) ? 0.f : m_used;
-      // P_{j-1} and O are free once PV_{j-1} has completed.
-      bool wok = true;
-      if (j > 0) wok = wait_bar(pv_done, (j - 1) & 1, limit, abort_flag);
-      ok = group_all(wok);
-      if (!ok) break;
-      tc_fence_after();
+      const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
+      // O and the row sums are stable: PV_{j-1} finished before s_full flipped.
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < D + 32; c0 += 32) {
           uint32_t ov[32];
-          CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);
+          CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);   // last chunk: 16 row-sum columns + 16 spare
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
           CA_TMEM_ST32(lane_addr + Cfg::kOCol + c0, ov);
         }
       }
-      // pass 2: P = 2^(x - mref) as bf16 pairs, row sum in fp32
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-      const float nb = -mref;
+      // pass 2: P = 2^(x - m) as bf16 pairs written over the front of S
 #pragma unroll
       for (int c0 = 0; c0 < KB; c0 += 32) {
         float sv[32];
@@ -527,25 +537,26 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         CA_TMEM_LD32(lane_addr + Cfg::kSCol + (uint32_t)c0, r);
         tmem_wait_ld();
         uint32_t pk[16];
+        if (mode == 0) {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          float x0 = sv[2 * q], x1 = sv[2 * q + 1];
-          float p0, p1;
-          if (cent) {
-            p0 = ex2(fmaf(x0, sc, bias[c0 + 2 * q]) + nb);
-            p1 = ex2(fmaf(x1, sc, bias[c0 + 2 * q + 1]) + nb);
-          } else {
-            p0 = (c0 + 2 * q < valid) ? ex2(fmaf(x0, sc, nb)) : 0.f;
-            p1 = (c0 + 2 * q + 1 < valid) ? ex2(fmaf(x1, sc, nb)) : 0.f;
+          for (int q = 0; q < 16; ++q)
+            pk[q] = pack_bf16(ex2(fmaf(sv[2 * q], sc, nb)), ex2(fmaf(sv[2 * q + 1], sc, nb)));
+        } else if (mode == 1) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float p0 = (c0 + 2 * q < valid) ? ex2(fmaf(sv[2 * q], sc, nb)) : 0.f;
+            const float p1 = (c0 + 2 * q + 1 < valid) ? ex2(fmaf(sv[2 * q + 1], sc, nb)) : 0.f;
+            pk[q] = pack_bf16(p0, p1);
           }
-          rs4[q & 3] += p0 + p1;
-          pk[q] = pack_bf16(p0, p1);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            pk[q] = pack_bf16(ex2(fmaf(sv[2 * q], sc, bias[c0 + 2 * q]) + nb),
+                              ex2(fmaf(sv[2 * q + 1], sc, bias[c0 + 2 * q + 1]) + nb));
         }
-        CA_TMEM_ST16(lane_addr + Cfg::kPCol + (uint32_t)(c0 / 2), pk);
+        // columns [c0/2, c0/2+16) of S were read by this or an earlier chunk
+        CA_TMEM_ST16(lane_addr + Cfg::kSCol + (uint32_t)(c0 / 2), pk);
       }
-      tc_fence_before();
-      mbar_arrive(s_free);                   // S_j fully read: the MMA may compute S_{j+1}
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -558,6 +569,10 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (p.dense) orow = tile * 128 + row < p.n_valid ? tile * 128 + row : -1;
       else orow = row < p.rows_per_tile ? p.perm_q[(size_t)bh * p.C * p.c + (size_t)a * p.c + sub_tile * 128 + row]
                                         : -1;
+      uint32_t lv[32];
+      CA_TMEM_LD32(lane_addr + Cfg::kLCol, lv);
+      tmem_wait_ld();
+      const float l = __uint_as_float(lv[0]);
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D;
 #pragma unroll
