@@ -153,15 +153,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// AND of a predicate over the 128 softmax threads (named barrier 1); every
+// AND of a predicate over the n softmax threads (named barrier 1); every
 // softmax thread executes the same sequence of these, so none can be left
 // waiting at the barrier.
-__device__ __forceinline__ bool group_all(bool v) {
+__device__ __forceinline__ bool group_all_n(bool v, int n) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "r"(n)
       : "memory");
   return r != 0;
 }
@@ -243,19 +243,27 @@ struct TcCfg {
   static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kOnesBytes = 16 * KB * 2;                       // B operand of the row sums
-  // as many stages as fit in ~100 KB, so that two CTAs share an SM
-  static constexpr int kStagesFit = (100 * 1024 - kQBytes - kOnesBytes) / kStageBytes;
+  static constexpr int kMaxKeptSmem = 1024;                            // kept list staged in shared memory
+  static constexpr int kStagesFit = (200 * 1024 - kQBytes - kOnesBytes - 2 * kMaxKeptSmem * 4) / kStageBytes;
   static constexpr int kStages = kStagesFit > 4 ? 4 : (kStagesFit < 2 ? 2 : kStagesFit);
   static constexpr int kOnesOff = kQBytes + kStages * kStageBytes;
   static constexpr int kBarOff = kOnesOff + kOnesBytes;
-  static constexpr int kSmem = kBarOff + 256 + KB * 4 + 1024;          // + barriers, bias, alignment slack
-  static constexpr int kThreads = 160;
-  static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kSCol = 0;       // S_j (fp32, KB columns); P_j (bf16 pairs) overwrites its front half
-  static constexpr uint32_t kOCol = KB;      // O (fp32, D columns)
-  static constexpr uint32_t kLCol = KB + D;  // row sums of P (fp32, 16 columns, column 0 used)
-  static_assert(kLCol + 16 <= kTmemCols, "S/P, O and the row sums must fit in 256 TMEM columns");
-  static_assert(kSmem <= 113 * 1024, "two CTAs per SM");
+  static constexpr int kBiasOff = kBarOff + 256;
+  static constexpr int kRedOff = kBiasOff + KB * 4;                    // row-max exchange [2][128]
+  static constexpr int kKeptOff = kRedOff + 2 * 128 * 4;
+  // + alignment slack; at least 116 KB so that one CTA (and its 512 TMEM
+  // columns) holds an SM
+  static constexpr int kSmemCalc = kKeptOff + 2 * kMaxKeptSmem * 4 + 1024;
+  static constexpr int kSmem = kSmemCalc > 116 * 1024 ? kSmemCalc : 116 * 1024;
+  static constexpr int kSoftmaxThreads = 256;                          // 8 warps, two threads per row
+  static constexpr int kThreads = 64 + kSoftmaxThreads;                // + producer warp + MMA warp
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kSCol = 0;        // S buffers at 0 and KB; P_j (bf16 pairs) over the front half
+  static constexpr uint32_t kOCol = 2 * KB;   // O (fp32, D columns)
+  static constexpr uint32_t kLCol = 2 * KB + D;  // row sums of P (fp32, 16 columns, column 0 used)
+  static constexpr int kHalf = KB / 2;        // columns of S per softmax thread
+  static_assert(kLCol + 32 <= kTmemCols, "S buffers, O and the row sums must fit in TMEM");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 // Items in load order: kept key sub-blocks (K,V), then per centroid block
@@ -263,13 +271,14 @@ struct TcCfg {
 struct Item { int kind; int row; };   // kind 0 KV, 1 KBAR, 2 VBAR
 
 template <int D, int KB>
-__global__ void __launch_bounds__(160, 2)
+__global__ void __launch_bounds__(TcCfg<D, KB>::kThreads, 1)
 tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khi,
                  const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_vhi,
                  const __grid_constant__ CUtensorMap tm_vlo, const TcParams p) {
   using Cfg = TcCfg<D, KB>;
   constexpr int NS = Cfg::kStages;
+  constexpr int HC = Cfg::kHalf;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -280,13 +289,16 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* full = bars;              // [NS] stage loaded
   uint64_t* empty = bars + NS;        // [NS] stage released
   uint64_t* q_full = bars + 2 * NS;   // Q tile loaded
-  uint64_t* s_full = q_full + 1;      // S_j computed (and every earlier MMA finished)
-  uint64_t* p_full = s_full + 1;      // P_j written
-  uint64_t* pv_done = p_full + 1;     // O += P_j V_j completed
+  uint64_t* s_full = q_full + 1;      // [2] S_j computed in buffer j&1
+  uint64_t* p_full = s_full + 2;      // [2] P_j written in buffer j&1
+  uint64_t* pv_done = p_full + 2;     // O += P_j V_j completed
   uint64_t* drain = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* bias = reinterpret_cast<float*>(smem + Cfg::kBarOff + 256);
+  float* bias = reinterpret_cast<float*>(smem + Cfg::kBiasOff);
+  float* red = reinterpret_cast<float*>(smem + Cfg::kRedOff);
+  int32_t* kept_s = reinterpret_cast<int32_t*>(smem + Cfg::kKeptOff);        // kept key clusters
+  int32_t* kcnt_s = kept_s + Cfg::kMaxKeptSmem;                               // their member counts
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
@@ -298,7 +310,16 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int J_cent = (p.compensate && !p.dense) ? p.Cpad / KB : 0;
   const int J = J_kept + J_cent;
   const int n_items = J_kept + 2 * J_cent;
-  const int32_t* kept = p.dense ? nullptr : p.kept_idx + ((size_t)bh * p.C + a) * p.k;
+  const int32_t* kept_g = p.dense ? nullptr : p.kept_idx + ((size_t)bh * p.C + a) * p.k;
+  const bool kept_in_smem = !p.dense && p.k <= Cfg::kMaxKeptSmem;
+  if (kept_in_smem) {
+    for (int i = threadIdx.x; i < p.k; i += Cfg::kThreads) {
+      const int b = kept_g[i];
+      kept_s[i] = b;
+      kcnt_s[i] = p.count_k[(size_t)bh * p.C + b];
+    }
+  }
+  const int32_t* kept = kept_in_smem ? kept_s : kept_g;
 
   // bf16 ones (0x3F80): the B operand that turns P into its row sums. Every
   // element is equal, so the swizzled layout needs no address arithmetic.
@@ -308,8 +329,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(q_full, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(&s_full[0], 1); mbar_init(&s_full[1], 1);
+    mbar_init(&p_full[0], Cfg::kSoftmaxThreads); mbar_init(&p_full[1], Cfg::kSoftmaxThreads);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -355,8 +376,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       for (int i = 0; i < n_items && ok; ++i) {
         const int s = i % NS, r = i / NS;
-        if (!wait_bar(&empty[s], (r & 1) ^ 1, limit, abort_flag)) { ok = false; break; }
         const Item it = item_of(i);
+        if (!wait_bar(&empty[s], (r & 1) ^ 1, limit, abort_flag)) { ok = false; break; }
         unsigned char* dst = sStage + s * Cfg::kStageBytes;
         mbar_expect_tx(&full[s], Cfg::kStageBytes);
         const CUtensorMap* m0 = it.kind == 0 ? &tm_k : (it.kind == 1 ? &tm_khi : &tm_vhi);
@@ -378,8 +399,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) drain_bar(&full[i % NS], (i / NS) & 1);
       }
     }
+  } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 1) {
+    if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
       constexpr uint32_t id_l = idesc_bf16(128, 16, 0);
@@ -395,6 +417,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_bar(&full[s], r & 1, limit, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
+        const uint32_t d_tmem = tmem + Cfg::kSCol + (uint32_t)((j & 1) * KB);
         const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
         for (int mtx = 0; mtx < nmat; ++mtx) {
           const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
@@ -403,18 +426,19 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t off = (uint32_t)((kk & 3) * 32);   // 16 bf16 along K inside the 128B row
             const uint64_t ad = sdesc(q_base + (kk >> 2) * 128 * 128 + off, 16, 1024);
             const uint64_t bd = sdesc(bbase + (kk >> 2) * KB * 128 + off, 16, 1024);
-            mma_ss(tmem + Cfg::kSCol, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        // Commits track every earlier MMA of this thread too: when s_full
-        // flips, PV_{j-1} (and its reads of P_{j-1}) has completed as well.
-        tc_commit(s_full);
+        // Commits track every earlier MMA of this thread too: when s_full[b]
+        // flips for S_j, PV_{j-2} (the last reader of that buffer) is done.
+        tc_commit(&s_full[j & 1]);
         if (j >= J_kept) tc_commit(&empty[s]);   // kbar stage is free once S is computed
         return true;
       };
       if (ok && J > 0) ok = issue_qk(0);
+      if (ok && J > 1) ok = issue_qk(1);
       for (int j = 0; j < J && ok; ++j) {
-        if (!wait_bar(p_full, j & 1, limit, abort_flag)) { ok = false; break; }
+        if (!wait_bar(&p_full[j & 1], (j >> 1) & 1, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int i = pv_item(j);
         const int s = i % NS, r = i / NS;
@@ -423,27 +447,27 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_fence_after();
         }
         const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
+        const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j & 1) * KB);
         const int nmat = (j < J_kept) ? 1 : 2;
         for (int mtx = 0; mtx < nmat; ++mtx) {
           const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < KB / 16; ++kk) {
             const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
-            mma_ts(tmem + Cfg::kOCol, tmem + Cfg::kSCol + kk * 8, bd, id_pv,
-                   (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
         // row sums: L += P_j 1 (the bf16 P the numerator used)
 #pragma unroll
         for (int kk = 0; kk < KB / 16; ++kk) {
           const uint64_t bd = sdesc(ones + (kk >> 2) * 16 * 128 + (kk & 3) * 32, 16, 1024);
-          mma_ts(tmem + Cfg::kLCol, tmem + Cfg::kSCol + kk * 8, bd, id_l, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + Cfg::kLCol, p_tmem + kk * 8, bd, id_l, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(pv_done);
         tc_commit(&empty[s]);
-        // S_{j+1} overwrites P_j: ordered after PV_j in this thread's MMA stream.
-        if (j + 1 < J) {
-          ok = issue_qk(j + 1);
+        // S_{j+2} overwrites P_j: ordered after PV_j in this thread's MMA stream.
+        if (j + 2 < J) {
+          ok = issue_qk(j + 2);
           if (!ok) break;
         }
       }
@@ -453,61 +477,77 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------- softmax
+    const int st = threadIdx.x - 64;          // 0..255 within the softmax group
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
+    const int half = st >> 7;                 // which half of the columns of its row
     const int row = q4 * 32 + lane;           // row of the query tile
-    const int st = threadIdx.x - 32;          // 0..127 within the softmax group
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     float m_used = -INFINITY;
     bool ok = true;
     const uint32_t* kb_row = p.dense ? nullptr : p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
     const float log2e = 1.4426950408889634f;
     const float sc = p.scale_log2;
+    const int col0 = half * HC;               // first S column of this thread
     for (int j = 0; j < J; ++j) {
       const bool cent = j >= J_kept;
+      const uint32_t sbuf = Cfg::kSCol + (uint32_t)((j & 1) * KB);
       if (cent) {
         // per-column compensation bias of this centroid block (log2 units)
-        named_sync(1, 128);
+        named_sync(1, Cfg::kSoftmaxThreads);
         if (st < KB) {
           const int e = (j - J_kept) * KB + st;
           float bv = -INFINITY;
           if (e < p.C && !((kb_row[e >> 5] >> (e & 31)) & 1u)) bv = p.logcnt[(size_t)bh * p.Cpad + e] * log2e;
           bias[st] = bv;
         }
-        named_sync(1, 128);
+        named_sync(1, Cfg::kSoftmaxThreads);
       }
       int valid = KB;   // real keys in a kept block
       if (!cent) {
         if (p.dense) valid = min(KB, p.n_valid - j * KB);
         else {
-          const int b = kept[j / nsb];
-          valid = min(KB, p.count_k[(size_t)bh * p.C + b] - (j % nsb) * KB);
+          const int cnt = kept_in_smem ? kcnt_s[j / nsb] : p.count_k[(size_t)bh * p.C + kept[j / nsb]];
+          valid = min(KB, cnt - (j % nsb) * KB);
         }
       }
-      ok = group_all(wait_bar(s_full, j & 1, limit, abort_flag));
+      const int vloc = valid - col0;             // valid columns among this thread's
+      const int mode = cent ? 2 : (vloc < HC ? 1 : 0);   // 0 full, 1 partial, 2 centroids
+      ok = group_all_n(wait_bar(&s_full[j & 1], (j >> 1) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
       if (!ok) break;
       tc_fence_after();
-      const int mode = cent ? 2 : (valid < KB ? 1 : 0);   // 0 full block, 1 partial block, 2 centroids
-      // pass 1: row max of the logits, 32 columns at a time
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      float sv[HC];
 #pragma unroll
-      for (int c0 = 0; c0 < KB; c0 += 32) {
-        float sv[32];
-        uint32_t* r = reinterpret_cast<uint32_t*>(sv);
-        CA_TMEM_LD32(lane_addr + Cfg::kSCol + (uint32_t)c0, r);
-        tmem_wait_ld();
-        if (mode == 0) {
+      for (int c0 = 0; c0 < HC; c0 += 32) {
+        uint32_t* r = reinterpret_cast<uint32_t*>(&sv[c0]);
+        CA_TMEM_LD32(lane_addr + sbuf + (uint32_t)(col0 + c0), r);
+      }
+      tmem_wait_ld();
+      float m8[8];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) m4[q & 3] = fmaxf(m4[q & 3], sv[q]);
-        } else if (mode == 1) {
+      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+      if (mode == 0) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) if (c0 + q < valid) m4[q & 3] = fmaxf(m4[q & 3], sv[q]);
-        } else {
+        for (int q = 0; q < HC; ++q) m8[q & 7] = fmaxf(m8[q & 7], sv[q]);
+      } else if (mode == 1) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) m4[q & 3] = fmaxf(m4[q & 3], fmaf(sv[q], sc, bias[c0 + q]));
+        for (int q = 0; q < HC; ++q) {
+          if (q >= vloc) sv[q] = -INFINITY;
+          m8[q & 7] = fmaxf(m8[q & 7], sv[q]);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < HC; ++q) {
+          sv[q] = fmaf(sv[q], sc, bias[col0 + q]);
+          m8[q & 7] = fmaxf(m8[q & 7], sv[q]);
         }
       }
-      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      if (mode != 2) mx *= sc;             // log2 units
+      float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      if (mode != 2) pm *= sc;             // log2 units
+      // combine the two halves of the row; after this barrier every S column
+      // of the block is in registers, so P may overwrite S.
+      red[half * 128 + row] = pm;
+      named_sync(1, Cfg::kSoftmaxThreads);
+      const float mx = fmaxf(red[row], red[128 + row]);
       // lazy rescale: move the reference max only when it grows by > 8 (x 256)
       bool need = false;
       float factor = 1.f;
@@ -517,52 +557,50 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         m_used = mx;
       }
       const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
-      // O and the row sums are stable: PV_{j-1} finished before s_full flipped.
-      if (__any_sync(0xffffffffu, need)) {
+      // O correction (rare) once PV_{j-1} has finished; each half scales its
+      // half of O, the second half also the row sums.
+      bool wok = true;
+      const bool wneed = __any_sync(0xffffffffu, need);
+      if (wneed) wok = __all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, limit, abort_flag));
+      ok = group_all_n(wok, Cfg::kSoftmaxThreads);
+      if (!ok) break;
+      if (wneed) {
+        tc_fence_after();
+        constexpr int OH = D / 2;
 #pragma unroll
-        for (int c0 = 0; c0 < D + 32; c0 += 32) {
+        for (int c0 = 0; c0 < OH; c0 += 32) {
           uint32_t ov[32];
-          CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);   // last chunk: 16 row-sum columns + 16 spare
+          CA_TMEM_LD32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
-          CA_TMEM_ST32(lane_addr + Cfg::kOCol + c0, ov);
+          CA_TMEM_ST32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
+        }
+        if (half == 1) {
+          uint32_t ov[32];
+          CA_TMEM_LD32(lane_addr + Cfg::kLCol, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
+          CA_TMEM_ST32(lane_addr + Cfg::kLCol, ov);
         }
       }
-      // pass 2: P = 2^(x - m) as bf16 pairs written over the front of S
+      // P = 2^(x - m) as bf16 pairs over the front half of this S buffer
+      const float xs = (mode == 2) ? 1.f : sc;
 #pragma unroll
-      for (int c0 = 0; c0 < KB; c0 += 32) {
-        float sv[32];
-        uint32_t* r = reinterpret_cast<uint32_t*>(sv);
-        CA_TMEM_LD32(lane_addr + Cfg::kSCol + (uint32_t)c0, r);
-        tmem_wait_ld();
+      for (int c0 = 0; c0 < HC; c0 += 32) {
         uint32_t pk[16];
-        if (mode == 0) {
 #pragma unroll
-          for (int q = 0; q < 16; ++q)
-            pk[q] = pack_bf16(ex2(fmaf(sv[2 * q], sc, nb)), ex2(fmaf(sv[2 * q + 1], sc, nb)));
-        } else if (mode == 1) {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float p0 = (c0 + 2 * q < valid) ? ex2(fmaf(sv[2 * q], sc, nb)) : 0.f;
-            const float p1 = (c0 + 2 * q + 1 < valid) ? ex2(fmaf(sv[2 * q + 1], sc, nb)) : 0.f;
-            pk[q] = pack_bf16(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            pk[q] = pack_bf16(ex2(fmaf(sv[2 * q], sc, bias[c0 + 2 * q]) + nb),
-                              ex2(fmaf(sv[2 * q + 1], sc, bias[c0 + 2 * q + 1]) + nb));
-        }
-        // columns [c0/2, c0/2+16) of S were read by this or an earlier chunk
-        CA_TMEM_ST16(lane_addr + Cfg::kSCol + (uint32_t)(c0 / 2), pk);
+        for (int q = 0; q < 16; ++q)
+          pk[q] = pack_bf16(ex2(fmaf(sv[c0 + 2 * q], xs, nb)), ex2(fmaf(sv[c0 + 2 * q + 1], xs, nb)));
+        CA_TMEM_ST16(lane_addr + sbuf + (uint32_t)((col0 + c0) / 2), pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
-    // epilogue: O / l to the query's original row
-    if (ok && J > 0) ok = group_all(wait_bar(pv_done, (J - 1) & 1, limit, abort_flag));
+    // epilogue: O / l to the query's original row; each half writes D/2 columns
+    if (ok && J > 0) ok = group_all_n(wait_bar(pv_done, (J - 1) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
     if (ok && J > 0) {
       tc_fence_after();
       int orow;
@@ -574,11 +612,12 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tmem_wait_ld();
       const float l = __uint_as_float(lv[0]);
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D;
+      constexpr int OH = D / 2;
+      __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D + half * OH;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < OH; c0 += 32) {
         uint32_t ov[32];
-        CA_TMEM_LD32(lane_addr + Cfg::kOCol + c0, ov);
+        CA_TMEM_LD32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
         tmem_wait_ld();
         if (orow >= 0) {
           uint4 w[4];
@@ -657,14 +696,12 @@ cudaError_t launch_tc(const CUtensorMap maps[7], const TcParams& p, dim3 grid, c
   return cudaGetLastError();
 }
 
-// Key-block width: 128 keys for d = 64; 64 keys for d = 128 (and for c = 64),
-// so that S, P and O fit in 256 TMEM columns.
-int key_block(int D, int c) { return (D == 64 && c >= 128) ? 128 : 64; }
+// Key-block width: 128 keys, or 64 when the cluster size is 64.
+int key_block(int D, int c) { return c >= 128 ? 128 : 64; (void)D; }
 
 cudaError_t dispatch(int D, int KB, const CUtensorMap maps[7], const TcParams& p, dim3 grid, cudaStream_t st) {
-  if (D == 64 && KB == 128) return launch_tc<64, 128>(maps, p, grid, st);
-  if (D == 64) return launch_tc<64, 64>(maps, p, grid, st);
-  return launch_tc<128, 64>(maps, p, grid, st);
+  if (D == 64) return KB == 128 ? launch_tc<64, 128>(maps, p, grid, st) : launch_tc<64, 64>(maps, p, grid, st);
+  return KB == 128 ? launch_tc<128, 128>(maps, p, grid, st) : launch_tc<128, 64>(maps, p, grid, st);
 }
 
 }  // namespace
