@@ -7,17 +7,21 @@
 // q . kbar_b / sqrt(d) + ln|b| and value vbar_b). The dense form (eq. 1) is
 // the same kernel with every key block kept and no compensation.
 //
-// One CTA handles one 128-row query tile of one head:
-//   warp 0      TMA producer: Q tile once, then a ring of stages holding
-//               (K, V) of a kept key block, (kbar_hi, kbar_lo) or
-//               (vbar_hi, vbar_lo) of a centroid block;
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
-//               S buffers; O += P_j V_j with P_j read from TMEM;
-//   warps 2..5  softmax: one thread per query row reads S_j from TMEM,
-//               applies the key mask / compensation bias, keeps a running
-//               max (rescaling O only when the max grows by more than 2^8),
-//               writes P_j as bf16 over S_j, and finally writes O / l to the
-//               query's original row.
+// One CTA handles one 128-row query tile of one head and holds an SM (512
+// TMEM columns: two S buffers and O):
+//   warp 0      TMA producer (one thread): Q tile once, then a ring of
+//               stages holding (K, V) of a kept key block, (kbar_hi,
+//               kbar_lo) or (vbar_hi, vbar_lo) of a centroid block;
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into TMEM buffer
+//               j % 2, so S_{j+1} is computed while the softmax works on S_j;
+//               O += P_j V_j with P_j read from TMEM;
+//   warps 2..9  softmax, two threads per query row (one per half of the key
+//               block): read S_j from TMEM, apply the key mask /
+//               compensation bias, exchange the row max through shared
+//               memory, keep a running max (rescaling O only when the max
+//               grows by more than 2^8), write P_j as bf16 over the front of
+//               S_j, accumulate the row sums in registers, and finally write
+//               O / l to the query's original row.
 // Centroids are split into bf16 hi + lo parts and enter as two MMAs each.
 // Every wait is bounded: on a timeout the CTA sets the library's device error
 // word (CA_ERR_TIMEOUT), drains what it issued, frees TMEM and returns.
@@ -236,18 +240,25 @@ struct TcParams {
   uint64_t wait_limit;
 };
 
+#ifndef CA_TC_SPLIT
+#define CA_TC_SPLIT 2   // softmax threads per query row
+#endif
+#ifndef CA_TC_NBUF
+#define CA_TC_NBUF 2    // S buffers in TMEM
+#endif
+
 template <int D, int KB>
 struct TcCfg {
+  static constexpr int kSplit = CA_TC_SPLIT;
+  static constexpr int kNBuf = CA_TC_NBUF;
   static constexpr int kSub = D / 64;                                  // 64-column sub-tiles per row
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kOnesBytes = 16 * KB * 2;                       // B operand of the row sums
   static constexpr int kMaxKeptSmem = 1024;                            // kept list staged in shared memory
-  static constexpr int kStagesFit = (200 * 1024 - kQBytes - kOnesBytes - 2 * kMaxKeptSmem * 4) / kStageBytes;
+  static constexpr int kStagesFit = (200 * 1024 - kQBytes - 2 * kMaxKeptSmem * 4) / kStageBytes;
   static constexpr int kStages = kStagesFit > 4 ? 4 : (kStagesFit < 2 ? 2 : kStagesFit);
-  static constexpr int kOnesOff = kQBytes + kStages * kStageBytes;
-  static constexpr int kBarOff = kOnesOff + kOnesBytes;
+  static constexpr int kBarOff = kQBytes + kStages * kStageBytes;
   static constexpr int kBiasOff = kBarOff + 256;
   static constexpr int kRedOff = kBiasOff + KB * 4;                    // row-max exchange [2][128]
   static constexpr int kKeptOff = kRedOff + 2 * 128 * 4;
@@ -255,14 +266,13 @@ struct TcCfg {
   // columns) holds an SM
   static constexpr int kSmemCalc = kKeptOff + 2 * kMaxKeptSmem * 4 + 1024;
   static constexpr int kSmem = kSmemCalc > 116 * 1024 ? kSmemCalc : 116 * 1024;
-  static constexpr int kSoftmaxThreads = 256;                          // 8 warps, two threads per row
+  static constexpr int kSoftmaxThreads = 128 * kSplit;                 // kSplit threads per row
   static constexpr int kThreads = 64 + kSoftmaxThreads;                // + producer warp + MMA warp
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSCol = 0;        // S buffers at 0 and KB; P_j (bf16 pairs) over the front half
-  static constexpr uint32_t kOCol = 2 * KB;   // O (fp32, D columns)
-  static constexpr uint32_t kLCol = 2 * KB + D;  // row sums of P (fp32, 16 columns, column 0 used)
-  static constexpr int kHalf = KB / 2;        // columns of S per softmax thread
-  static_assert(kLCol + 32 <= kTmemCols, "S buffers, O and the row sums must fit in TMEM");
+  static constexpr uint32_t kOCol = kNBuf * KB;      // O (fp32, D columns)
+  static constexpr int kHalf = KB / kSplit;          // columns of S per softmax thread
+  static_assert(kOCol + D <= kTmemCols, "S buffers and O must fit in TMEM");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
@@ -284,7 +294,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                          ~static_cast<uintptr_t>(1023));
   unsigned char* sQ = smem;
   unsigned char* sStage = smem + Cfg::kQBytes;
-  unsigned char* sOnes = smem + Cfg::kOnesOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
   uint64_t* full = bars;              // [NS] stage loaded
   uint64_t* empty = bars + NS;        // [NS] stage released
@@ -321,11 +330,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   const int32_t* kept = kept_in_smem ? kept_s : kept_g;
 
-  // bf16 ones (0x3F80): the B operand that turns P into its row sums. Every
-  // element is equal, so the swizzled layout needs no address arithmetic.
-  for (int i = threadIdx.x; i < Cfg::kOnesBytes / 4; i += Cfg::kThreads)
-    reinterpret_cast<uint32_t*>(sOnes)[i] = 0x3F803F80u;
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> tensor-core reads
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(q_full, 1);
@@ -404,9 +408,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
       constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
-      constexpr uint32_t id_l = idesc_bf16(128, 16, 0);
       const uint32_t q_base = su32(sQ);
-      const uint32_t ones = su32(sOnes);
       bool ok = wait_bar(q_full, 0, limit, abort_flag);
       // item index of block j's QK and PV operands
       auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
@@ -417,7 +419,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!wait_bar(&full[s], r & 1, limit, abort_flag)) return false;
         tc_fence_after();
         const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
-        const uint32_t d_tmem = tmem + Cfg::kSCol + (uint32_t)((j & 1) * KB);
+        const uint32_t d_tmem = tmem + Cfg::kSCol + (uint32_t)((j % Cfg::kNBuf) * KB);
         const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
         for (int mtx = 0; mtx < nmat; ++mtx) {
           const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
@@ -431,14 +433,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // Commits track every earlier MMA of this thread too: when s_full[b]
         // flips for S_j, PV_{j-2} (the last reader of that buffer) is done.
-        tc_commit(&s_full[j & 1]);
+        tc_commit(&s_full[j % Cfg::kNBuf]);
         if (j >= J_kept) tc_commit(&empty[s]);   // kbar stage is free once S is computed
         return true;
       };
-      if (ok && J > 0) ok = issue_qk(0);
-      if (ok && J > 1) ok = issue_qk(1);
+      constexpr int NB = Cfg::kNBuf;
+      for (int j = 0; j < NB && j < J && ok; ++j) ok = issue_qk(j);
       for (int j = 0; j < J && ok; ++j) {
-        if (!wait_bar(&p_full[j & 1], (j >> 1) & 1, limit, abort_flag)) { ok = false; break; }
+        if (!wait_bar(&p_full[j % NB], (j / NB) & 1, limit, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const int i = pv_item(j);
         const int s = i % NS, r = i / NS;
@@ -447,7 +449,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tc_fence_after();
         }
         const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
-        const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j & 1) * KB);
+        const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
         const int nmat = (j < J_kept) ? 1 : 2;
         for (int mtx = 0; mtx < nmat; ++mtx) {
           const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
@@ -457,17 +459,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        // row sums: L += P_j 1 (the bf16 P the numerator used)
-#pragma unroll
-        for (int kk = 0; kk < KB / 16; ++kk) {
-          const uint64_t bd = sdesc(ones + (kk >> 2) * 16 * 128 + (kk & 3) * 32, 16, 1024);
-          mma_ts(tmem + Cfg::kLCol, p_tmem + kk * 8, bd, id_l, (j > 0 || kk > 0) ? 1u : 0u);
-        }
         tc_commit(pv_done);
         tc_commit(&empty[s]);
-        // S_{j+2} overwrites P_j: ordered after PV_j in this thread's MMA stream.
-        if (j + 2 < J) {
-          ok = issue_qk(j + 2);
+        // S_{j+NB} overwrites P_j: issue it only once PV_j (the last reader of
+        // that buffer) has completed.
+        if (j + NB < J) {
+          if (!wait_bar(pv_done, j & 1, limit, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          ok = issue_qk(j + NB);
           if (!ok) break;
         }
       }
@@ -479,10 +478,10 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ------------------------------------------------------------- softmax
     const int st = threadIdx.x - 64;          // 0..255 within the softmax group
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
-    const int half = st >> 7;                 // which half of the columns of its row
+    const int half = st >> 7;                 // which part of the columns of its row
     const int row = q4 * 32 + lane;           // row of the query tile
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
-    float m_used = -INFINITY;
+    float m_used = -INFINITY, lreg = 0.f;
     bool ok = true;
     const uint32_t* kb_row = p.dense ? nullptr : p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
     const float log2e = 1.4426950408889634f;
@@ -490,7 +489,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int col0 = half * HC;               // first S column of this thread
     for (int j = 0; j < J; ++j) {
       const bool cent = j >= J_kept;
-      const uint32_t sbuf = Cfg::kSCol + (uint32_t)((j & 1) * KB);
+      constexpr int NB = Cfg::kNBuf;
+      const uint32_t sbuf = Cfg::kSCol + (uint32_t)((j % NB) * KB);
       if (cent) {
         // per-column compensation bias of this centroid block (log2 units)
         named_sync(1, Cfg::kSoftmaxThreads);
@@ -512,7 +512,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       const int vloc = valid - col0;             // valid columns among this thread's
       const int mode = cent ? 2 : (vloc < HC ? 1 : 0);   // 0 full, 1 partial, 2 centroids
-      ok = group_all_n(wait_bar(&s_full[j & 1], (j >> 1) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
+      ok = group_all_n(wait_bar(&s_full[j % NB], (j / NB) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
       if (!ok) break;
       tc_fence_after();
       float sv[HC];
@@ -545,9 +545,12 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (mode != 2) pm *= sc;             // log2 units
       // combine the two halves of the row; after this barrier every S column
       // of the block is in registers, so P may overwrite S.
-      red[half * 128 + row] = pm;
-      named_sync(1, Cfg::kSoftmaxThreads);
-      const float mx = fmaxf(red[row], red[128 + row]);
+      float mx = pm;
+      if (Cfg::kSplit == 2) {
+        red[half * 128 + row] = pm;
+        named_sync(1, Cfg::kSoftmaxThreads);
+        mx = fmaxf(red[row], red[128 + row]);
+      }
       // lazy rescale: move the reference max only when it grows by > 8 (x 256)
       bool need = false;
       float factor = 1.f;
@@ -555,10 +558,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - mx);
         need = (j > 0);
         m_used = mx;
+        lreg *= factor;
       }
       const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
       // O correction (rare) once PV_{j-1} has finished; each half scales its
-      // half of O, the second half also the row sums.
+      // half of O.
       bool wok = true;
       const bool wneed = __any_sync(0xffffffffu, need);
       if (wneed) wok = __all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, limit, abort_flag));
@@ -566,7 +570,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!ok) break;
       if (wneed) {
         tc_fence_after();
-        constexpr int OH = D / 2;
+        constexpr int OH = D / Cfg::kSplit;
 #pragma unroll
         for (int c0 = 0; c0 < OH; c0 += 32) {
           uint32_t ov[32];
@@ -576,14 +580,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
           CA_TMEM_ST32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
         }
-        if (half == 1) {
-          uint32_t ov[32];
-          CA_TMEM_LD32(lane_addr + Cfg::kLCol, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
-          CA_TMEM_ST32(lane_addr + Cfg::kLCol, ov);
-        }
       }
       // P = 2^(x - m) as bf16 pairs over the front half of this S buffer
       const float xs = (mode == 2) ? 1.f : sc;
@@ -591,13 +587,16 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int c0 = 0; c0 < HC; c0 += 32) {
         uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          pk[q] = pack_bf16(ex2(fmaf(sv[c0 + 2 * q], xs, nb)), ex2(fmaf(sv[c0 + 2 * q + 1], xs, nb)));
+        for (int q = 0; q < 16; ++q) {
+          const float p0 = ex2(fmaf(sv[c0 + 2 * q], xs, nb)), p1 = ex2(fmaf(sv[c0 + 2 * q + 1], xs, nb));
+          lreg += p0 + p1;
+          pk[q] = pack_bf16(p0, p1);
+        }
         CA_TMEM_ST16(lane_addr + sbuf + (uint32_t)((col0 + c0) / 2), pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[j % NB]);
     }
     // epilogue: O / l to the query's original row; each half writes D/2 columns
     if (ok && J > 0) ok = group_all_n(wait_bar(pv_done, (J - 1) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
@@ -607,12 +606,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (p.dense) orow = tile * 128 + row < p.n_valid ? tile * 128 + row : -1;
       else orow = row < p.rows_per_tile ? p.perm_q[(size_t)bh * p.C * p.c + (size_t)a * p.c + sub_tile * 128 + row]
                                         : -1;
-      uint32_t lv[32];
-      CA_TMEM_LD32(lane_addr + Cfg::kLCol, lv);
-      tmem_wait_ld();
-      const float l = __uint_as_float(lv[0]);
+      red[half * 128 + row] = lreg;
+      named_sync(1, Cfg::kSoftmaxThreads);
+      const float l = Cfg::kSplit == 2 ? red[row] + red[128 + row] : lreg;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      constexpr int OH = D / 2;
+      constexpr int OH = D / Cfg::kSplit;
       __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D + half * OH;
 #pragma unroll
       for (int c0 = 0; c0 < OH; c0 += 32) {
