@@ -166,6 +166,27 @@ def run_reference(args):
     return 0
 
 
+def rank_seed(rank: int) -> int:
+    """Seed of the independent layer a rank runs (rank 0: the standard workload)."""
+    return 1000 + CONFIG_ID + 7919 * rank
+
+
+def whole_job_value(world: int, steps: int, total_ms: float) -> float:
+    """Layer forwards per second over all ranks, from the max-over-ranks time."""
+    return world * steps / (total_ms / 1e3)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank time over the process group (identity on one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -186,15 +207,11 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(x):
+        return max_over_ranks(x, world, "cuda")
 
     # Each rank: an independent layer (its own seeded inputs).
-    w = wl.config_workload(CONFIG_ID, seed=1000 + CONFIG_ID + 7919 * rank)
+    w = wl.config_workload(CONFIG_ID, seed=rank_seed(rank))
 
     def dev(x):
         return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).cuda().contiguous()
@@ -234,12 +251,12 @@ def run_ours(args):
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
-    total_ms = max_over_ranks(start.elapsed_time(end))
+    total_ms = ranks_max(start.elapsed_time(end))
     clocks = clk.summary()
     stage = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
              for j, name in enumerate(("cluster", "route", "attend"))}
     ms_per_step = total_ms / args.steps
-    value = world * args.steps / (total_ms / 1e3)
+    value = whole_job_value(world, args.steps, total_ms)
 
     # Dense attention (this build's own kernel) on the same inputs, for the speedup.
     Od = torch.empty_like(Q)
@@ -252,7 +269,7 @@ def run_ours(args):
         layer.dense(Q, K, V, Od)
     d1.record(stream)
     torch.cuda.synchronize()
-    dense_ms = max_over_ranks(d0.elapsed_time(d1) / dense_iters)
+    dense_ms = ranks_max(d0.elapsed_time(d1) / dense_iters)
 
     # End to end through the C ABI with host buffers (pinned), copies inside the region.
     shape = layer.shape
@@ -269,8 +286,8 @@ def run_ours(args):
         ca.ca_forward_host(hQ, hK, hV, shape, layer.params, w.k, w.compensate, hO, wsh)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * args.steps / (e2e_ms / 1e3)
+    e2e_ms = ranks_max(e0.elapsed_time(e1))
+    e2e_value = whole_job_value(world, args.steps, e2e_ms)
     in_bytes = 3 * Q.numel() * Q.element_size()
     out_bytes = O.numel() * O.element_size()
 
