@@ -27,6 +27,7 @@ EXPORTED = [
     "ca_dense_workspace_bytes", "ca_forward_workspace_bytes", "ca_cluster", "ca_route", "ca_attend",
     "ca_dense_attend", "ca_forward", "ca_forward_host_workspace_bytes", "ca_forward_host",
     "ca_get_device_error", "ca_set_wait_limit", "ca_status_string", "ca_version", "ca_launch_count",
+    "ca_cluster_noalloc",
 ]
 
 
@@ -91,6 +92,7 @@ def lib():
             "ca_status_string": (ctypes.c_char_p, [i32]),
             "ca_version": (ctypes.c_char_p, []),
             "ca_launch_count": (i32, [P(ca_shape), i32]),
+            "ca_cluster_noalloc": (i32, [vp, vp, P(ca_shape), P(ca_cluster_params), P(ca_clusters), vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -168,6 +170,16 @@ def ca_cluster(Q, K, shape: ca_shape, params: Optional[ca_cluster_params], clust
                           0 if workspace is None else workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _check(st, "ca_cluster")
+
+
+def ca_cluster_noalloc(Q, K, shape: ca_shape, params: Optional[ca_cluster_params], clusters: ca_clusters,
+                       stream=None):
+    """ca_cluster with the library's fixed 16 MiB device scratch instead of a
+    workspace, for callers that cannot allocate device memory."""
+    st = lib().ca_cluster_noalloc(_ptr(Q), _ptr(K), ctypes.byref(shape),
+                                  ctypes.byref(params) if params is not None else None,
+                                  ctypes.byref(clusters), _stream(stream))
+    _check(st, "ca_cluster_noalloc")
 
 
 def ca_route(shape: ca_shape, centroids: ca_clusters, routes: ca_routes, stream=None):

@@ -134,6 +134,28 @@ ca_status ca_cluster(const void* Q, const void* K, const ca_shape* shape,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * ca_cluster_noalloc -- ca_cluster for callers that cannot allocate device
+ * memory: plugins inside another framework that owns every device allocation
+ * and gives no scratch buffer, and latency-critical loops that must not call
+ * cudaMalloc (it can synchronise the device and can fail mid-run). The paper
+ * has no counterpart; this is a deployment convenience of this library.
+ * Same arguments and results as ca_cluster, without the workspace: the
+ * scratch is a fixed 16 MiB array in device memory that belongs to the
+ * library (every GPU on which it is loaded holds those 16 MiB until the
+ * process exits). Shapes whose ca_cluster_workspace_bytes() exceeds 16 MiB
+ * are rejected with CA_ERR_WORKSPACE before any launch (e.g. two
+ * 65,536-token heads at d = 64 fit, eight do not). Nothing here calls
+ * cudaMalloc, cudaFree or any allocating routine. The first call on a device
+ * looks up the array's device address (with that device current), so make
+ * that first call before any stream capture. All calls share the one array:
+ * calls whose work overlaps on the GPU (different streams, or several host
+ * threads) race on it and must be serialised by the caller.
+ */
+ca_status ca_cluster_noalloc(const void* Q, const void* K, const ca_shape* shape,
+                             const ca_cluster_params* params, const ca_clusters* out,
+                             void* stream);
+
+/*
  * ca_route -- centroid scores and top-k selection.
  * Paper Section 3.3.1 (score s_ab = qbar_a . kbar_b, eq. 18, computed in fp64)
  * and Section 3.3.2 (keep the k best-scoring key clusters per query cluster).
