@@ -30,10 +30,76 @@ __device__ __forceinline__ double warp_sum(double v) {
 }
 
 // ---------------------------------------------------------------------------
-// Tree tables on the device (one thread; the host runs the same function).
+// Tree tables on the device: breadth first, one level at a time; the
+// children of node i land at (level end + exclusive prefix of the child
+// counts), which reproduces the host's sequential plan_tree order exactly.
+// One block of 1024 threads.
 // ---------------------------------------------------------------------------
-__global__ void plan_kernel(int n, int c, TreeNode* nodes, int* level_begin) {
-  if (threadIdx.x == 0 && blockIdx.x == 0) plan_tree(n, c, nodes, level_begin, kMaxLevels);
+__global__ void __launch_bounds__(1024) plan_kernel(int n, int c, TreeNode* nodes, int* level_begin) {
+  __shared__ int warp_tot[32];
+  __shared__ int s_total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (n <= c) {
+    if (tid == 0) level_begin[0] = 0;
+    return;
+  }
+  if (tid == 0) {
+    TreeNode r;
+    r.off = 0; r.size = n; r.t = split_count(n, c); r.parent = -1; r.heap = 1;
+    nodes[0] = r;
+  }
+  __syncthreads();
+  int begin = 0, end = 1, count = 1, lvl = 0;
+  while (begin < end && lvl < kMaxLevels) {
+    if (tid == 0) level_begin[lvl] = begin;
+    for (int chunk = begin; chunk < end; chunk += 1024) {
+      const int i = chunk + tid;
+      TreeNode nd;
+      int ls = 0, rs = 0, nch = 0;
+      if (i < end) {
+        nd = nodes[i];
+        ls = nd.t; rs = nd.size - nd.t;
+        nch = (ls > c) + (rs > c);
+      }
+      int x = nch;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) warp_tot[warp] = x;
+      __syncthreads();
+      if (warp == 0) {
+        int t = warp_tot[lane];
+        int u = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, u, o);
+          if (lane >= o) u += y;
+        }
+        warp_tot[lane] = u - t;
+        if (lane == 31) s_total = u;
+      }
+      __syncthreads();
+      if (i < end) {
+        int pos = count + warp_tot[warp] + x - nch;
+        if (ls > c) {
+          TreeNode ch;
+          ch.off = nd.off; ch.size = ls; ch.t = split_count(ls, c); ch.parent = i; ch.heap = 2 * nd.heap;
+          nodes[pos++] = ch;
+        }
+        if (rs > c) {
+          TreeNode ch;
+          ch.off = nd.off + ls; ch.size = rs; ch.t = split_count(rs, c); ch.parent = i; ch.heap = 2 * nd.heap + 1;
+          nodes[pos] = ch;
+        }
+      }
+      count += s_total;
+      __syncthreads();
+    }
+    begin = end; end = count; ++lvl;
+  }
+  if (tid == 0) level_begin[lvl] = count;
 }
 
 // ---------------------------------------------------------------------------
@@ -211,38 +277,6 @@ __global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int
 // random normal vector of unit norm; g is drawn in the untransformed
 // coordinates and mapped through R: g_hat = R g / |R g|, i.e. z_g = g / sqrt(g^T M g).
 // ---------------------------------------------------------------------------
-template <int D>
-__device__ void block_matvec_sym(const double* Ms, const double* x, double* y, double* red) {
-  // y = M x with M symmetric: y_a = sum_b M[b][a] x_b, column access.
-  constexpr int G = 256 / D;
-  const int a = threadIdx.x % D, p = threadIdx.x / D;
-  double s = 0.0;
-  for (int b = p; b < D; b += G) s = fma(Ms[b * D + a], x[b], s);
-  red[p * D + a] = s;
-  __syncthreads();
-  if (threadIdx.x < D) {
-    double t = 0.0;
-    for (int q = 0; q < G; ++q) t += red[q * D + threadIdx.x];
-    y[threadIdx.x] = t;
-  }
-  __syncthreads();
-}
-
-template <int D>
-__device__ double block_dot(const double* x, const double* y, double* bc) {
-  // Warp 0 sums; result broadcast through bc[0].
-  if (threadIdx.x < 32) {
-    double s = 0.0;
-    for (int i = threadIdx.x; i < D; i += 32) s = fma(x[i], y[i], s);
-    s = warp_sum(s);
-    if (threadIdx.x == 0) bc[0] = s;
-  }
-  __syncthreads();
-  double r = bc[0];
-  __syncthreads();
-  return r;
-}
-
 template <typename T, int D>
 __global__ void __launch_bounds__(256) dir_kernel(const T* __restrict__ Q, const T* __restrict__ K,
                                                   int N_alloc, int n, const TreeNode* __restrict__ nodes,
@@ -252,112 +286,197 @@ __global__ void __launch_bounds__(256) dir_kernel(const T* __restrict__ Q, const
                                                   double* __restrict__ zvec, double* __restrict__ wvec,
                                                   uint64_t seed, int power_iters, int sample_factor) {
   constexpr int XS = D + 1;            // padded fp32 row stride of the sample
+  constexpr int G = 256 / D;           // threads sharing one output coordinate
+  constexpr int NW = D / 32;           // warps holding the D coordinates
   const int node_id = lvl_begin + blockIdx.x;
   const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const TreeNode nd = nodes[node_id];
   const int m_cap = sample_factor * D;
   const int m = min(m_cap, nd.size);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* Ms = reinterpret_cast<double*>(smem_raw);   // D*D
-  double* red = Ms + D * D;                           // 256
+  double* red = Ms + D * D;                           // 256 partial sums
   double* scale = red + 256;                          // m_cap
   double* xbar = scale + m_cap;                       // D
   double* z = xbar + D;                               // D
   double* w = z + D;                                  // D
   double* g = w + D;                                  // D
   double* v = g + D;                                  // m_cap
-  double* bc = v + m_cap;                             // 2
-  float* Xs = reinterpret_cast<float*>(bc + 2);       // m_cap * XS
+  double* dotp = v + m_cap;                           // 2 * NW + 8
+  float* Xs = reinterpret_cast<float*>(dotp + 2 * NW + 8);   // m_cap * XS
 
-  for (int e = threadIdx.x; e < D * D; e += 256) Ms[e] = M[(size_t)th * D * D + e];
+  for (int e = tid; e < D * D; e += 256) Ms[e] = M[(size_t)th * D * D + e];
   const uint64_t key = node_stream(seed, (uint64_t)bh, (uint64_t)tensor, nd.heap);
   const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
   const int* idx_th = idx ? idx + (size_t)th * n : nullptr;
-  for (int e = threadIdx.x; e < m * D; e += 256) {
+  for (int e = tid; e < m * D; e += 256) {
     const int j = e / D, col = e % D;
     const int pos = (nd.size > m) ? (int)(((uint64_t)j * (uint64_t)nd.size + r) / (uint64_t)m) : j;
     const int row = idx_th ? idx_th[nd.off + pos] : nd.off + pos;
     Xs[j * XS + col] = to_f(X[(size_t)row * D + col]);
     if (col == 0) scale[j] = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
   }
-  if (threadIdx.x < D) {
+  if (tid < D) {
     // Box-Muller on two SplitMix64 draws per coordinate.
-    const uint64_t ua = splitmix64(key + 2ull * threadIdx.x + 1ull);
-    const uint64_t ub = splitmix64(key + 2ull * threadIdx.x + 2ull);
+    const uint64_t ua = splitmix64(key + 2ull * tid + 1ull);
+    const uint64_t ub = splitmix64(key + 2ull * tid + 2ull);
     const double u1 = (double)((ua >> 11) + 1ull) * 0x1.0p-53;
     const double u2 = (double)(ub >> 11) * 0x1.0p-53;
-    g[threadIdx.x] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+    g[tid] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
   }
   __syncthreads();
-  if (threadIdx.x < D) {
-    double s = 0.0;
-    for (int j = 0; j < m; ++j) s = fma(scale[j], (double)Xs[j * XS + threadIdx.x], s);
-    xbar[threadIdx.x] = s / (double)m;
-  }
-  // z0 = (z_parent + g / sqrt(g^T M g)) / 2, or g / sqrt(g^T M g) at the root.
-  block_matvec_sym<D>(Ms, g, w, red);
+  const int a = tid % D, part = tid / D;     // coordinate and partial-sum slot of this thread
+  // sample mean: xbar_a = sum_j scale_j X_ja / m
   {
-    const double gq = block_dot<D>(g, w, bc);
+    double s0 = 0.0, s1 = 0.0;
+    int j = part;
+    for (; j + G < m; j += 2 * G) {
+      s0 = fma(scale[j], (double)Xs[j * XS + a], s0);
+      s1 = fma(scale[j + G], (double)Xs[(j + G) * XS + a], s1);
+    }
+    if (j < m) s0 = fma(scale[j], (double)Xs[j * XS + a], s0);
+    red[part * D + a] = s0 + s1;
+  }
+  __syncthreads();
+  if (tid < D) {
+    double t = 0.0;
+    for (int q = 0; q < G; ++q) t += red[q * D + tid];
+    xbar[tid] = t / (double)m;
+  }
+  __syncthreads();
+
+  // w = M x into w[], partial sums over b = part (mod G); M is symmetric.
+  auto matvec = [&](const double* x) {
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll 4
+    for (int b = part; b < D; b += 4 * G) {
+      s0 = fma(Ms[b * D + a], x[b], s0);
+      s1 = fma(Ms[(b + G) * D + a], x[b + G], s1);
+      s2 = fma(Ms[(b + 2 * G) * D + a], x[b + 2 * G], s2);
+      s3 = fma(Ms[(b + 3 * G) * D + a], x[b + 3 * G], s3);
+    }
+    red[part * D + a] = (s0 + s1) + (s2 + s3);
+    __syncthreads();
+    if (tid < D) {
+      double t = 0.0;
+      for (int q = 0; q < G; ++q) t += red[q * D + tid];
+      w[tid] = t;
+    }
+  };
+  // two dot products with w over the D coordinates (threads < D), result in
+  // every thread; deterministic fixed-order combination of warp partials.
+  auto dots = [&](const double* x, const double* y, double* r0, double* r1) {
+    if (tid < D) {
+      double p0 = x[tid] * w[tid], p1 = y ? y[tid] * w[tid] : 0.0;
+      p0 = warp_sum(p0);
+      p1 = warp_sum(p1);
+      if (lane == 0) { dotp[2 * warp] = p0; dotp[2 * warp + 1] = p1; }
+    }
+    __syncthreads();
+    double t0 = 0.0, t1 = 0.0;
+#pragma unroll
+    for (int q = 0; q < NW; ++q) { t0 += dotp[2 * q]; t1 += dotp[2 * q + 1]; }
+    *r0 = t0; *r1 = t1;
+  };
+
+  // z0 = (z_parent + g / sqrt(g^T M g)) / 2, or g / sqrt(g^T M g) at the root.
+  matvec(g);
+  {
+    double gq, unused;
+    dots(g, nullptr, &gq, &unused);
     const double gi = (gq > 0.0) ? 1.0 / sqrt(gq) : 0.0;
-    if (threadIdx.x < D) {
-      const double gh = g[threadIdx.x] * gi;
-      z[threadIdx.x] = (nd.parent < 0)
-                           ? gh
-                           : 0.5 * (zvec[((size_t)th * NI + nd.parent) * D + threadIdx.x] + gh);
+    if (tid < D) {
+      const double gh = g[tid] * gi;
+      z[tid] = (nd.parent < 0) ? gh : 0.5 * (zvec[((size_t)th * NI + nd.parent) * D + tid] + gh);
     }
     __syncthreads();
   }
+  // power iteration in z-form: z <- C_x M z, normalised by sqrt(z^T M z)
+  constexpr int TPJ = G;                 // threads per sample row (m <= D)
   for (int it = 0; it < power_iters; ++it) {
-    block_matvec_sym<D>(Ms, z, w, red);       // w = M z
-    if (it > 0) {                              // normalise: |u|^2 = z^T M z
-      const double q = block_dot<D>(z, w, bc);
-      const double qi = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
-      if (threadIdx.x < D) { z[threadIdx.x] *= qi; w[threadIdx.x] *= qi; }
-      __syncthreads();
-    }
-    const double xw = block_dot<D>(xbar, w, bc);
-    // v_j = (x_j - xbar) . w over the sample
-    for (int j = threadIdx.x; j < m; j += 256) {
-      double s = 0.0;
-      for (int col = 0; col < D; ++col) s = fma((double)Xs[j * XS + col], w[col], s);
-      v[j] = fma(scale[j], s, -xw);
+    matvec(z);                            // w = M z (unnormalised)
+    double q, xw;
+    dots(z, xbar, &q, &xw);               // q = z.w, xw = xbar.w
+    const double s = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
+    // v_j = (x_j - xbar) . (s w), TPJ threads per j
+    {
+      const int pj = tid % TPJ;
+      double vs = 0.0;                     // sum of v over this thread's rows (pj == 0 only)
+      for (int j0 = 0; j0 < m; j0 += 256 / TPJ) {
+        const int j = j0 + tid / TPJ;
+        double d0 = 0.0, d1 = 0.0;
+        if (j < m) {
+#pragma unroll 4
+          for (int col = pj; col < D; col += 2 * TPJ) {
+            d0 = fma((double)Xs[j * XS + col], w[col], d0);
+            d1 = fma((double)Xs[j * XS + col + TPJ], w[col + TPJ], d1);
+          }
+        }
+        double dsum = d0 + d1;
+#pragma unroll
+        for (int o = TPJ / 2; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+        if (j < m && pj == 0) {
+          const double vj = s * fma(scale[j], dsum, -xw);
+          v[j] = vj;
+          vs += vj;
+        }
+      }
+      vs = warp_sum(vs);
+      if (lane == 0) dotp[2 * NW + warp] = vs;
     }
     __syncthreads();
-    // z' = sum_j v_j (x_j - xbar) / m
-    if (threadIdx.x < D) {
-      double s = 0.0, sv = 0.0;
-      for (int j = 0; j < m; ++j) {
-        s = fma(v[j] * scale[j], (double)Xs[j * XS + threadIdx.x], s);
-        sv += v[j];
+    double vsum = 0.0;
+#pragma unroll
+    for (int q8 = 0; q8 < 8; ++q8) vsum += dotp[2 * NW + q8];
+    // z'_a = (sum_j v_j scale_j X_ja - xbar_a sum_j v_j) / m
+    {
+      double s0 = 0.0, s1 = 0.0;
+      int j = part;
+      for (; j + G < m; j += 2 * G) {
+        s0 = fma(v[j] * scale[j], (double)Xs[j * XS + a], s0);
+        s1 = fma(v[j + G] * scale[j + G], (double)Xs[(j + G) * XS + a], s1);
       }
-      z[threadIdx.x] = (s - xbar[threadIdx.x] * sv) / (double)m;
+      if (j < m) s0 = fma(v[j] * scale[j], (double)Xs[j * XS + a], s0);
+      red[part * D + a] = s0 + s1;
+    }
+    __syncthreads();
+    if (tid < D) {
+      double t = 0.0;
+      for (int q2 = 0; q2 < G; ++q2) t += red[q2 * D + tid];
+      z[tid] = (t - xbar[tid] * vsum) / (double)m;
     }
     __syncthreads();
   }
-  block_matvec_sym<D>(Ms, z, w, red);
-  const double q = block_dot<D>(z, w, bc);
+  matvec(z);
+  double q, unused;
+  dots(z, nullptr, &q, &unused);
   const double qi = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
-  if (threadIdx.x < D) {
-    const size_t o = ((size_t)th * NI + node_id) * D + threadIdx.x;
-    zvec[o] = z[threadIdx.x] * qi;
-    wvec[o] = w[threadIdx.x] * qi;
+  if (tid < D) {
+    const size_t o = ((size_t)th * NI + node_id) * D + tid;
+    zvec[o] = z[tid] * qi;
+    wvec[o] = w[tid] * qi;
   }
 }
 
 // ---------------------------------------------------------------------------
 // K2a: projection key_i = x_i . w_node for every position of the level's
-// internal nodes, stored as order-preserving uint64. One group of G lanes
-// reads one row (16 bytes per lane, coalesced).
+// internal nodes, stored as order-preserving uint64. A block covers 256
+// consecutive positions, which meet at most a handful of nodes (every
+// internal node holds more than c >= 64 vectors); their directions are staged
+// in shared memory. One group of G lanes reads one row (16 bytes per lane,
+// coalesced).
 // ---------------------------------------------------------------------------
+constexpr int kProjNodes = 8;   // > 256 / 65 + 2
+
 __device__ __forceinline__ int find_node(const TreeNode* nodes, int lb, int le, int pos) {
-  // last node in [lb, le) with off <= pos; -1 if none covers pos
-  int lo = lb, hi = le - 1, ans = -1;
+  // last node in [lb, le) with off <= pos (lb - 1 if none)
+  int lo = lb, hi = le - 1, ans = lb - 1;
   while (lo <= hi) {
     const int mid = (lo + hi) >> 1;
     if (nodes[mid].off <= pos) { ans = mid; lo = mid + 1; } else hi = mid - 1;
   }
-  if (ans >= 0 && pos >= nodes[ans].off + nodes[ans].size) ans = -1;
   return ans;
 }
 
@@ -371,22 +490,44 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   constexpr int EPL = 16 / sizeof(T);        // elements per lane (16 bytes)
   constexpr int G = D / EPL;                 // lanes per row
   constexpr int RPW = 32 / G;                // rows per warp step
+  __shared__ double ws[kProjNodes][D];
+  __shared__ int n_off[kProjNodes], n_end[kProjNodes], n_id[kProjNodes];
+  __shared__ int s_first, s_count;
   const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const int base = blockIdx.x * 256;
+  if (threadIdx.x == 0) {
+    const int f = find_node(nodes, lb, le, base);
+    int first = f < lb ? lb : f, cnt = 0;
+    for (int i = first; i < le && cnt < kProjNodes && nodes[i].off < base + 256; ++i) {
+      if (nodes[i].off + nodes[i].size <= base) { ++first; continue; }
+      n_off[cnt] = nodes[i].off; n_end[cnt] = nodes[i].off + nodes[i].size; n_id[cnt] = i;
+      ++cnt;
+    }
+    s_first = first; s_count = cnt;
+  }
+  __syncthreads();
+  const int cnt = s_count;
+  for (int e = threadIdx.x; e < cnt * D; e += 256)
+    ws[e / D][e % D] = wvec[((size_t)th * NI + n_id[e / D]) * D + (e % D)];
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / G, gl = lane % G;
-  const int base = blockIdx.x * 256;
   for (int rr = warp * RPW + sub; rr < 256; rr += 8 * RPW) {
     const int pos = base + rr;
     int node = -1;
-    if (pos < n) node = find_node(nodes, lb, le, pos);
+    if (pos < n) {
+#pragma unroll
+      for (int q = 0; q < kProjNodes; ++q)
+        if (q < cnt && pos >= n_off[q] && pos < n_end[q]) node = q;
+    }
     double s = 0.0;
     int row = 0;
     if (node >= 0) {
       row = idx ? idx[(size_t)th * n + pos] : pos;
       const uint4 raw = *reinterpret_cast<const uint4*>(X + (size_t)row * D + gl * EPL);
       const T* e = reinterpret_cast<const T*>(&raw);
-      const double* wn = wvec + ((size_t)th * NI + node) * D + gl * EPL;
+      const double* wn = &ws[node][gl * EPL];
 #pragma unroll
       for (int q = 0; q < EPL; ++q) s = fma((double)to_f(e[q]), wn[q], s);
     }
@@ -401,17 +542,20 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
 
 // ---------------------------------------------------------------------------
 // K2b: the t-th smallest key of a node (MSD radix select, 8-bit digits).
-// Candidates move to shared memory once they fit. Output: the threshold key T
-// and eq_left = how many keys equal to T go below the split (the first ones
-// in row order, so equal projections are ordered by row index).
+// Nodes of at most kSelCap keys are read into shared memory once; larger
+// nodes are scanned in global memory until the candidates sharing the
+// selected prefix fit. Output: the threshold key T and eq_left = how many
+// keys equal to T go below the split (the first ones in row order, so equal
+// projections are ordered by row index).
 // ---------------------------------------------------------------------------
 struct SelectResult { uint64_t T; int eq_left; int pad; };
 constexpr int kSelCap = 8192;
 
-__global__ void __launch_bounds__(1024) select_kernel(const TreeNode* __restrict__ nodes, int lb,
-                                                      int nodes_in_level, int n,
-                                                      const uint64_t* __restrict__ keys,
-                                                      SelectResult* __restrict__ sel) {
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__ nodes, int lb,
+                                                    int nodes_in_level, int n,
+                                                    const uint64_t* __restrict__ keys,
+                                                    SelectResult* __restrict__ sel) {
   __shared__ unsigned int hist[256];
   __shared__ int s_digit, s_rank, s_cnt, s_ncand;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -420,16 +564,19 @@ __global__ void __launch_bounds__(1024) select_kernel(const TreeNode* __restrict
   const TreeNode nd = nodes[lb + blockIdx.x];
   const uint64_t* base = keys + (size_t)th * n + nd.off;
   const int size = nd.size;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int rank = nd.t - 1;
   uint64_t prefix = 0, mask = 0;
-  bool global_mode = true;
-  int ncand = 0;
-  const int lane = threadIdx.x & 31;
+  bool global_mode = size > kSelCap;
+  int ncand = size;
+  if (!global_mode) {
+    for (int i = threadIdx.x; i < size; i += NT) cand[i] = base[i];
+  }
   for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
     const int cnt_total = global_mode ? size : ncand;
-    for (int i0 = 0; i0 < cnt_total; i0 += blockDim.x) {
+    for (int i0 = 0; i0 < cnt_total; i0 += NT) {
       const int i = i0 + threadIdx.x;
       bool ok = false;
       unsigned dg = 0;
@@ -446,16 +593,27 @@ __global__ void __launch_bounds__(1024) select_kernel(const TreeNode* __restrict
       }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      unsigned cum = 0;
-      int dsel = 255, rsel = rank;
-      unsigned csel = 0;
-      for (int dgt = 0; dgt < 256; ++dgt) {
-        const unsigned h = hist[dgt];
-        if ((unsigned)rank < cum + h) { dsel = dgt; rsel = rank - (int)cum; csel = h; break; }
-        cum += h;
+    if (warp == 0) {
+      // digit holding the rank: lane L owns bins 8L..8L+7
+      unsigned h[8], local = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) { h[q] = hist[lane * 8 + q]; local += h[q]; }
+      unsigned incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      s_digit = dsel; s_rank = rsel; s_cnt = (int)csel;
+      const unsigned excl = incl - local;
+      const bool mine = excl <= (unsigned)rank && (unsigned)rank < incl;
+      if (mine) {
+        unsigned r = (unsigned)rank - excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (r < h[q]) { s_digit = lane * 8 + q; s_rank = (int)r; s_cnt = (int)h[q]; break; }
+          r -= h[q];
+        }
+      }
     }
     __syncthreads();
     rank = s_rank;
@@ -463,12 +621,25 @@ __global__ void __launch_bounds__(1024) select_kernel(const TreeNode* __restrict
     mask |= (uint64_t)0xFF << shift;
     const int cnt = s_cnt;
     __syncthreads();
-    if (global_mode && cnt <= kSelCap && shift > 0) {
+    if (shift > 0 && cnt <= kSelCap && (global_mode || cnt < ncand)) {
+      // keep only the candidates that share the prefix
       if (threadIdx.x == 0) s_ncand = 0;
       __syncthreads();
-      for (int i = threadIdx.x; i < size; i += blockDim.x) {
-        const uint64_t k = base[i];
-        if ((k & mask) == prefix) cand[atomicAdd(&s_ncand, 1)] = k;
+      if (global_mode) {
+        for (int i = threadIdx.x; i < size; i += NT) {
+          const uint64_t k = base[i];
+          if ((k & mask) == prefix) cand[atomicAdd(&s_ncand, 1)] = k;
+        }
+      } else {
+        // in place: read all candidates first, then write the survivors
+        uint64_t mine[kSelCap / NT];
+        int nm = 0;
+        for (int i = threadIdx.x; i < ncand; i += NT) {
+          const uint64_t k = cand[i];
+          if ((k & mask) == prefix) mine[nm++] = k;
+        }
+        __syncthreads();
+        for (int q = 0; q < nm; ++q) cand[atomicAdd(&s_ncand, 1)] = mine[q];
       }
       __syncthreads();
       ncand = s_ncand;
@@ -667,7 +838,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
   const int transform = p->transform;
 
   if (plan.levels > 0) {
-    plan_kernel<<<1, 1, 0, st>>>(n, c, nodes, level_begin);
+    plan_kernel<<<1, 1024, 0, st>>>(n, c, nodes, level_begin);
     colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
     syrk_kernel<T, D><<<dim3(nch, BH, 2), 256, 0, st>>>(Q, K, N_alloc, n, nch, colpart, metpart);
     metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
@@ -675,10 +846,11 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
     qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, transform, inv_s);
     const int m_cap = sample_factor * D;
-    const size_t dir_smem = (size_t)D * D * 8 + 256 * 8 + (size_t)m_cap * 8 * 2 + (size_t)D * 8 * 4 + 16 +
-                            (size_t)m_cap * (D + 1) * 4;
+    const size_t dir_smem = (size_t)D * D * 8 + 256 * 8 + (size_t)m_cap * 8 * 2 + (size_t)D * 8 * 4 +
+                            (size_t)(2 * (D / 32) + 8) * 8 + (size_t)m_cap * (D + 1) * 4;
     cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
-    cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
+    cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
+    cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
     for (int l = 0; l < plan.levels; ++l) {
       const int lb = plan.level_begin[l], le = plan.level_begin[l + 1], nl = le - lb;
       const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
@@ -688,7 +860,10 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
                                                             sample_factor);
       project_kernel<T, D><<<dim3((n + 255) / 256, TH), 256, 0, st>>>(Q, K, N_alloc, n, nodes, lb, le,
                                                                       inv_s, idx_in, NI, wvec, keys);
-      select_kernel<<<dim3(nl, TH), 1024, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
+      if (plan.level_max_size[l] <= kSelCap)
+        select_kernel<256><<<dim3(nl, TH), 256, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
+      else
+        select_kernel<1024><<<dim3(nl, TH), 1024, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
       const int pch = (plan.level_max_size[l] + kPartChunk - 1) / kPartChunk;
       part_count_kernel<<<dim3(pch, nl, TH), kPartThreads, 0, st>>>(nodes, lb, nl, n, pch, keys, sel, ccnt);
       part_scatter_kernel<<<dim3(pch, nl, TH), kPartThreads, 0, st>>>(nodes, lb, nl, n, c, pch, keys, sel,
