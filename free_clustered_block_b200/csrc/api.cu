@@ -36,9 +36,9 @@ ca_status check_shape(const ca_shape* s) {
 bool plan_for(const ca_shape* s, TreePlan* plan) { return host_plan(s->n_valid, s->c, plan); }
 
 size_t dir_smem(int d, int a) {
+  // one warp's share of the per-node kernel (fp32 sample rows, the larger case) plus M
   const size_t m_cap = (size_t)a * d;
-  return (size_t)d * d * 8 + 256 * 8 + m_cap * 16 + (size_t)d * 32 + (size_t)(2 * (d / 32) + 8) * 8 +
-         m_cap * (d + 1) * 4;
+  return (size_t)d * d * 8 + m_cap * (d + 1) * 4 + (2 * d + 2 * m_cap) * 8 + m_cap * 4;
 }
 
 ca_status check_params(const ca_shape* s, const ca_cluster_params* p) {

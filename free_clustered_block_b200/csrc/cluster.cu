@@ -277,208 +277,233 @@ __global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int
 // random normal vector of unit norm; g is drawn in the untransformed
 // coordinates and mapped through R: g_hat = R g / |R g|, i.e. z_g = g / sqrt(g^T M g).
 // ---------------------------------------------------------------------------
+// One warp per node: the block's warps take consecutive nodes of one
+// tensor-head and share its M in shared memory; each warp stages its node's
+// sample rows (in the input type, exact) in shared memory with a padded row
+// stride (odd number of 32-bit words, conflict-free both along rows and
+// along columns). Every reduction is a warp shuffle: after M is staged no
+// block barrier is needed.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) dir_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                  int N_alloc, int n, const TreeNode* __restrict__ nodes,
-                                                  int lvl_begin, const double* __restrict__ M,
-                                                  const double* __restrict__ inv_s,
-                                                  const int* __restrict__ idx, int NI,
-                                                  double* __restrict__ zvec, double* __restrict__ wvec,
-                                                  uint64_t seed, int power_iters, int sample_factor) {
-  constexpr int XS = D + 1;            // padded fp32 row stride of the sample
-  constexpr int G = 256 / D;           // threads sharing one output coordinate
-  constexpr int NW = D / 32;           // warps holding the D coordinates
-  const int node_id = lvl_begin + blockIdx.x;
-  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
-  const TreeNode nd = nodes[node_id];
-  const int m_cap = sample_factor * D;
-  const int m = min(m_cap, nd.size);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  double* Ms = reinterpret_cast<double*>(smem_raw);   // D*D
-  double* red = Ms + D * D;                           // 256 partial sums
-  double* scale = red + 256;                          // m_cap
-  double* xbar = scale + m_cap;                       // D
-  double* z = xbar + D;                               // D
-  double* w = z + D;                                  // D
-  double* g = w + D;                                  // D
-  double* v = g + D;                                  // m_cap
-  double* dotp = v + m_cap;                           // 2 * NW + 8
-  float* Xs = reinterpret_cast<float*>(dotp + 2 * NW + 8);   // m_cap * XS
+struct DirCfg {
+  static constexpr int kRowPad = (sizeof(T) == 2) ? 2 : 1;             // elements
+  static constexpr int kRowStride = D + kRowPad;                       // elements; odd word count
+  __host__ __device__ static size_t warp_bytes(int m_cap) {
+    return (size_t)m_cap * kRowStride * sizeof(T) + (size_t)(2 * D + 2 * m_cap) * 8 + (size_t)m_cap * 4;
+  }
+  static int warps(int m_cap) {
+    const long long per = (long long)warp_bytes(m_cap);
+    const long long two = 112 * 1024 - (long long)D * D * 8;   // two blocks per SM when it fits
+    long long w = two > 0 ? two / per : 0;
+    if (w < 1) w = (220 * 1024 - (long long)D * D * 8) / per;  // one block per SM
+    if (w < 1) w = 1;
+    return (int)(w > 16 ? 16 : w);
+  }
+};
 
-  for (int e = tid; e < D * D; e += 256) Ms[e] = M[(size_t)th * D * D + e];
+template <typename T, int D>
+__global__ void __launch_bounds__(512) dir_kernel(
+    const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
+    int lvl_begin, int nodes_in_level, const double* __restrict__ M, const double* __restrict__ inv_s,
+    const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
+    int power_iters, int sample_factor) {
+  using Cfg = DirCfg<T, D>;
+  constexpr int CPL = D / 32;                      // coordinates per lane: a = lane + 32 c
+  constexpr int RS = Cfg::kRowStride;
+  const int m_cap = sample_factor * D;
+  const int nwarps = blockDim.x >> 5;
+  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* Ms = reinterpret_cast<double*>(smem_raw);                          // D*D
+  unsigned char* wbase = smem_raw + (size_t)D * D * 8 + (size_t)warp * Cfg::warp_bytes(m_cap);
+  double* vz = reinterpret_cast<double*>(wbase);   // z (D)
+  double* vw = vz + D;                             // w (D)
+  double* vv = vw + D;                             // v over the sample (m_cap)
+  double* vs = vv + m_cap;                         // sample scales (m_cap)
+  int* srow = reinterpret_cast<int*>(vs + m_cap);  // sample rows (m_cap)
+  T* Xs = reinterpret_cast<T*>(srow + m_cap);      // m_cap x RS sample (4-byte aligned)
+  for (int e = threadIdx.x; e < D * D; e += nwarps * 32) Ms[e] = M[(size_t)th * D * D + e];
+  __syncthreads();
+  const int local = blockIdx.x * nwarps + warp;
+  if (local >= nodes_in_level) return;             // whole warp leaves; no block barrier follows
+  const int node_id = lvl_begin + local;
+  const TreeNode nd = nodes[node_id];
+  const int m = min(m_cap, nd.size);
   const uint64_t key = node_stream(seed, (uint64_t)bh, (uint64_t)tensor, nd.heap);
   const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
   const int* idx_th = idx ? idx + (size_t)th * n : nullptr;
-  for (int e = tid; e < m * D; e += 256) {
-    const int j = e / D, col = e % D;
+  for (int j = lane; j < m; j += 32) {
     const int pos = (nd.size > m) ? (int)(((uint64_t)j * (uint64_t)nd.size + r) / (uint64_t)m) : j;
     const int row = idx_th ? idx_th[nd.off + pos] : nd.off + pos;
-    Xs[j * XS + col] = to_f(X[(size_t)row * D + col]);
-    if (col == 0) scale[j] = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
+    srow[j] = row;
+    vs[j] = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
   }
-  if (tid < D) {
-    // Box-Muller on two SplitMix64 draws per coordinate.
-    const uint64_t ua = splitmix64(key + 2ull * tid + 1ull);
-    const uint64_t ub = splitmix64(key + 2ull * tid + 2ull);
+  __syncwarp();
+  // stage the sample: 16-byte chunks, several rows per warp instruction, up to
+  // four instructions' loads in flight before their stores
+  {
+    constexpr int CPR = D * (int)sizeof(T) / 16;    // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;                   // rows per warp instruction
+    constexpr int WRS = RS * (int)sizeof(T) / 4;    // padded row stride in 32-bit words
+    uint32_t* xw = reinterpret_cast<uint32_t*>(Xs);
+    const int sub = lane / CPR, part = lane % CPR;
+    for (int j0 = 0; j0 < m; j0 += 4 * RPI) {
+      uint4 v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * RPI + sub;
+        v4[u] = make_uint4(0, 0, 0, 0);
+        if (j < m) v4[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * D + part * (16 / sizeof(T)));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * RPI + sub;
+        if (j < m) {
+          uint32_t* dst = xw + (size_t)j * WRS + part * 4;
+          dst[0] = v4[u].x; dst[1] = v4[u].y; dst[2] = v4[u].z; dst[3] = v4[u].w;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  // sample mean
+  double xbar[CPL];
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) xbar[cc] = 0.0;
+  for (int j = 0; j < m; ++j) {
+    const double sj = vs[j];
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) xbar[cc] = fma(sj, (double)to_f(Xs[j * RS + lane + 32 * cc]), xbar[cc]);
+  }
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) xbar[cc] /= (double)m;
+  // w = M z with z in vz; M symmetric, column access is conflict-free
+  auto matvec = [&](double* out) {
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int a = lane + 32 * cc;
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll 4
+      for (int b = 0; b < D; b += 4) {
+        s0 = fma(Ms[b * D + a], vz[b], s0);
+        s1 = fma(Ms[(b + 1) * D + a], vz[b + 1], s1);
+        s2 = fma(Ms[(b + 2) * D + a], vz[b + 2], s2);
+        s3 = fma(Ms[(b + 3) * D + a], vz[b + 3], s3);
+      }
+      out[cc] = (s0 + s1) + (s2 + s3);
+    }
+  };
+  // z0 = (z_parent + g / sqrt(g^T M g)) / 2, or g / sqrt(g^T M g) at the root
+  double g[CPL], w[CPL], z[CPL];
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) {
+    const int a = lane + 32 * cc;
+    // Box-Muller on two SplitMix64 draws per coordinate
+    const uint64_t ua = splitmix64(key + 2ull * a + 1ull);
+    const uint64_t ub = splitmix64(key + 2ull * a + 2ull);
     const double u1 = (double)((ua >> 11) + 1ull) * 0x1.0p-53;
     const double u2 = (double)(ub >> 11) * 0x1.0p-53;
-    g[tid] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+    g[cc] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+    vz[a] = g[cc];
   }
-  __syncthreads();
-  const int a = tid % D, part = tid / D;     // coordinate and partial-sum slot of this thread
-  // sample mean: xbar_a = sum_j scale_j X_ja / m
-  {
-    double s0 = 0.0, s1 = 0.0;
-    int j = part;
-    for (; j + G < m; j += 2 * G) {
-      s0 = fma(scale[j], (double)Xs[j * XS + a], s0);
-      s1 = fma(scale[j + G], (double)Xs[(j + G) * XS + a], s1);
-    }
-    if (j < m) s0 = fma(scale[j], (double)Xs[j * XS + a], s0);
-    red[part * D + a] = s0 + s1;
-  }
-  __syncthreads();
-  if (tid < D) {
-    double t = 0.0;
-    for (int q = 0; q < G; ++q) t += red[q * D + tid];
-    xbar[tid] = t / (double)m;
-  }
-  __syncthreads();
-
-  // w = M x into w[], partial sums over b = part (mod G); M is symmetric.
-  auto matvec = [&](const double* x) {
-    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-#pragma unroll 4
-    for (int b = part; b < D; b += 4 * G) {
-      s0 = fma(Ms[b * D + a], x[b], s0);
-      s1 = fma(Ms[(b + G) * D + a], x[b + G], s1);
-      s2 = fma(Ms[(b + 2 * G) * D + a], x[b + 2 * G], s2);
-      s3 = fma(Ms[(b + 3 * G) * D + a], x[b + 3 * G], s3);
-    }
-    red[part * D + a] = (s0 + s1) + (s2 + s3);
-    __syncthreads();
-    if (tid < D) {
-      double t = 0.0;
-      for (int q = 0; q < G; ++q) t += red[q * D + tid];
-      w[tid] = t;
-    }
-  };
-  // two dot products with w over the D coordinates (threads < D), result in
-  // every thread; deterministic fixed-order combination of warp partials.
-  auto dots = [&](const double* x, const double* y, double* r0, double* r1) {
-    if (tid < D) {
-      double p0 = x[tid] * w[tid], p1 = y ? y[tid] * w[tid] : 0.0;
-      p0 = warp_sum(p0);
-      p1 = warp_sum(p1);
-      if (lane == 0) { dotp[2 * warp] = p0; dotp[2 * warp + 1] = p1; }
-    }
-    __syncthreads();
-    double t0 = 0.0, t1 = 0.0;
+  __syncwarp();
+  matvec(w);
+  double gq = 0.0;
 #pragma unroll
-    for (int q = 0; q < NW; ++q) { t0 += dotp[2 * q]; t1 += dotp[2 * q + 1]; }
-    *r0 = t0; *r1 = t1;
-  };
-
-  // z0 = (z_parent + g / sqrt(g^T M g)) / 2, or g / sqrt(g^T M g) at the root.
-  matvec(g);
-  {
-    double gq, unused;
-    dots(g, nullptr, &gq, &unused);
-    const double gi = (gq > 0.0) ? 1.0 / sqrt(gq) : 0.0;
-    if (tid < D) {
-      const double gh = g[tid] * gi;
-      z[tid] = (nd.parent < 0) ? gh : 0.5 * (zvec[((size_t)th * NI + nd.parent) * D + tid] + gh);
-    }
-    __syncthreads();
+  for (int cc = 0; cc < CPL; ++cc) gq = fma(g[cc], w[cc], gq);
+  gq = warp_sum(gq);
+  const double gi = (gq > 0.0) ? 1.0 / sqrt(gq) : 0.0;
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) {
+    const double gh = g[cc] * gi;
+    z[cc] = (nd.parent < 0) ? gh : 0.5 * (zvec[((size_t)th * NI + nd.parent) * D + lane + 32 * cc] + gh);
   }
+  __syncwarp();
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) vz[lane + 32 * cc] = z[cc];
+  __syncwarp();
   // power iteration in z-form: z <- C_x M z, normalised by sqrt(z^T M z)
-  constexpr int TPJ = G;                 // threads per sample row (m <= D)
   for (int it = 0; it < power_iters; ++it) {
-    matvec(z);                            // w = M z (unnormalised)
-    double q, xw;
-    dots(z, xbar, &q, &xw);               // q = z.w, xw = xbar.w
+    matvec(w);
+    double q = 0.0, xw = 0.0;
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) { q = fma(z[cc], w[cc], q); xw = fma(xbar[cc], w[cc], xw); }
+    q = warp_sum(q);
+    xw = warp_sum(xw);
     const double s = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
-    // v_j = (x_j - xbar) . (s w), TPJ threads per j
-    {
-      const int pj = tid % TPJ;
-      double vs = 0.0;                     // sum of v over this thread's rows (pj == 0 only)
-      for (int j0 = 0; j0 < m; j0 += 256 / TPJ) {
-        const int j = j0 + tid / TPJ;
-        double d0 = 0.0, d1 = 0.0;
-        if (j < m) {
-#pragma unroll 4
-          for (int col = pj; col < D; col += 2 * TPJ) {
-            d0 = fma((double)Xs[j * XS + col], w[col], d0);
-            d1 = fma((double)Xs[j * XS + col + TPJ], w[col + TPJ], d1);
-          }
-        }
-        double dsum = d0 + d1;
 #pragma unroll
-        for (int o = TPJ / 2; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-        if (j < m && pj == 0) {
-          const double vj = s * fma(scale[j], dsum, -xw);
-          v[j] = vj;
-          vs += vj;
-        }
-      }
-      vs = warp_sum(vs);
-      if (lane == 0) dotp[2 * NW + warp] = vs;
-    }
-    __syncthreads();
+    for (int cc = 0; cc < CPL; ++cc) vw[lane + 32 * cc] = w[cc];
+    __syncwarp();
+    // v_j = s (scale_j X_j . w - xbar . w); lane takes rows j = lane + 32 q
     double vsum = 0.0;
-#pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8) vsum += dotp[2 * NW + q8];
-    // z'_a = (sum_j v_j scale_j X_ja - xbar_a sum_j v_j) / m
-    {
-      double s0 = 0.0, s1 = 0.0;
-      int j = part;
-      for (; j + G < m; j += 2 * G) {
-        s0 = fma(v[j] * scale[j], (double)Xs[j * XS + a], s0);
-        s1 = fma(v[j + G] * scale[j + G], (double)Xs[(j + G) * XS + a], s1);
+    for (int j = lane; j < m; j += 32) {
+      const T* xr = Xs + j * RS;
+      double d0 = 0.0, d1 = 0.0, d2 = 0.0, d3 = 0.0;
+#pragma unroll 4
+      for (int e = 0; e < D; e += 4) {
+        d0 = fma((double)to_f(xr[e]), vw[e], d0);
+        d1 = fma((double)to_f(xr[e + 1]), vw[e + 1], d1);
+        d2 = fma((double)to_f(xr[e + 2]), vw[e + 2], d2);
+        d3 = fma((double)to_f(xr[e + 3]), vw[e + 3], d3);
       }
-      if (j < m) s0 = fma(v[j] * scale[j], (double)Xs[j * XS + a], s0);
-      red[part * D + a] = s0 + s1;
+      const double vj = s * fma(vs[j], (d0 + d1) + (d2 + d3), -xw);
+      vv[j] = vj;
+      vsum += vj;
     }
-    __syncthreads();
-    if (tid < D) {
-      double t = 0.0;
-      for (int q2 = 0; q2 < G; ++q2) t += red[q2 * D + tid];
-      z[tid] = (t - xbar[tid] * vsum) / (double)m;
+    vsum = warp_sum(vsum);
+    __syncwarp();
+    // z'_a = (sum_j v_j scale_j X_ja - xbar_a sum_j v_j) / m
+    double acc0[CPL], acc1[CPL];
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) { acc0[cc] = 0.0; acc1[cc] = 0.0; }
+    int j = 0;
+    for (; j + 1 < m; j += 2) {
+      const double f0 = vv[j] * vs[j], f1 = vv[j + 1] * vs[j + 1];
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) {
+        acc0[cc] = fma(f0, (double)to_f(Xs[j * RS + lane + 32 * cc]), acc0[cc]);
+        acc1[cc] = fma(f1, (double)to_f(Xs[(j + 1) * RS + lane + 32 * cc]), acc1[cc]);
+      }
     }
-    __syncthreads();
+    if (j < m) {
+      const double f0 = vv[j] * vs[j];
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) acc0[cc] = fma(f0, (double)to_f(Xs[j * RS + lane + 32 * cc]), acc0[cc]);
+    }
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) z[cc] = ((acc0[cc] + acc1[cc]) - xbar[cc] * vsum) / (double)m;
+    __syncwarp();
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) vz[lane + 32 * cc] = z[cc];
+    __syncwarp();
   }
-  matvec(z);
-  double q, unused;
-  dots(z, nullptr, &q, &unused);
+  matvec(w);
+  double q = 0.0;
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) q = fma(z[cc], w[cc], q);
+  q = warp_sum(q);
   const double qi = (q > 0.0) ? 1.0 / sqrt(q) : 0.0;
-  if (tid < D) {
-    const size_t o = ((size_t)th * NI + node_id) * D + tid;
-    zvec[o] = z[tid] * qi;
-    wvec[o] = w[tid] * qi;
+#pragma unroll
+  for (int cc = 0; cc < CPL; ++cc) {
+    const size_t o = ((size_t)th * NI + node_id) * D + lane + 32 * cc;
+    zvec[o] = z[cc] * qi;
+    wvec[o] = w[cc] * qi;
   }
 }
 
 // ---------------------------------------------------------------------------
 // K2a: projection key_i = x_i . w_node for every position of the level's
-// internal nodes, stored as order-preserving uint64. A block covers 256
-// consecutive positions, which meet at most a handful of nodes (every
+// internal nodes, stored as order-preserving uint64. A block covers
+// kProjSpan consecutive positions, which meet at most kProjNodes nodes (every
 // internal node holds more than c >= 64 vectors); their directions are staged
-// in shared memory. One group of G lanes reads one row (16 bytes per lane,
-// coalesced).
+// in shared memory with a position -> node table. A group of G lanes reads
+// one row (16 bytes per lane, coalesced); each group keeps kProjU rows in
+// flight.
 // ---------------------------------------------------------------------------
-constexpr int kProjNodes = 8;   // > 256 / 65 + 2
-
-__device__ __forceinline__ int find_node(const TreeNode* nodes, int lb, int le, int pos) {
-  // last node in [lb, le) with off <= pos (lb - 1 if none)
-  int lo = lb, hi = le - 1, ans = lb - 1;
-  while (lo <= hi) {
-    const int mid = (lo + hi) >> 1;
-    if (nodes[mid].off <= pos) { ans = mid; lo = mid + 1; } else hi = mid - 1;
-  }
-  return ans;
-}
+constexpr int kProjSpan = 1024;
+constexpr int kProjNodes = 20;   // > kProjSpan / 65 + 2
+constexpr int kProjU = 4;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, const T* __restrict__ K,
@@ -490,52 +515,107 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   constexpr int EPL = 16 / sizeof(T);        // elements per lane (16 bytes)
   constexpr int G = D / EPL;                 // lanes per row
   constexpr int RPW = 32 / G;                // rows per warp step
+  constexpr int STEP = 8 * RPW;              // rows per block step (8 warps)
   __shared__ double ws[kProjNodes][D];
   __shared__ int n_off[kProjNodes], n_end[kProjNodes], n_id[kProjNodes];
-  __shared__ int s_first, s_count;
+  __shared__ unsigned char slot_of[kProjSpan];
+  __shared__ int s_cnt;
   const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
-  const int base = blockIdx.x * 256;
-  if (threadIdx.x == 0) {
-    const int f = find_node(nodes, lb, le, base);
-    int first = f < lb ? lb : f, cnt = 0;
-    for (int i = first; i < le && cnt < kProjNodes && nodes[i].off < base + 256; ++i) {
-      if (nodes[i].off + nodes[i].size <= base) { ++first; continue; }
-      n_off[cnt] = nodes[i].off; n_end[cnt] = nodes[i].off + nodes[i].size; n_id[cnt] = i;
-      ++cnt;
+  const int base = blockIdx.x * kProjSpan;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    // last node with off <= base (32-ary search), lb - 1 if none
+    int lo = lb, hi = le, f = lb - 1;
+    while (hi > lo) {
+      const int step = (hi - lo + 31) / 32;
+      const int probe = lo + lane * step;
+      const bool ok = probe < hi && nodes[probe].off <= base;
+      const unsigned b = __ballot_sync(0xffffffffu, ok);
+      if (b == 0) break;
+      const int L = 31 - __clz(b);
+      f = lo + L * step;
+      if (step == 1) break;
+      lo = f;
+      hi = min(hi, f + step);
     }
-    s_first = first; s_count = cnt;
+    const int start = f < lb ? lb : f;
+    const int i = start + lane;
+    bool take = false;
+    int off = 0, end = 0;
+    if (lane < kProjNodes && i < le) {
+      off = nodes[i].off;
+      end = off + nodes[i].size;
+      take = off < base + kProjSpan && end > base;
+    }
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int sl = __popc(tb & ((1u << lane) - 1u));
+      n_off[sl] = off; n_end[sl] = end; n_id[sl] = i;
+    }
+    if (lane == 0) s_cnt = __popc(tb);
   }
   __syncthreads();
-  const int cnt = s_count;
+  const int cnt = s_cnt;
+  for (int p = threadIdx.x; p < kProjSpan; p += 256) {
+    const int pos = base + p;
+    unsigned char sl = 255;
+    for (int q = 0; q < cnt; ++q)
+      if (pos >= n_off[q] && pos < n_end[q]) sl = (unsigned char)q;
+    slot_of[p] = sl;
+  }
   for (int e = threadIdx.x; e < cnt * D; e += 256)
     ws[e / D][e % D] = wvec[((size_t)th * NI + n_id[e / D]) * D + (e % D)];
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / G, gl = lane % G;
-  for (int rr = warp * RPW + sub; rr < 256; rr += 8 * RPW) {
-    const int pos = base + rr;
-    int node = -1;
-    if (pos < n) {
+  // this lane's EPL direction values of the current node, reloaded only when
+  // the node changes (rows are in position order, so rarely)
+  int wslot = -1;
+  double wr[EPL];
 #pragma unroll
-      for (int q = 0; q < kProjNodes; ++q)
-        if (q < cnt && pos >= n_off[q] && pos < n_end[q]) node = q;
+  for (int q = 0; q < EPL; ++q) wr[q] = 0.0;
+  for (int r0 = warp * RPW + sub; r0 < kProjSpan; r0 += STEP * kProjU) {
+    int slot[kProjU], row[kProjU];
+    uint4 raw[kProjU];
+    double sc[kProjU];
+#pragma unroll
+    for (int u = 0; u < kProjU; ++u) {
+      const int rr = r0 + u * STEP;
+      const int pos = base + rr;
+      slot[u] = (rr < kProjSpan && pos < n) ? slot_of[rr] : 255;
+      row[u] = 0;
+      if (slot[u] != 255) row[u] = idx ? idx[(size_t)th * n + pos] : pos;
     }
-    double s = 0.0;
-    int row = 0;
-    if (node >= 0) {
-      row = idx ? idx[(size_t)th * n + pos] : pos;
-      const uint4 raw = *reinterpret_cast<const uint4*>(X + (size_t)row * D + gl * EPL);
-      const T* e = reinterpret_cast<const T*>(&raw);
-      const double* wn = &ws[node][gl * EPL];
 #pragma unroll
-      for (int q = 0; q < EPL; ++q) s = fma((double)to_f(e[q]), wn[q], s);
+    for (int u = 0; u < kProjU; ++u) {
+      raw[u] = make_uint4(0, 0, 0, 0);
+      sc[u] = 1.0;
+      if (slot[u] != 255) {
+        raw[u] = *reinterpret_cast<const uint4*>(X + (size_t)row[u] * D + gl * EPL);
+        if (tensor == 0) sc[u] = inv_s[(size_t)bh * n + row[u]];
+      }
     }
 #pragma unroll
-    for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (node >= 0 && gl == 0) {
-      const double sc = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
-      keys[(size_t)th * n + pos] = ordered_key(s * sc);
+    for (int u = 0; u < kProjU; ++u) {
+      double s = 0.0;
+      if (slot[u] != 255) {
+        if (slot[u] != wslot) {
+          wslot = slot[u];
+#pragma unroll
+          for (int q = 0; q < EPL; ++q) wr[q] = ws[wslot][gl * EPL + q];
+        }
+        const T* e = reinterpret_cast<const T*>(&raw[u]);
+        double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+        for (int q = 0; q < EPL; q += 2) {
+          s0 = fma((double)to_f(e[q]), wr[q], s0);
+          s1 = fma((double)to_f(e[q + 1]), wr[q + 1], s1);
+        }
+        s = s0 + s1;
+      }
+#pragma unroll
+      for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (slot[u] != 255 && gl == 0) keys[(size_t)th * n + base + r0 + u * STEP] = ordered_key(s * sc[u]);
     }
   }
 }
@@ -846,8 +926,8 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
     qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, transform, inv_s);
     const int m_cap = sample_factor * D;
-    const size_t dir_smem = (size_t)D * D * 8 + 256 * 8 + (size_t)m_cap * 8 * 2 + (size_t)D * 8 * 4 +
-                            (size_t)(2 * (D / 32) + 8) * 8 + (size_t)m_cap * (D + 1) * 4;
+    const int dir_warps = DirCfg<T, D>::warps(m_cap);
+    const size_t dir_smem = (size_t)D * D * 8 + (size_t)dir_warps * DirCfg<T, D>::warp_bytes(m_cap);
     cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
     cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
     cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
@@ -855,10 +935,9 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       const int lb = plan.level_begin[l], le = plan.level_begin[l + 1], nl = le - lb;
       const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
       int* idx_out = idxbuf[(l + 1) & 1];
-      dir_kernel<T, D><<<dim3(nl, TH), 256, dir_smem, st>>>(Q, K, N_alloc, n, nodes, lb, M, inv_s, idx_in,
-                                                            NI, zvec, wvec, p->seed, power_iters,
-                                                            sample_factor);
-      project_kernel<T, D><<<dim3((n + 255) / 256, TH), 256, 0, st>>>(Q, K, N_alloc, n, nodes, lb, le,
+      dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(
+          Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters, sample_factor);
+      project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(Q, K, N_alloc, n, nodes, lb, le,
                                                                       inv_s, idx_in, NI, wvec, keys);
       if (plan.level_max_size[l] <= kSelCap)
         select_kernel<256><<<dim3(nl, TH), 256, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
