@@ -154,6 +154,7 @@ ca_status ca_route(const ca_shape* s, const ca_clusters* cen, const ca_routes* o
   ca_status st = check_shape(s);
   if (st != CA_OK) return st;
   if (!cen || !cen->qbar || !cen->kbar || !out || !out->kept_idx || !out->kept_bits) return CA_ERR_INVALID_ARG;
+  if (!aligned16(cen->qbar) || !aligned16(cen->kbar)) return CA_ERR_INVALID_ARG;
   const int C = (s->n_valid + s->c - 1) / s->c;
   if (out->k < 1 || out->k > C) return CA_ERR_INVALID_ARG;
   if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;

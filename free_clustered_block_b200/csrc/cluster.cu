@@ -128,60 +128,139 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, in
 // ---------------------------------------------------------------------------
 // S1: partial second-moment matrices over a row chunk.
 // z = 0: Q^T Q (uncentred); z = 1: (K - kmean)^T (K - kmean).
-// Thread (ty, tx) owns entries (ty + 16 i, tx + 16 j).
+// Only the upper triangle of 8 x 8 tiles is accumulated (the matrix is
+// symmetric): thread t of row group g owns tile t over the staged rows
+// g, g + R, g + 2R, ... The R groups are then summed in a fixed order through
+// shared memory, so the result does not depend on scheduling.
+// Rows arrive by 16-byte cp.async into a raw tile while the previous tile is
+// being multiplied, and are converted (minus the mean) into an fp64 tile whose
+// 16-byte chunks are rotated within each 8-column group, so that the lanes of
+// a warp reading chunk i of different column groups hit different banks.
 // ---------------------------------------------------------------------------
+template <int D>
+struct SyrkCfg {
+  static constexpr int TT = D / 8;                 // tile rows
+  static constexpr int NT = TT * (TT + 1) / 2;     // upper tiles incl. diagonal
+  static constexpr int R = D == 64 ? 4 : 1;        // row groups
+  static constexpr int kThreads = NT * R;          // 144 (d = 64), 136 (d = 128)
+  static constexpr int kRows = D == 64 ? 64 : 32;  // rows staged per step
+  static constexpr size_t kXsBytes = (size_t)kRows * D * 8 > (R > 1 ? (size_t)D * D * 8 : 0)
+                                         ? (size_t)kRows * D * 8
+                                         : (size_t)D * D * 8;
+  template <typename T>
+  static constexpr size_t smem() { return kXsBytes + (size_t)kRows * D * sizeof(T); }
+};
+
+// position (in doubles) of column col inside a staged fp64 row
+__device__ __forceinline__ int syrk_pos(int col) {
+  const int I = col >> 3, i = (col >> 1) & 3;
+  return ((4 * I + ((i + (I >> 1)) & 3)) << 1) | (col & 1);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) syrk_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                   int N_alloc, int n, int nch,
-                                                   const double* __restrict__ colpart,
-                                                   double* __restrict__ part) {
-  constexpr int TR = 32;
-  constexpr int B = D / 16;
-  __shared__ double xs[TR][D];
+__global__ void __maxnreg__(200) syrk_kernel(const T* __restrict__ Q,
+                                                                    const T* __restrict__ K, int N_alloc,
+                                                                    int n, int nch,
+                                                                    const double* __restrict__ colpart,
+                                                                    double* __restrict__ part) {
+  using Cfg = SyrkCfg<D>;
+  constexpr int R = Cfg::R, NTH = Cfg::kThreads, ROWS = Cfg::kRows;
+  constexpr int VEC = 16 / sizeof(T);                 // elements per 16-byte chunk
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* xs = reinterpret_cast<double*>(smem_raw);   // ROWS x D (rotated), later D x D for the group sum
+  T* raw = reinterpret_cast<T*>(smem_raw + Cfg::kXsBytes);   // ROWS x D as loaded
   __shared__ double mean[D];
   const int bh = blockIdx.y, z = blockIdx.z, ch = blockIdx.x;
   const T* X = (z == 0 ? Q : K) + (size_t)bh * N_alloc * D;
-  if (threadIdx.x < D) {
+  const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
+
+  auto issue = [&](int rt) {
+    const int rows = min(ROWS, r1 - rt);
+    for (int e = threadIdx.x; e < rows * (D / VEC); e += NTH)
+      cp_async16(raw + e * VEC, X + (size_t)rt * D + (size_t)e * VEC);
+    cp_async_commit();
+  };
+  if (r0 < r1) issue(r0);
+  for (int c = threadIdx.x; c < D; c += NTH) {
     double m = 0.0;
     if (z == 1) {
-      for (int i = 0; i < nch; ++i) m += colpart[((size_t)bh * nch + i) * D + threadIdx.x];
+      for (int i = 0; i < nch; ++i) m += colpart[((size_t)bh * nch + i) * D + c];
       m /= (double)n;
     }
-    mean[threadIdx.x] = m;
+    mean[c] = m;
   }
-  __syncthreads();
-  const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  double acc[B][B];
+  // tile t -> (I, J), I <= J, row-major over the upper triangle
+  const int g = threadIdx.x / Cfg::NT, t = threadIdx.x % Cfg::NT;
+  int I = 0, rem = t;
+  while (rem >= Cfg::TT - I) { rem -= Cfg::TT - I; ++I; }
+  const int J = I + rem;
+  double acc[8][8];
 #pragma unroll
-  for (int i = 0; i < B; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < B; ++j) acc[i][j] = 0.0;
-  const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
-  for (int rt = r0; rt < r1; rt += TR) {
-    for (int e = threadIdx.x; e < TR * D; e += 256) {
-      const int rr = e / D, cc = e % D, r = rt + rr;
-      xs[rr][cc] = (r < r1) ? (double)to_f(X[(size_t)r * D + cc]) - mean[cc] : 0.0;
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+  for (int rt = r0; rt < r1; rt += ROWS) {
+    cp_async_wait_all();
+    __syncthreads();   // raw tile complete, mean written, previous tile's products done
+    const int rows = min(ROWS, r1 - rt);
+    for (int e = threadIdx.x; e < ROWS * D; e += NTH) {
+      const int rr = e / D, cc = e % D;
+      xs[rr * D + syrk_pos(cc)] = rr < rows ? (double)to_f(raw[e]) - mean[cc] : 0.0;
     }
     __syncthreads();
-#pragma unroll 4
-    for (int rr = 0; rr < TR; ++rr) {
-      double a[B], b[B];
+    if (rt + ROWS < r1) issue(rt + ROWS);
+#pragma unroll 2
+    for (int rr = g; rr < ROWS; rr += R) {
+      const double2* row = reinterpret_cast<const double2*>(xs + rr * D);
+      double a[8], b[8];
 #pragma unroll
-      for (int i = 0; i < B; ++i) a[i] = xs[rr][ty + 16 * i];
+      for (int i = 0; i < 4; ++i) {
+        const double2 va = row[4 * I + ((i + (I >> 1)) & 3)];
+        const double2 vb = row[4 * J + ((i + (J >> 1)) & 3)];
+        a[2 * i] = va.x; a[2 * i + 1] = va.y; b[2 * i] = vb.x; b[2 * i + 1] = vb.y;
+      }
 #pragma unroll
-      for (int j = 0; j < B; ++j) b[j] = xs[rr][tx + 16 * j];
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int i = 0; i < B; ++i)
-#pragma unroll
-        for (int j = 0; j < B; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
-    __syncthreads();
   }
   double* out = part + (((size_t)bh * 2 + z) * nch + ch) * D * D;
+  if constexpr (R == 1) {
 #pragma unroll
-  for (int i = 0; i < B; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < B; ++j) out[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+      for (int j = 0; j < 8; ++j) {
+        out[(8 * I + i) * D + 8 * J + j] = acc[i][j];
+        out[(8 * J + j) * D + 8 * I + i] = acc[i][j];
+      }
+  } else {
+    __syncthreads();    // last tile's products done before xs becomes the group-sum buffer
+    double* red = xs;   // D x D, upper tiles only
+    for (int gg = 0; gg < R; ++gg) {
+      if (g == gg) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            double* dst = red + (8 * I + i) * D + 8 * J + j;
+            *dst = (gg == 0 ? 0.0 : *dst) + acc[i][j];
+          }
+      }
+      __syncthreads();
+    }
+    for (int e = threadIdx.x; e < D * D; e += NTH) {
+      const int i = e / D, j = e % D;
+      out[e] = (i / 8 <= j / 8) ? red[e] : red[j * D + i];
+    }
+  }
 }
 
 // M[th] for tensor-head th = 2 bh + tensor: queries (tensor 0) are split in
@@ -920,7 +999,10 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
   if (plan.levels > 0) {
     plan_kernel<<<1, 1024, 0, st>>>(n, c, nodes, level_begin);
     colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
-    syrk_kernel<T, D><<<dim3(nch, BH, 2), 256, 0, st>>>(Q, K, N_alloc, n, nch, colpart, metpart);
+    const size_t syrk_smem = SyrkCfg<D>::template smem<T>();
+    cudaFuncSetAttribute(syrk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
+    syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
+                                                                                metpart);
     metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
     const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
     cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);

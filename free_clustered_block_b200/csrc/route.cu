@@ -5,136 +5,208 @@
 // "Selection": each query cluster keeps its k best-scoring key clusters.
 // Scores are fp64; the selection is exact, equal scores ordered by the lower
 // key-cluster index, and the kept list is written in ascending order.
+//
+// A block handles QA query clusters of one head.
+//  * Scores: thread t holds key centroid b = t, t + 256, ... in registers (64
+//    columns at a time) and forms its QA dot products against the query
+//    centroids, which every lane reads from shared memory as broadcasts. The
+//    dot product runs over the columns in order with one fma chain.
+//  * Selection: one warp per query cluster runs a radix select over the
+//    order-preserving 64-bit keys of the scores, 8 bits per pass from the top,
+//    starting below the prefix that all C keys share. A pass histograms the
+//    keys that still match the decided prefix and picks the digit where the
+//    running count from the top reaches the number still to take; it stops as
+//    soon as that whole digit bin is taken. Keys above the final prefix are
+//    kept; keys equal to it are kept in ascending index order until k are
+//    kept. The kept bitmask word w is the warp's ballot over keys 32w..32w+31.
 #include "ca_internal.cuh"
 
 namespace ca {
 namespace {
 
 constexpr int kRouteThreads = 256;
-constexpr int kRouteTile = 64;   // key centroids staged per step
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr size_t kRouteSmemBudget = 120 * 1024;
 
-template <int D>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(const double* __restrict__ qbar,
-                                                              const double* __restrict__ kbar, int C,
-                                                              int Cpad, int k, int32_t* __restrict__ kept_idx,
-                                                              uint32_t* __restrict__ kept_bits) {
-  constexpr int P = kRouteThreads / kRouteTile;   // partial sums per score
-  constexpr int DP = D / P;
+template <int D, int QA>
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* __restrict__ qbar,
+                                                                 const double* __restrict__ kbar, int C, int k,
+                                                                 int32_t* __restrict__ kept_idx,
+                                                                 uint32_t* __restrict__ kept_bits) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  double* qa = reinterpret_cast<double*>(smem_raw);        // D
-  double* kt = qa + D;                                     // kRouteTile * (D + 1)
-  double* part = kt + kRouteTile * (D + 1);                // kRouteThreads
-  double* sc = part + kRouteThreads;                       // Cpad
-  int* id = reinterpret_cast<int*>(sc + Cpad);             // Cpad
-  uint32_t* bits = reinterpret_cast<uint32_t*>(id + Cpad); // Cpad / 32
-  __shared__ int woff[kRouteThreads + 1];
+  double* qs = reinterpret_cast<double*>(smem_raw);   // QA x D
+  double* sc = qs + QA * D;                           // QA x C scores
+  __shared__ uint32_t hist[kRouteWarps][256];
 
-  const int a = blockIdx.x, bh = blockIdx.y;
-  const double* kb = kbar + (size_t)bh * C * D;
-  if (threadIdx.x < D) qa[threadIdx.x] = qbar[((size_t)bh * C + a) * D + threadIdx.x];
-  const int bl = threadIdx.x % kRouteTile, pp = threadIdx.x / kRouteTile;
-  for (int b0 = 0; b0 < Cpad; b0 += kRouteTile) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < kRouteTile * D; e += kRouteThreads) {
-      const int r = e / D, col = e % D, b = b0 + r;
-      kt[r * (D + 1) + col] = (b < C) ? kb[(size_t)b * D + col] : 0.0;
-    }
-    __syncthreads();
-    double s = 0.0;
-#pragma unroll 8
-    for (int j = pp * DP; j < (pp + 1) * DP; ++j) s = fma(qa[j], kt[bl * (D + 1) + j], s);
-    part[threadIdx.x] = s;
-    __syncthreads();
-    if (threadIdx.x < kRouteTile) {
-      const int b = b0 + threadIdx.x;
-      double t = 0.0;
-      for (int q = 0; q < P; ++q) t += part[q * kRouteTile + threadIdx.x];
-      sc[b] = (b < C) ? t : -INFINITY;
-      id[b] = (b < C) ? b : 0x7fffffff;
-    }
+  const int a0 = blockIdx.x * QA, bh = blockIdx.y;
+  const int nq = min(QA, C - a0);
+  for (int e = threadIdx.x; e < QA * D; e += kRouteThreads) {
+    const int r = e / D;
+    qs[e] = r < nq ? qbar[((size_t)bh * C + a0 + r) * D + (e % D)] : 0.0;
   }
   __syncthreads();
-  // Bitonic sort: descending score, ascending index.
-  for (int size = 2; size <= Cpad; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < Cpad; i += kRouteThreads) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const double si = sc[i], sj = sc[j];
-          const int ii = id[i], ij = id[j];
-          const bool i_first = (si > sj) || (si == sj && ii < ij);
-          const bool up = ((i & size) == 0);
-          if (up ? !i_first : i_first) { sc[i] = sj; sc[j] = si; id[i] = ij; id[j] = ii; }
+
+  // ---- scores ----
+  const double* kb = kbar + (size_t)bh * C * D;
+  for (int b = threadIdx.x; b < C; b += kRouteThreads) {
+    double s[QA];
+#pragma unroll
+    for (int r = 0; r < QA; ++r) s[r] = 0.0;
+#pragma unroll
+    for (int h = 0; h < D; h += 64) {
+      double kr[64];
+      const double2* src = reinterpret_cast<const double2*>(kb + (size_t)b * D + h);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const double2 v = __ldg(src + i);
+        kr[2 * i] = v.x; kr[2 * i + 1] = v.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+#pragma unroll
+        for (int r = 0; r < QA; ++r) {
+          const double2 q2 = *reinterpret_cast<const double2*>(qs + r * D + h + 2 * i);
+          s[r] = fma(q2.x, kr[2 * i], s[r]);
+          s[r] = fma(q2.y, kr[2 * i + 1], s[r]);
         }
       }
-      __syncthreads();
     }
+#pragma unroll
+    for (int r = 0; r < QA; ++r) sc[(size_t)r * C + b] = s[r];
   }
+  __syncthreads();
+
+  // ---- selection, one warp per query cluster ----
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
   const int W = (C + 31) / 32;
-  for (int w = threadIdx.x; w < W; w += kRouteThreads) bits[w] = 0u;
-  __syncthreads();
-  for (int i = threadIdx.x; i < k; i += kRouteThreads) atomicOr(&bits[id[i] >> 5], 1u << (id[i] & 31));
-  __syncthreads();
-  uint32_t* brow = kept_bits + ((size_t)bh * C + a) * W;
-  for (int w = threadIdx.x; w < W; w += kRouteThreads) brow[w] = bits[w];
-  // Ascending kept list from the bitmask (W <= 256 words per pass).
-  int32_t* krow = kept_idx + ((size_t)bh * C + a) * k;
-  for (int w0 = 0, base = 0; w0 < W; w0 += kRouteThreads) {
-    const int w = w0 + threadIdx.x;
-    const int pc = (w < W) ? __popc(bits[w]) : 0;
-    if (threadIdx.x == 0) woff[0] = 0;
-    __syncthreads();
-    // serial exclusive scan (W is small)
-    if (threadIdx.x == 0) {
-      int s = 0;
-      for (int i = 0; i < kRouteThreads; ++i) {
-        const int ww = w0 + i;
-        woff[i] = s;
-        s += (ww < W) ? __popc(bits[ww]) : 0;
-      }
-      woff[kRouteThreads] = s;
+  uint32_t* h = hist[warp];
+  for (int r = warp; r < nq; r += kRouteWarps) {
+    const double* row = sc + (size_t)r * C;
+    // common prefix of all keys
+    uint64_t kand = ~0ull, kor = 0ull;
+    for (int b = lane; b < C; b += 32) {
+      const uint64_t key = ordered_key(row[b]);
+      kand &= key; kor |= key;
     }
-    __syncthreads();
-    if (w < W) {
-      uint32_t m = bits[w];
-      int o = base + woff[threadIdx.x];
-      while (m) {
-        const int bpos = __ffs(m) - 1;
-        krow[o++] = w * 32 + bpos;
-        m &= m - 1;
-      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+      kor |= __shfl_xor_sync(0xffffffffu, kor, o);
     }
-    (void)pc;
-    base += woff[kRouteThreads];
-    __syncthreads();
+    const uint64_t diff = kand ^ kor;
+    int L = diff ? (__clzll((long long)diff) & ~7) : 64;   // decided prefix length (bits)
+    uint64_t P = L == 0 ? 0ull : (L == 64 ? kand : kand >> (64 - L));
+    int krem = k;                     // still to take among keys whose prefix equals P
+    bool all = (k >= C);              // every key matching P is kept
+    while (!all && L < 64) {
+      for (int i = lane; i < 256; i += 32) h[i] = 0u;
+      __syncwarp();
+      const int shift = 56 - L;
+      for (int b0 = 0; b0 < C; b0 += 32) {
+        const int b = b0 + lane;
+        int dig = 256 + lane;          // no bin
+        if (b < C) {
+          const uint64_t key = ordered_key(row[b]);
+          if (L == 0 || (key >> (64 - L)) == P) dig = (int)((key >> shift) & 255u);
+        }
+        const unsigned grp = __match_any_sync(0xffffffffu, dig);
+        if (dig < 256 && (grp & lt) == 0u) atomicAdd(&h[dig], (uint32_t)__popc(grp));
+      }
+      __syncwarp();
+      // lane l owns bins 255 - 8l ... 248 - 8l, scanned from the top
+      uint32_t cnt[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cnt[j] = h[255 - 8 * lane - j]; tot += cnt[j]; }
+      uint32_t inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+      }
+      const uint32_t exc = inc - tot;
+      const bool mine = exc < (uint32_t)krem && (uint32_t)krem <= inc;
+      const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+      int dsel = 0;
+      uint32_t above = 0, inbin = 0;
+      if (mine) {
+        uint32_t c = exc;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (inbin == 0u && c + cnt[j] >= (uint32_t)krem) { dsel = 255 - 8 * lane - j; above = c; inbin = cnt[j]; }
+          c += cnt[j];
+        }
+      }
+      dsel = __shfl_sync(0xffffffffu, dsel, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      inbin = __shfl_sync(0xffffffffu, inbin, src);
+      krem -= (int)above;
+      P = (P << 8) | (uint64_t)dsel;
+      L += 8;
+      if (inbin == (uint32_t)krem) all = true;
+      __syncwarp();
+    }
+    // membership, bitmask and ascending kept list
+    int32_t* krow = kept_idx + ((size_t)bh * C + a0 + r) * k;
+    uint32_t* brow = kept_bits + ((size_t)bh * C + a0 + r) * W;
+    int base = 0, eqseen = 0;
+    for (int i = 0; i < W; ++i) {
+      const int b = i * 32 + lane;
+      bool take = false, eq = false;
+      if (b < C) {
+        const uint64_t key = ordered_key(row[b]);
+        const uint64_t top = L == 0 ? 0ull : (L == 64 ? key : key >> (64 - L));
+        take = top > P;
+        eq = top == P;
+      }
+      const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      if (eq) take = all || (eqseen + __popc(eqb & lt) < krem);
+      eqseen += __popc(eqb);
+      const unsigned tb = __ballot_sync(0xffffffffu, take);
+      if (lane == 0) brow[i] = tb;
+      if (take) krow[base + __popc(tb & lt)] = b;
+      base += __popc(tb);
+    }
   }
+}
+
+template <int D, int QA>
+size_t route_smem(int C) {
+  return (size_t)QA * D * 8 + (size_t)QA * C * 8;
+}
+
+template <int D, int QA>
+cudaError_t launch_qa(const ca_shape* s, int C, const double* qbar, const double* kbar, int k, int32_t* kept_idx,
+                      uint32_t* kept_bits, cudaStream_t st) {
+  const size_t smem = route_smem<D, QA>(C);
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((C + QA - 1) / QA, s->B * s->H);
+  route_kernel<D, QA><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, k, kept_idx, kept_bits);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const ca_shape* s, int C, const double* qbar, const double* kbar, int k, int32_t* kept_idx,
+                     uint32_t* kept_bits, cudaStream_t st) {
+  // as many query clusters per block as the score rows allow in the budget
+  if (route_smem<D, 16>(C) <= kRouteSmemBudget) return launch_qa<D, 16>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+  if (route_smem<D, 8>(C) <= kRouteSmemBudget) return launch_qa<D, 8>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+  if (route_smem<D, 4>(C) <= kRouteSmemBudget) return launch_qa<D, 4>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+  if (route_smem<D, 2>(C) <= kRouteSmemBudget) return launch_qa<D, 2>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+  return launch_qa<D, 1>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
 }
 
 }  // namespace
 
 size_t route_smem_bytes(int C, int D) {
-  int Cpad = 1;
-  while (Cpad < C) Cpad <<= 1;
-  if (Cpad < kRouteTile) Cpad = kRouteTile;
-  return (size_t)D * 8 + (size_t)kRouteTile * (D + 1) * 8 + kRouteThreads * 8 + (size_t)Cpad * 12 +
-         (size_t)(Cpad / 32 + 1) * 4;
+  return D == 64 ? route_smem<64, 1>(C) : route_smem<128, 1>(C);
 }
 
 cudaError_t launch_route(const ca_shape* s, int C, const double* qbar, const double* kbar, int k,
                          int32_t* kept_idx, uint32_t* kept_bits, cudaStream_t st) {
-  int Cpad = 1;
-  while (Cpad < C) Cpad <<= 1;
-  if (Cpad < kRouteTile) Cpad = kRouteTile;
-  const size_t smem = route_smem_bytes(C, s->d);
-  const dim3 grid(C, s->B * s->H);
-  if (s->d == 64) {
-    cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    route_kernel<64><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, Cpad, k, kept_idx, kept_bits);
-  } else {
-    cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    route_kernel<128><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, Cpad, k, kept_idx, kept_bits);
-  }
-  return cudaGetLastError();
+  if (s->d == 64) return launch_d<64>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+  return launch_d<128>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
 }
 
 }  // namespace ca

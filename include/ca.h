@@ -161,7 +161,8 @@ ca_status ca_cluster_noalloc(const void* Q, const void* K, const ca_shape* shape
  * and Section 3.3.2 (keep the k best-scoring key clusters per query cluster).
  * Exact top-k; equal scores go to the lower key-cluster index.
  * centroids: device qbar/kbar (fp64) as produced by ca_cluster or supplied by
- * the caller; only qbar and kbar are read. out: device kept_idx and kept_bits;
+ * the caller; only qbar and kbar are read, and both must be 16-byte aligned
+ * (CA_ERR_INVALID_ARG otherwise). out: device kept_idx and kept_bits;
  * out->k is k. 1 <= k <= C, C <= 8192.
  */
 ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
