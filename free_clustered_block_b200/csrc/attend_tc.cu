@@ -8,13 +8,15 @@
 // the same kernel with every key block kept and no compensation.
 //
 // One CTA handles one 128-row query tile of one head and holds an SM (512
-// TMEM columns: two S buffers and O):
+// TMEM columns: three S buffers and O):
 //   warp 0      TMA producer (one thread): Q tile once, then a ring of
 //               stages holding (K, V) of a kept key block, (kbar_hi,
 //               kbar_lo) or (vbar_hi, vbar_lo) of a centroid block;
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into TMEM buffer
-//               j % 2, so S_{j+1} is computed while the softmax works on S_j;
-//               O += P_j V_j with P_j read from TMEM;
+//   warp 1      MMA issuer (the converged warp, one elected lane issuing):
+//               S_j = Q K_j^T into TMEM buffer j % 3 and O += P_j V_j with
+//               P_j read from TMEM. S_{j+2} is issued right behind PV_j: its
+//               buffer was last read by PV_{j-1}, so the tensor pipe gets both
+//               without waiting for PV_j, and the softmax of S_{j+1} overlaps;
 //   warps 2..9  softmax, two threads per query row (one per half of the key
 //               block): read S_j from TMEM, apply the key mask /
 //               compensation bias, exchange the row max through shared
@@ -96,22 +98,27 @@ __device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, uint64
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t* b) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
-               : "memory");
-}
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// tcgen05.mma (A and B from shared memory, or A from TMEM) and commit, issued
+// by one elected lane of a converged warp: the whole warp computes the
+// (warp-uniform) operands, so issue needs no divergent single-lane code.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u)
       : "memory");
 }
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void mma_ts_elect(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
+      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint64_t* b) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(su32(b))
       : "memory");
 }
 
@@ -149,6 +156,30 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// packed pairs of f32 (sm_100 f32x2 arithmetic) and the three-input max
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -200,8 +231,8 @@ __device__ __forceinline__ void raise_timeout(volatile int* abort_flag) {
   *abort_flag = 1;
 }
 // Bounded wait (limit in ns); false on timeout or when another role aborted.
-__device__ __noinline__ bool wait_bar(uint64_t* b, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
-  if (mbar_try(b, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, uint64_t limit_ns,
+                                           volatile int* abort_flag) {
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(b, parity)) return true;
@@ -210,6 +241,11 @@ __device__ __noinline__ bool wait_bar(uint64_t* b, uint32_t parity, uint64_t lim
       if (now_ns() - t0 > limit_ns) { raise_timeout(abort_flag); return false; }
     }
   }
+}
+// The first probe is inline: a barrier that has already flipped costs no call.
+__device__ __forceinline__ bool wait_bar(uint64_t* b, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
+  if (mbar_try(b, parity)) return true;
+  return wait_bar_slow(b, parity, limit_ns, abort_flag);
 }
 // Bounded wait used while draining: ignores the abort flag, fixed limit.
 __device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
@@ -244,7 +280,7 @@ struct TcParams {
 #define CA_TC_SPLIT 2   // softmax threads per query row
 #endif
 #ifndef CA_TC_NBUF
-#define CA_TC_NBUF 2    // S buffers in TMEM
+#define CA_TC_NBUF 3    // S buffers in TMEM
 #endif
 
 template <int D, int KB>
@@ -269,7 +305,7 @@ struct TcCfg {
   static constexpr int kSoftmaxThreads = 128 * kSplit;                 // kSplit threads per row
   static constexpr int kThreads = 64 + kSoftmaxThreads;                // + producer warp + MMA warp
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kSCol = 0;        // S buffers at 0 and KB; P_j (bf16 pairs) over the front half
+  static constexpr uint32_t kSCol = 0;        // S buffers at 0, KB, 2 KB; P_j (bf16 pairs) over the front half
   static constexpr uint32_t kOCol = kNBuf * KB;      // O (fp32, D columns)
   static constexpr int kHalf = KB / kSplit;          // columns of S per softmax thread
   static_assert(kOCol + D <= kTmemCols, "S buffers and O must fit in TMEM");
@@ -298,10 +334,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* full = bars;              // [NS] stage loaded
   uint64_t* empty = bars + NS;        // [NS] stage released
   uint64_t* q_full = bars + 2 * NS;   // Q tile loaded
-  uint64_t* s_full = q_full + 1;      // [2] S_j computed in buffer j&1
-  uint64_t* p_full = s_full + 2;      // [2] P_j written in buffer j&1
-  uint64_t* pv_done = p_full + 2;     // O += P_j V_j completed
-  uint64_t* drain = pv_done + 1;
+  constexpr int NB = Cfg::kNBuf;
+  uint64_t* s_full = q_full + 1;      // [NB] S_j computed in buffer j % NB
+  uint64_t* p_full = s_full + NB;     // [NB] P_j written in buffer j % NB
+  uint64_t* pv_done = p_full + NB;    // [NB] O += P_j V_j completed (j % NB)
+  uint64_t* drain = pv_done + NB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias = reinterpret_cast<float*>(smem + Cfg::kBiasOff);
@@ -333,9 +370,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(q_full, 1);
-    mbar_init(&s_full[0], 1); mbar_init(&s_full[1], 1);
-    mbar_init(&p_full[0], Cfg::kSoftmaxThreads); mbar_init(&p_full[1], Cfg::kSoftmaxThreads);
-    mbar_init(pv_done, 1);
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], Cfg::kSoftmaxThreads);
+      mbar_init(&pv_done[b], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -405,75 +444,76 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
-      constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
-      const uint32_t q_base = su32(sQ);
-      bool ok = wait_bar(q_full, 0, limit, abort_flag);
-      // item index of block j's QK and PV operands
-      auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
-      auto pv_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept) + 1; };
-      auto issue_qk = [&](int j) -> bool {
-        const int i = qk_item(j);
-        const int s = i % NS, r = i / NS;
-        if (!wait_bar(&full[s], r & 1, limit, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
-        const uint32_t d_tmem = tmem + Cfg::kSCol + (uint32_t)((j % Cfg::kNBuf) * KB);
-        const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
-        for (int mtx = 0; mtx < nmat; ++mtx) {
-          const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
+    // The whole warp runs this loop (so descriptors are warp-uniform); one
+    // elected lane issues each tcgen05 instruction and every commit.
+    constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
+    constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
+    const uint32_t q_base = su32(sQ);
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, limit, abort_flag));
+    };
+    bool ok = wwait(q_full, 0);
+    // item index of block j's QK and PV operands
+    auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
+    auto pv_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept) + 1; };
+    auto issue_qk = [&](int j) -> bool {
+      const int i = qk_item(j);
+      const int s = i % NS, r = i / NS;
+      if (!wwait(&full[s], r & 1)) return false;
+      tc_fence_after();
+      const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
+      const uint32_t d_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
+      const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
+      for (int mtx = 0; mtx < nmat; ++mtx) {
+        const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (uint32_t)((kk & 3) * 32);   // 16 bf16 along K inside the 128B row
-            const uint64_t ad = sdesc(q_base + (kk >> 2) * 128 * 128 + off, 16, 1024);
-            const uint64_t bd = sdesc(bbase + (kk >> 2) * KB * 128 + off, 16, 1024);
-            mma_ss(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        // Commits track every earlier MMA of this thread too: when s_full[b]
-        // flips for S_j, PV_{j-2} (the last reader of that buffer) is done.
-        tc_commit(&s_full[j % Cfg::kNBuf]);
-        if (j >= J_kept) tc_commit(&empty[s]);   // kbar stage is free once S is computed
-        return true;
-      };
-      constexpr int NB = Cfg::kNBuf;
-      for (int j = 0; j < NB && j < J && ok; ++j) ok = issue_qk(j);
-      for (int j = 0; j < J && ok; ++j) {
-        if (!wait_bar(&p_full[j % NB], (j / NB) & 1, limit, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const int i = pv_item(j);
-        const int s = i % NS, r = i / NS;
-        if (j >= J_kept) {
-          if (!wait_bar(&full[s], r & 1, limit, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-        }
-        const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
-        const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
-        const int nmat = (j < J_kept) ? 1 : 2;
-        for (int mtx = 0; mtx < nmat; ++mtx) {
-          const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < KB / 16; ++kk) {
-            const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
-            mma_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        tc_commit(pv_done);
-        tc_commit(&empty[s]);
-        // S_{j+NB} overwrites P_j: issue it only once PV_j (the last reader of
-        // that buffer) has completed.
-        if (j + NB < J) {
-          if (!wait_bar(pv_done, j & 1, limit, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          ok = issue_qk(j + NB);
-          if (!ok) break;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk & 3) * 32);   // 16 bf16 along K inside the 128B row
+          const uint64_t ad = sdesc(q_base + (kk >> 2) * 128 * 128 + off, 16, 1024);
+          const uint64_t bd = sdesc(bbase + (kk >> 2) * KB * 128 + off, 16, 1024);
+          mma_ss_elect(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
         }
       }
-      // Drain: every MMA issued so far has completed once `drain` flips.
-      tc_commit(drain);
-      drain_bar(drain, 0);
+      tc_commit_elect(&s_full[j % NB]);
+      if (j >= J_kept) tc_commit_elect(&empty[s]);   // kbar stage is free once S is computed
+      return true;
+    };
+    // S_0 .. S_{NB-2} ahead; afterwards S_{j+NB-1} follows PV_j. Its buffer
+    // was last read (as P_{j-1}) by PV_{j-1}, committed one step earlier.
+    for (int j = 0; j < NB - 1 && j < J && ok; ++j) ok = issue_qk(j);
+    for (int j = 0; j < J && ok; ++j) {
+      if (!wwait(&p_full[j % NB], (j / NB) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const int i = pv_item(j);
+      const int s = i % NS, r = i / NS;
+      if (j >= J_kept) {
+        if (!wwait(&full[s], r & 1)) { ok = false; break; }
+        tc_fence_after();
+      }
+      const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
+      const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
+      const int nmat = (j < J_kept) ? 1 : 2;
+      for (int mtx = 0; mtx < nmat; ++mtx) {
+        const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < KB / 16; ++kk) {
+          const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
+          mma_ts_elect(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      tc_commit_elect(&pv_done[j % NB]);
+      tc_commit_elect(&empty[s]);
+      const int jn = j + NB - 1;
+      if (jn < J) {
+        if (j > 0 && !wwait(&pv_done[(j - 1) % NB], ((j - 1) / NB) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (!issue_qk(jn)) { ok = false; break; }
+      }
     }
+    // Drain: every MMA issued so far has completed once `drain` flips.
+    tc_commit_elect(drain);
+    if (lane == 0) drain_bar(drain, 0);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
     const int st = threadIdx.x - 64;          // 0..255 within the softmax group
@@ -489,7 +529,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int col0 = half * HC;               // first S column of this thread
     for (int j = 0; j < J; ++j) {
       const bool cent = j >= J_kept;
-      constexpr int NB = Cfg::kNBuf;
       const uint32_t sbuf = Cfg::kSCol + (uint32_t)((j % NB) * KB);
       if (cent) {
         // per-column compensation bias of this centroid block (log2 units)
@@ -525,22 +564,16 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-      if (mode == 0) {
+      if (mode == 1) {
 #pragma unroll
-        for (int q = 0; q < HC; ++q) m8[q & 7] = fmaxf(m8[q & 7], sv[q]);
-      } else if (mode == 1) {
-#pragma unroll
-        for (int q = 0; q < HC; ++q) {
+        for (int q = 0; q < HC; ++q)
           if (q >= vloc) sv[q] = -INFINITY;
-          m8[q & 7] = fmaxf(m8[q & 7], sv[q]);
-        }
-      } else {
+      } else if (mode == 2) {
 #pragma unroll
-        for (int q = 0; q < HC; ++q) {
-          sv[q] = fmaf(sv[q], sc, bias[col0 + q]);
-          m8[q & 7] = fmaxf(m8[q & 7], sv[q]);
-        }
+        for (int q = 0; q < HC; ++q) sv[q] = fmaf(sv[q], sc, bias[col0 + q]);
       }
+#pragma unroll
+      for (int q = 0; q < HC; q += 2) m8[(q >> 1) & 7] = max3(m8[(q >> 1) & 7], sv[q], sv[q + 1]);
       float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       if (mode != 2) pm *= sc;             // log2 units
       // combine the two halves of the row; after this barrier every S column
@@ -565,7 +598,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // half of O.
       bool wok = true;
       const bool wneed = __any_sync(0xffffffffu, need);
-      if (wneed) wok = __all_sync(0xffffffffu, wait_bar(pv_done, (j - 1) & 1, limit, abort_flag));
+      if (wneed) wok = __all_sync(0xffffffffu, wait_bar(&pv_done[(j - 1) % NB], ((j - 1) / NB) & 1, limit, abort_flag));
       ok = group_all_n(wok, Cfg::kSoftmaxThreads);
       if (!ok) break;
       if (wneed) {
@@ -583,23 +616,33 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       // P = 2^(x - m) as bf16 pairs over the front half of this S buffer
       const float xs = (mode == 2) ? 1.f : sc;
+      const uint64_t xs2 = f2_pack(xs, xs), nb2 = f2_pack(nb, nb);
+      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};   // packed partial row sums
 #pragma unroll
       for (int c0 = 0; c0 < HC; c0 += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          const float p0 = ex2(fmaf(sv[c0 + 2 * q], xs, nb)), p1 = ex2(fmaf(sv[c0 + 2 * q + 1], xs, nb));
-          lreg += p0 + p1;
+          float t0, t1;
+          f2_unpack(fma2(f2_pack(sv[c0 + 2 * q], sv[c0 + 2 * q + 1]), xs2, nb2), t0, t1);
+          const float p0 = ex2(t0), p1 = ex2(t1);
+          ls2[q & 3] = add2(ls2[q & 3], f2_pack(p0, p1));
           pk[q] = pack_bf16(p0, p1);
         }
         CA_TMEM_ST16(lane_addr + sbuf + (uint32_t)((col0 + c0) / 2), pk);
+      }
+      {
+        float a0, a1;
+        f2_unpack(add2(add2(ls2[0], ls2[1]), add2(ls2[2], ls2[3])), a0, a1);
+        lreg += a0 + a1;
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[j % NB]);
     }
     // epilogue: O / l to the query's original row; each half writes D/2 columns
-    if (ok && J > 0) ok = group_all_n(wait_bar(pv_done, (J - 1) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
+    if (ok && J > 0)
+      ok = group_all_n(wait_bar(&pv_done[(J - 1) % NB], ((J - 1) / NB) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
     if (ok && J > 0) {
       tc_fence_after();
       int orow;

@@ -139,11 +139,12 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, in
 // ---------------------------------------------------------------------------
 template <int D>
 struct SyrkCfg {
-  static constexpr int TT = D / 8;                 // tile rows
-  static constexpr int NT = TT * (TT + 1) / 2;     // upper tiles incl. diagonal
-  static constexpr int R = D == 64 ? 4 : 1;        // row groups
-  static constexpr int kThreads = NT * R;          // 144 (d = 64), 136 (d = 128)
-  static constexpr int kRows = D == 64 ? 64 : 32;  // rows staged per step
+  static constexpr int TR = D / 8;                 // 8-row tile rows
+  static constexpr int TC = D / 4;                 // 4-column tile columns
+  static constexpr int NT = TR * TC - TR * (TR - 1);   // tiles (I, J) with 4J + 3 >= 8I: 72 / 272
+  static constexpr int R = D == 64 ? 3 : 1;        // row groups
+  static constexpr int kThreads = NT * R;          // 216 (d = 64), 272 (d = 128)
+  static constexpr int kRows = D == 64 ? 63 : 32;  // rows staged per step (a multiple of R)
   static constexpr size_t kXsBytes = (size_t)kRows * D * 8 > (R > 1 ? (size_t)D * D * 8 : 0)
                                          ? (size_t)kRows * D * 8
                                          : (size_t)D * D * 8;
@@ -165,11 +166,9 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 template <typename T, int D>
-__global__ void __maxnreg__(200) syrk_kernel(const T* __restrict__ Q,
-                                                                    const T* __restrict__ K, int N_alloc,
-                                                                    int n, int nch,
-                                                                    const double* __restrict__ colpart,
-                                                                    double* __restrict__ part) {
+__global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* __restrict__ K, int N_alloc,
+                                             int n, int nch, const double* __restrict__ colpart,
+                                             double* __restrict__ part) {
   using Cfg = SyrkCfg<D>;
   constexpr int R = Cfg::R, NTH = Cfg::kThreads, ROWS = Cfg::kRows;
   constexpr int VEC = 16 / sizeof(T);                 // elements per 16-byte chunk
@@ -196,16 +195,17 @@ __global__ void __maxnreg__(200) syrk_kernel(const T* __restrict__ Q,
     }
     mean[c] = m;
   }
-  // tile t -> (I, J), I <= J, row-major over the upper triangle
+  // tile t -> (I, J): rows 8I..8I+7, columns 4J..4J+3, J >= 2I (on or above the diagonal)
   const int g = threadIdx.x / Cfg::NT, t = threadIdx.x % Cfg::NT;
   int I = 0, rem = t;
-  while (rem >= Cfg::TT - I) { rem -= Cfg::TT - I; ++I; }
-  const int J = I + rem;
-  double acc[8][8];
+  while (rem >= Cfg::TC - 2 * I) { rem -= Cfg::TC - 2 * I; ++I; }
+  const int J = 2 * I + rem;
+  const int JI = J >> 1, Jc = 2 * (J & 1);             // 8-column group and first chunk of it
+  double acc[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
   for (int rt = r0; rt < r1; rt += ROWS) {
     cp_async_wait_all();
     __syncthreads();   // raw tile complete, mean written, previous tile's products done
@@ -216,49 +216,54 @@ __global__ void __maxnreg__(200) syrk_kernel(const T* __restrict__ Q,
     }
     __syncthreads();
     if (rt + ROWS < r1) issue(rt + ROWS);
-#pragma unroll 2
+#pragma unroll (D == 64 ? 2 : 1)
     for (int rr = g; rr < ROWS; rr += R) {
       const double2* row = reinterpret_cast<const double2*>(xs + rr * D);
-      double a[8], b[8];
+      double a[8], b[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const double2 va = row[4 * I + ((i + (I >> 1)) & 3)];
-        const double2 vb = row[4 * J + ((i + (J >> 1)) & 3)];
-        a[2 * i] = va.x; a[2 * i + 1] = va.y; b[2 * i] = vb.x; b[2 * i + 1] = vb.y;
+        a[2 * i] = va.x; a[2 * i + 1] = va.y;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const double2 vb = row[4 * JI + ((Jc + i + (JI >> 1)) & 3)];
+        b[2 * i] = vb.x; b[2 * i + 1] = vb.y;
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
     }
   }
   double* out = part + (((size_t)bh * 2 + z) * nch + ch) * D * D;
+  // an entry (r, c) with c >= r lies in exactly one tile; write it and its mirror
   if constexpr (R == 1) {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        out[(8 * I + i) * D + 8 * J + j] = acc[i][j];
-        out[(8 * J + j) * D + 8 * I + i] = acc[i][j];
+      for (int j = 0; j < 4; ++j) {
+        const int r = 8 * I + i, c = 4 * J + j;
+        if (c >= r) { out[r * D + c] = acc[i][j]; out[c * D + r] = acc[i][j]; }
       }
   } else {
-    __syncthreads();    // last tile's products done before xs becomes the group-sum buffer
-    double* red = xs;   // D x D, upper tiles only
+    __syncthreads();    // last tile's products done before xs becomes the group sum
+    double* red = xs;   // D x D, entries (r, c >= r)
     for (int gg = 0; gg < R; ++gg) {
       if (g == gg) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            double* dst = red + (8 * I + i) * D + 8 * J + j;
-            *dst = (gg == 0 ? 0.0 : *dst) + acc[i][j];
+          for (int j = 0; j < 4; ++j) {
+            const int r = 8 * I + i, c = 4 * J + j;
+            if (c >= r) red[r * D + c] = (gg == 0 ? 0.0 : red[r * D + c]) + acc[i][j];
           }
       }
       __syncthreads();
     }
     for (int e = threadIdx.x; e < D * D; e += NTH) {
       const int i = e / D, j = e % D;
-      out[e] = (i / 8 <= j / 8) ? red[e] : red[j * D + i];
+      out[e] = j >= i ? red[e] : red[j * D + i];
     }
   }
 }
@@ -342,6 +347,54 @@ __global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int
     const int r = r0 + ty + 16 * i;
     if (tx == 0 && r < n) inv_s[(size_t)bh * n + r] = (s > 0.0) ? 1.0 / sqrt(s) : 0.0;
   }
+}
+
+// d = 64 variant: one thread per query row, the row held in registers as
+// fp64. q^T M q = sum_i q_i (M_ii q_i + 2 sum_{j>i} M_ij q_j) uses only the
+// upper triangle of the symmetric M (2080 fma per row instead of 4160); every
+// lane reads the same M entries, so the shared-memory loads are broadcasts.
+template <typename T>
+__global__ void __launch_bounds__(128, 3) qnorm64_kernel(const T* __restrict__ Q, int N_alloc, int n,
+                                                      const double* __restrict__ M,
+                                                      double* __restrict__ inv_s) {
+  constexpr int D = 64;
+  __shared__ __align__(16) double Ms[D * D];
+  const int bh = blockIdx.y, r = blockIdx.x * 128 + threadIdx.x;
+  const double* Mh = M + (size_t)(bh * 2) * D * D;   // queries use M_k
+  for (int e = threadIdx.x; e < D * D / 2; e += 128)
+    reinterpret_cast<double2*>(Ms)[e] = reinterpret_cast<const double2*>(Mh)[e];
+  double x[D];
+  {
+    constexpr int VEC = 16 / sizeof(T);
+    const uint4* src = reinterpret_cast<const uint4*>(Q + ((size_t)bh * N_alloc + (r < n ? r : 0)) * D);
+    uint4 raw[D / VEC];
+#pragma unroll
+    for (int v = 0; v < D / VEC; ++v) raw[v] = __ldg(src + v);
+#pragma unroll
+    for (int v = 0; v < D / VEC; ++v) {
+      const T* e = reinterpret_cast<const T*>(&raw[v]);
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) x[v * VEC + u] = (double)to_f(e[u]);
+    }
+  }
+  __syncthreads();
+  if (r >= n) return;
+  double s = 0.0;
+#pragma unroll
+  for (int i = 0; i < D; ++i) {
+    const double* Mi = Ms + i * D;
+    double t0 = 0.0, t1 = 0.0;
+    int j = i + 1;
+    if (j & 1) { t0 = Mi[j] * x[j]; ++j; }
+#pragma unroll
+    for (; j < D; j += 2) {
+      const double2 m2 = *reinterpret_cast<const double2*>(Mi + j);
+      t0 = fma(m2.x, x[j], t0);
+      t1 = fma(m2.y, x[j + 1], t1);
+    }
+    s = fma(x[i], fma(2.0, t0 + t1, Mi[i] * x[i]), s);
+  }
+  inv_s[(size_t)bh * n + r] = (s > 0.0) ? 1.0 / sqrt(s) : 0.0;
 }
 
 // ---------------------------------------------------------------------------
@@ -1004,9 +1057,13 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
                                                                                 metpart);
     metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
-    const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
-    cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
-    qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, transform, inv_s);
+    if (D == 64 && transform) {
+      qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
+    } else {
+      const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
+      cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
+      qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, transform, inv_s);
+    }
     const int m_cap = sample_factor * D;
     const int dir_warps = DirCfg<T, D>::warps(m_cap);
     const size_t dir_smem = (size_t)D * D * 8 + (size_t)dir_warps * DirCfg<T, D>::warp_bytes(m_cap);
