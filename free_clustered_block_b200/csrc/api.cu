@@ -17,6 +17,7 @@ using namespace ca;
 namespace {
 
 constexpr int kMaxRouteC = 8192;
+constexpr int kMaxCompensatedC = 8192;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -173,6 +174,8 @@ ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape*
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return CA_ERR_INVALID_ARG;
   const int C = (s->n_valid + s->c - 1) / s->c;
   if (rt->k < 1 || rt->k > C) return CA_ERR_INVALID_ARG;
+  // the bf16 kernel keeps one compensation bias per key cluster on chip
+  if (compensate && s->dtype == CA_BF16 && C > kMaxCompensatedC) return CA_ERR_UNSUPPORTED;
   AttendWs L;
   attend_ws_layout(s, &L);
   if (workspace_bytes < L.total) return CA_ERR_WORKSPACE;

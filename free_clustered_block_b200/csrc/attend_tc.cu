@@ -188,18 +188,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// AND of a predicate over the n softmax threads (named barrier 1); every
-// softmax thread executes the same sequence of these, so none can be left
-// waiting at the barrier.
-__device__ __forceinline__ bool group_all_n(bool v, int n) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(n)
-      : "memory");
-  return r != 0;
-}
 
 // Shared-memory matrix descriptor, 128-byte swizzle (canonical layouts of the
 // tcgen05 matrix descriptor: start >> 4 in bits 0-13, leading byte offset >> 4
@@ -276,39 +264,38 @@ struct TcParams {
   uint64_t wait_limit;
 };
 
-#ifndef CA_TC_SPLIT
-#define CA_TC_SPLIT 2   // softmax threads per query row
-#endif
-#ifndef CA_TC_NBUF
-#define CA_TC_NBUF 3    // S buffers in TMEM
-#endif
-
 template <int D, int KB>
 struct TcCfg {
-  static constexpr int kSplit = CA_TC_SPLIT;
-  static constexpr int kNBuf = CA_TC_NBUF;
   static constexpr int kSub = D / 64;                                  // 64-column sub-tiles per row
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kMaxKeptSmem = 1024;                            // kept list staged in shared memory
-  static constexpr int kStagesFit = (200 * 1024 - kQBytes - 2 * kMaxKeptSmem * 4) / kStageBytes;
+  static constexpr int kMaxBias = 8192;                                // centroid columns (C <= 8192)
+  static constexpr int kFixedBytes = 256 + kMaxBias * 4 + 2 * 2 * 128 * 4 + 2 * kMaxKeptSmem * 4 + 1024;
+  static constexpr int kStagesFit = (200 * 1024 - kQBytes - kFixedBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 4 ? 4 : (kStagesFit < 2 ? 2 : kStagesFit);
   static constexpr int kBarOff = kQBytes + kStages * kStageBytes;
-  static constexpr int kBiasOff = kBarOff + 256;
-  static constexpr int kRedOff = kBiasOff + KB * 4;                    // row-max exchange [2][128]
-  static constexpr int kKeptOff = kRedOff + 2 * 128 * 4;
+  static constexpr int kBiasOff = kBarOff + 256;                       // compensation bias per centroid column
+  static constexpr int kXchOff = kBiasOff + kMaxBias * 4;              // (m, l) exchange [2 groups][2][128]
+  static constexpr int kKeptOff = kXchOff + 2 * 2 * 128 * 4;
   // + alignment slack; at least 116 KB so that one CTA (and its 512 TMEM
   // columns) holds an SM
   static constexpr int kSmemCalc = kKeptOff + 2 * kMaxKeptSmem * 4 + 1024;
   static constexpr int kSmem = kSmemCalc > 116 * 1024 ? kSmemCalc : 116 * 1024;
-  static constexpr int kSoftmaxThreads = 128 * kSplit;                 // kSplit threads per row
-  static constexpr int kThreads = 64 + kSoftmaxThreads;                // + producer warp + MMA warp
+  static constexpr int kGroupThreads = 128;                            // one softmax group: a thread per row
+  static constexpr int kSoftmaxThreads = 2 * kGroupThreads;
+  static constexpr int kThreads = 128 + kSoftmaxThreads;               // warps 0-3: producer, MMA, 2 idle
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kSCol = 0;        // S buffers at 0, KB, 2 KB; P_j (bf16 pairs) over the front half
-  static constexpr uint32_t kOCol = kNBuf * KB;      // O (fp32, D columns)
-  static constexpr int kHalf = KB / kSplit;          // columns of S per softmax thread
-  static_assert(kOCol + D <= kTmemCols, "S buffers and O must fit in TMEM");
+  // TMEM: NB S buffers of KB columns (P_j as bf16 pairs over the front half
+  // of its buffer), then O_0 and O_1 (fp32, D columns each)
+  static constexpr int kNBufFit = (512 - 2 * D) / KB;
+  static constexpr int kNBuf = kNBufFit > 4 ? 4 : kNBufFit;
+  static constexpr int kSPhase = (kNBuf % 2 == 0) ? kNBuf : 2 * kNBuf;   // blocks between uses of one s_full
+  static constexpr uint32_t kSCol = 0;
+  static constexpr uint32_t kOCol = kNBuf * KB;
+  static_assert(kNBuf >= 2, "two S buffers at least");
+  static_assert(kOCol + 2 * D <= kTmemCols, "S buffers and both O accumulators must fit in TMEM");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
@@ -324,7 +311,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_vlo, const TcParams p) {
   using Cfg = TcCfg<D, KB>;
   constexpr int NS = Cfg::kStages;
-  constexpr int HC = Cfg::kHalf;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
@@ -335,14 +321,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* empty = bars + NS;        // [NS] stage released
   uint64_t* q_full = bars + 2 * NS;   // Q tile loaded
   constexpr int NB = Cfg::kNBuf;
-  uint64_t* s_full = q_full + 1;      // [NB] S_j computed in buffer j % NB
-  uint64_t* p_full = s_full + NB;     // [NB] P_j written in buffer j % NB
-  uint64_t* pv_done = p_full + NB;    // [NB] O += P_j V_j completed (j % NB)
+  uint64_t* s_full = q_full + 1;      // [NB][2] S_j computed in buffer j % NB, for group j % 2
+  uint64_t* p_full = s_full + 2 * NB; // [NB] P_j written in buffer j % NB
+  uint64_t* pv_done = p_full + NB;    // [NB] O_{j%2} += P_j V_j completed (j % NB)
   uint64_t* drain = pv_done + NB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* bias = reinterpret_cast<float*>(smem + Cfg::kBiasOff);
-  float* red = reinterpret_cast<float*>(smem + Cfg::kRedOff);
+  float* bias_all = reinterpret_cast<float*>(smem + Cfg::kBiasOff);
+  float* xch = reinterpret_cast<float*>(smem + Cfg::kXchOff);
   int32_t* kept_s = reinterpret_cast<int32_t*>(smem + Cfg::kKeptOff);        // kept key clusters
   int32_t* kcnt_s = kept_s + Cfg::kMaxKeptSmem;                               // their member counts
 
@@ -371,8 +357,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(q_full, 1);
     for (int b = 0; b < NB; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], Cfg::kSoftmaxThreads);
+      mbar_init(&s_full[2 * b], 1);
+      mbar_init(&s_full[2 * b + 1], 1);
+      mbar_init(&p_full[b], Cfg::kGroupThreads);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(drain, 1);
@@ -474,13 +461,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mma_ss_elect(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
         }
       }
-      tc_commit_elect(&s_full[j % NB]);
+      tc_commit_elect(&s_full[(j % NB) * 2 + (j & 1)]);
       if (j >= J_kept) tc_commit_elect(&empty[s]);   // kbar stage is free once S is computed
       return true;
     };
-    // S_0 .. S_{NB-2} ahead; afterwards S_{j+NB-1} follows PV_j. Its buffer
-    // was last read (as P_{j-1}) by PV_{j-1}, committed one step earlier.
-    for (int j = 0; j < NB - 1 && j < J && ok; ++j) ok = issue_qk(j);
+    // S_0 .. S_{NB-1} ahead; S_{j+NB} reuses buffer j % NB once PV_j (its
+    // last reader) has completed. Blocks alternate between the two softmax
+    // groups, so the other group works on S_{j+1} meanwhile.
+    for (int j = 0; j < NB && j < J && ok; ++j) ok = issue_qk(j);
     for (int j = 0; j < J && ok; ++j) {
       if (!wwait(&p_full[j % NB], (j / NB) & 1)) { ok = false; break; }
       tc_fence_after();
@@ -492,55 +480,54 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
       const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
+      const uint32_t o_tmem = tmem + Cfg::kOCol + (uint32_t)((j & 1) * D);   // O of the block's group
       const int nmat = (j < J_kept) ? 1 : 2;
       for (int mtx = 0; mtx < nmat; ++mtx) {
         const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < KB / 16; ++kk) {
           const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
-          mma_ts_elect(tmem + Cfg::kOCol, p_tmem + kk * 8, bd, id_pv, (j > 0 || mtx > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_elect(o_tmem, p_tmem + kk * 8, bd, id_pv, (j >= 2 || mtx > 0 || kk > 0) ? 1u : 0u);
         }
       }
       tc_commit_elect(&pv_done[j % NB]);
       tc_commit_elect(&empty[s]);
-      const int jn = j + NB - 1;
-      if (jn < J) {
-        if (j > 0 && !wwait(&pv_done[(j - 1) % NB], ((j - 1) / NB) & 1)) { ok = false; break; }
+      if (j + NB < J) {
+        if (!wwait(&pv_done[j % NB], (j / NB) & 1)) { ok = false; break; }
         tc_fence_after();
-        if (!issue_qk(jn)) { ok = false; break; }
+        if (!issue_qk(j + NB)) { ok = false; break; }
       }
     }
     // Drain: every MMA issued so far has completed once `drain` flips.
     tc_commit_elect(drain);
     if (lane == 0) drain_bar(drain, 0);
     __syncwarp();
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
-    const int st = threadIdx.x - 64;          // 0..255 within the softmax group
+    // Group g (warps 4-7 or 8-11) takes the blocks j with j % 2 == g, one
+    // thread per query row, and accumulates them in its own O_g.
+    const int g = (warp - 4) >> 2;
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
-    const int half = st >> 7;                 // which part of the columns of its row
     const int row = q4 * 32 + lane;           // row of the query tile
+    const int sth = threadIdx.x - 128;        // 0..255 over both groups
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+    const float sc = p.scale_log2;
+    // compensation bias of every centroid column (log2 units; -inf where the
+    // key cluster is kept or is padding), once per CTA
+    if (J_cent > 0) {
+      const uint32_t* kb_row = p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
+      const float log2e = 1.4426950408889634f;
+      for (int e = sth; e < J_cent * KB; e += Cfg::kSoftmaxThreads) {
+        float bv = -INFINITY;
+        if (e < p.C && !((kb_row[e >> 5] >> (e & 31)) & 1u)) bv = p.logcnt[(size_t)bh * p.Cpad + e] * log2e;
+        bias_all[e] = bv;
+      }
+    }
+    named_sync(1, Cfg::kSoftmaxThreads);
     float m_used = -INFINITY, lreg = 0.f;
     bool ok = true;
-    const uint32_t* kb_row = p.dense ? nullptr : p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
-    const float log2e = 1.4426950408889634f;
-    const float sc = p.scale_log2;
-    const int col0 = half * HC;               // first S column of this thread
-    for (int j = 0; j < J; ++j) {
+    for (int j = g; j < J; j += 2) {
       const bool cent = j >= J_kept;
-      const uint32_t sbuf = Cfg::kSCol + (uint32_t)((j % NB) * KB);
-      if (cent) {
-        // per-column compensation bias of this centroid block (log2 units)
-        named_sync(1, Cfg::kSoftmaxThreads);
-        if (st < KB) {
-          const int e = (j - J_kept) * KB + st;
-          float bv = -INFINITY;
-          if (e < p.C && !((kb_row[e >> 5] >> (e & 31)) & 1u)) bv = p.logcnt[(size_t)bh * p.Cpad + e] * log2e;
-          bias[st] = bv;
-        }
-        named_sync(1, Cfg::kSoftmaxThreads);
-      }
       int valid = KB;   // real keys in a kept block
       if (!cent) {
         if (p.dense) valid = min(KB, p.n_valid - j * KB);
@@ -549,87 +536,88 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           valid = min(KB, cnt - (j % nsb) * KB);
         }
       }
-      const int vloc = valid - col0;             // valid columns among this thread's
-      const int mode = cent ? 2 : (vloc < HC ? 1 : 0);   // 0 full, 1 partial, 2 centroids
-      ok = group_all_n(wait_bar(&s_full[j % NB], (j / NB) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
+      const float* bias = bias_all + (cent ? (j - J_kept) * KB : 0);
+      const uint32_t sbuf = lane_addr + Cfg::kSCol + (uint32_t)((j % NB) * KB);
+      ok = __all_sync(0xffffffffu, wait_bar(&s_full[(j % NB) * 2 + g], (j / Cfg::kSPhase) & 1, limit, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      float sv[HC];
-#pragma unroll
-      for (int c0 = 0; c0 < HC; c0 += 32) {
-        uint32_t* r = reinterpret_cast<uint32_t*>(&sv[c0]);
-        CA_TMEM_LD32(lane_addr + sbuf + (uint32_t)(col0 + c0), r);
-      }
-      tmem_wait_ld();
+      // pass 1: the row maximum, 64 columns per TMEM round trip
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-      if (mode == 1) {
 #pragma unroll
-        for (int q = 0; q < HC; ++q)
-          if (q >= vloc) sv[q] = -INFINITY;
-      } else if (mode == 2) {
+      for (int c0 = 0; c0 < KB; c0 += 64) {
+        float v[64];
+        CA_TMEM_LD32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
+        CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(v + 32));
+        tmem_wait_ld();
+        if (cent) {
 #pragma unroll
-        for (int q = 0; q < HC; ++q) sv[q] = fmaf(sv[q], sc, bias[col0 + q]);
+          for (int q = 0; q < 64; ++q) v[q] = fmaf(v[q], sc, bias[c0 + q]);
+        } else if (valid < KB) {
+#pragma unroll
+          for (int q = 0; q < 64; ++q)
+            if (c0 + q >= valid) v[q] = -INFINITY;
+        }
+#pragma unroll
+        for (int q = 0; q < 64; q += 2) m8[(q >> 1) & 7] = max3(m8[(q >> 1) & 7], v[q], v[q + 1]);
       }
-#pragma unroll
-      for (int q = 0; q < HC; q += 2) m8[(q >> 1) & 7] = max3(m8[(q >> 1) & 7], sv[q], sv[q + 1]);
-      float pm = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      if (mode != 2) pm *= sc;             // log2 units
-      // combine the two halves of the row; after this barrier every S column
-      // of the block is in registers, so P may overwrite S.
-      float mx = pm;
-      if (Cfg::kSplit == 2) {
-        red[half * 128 + row] = pm;
-        named_sync(1, Cfg::kSoftmaxThreads);
-        mx = fmaxf(red[row], red[128 + row]);
-      }
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      if (!cent) mx *= sc;                   // log2 units
       // lazy rescale: move the reference max only when it grows by > 8 (x 256)
-      bool need = false;
       float factor = 1.f;
-      if (mx > m_used + 8.f) {
+      const bool need = mx > m_used + 8.f;
+      if (need) {
         factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - mx);
-        need = (j > 0);
         m_used = mx;
         lreg *= factor;
       }
-      const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
-      // O correction (rare) once PV_{j-1} has finished; each half scales its
-      // half of O.
-      bool wok = true;
-      const bool wneed = __any_sync(0xffffffffu, need);
-      if (wneed) wok = __all_sync(0xffffffffu, wait_bar(&pv_done[(j - 1) % NB], ((j - 1) / NB) & 1, limit, abort_flag));
-      ok = group_all_n(wok, Cfg::kSoftmaxThreads);
-      if (!ok) break;
-      if (wneed) {
+      // O_g already holds blocks j-2, j-4, ...: rescale it (whole warp, as
+      // TMEM loads and stores are warp-wide) once PV_{j-2} has completed.
+      if (j >= 2 && __any_sync(0xffffffffu, need)) {
+        ok = __all_sync(0xffffffffu, wait_bar(&pv_done[(j - 2) % NB], ((j - 2) / NB) & 1, limit, abort_flag));
+        if (!ok) break;
         tc_fence_after();
-        constexpr int OH = D / Cfg::kSplit;
+        const uint32_t oaddr = lane_addr + Cfg::kOCol + (uint32_t)(g * D);
 #pragma unroll
-        for (int c0 = 0; c0 < OH; c0 += 32) {
+        for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t ov[32];
-          CA_TMEM_LD32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
+          CA_TMEM_LD32(oaddr + (uint32_t)c0, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
-          CA_TMEM_ST32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
+          CA_TMEM_ST32(oaddr + (uint32_t)c0, ov);
         }
       }
-      // P = 2^(x - m) as bf16 pairs over the front half of this S buffer
-      const float xs = (mode == 2) ? 1.f : sc;
+      const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
+      // pass 2: P = 2^(x - m) as bf16 pairs over the front half of the buffer
+      // (the pairs of columns c0.. land on columns c0/2.., already read)
+      const float xs = cent ? 1.f : sc;
       const uint64_t xs2 = f2_pack(xs, xs), nb2 = f2_pack(nb, nb);
       uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};   // packed partial row sums
 #pragma unroll
-      for (int c0 = 0; c0 < HC; c0 += 32) {
+      for (int c0 = 0; c0 < KB; c0 += 32) {
+        float v[32];
+        CA_TMEM_LD32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
+        tmem_wait_ld();
+        if (cent) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = fmaf(v[q], sc, bias[c0 + q]);
+        } else if (valid < KB) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            if (c0 + q >= valid) v[q] = -INFINITY;
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           float t0, t1;
-          f2_unpack(fma2(f2_pack(sv[c0 + 2 * q], sv[c0 + 2 * q + 1]), xs2, nb2), t0, t1);
+          f2_unpack(fma2(f2_pack(v[2 * q], v[2 * q + 1]), xs2, nb2), t0, t1);
           const float p0 = ex2(t0), p1 = ex2(t1);
           ls2[q & 3] = add2(ls2[q & 3], f2_pack(p0, p1));
           pk[q] = pack_bf16(p0, p1);
         }
-        CA_TMEM_ST16(lane_addr + sbuf + (uint32_t)((col0 + c0) / 2), pk);
+        CA_TMEM_ST16(sbuf + (uint32_t)(c0 / 2), pk);
       }
       {
         float a0, a1;
@@ -640,35 +628,52 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       mbar_arrive(&p_full[j % NB]);
     }
-    // epilogue: O / l to the query's original row; each half writes D/2 columns
-    if (ok && J > 0)
-      ok = group_all_n(wait_bar(&pv_done[(J - 1) % NB], ((J - 1) / NB) & 1, limit, abort_flag), Cfg::kSoftmaxThreads);
-    if (ok && J > 0) {
+    // epilogue: merge the two groups' (m, l, O) and write O / l to the
+    // query's original row; group g writes columns [g D/2, (g+1) D/2)
+    const int jl0 = (J >= 1) ? ((J - 1) & ~1) : -1;          // last block of group 0
+    const int jl1 = (J >= 2) ? (((J - 2) & ~1) + 1) : -1;    // last block of group 1
+    const int jl = g ? jl1 : jl0;
+    if (ok && jl >= 0)
+      ok = __all_sync(0xffffffffu, wait_bar(&pv_done[jl % NB], (jl / NB) & 1, limit, abort_flag));
+    xch[(g * 2 + 0) * 128 + row] = jl >= 0 ? m_used : -INFINITY;
+    xch[(g * 2 + 1) * 128 + row] = jl >= 0 ? lreg : 0.f;
+    named_sync(1, Cfg::kSoftmaxThreads);
+    if (ok) {
       tc_fence_after();
+      const float m0 = xch[0 * 128 + row], l0 = xch[1 * 128 + row];
+      const float m1 = xch[2 * 128 + row], l1 = xch[3 * 128 + row];
+      const float M = fmaxf(m0, m1);
+      const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
+      const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+      const float l = l0 * f0 + l1 * f1;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float w0 = f0 * inv, w1 = f1 * inv;
       int orow;
       if (p.dense) orow = tile * 128 + row < p.n_valid ? tile * 128 + row : -1;
       else orow = row < p.rows_per_tile ? p.perm_q[(size_t)bh * p.C * p.c + (size_t)a * p.c + sub_tile * 128 + row]
                                         : -1;
-      red[half * 128 + row] = lreg;
-      named_sync(1, Cfg::kSoftmaxThreads);
-      const float l = Cfg::kSplit == 2 ? red[row] + red[128 + row] : lreg;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      constexpr int OH = D / Cfg::kSplit;
-      __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D + half * OH;
+      constexpr int OH = D / 2;
+      __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D + g * OH;
 #pragma unroll
       for (int c0 = 0; c0 < OH; c0 += 32) {
-        uint32_t ov[32];
-        CA_TMEM_LD32(lane_addr + Cfg::kOCol + half * OH + c0, ov);
+        uint32_t o0[32], o1[32];
+        // an accumulator whose group had no block was never written
+        if (jl0 >= 0) CA_TMEM_LD32(lane_addr + Cfg::kOCol + (uint32_t)(g * OH + c0), o0);
+        if (jl1 >= 0) CA_TMEM_LD32(lane_addr + Cfg::kOCol + (uint32_t)(D + g * OH + c0), o1);
         tmem_wait_ld();
         if (orow >= 0) {
           uint4 w[4];
           uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-          for (int q = 0; q < 16; ++q)
-            wp[q] = pack_bf16(__uint_as_float(ov[2 * q]) * inv, __uint_as_float(ov[2 * q + 1]) * inv);
-          uint4* g = reinterpret_cast<uint4*>(dst + c0);
+          for (int q = 0; q < 16; ++q) {
+            float x0 = 0.f, x1 = 0.f;
+            if (jl0 >= 0) { x0 = __uint_as_float(o0[2 * q]) * w0; x1 = __uint_as_float(o0[2 * q + 1]) * w0; }
+            if (jl1 >= 0) { x0 = fmaf(__uint_as_float(o1[2 * q]), w1, x0); x1 = fmaf(__uint_as_float(o1[2 * q + 1]), w1, x1); }
+            wp[q] = pack_bf16(x0, x1);
+          }
+          uint4* gp = reinterpret_cast<uint4*>(dst + c0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) g[q] = w[q];
+          for (int q = 0; q < 4; ++q) gp[q] = w[q];
         }
       }
     }

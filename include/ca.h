@@ -180,6 +180,8 @@ ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
  * Reads clusters->perm_q/perm_k/count_k/kbar and routes->kept_idx/kept_bits;
  * vbar is computed here. O: device [B][H][N_alloc][d], written in original
  * row order (padding rows 0). workspace >= ca_attend_workspace_bytes(shape).
+ * bf16 with compensate != 0 supports C <= 8192 key clusters
+ * (CA_ERR_UNSUPPORTED beyond).
  */
 ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* shape,
                     const ca_clusters* clusters, const ca_routes* routes, int compensate,
