@@ -181,6 +181,30 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// 2^t0, 2^t1 (t <= 8) on the FMA pipe, to take part of the load off the
+// MUFU ex2 unit: t = n + f with n = round(t) (adding and subtracting 1.5 * 2^23
+// leaves the rounded integer in the low mantissa bits), 2^f on [-1/2, 1/2] by
+// a cubic fitted to the least maximum relative error on that interval
+// (< 8e-5, far below the bf16 rounding of P), and n added into the exponent
+// field with one integer multiply-add. t is clamped at -126 (2^-126 is as good
+// as 0 in a bf16 P).
+__device__ __forceinline__ void exp2_poly2(float t0, float t1, float& r0, float& r1) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  constexpr float c0 = 0.9999281168f, c1 = 0.6932609677f, c2 = 0.2426105440f, c3 = 0.0551713221f;
+  const uint64_t t2 = f2_pack(fmaxf(t0, -126.f), fmaxf(t1, -126.f));
+  const uint64_t y2 = add2(t2, f2_pack(kRound, kRound));
+  const uint64_t n2 = add2(y2, f2_pack(-kRound, -kRound));
+  const uint64_t f2 = fma2(n2, f2_pack(-1.f, -1.f), t2);
+  uint64_t q2 = fma2(f2_pack(c3, c3), f2, f2_pack(c2, c2));
+  q2 = fma2(q2, f2, f2_pack(c1, c1));
+  q2 = fma2(q2, f2, f2_pack(c0, c0));
+  float y0, y1, q0, q1;
+  f2_unpack(y2, y0, y1);
+  f2_unpack(q2, q0, q1);
+  // low mantissa bits of y hold n (two's complement); times 2^23 moves them to the exponent
+  r0 = __int_as_float(__float_as_int(y0) * 8388608 + __float_as_int(q0));
+  r1 = __int_as_float(__float_as_int(y1) * 8388608 + __float_as_int(q1));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -298,6 +322,13 @@ struct TcCfg {
   static_assert(kOCol + 2 * D <= kTmemCols, "S buffers and both O accumulators must fit in TMEM");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
+
+// Pairs of P columns (bit q % 8) whose exponentials run on the FMA pipe
+// instead of the MUFU unit.
+#ifndef CA_TC_POLY_PAIRS
+#define CA_TC_POLY_PAIRS 0x00
+#endif
+constexpr unsigned kPolyPairs = CA_TC_POLY_PAIRS;
 
 // Items in load order: kept key sub-blocks (K,V), then per centroid block
 // (kbar hi, lo) and (vbar hi, vbar lo).
@@ -541,29 +572,36 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       ok = __all_sync(0xffffffffu, wait_bar(&s_full[(j % NB) * 2 + g], (j / Cfg::kSPhase) & 1, limit, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      // pass 1: the row maximum, 64 columns per TMEM round trip
+      // pass 1: the row maximum, 64 columns per TMEM round trip. Partial and
+      // centroid blocks (rare) get their mask / bias here and are written
+      // back, so that pass 2 has a single path.
+      const bool special = cent || valid < KB;
       float m8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-#pragma unroll
+#pragma unroll 1
       for (int c0 = 0; c0 < KB; c0 += 64) {
         float v[64];
         CA_TMEM_LD32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
         CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(v + 32));
         tmem_wait_ld();
-        if (cent) {
+        if (special) {
+          if (cent) {
 #pragma unroll
-          for (int q = 0; q < 64; ++q) v[q] = fmaf(v[q], sc, bias[c0 + q]);
-        } else if (valid < KB) {
+            for (int q = 0; q < 64; ++q) v[q] = fmaf(v[q], sc, bias[c0 + q]);
+          } else {
 #pragma unroll
-          for (int q = 0; q < 64; ++q)
-            if (c0 + q >= valid) v[q] = -INFINITY;
+            for (int q = 0; q < 64; ++q) v[q] = (c0 + q < valid) ? v[q] : -INFINITY;
+          }
+          CA_TMEM_ST32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
+          CA_TMEM_ST32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(v + 32));
         }
 #pragma unroll
         for (int q = 0; q < 64; q += 2) m8[(q >> 1) & 7] = max3(m8[(q >> 1) & 7], v[q], v[q + 1]);
       }
+      if (special) tmem_wait_st();
       float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      if (!cent) mx *= sc;                   // log2 units
+      if (!cent) mx *= sc;                   // log2 units (centroid values already are)
       // lazy rescale: move the reference max only when it grows by > 8 (x 256)
       float factor = 1.f;
       const bool need = mx > m_used + 8.f;
@@ -595,29 +633,31 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float xs = cent ? 1.f : sc;
       const uint64_t xs2 = f2_pack(xs, xs), nb2 = f2_pack(nb, nb);
       uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};   // packed partial row sums
-#pragma unroll
-      for (int c0 = 0; c0 < KB; c0 += 32) {
-        float v[32];
-        CA_TMEM_LD32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
-        tmem_wait_ld();
-        if (cent) {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) v[q] = fmaf(v[q], sc, bias[c0 + q]);
-        } else if (valid < KB) {
-#pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (c0 + q >= valid) v[q] = -INFINITY;
-        }
+      // 32 columns per step, two steps per loop turn; the next step's TMEM
+      // load is in flight while a step computes
+      auto p_step = [&](const float* v, int c0) {
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          float t0, t1;
+          float t0, t1, p0, p1;
           f2_unpack(fma2(f2_pack(v[2 * q], v[2 * q + 1]), xs2, nb2), t0, t1);
-          const float p0 = ex2(t0), p1 = ex2(t1);
+          if ((kPolyPairs >> (q & 7)) & 1) exp2_poly2(t0, t1, p0, p1);
+          else { p0 = ex2(t0); p1 = ex2(t1); }
           ls2[q & 3] = add2(ls2[q & 3], f2_pack(p0, p1));
           pk[q] = pack_bf16(p0, p1);
         }
         CA_TMEM_ST16(sbuf + (uint32_t)(c0 / 2), pk);
+      };
+      float va[32], vb[32];
+      CA_TMEM_LD32(sbuf, reinterpret_cast<uint32_t*>(va));
+#pragma unroll 1
+      for (int c0 = 0; c0 < KB; c0 += 64) {
+        tmem_wait_ld();
+        CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(vb));
+        p_step(va, c0);
+        tmem_wait_ld();
+        if (c0 + 64 < KB) CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 64), reinterpret_cast<uint32_t*>(va));
+        p_step(vb, c0 + 32);
       }
       {
         float a0, a1;
