@@ -35,6 +35,25 @@ UNIT = "layer-fwd/s"
 CONFIG_ID = 2
 
 
+# DRAM traffic (read + write bytes) of one attention-kernel launch on this
+# workload, from the ncu capture summarised in
+# profiles/tc_attend_kernel_64_128_layer_B1_H8_N65536.md. It describes the
+# kernel source whose SHA-256 starts with `source_sha256`; for any other source
+# the bench reports null.
+ATTN_TRAFFIC = {"bytes": 205448192 + 52447232, "source_sha256": "1f30034b366e1e6c"}
+
+
+def attention_traffic():
+    import hashlib
+    src = os.path.join(ROOT, "free_clustered_block_b200", "csrc", "attend_tc.cu")
+    try:
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    return ATTN_TRAFFIC["bytes"] if h.startswith(ATTN_TRAFFIC["source_sha256"]) else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -306,7 +325,8 @@ def run_ours(args):
         "speedup_vs_dense": dense_ms / ms_per_step,
         "roofline": {"kernel": "attention (ca_attend span: prep + attention)", "bound": "tensor",
                      "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_sus"], "traffic": None,
+                     "frac": achieved / pk["bf16_sus"], "traffic": attention_traffic(),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read + dram__bytes_write)",
                      "peak_source": f"bf16 dense sustained, {pk['source']}",
                      "algorithmic_flops": kept_f + smc_f},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
