@@ -64,10 +64,29 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+L2_BYTES = 126 * 2 ** 20
+
+
+def input_bytes(w):
+    return 3 * w.B * w.H * w.N_alloc * w.d * (2 if w.dtype == "bf16" else 4)
+
+
+def needs_flush(w):
+    """Inputs that fit in L2 get an L2 flush before every timed step."""
+    return input_bytes(w) < 2 * L2_BYTES
+
+
 def workload_config(w):
+    mb = input_bytes(w) / 3 / 1e6
+    l2 = (f"L2 flushed (512 MB write) before every timed step: Q, K, V are 3 x {mb:.1f} MB" if needs_flush(w)
+          else f"inputs larger than L2: Q, K, V are 3 x {mb:.0f} MB per layer (L2 126 MB)")
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N_alloc, "n_valid": w.n_valid, "d": w.d, "c": w.c,
-            "k": w.k, "clusters": w.C, "compensate": bool(w.compensate), "input_dtype": w.dtype,
-            "l2": "inputs larger than L2: Q, K, V are 3 x 67 MB per layer (L2 126 MB)"}
+            "k": w.k, "clusters": w.C, "compensate": bool(w.compensate), "input_dtype": w.dtype, "l2": l2}
+
+
+def dense_flops(w):
+    """FLOPs of dense attention over the valid tokens (QK^T and PV)."""
+    return 4.0 * w.n_valid * w.n_valid * w.d * w.H * w.B
 
 
 def attention_flops(w):
@@ -136,11 +155,12 @@ def blas_threads():
         return 1
 
 
-def oracle_sample(w, n_clusters=48, heads=(0,)):
+def oracle_sample(w, n_clusters=48, heads=(0,), keep=None):
     """Time the oracle on a bounded sample and extrapolate to one whole layer.
     Per sampled head: full clustering of queries and keys, routing, and the
     attention of `n_clusters` query clusters (work per query cluster is the
-    same k kept blocks plus compensation). Returns seconds per layer."""
+    same k kept blocks plus compensation). Returns seconds per layer and, when
+    `keep` is a dict, stores head 0's oracle output and sampled clusters there."""
     import numpy as np
     from oracle import ca_oracle as orc
     t_head = []
@@ -151,11 +171,35 @@ def oracle_sample(w, n_clusters=48, heads=(0,)):
         kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
         t1 = time.perf_counter()
         sample = list(range(0, w.C, max(1, w.C // n_clusters)))[:n_clusters]
-        orc.compensated_attention(Qf, Kf, Vf, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, w.c,
-                                  compensate=w.compensate, clusters=sample)
+        out = orc.compensated_attention(Qf, Kf, Vf, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, w.c,
+                                        compensate=w.compensate, clusters=sample)
         t2 = time.perf_counter()
         t_head.append((t1 - t0) + (t2 - t1) * w.C / len(sample))
+        if keep is not None and h == heads[0]:
+            keep.update(head=h, out=out, perm_q=hc.perm_q, sample=sample)
     return statistics.mean(t_head) * w.H * w.B, {"heads": list(heads), "query_clusters": n_clusters}
+
+
+def error_vs_dense(w, O_gpu_head, kept, n_clusters=8):
+    """Max-abs and relative-L2 error against fp64 dense attention on the rows
+    of `n_clusters` of the oracle's sampled query clusters of one head, for
+    the GPU output and for the oracle's output."""
+    import numpy as np
+    from oracle import ca_oracle as orc
+    h = kept["head"]
+    Qf, Kf, Vf = (x[0, h, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
+    rows = []
+    for a in kept["sample"][:n_clusters]:
+        r = kept["perm_q"][a * w.c:(a + 1) * w.c]
+        rows.extend(int(x) for x in r if x >= 0)
+    rows = np.array(rows)
+    ref = orc.dense_attention(Qf, Kf, Vf, rows=rows)
+    res = {"rows": int(rows.size), "reference": "fp64 dense softmax attention over all valid keys"}
+    for name, got in (("gpu", O_gpu_head[rows].astype(np.float64)), ("oracle", kept["out"][rows])):
+        d = got - ref
+        res[name] = {"max_abs": float(np.abs(d).max()),
+                     "rel_l2": float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-300))}
+    return res
 
 
 def run_reference(args):
@@ -163,7 +207,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     import workloads as wl
-    w = wl.config_workload(CONFIG_ID)
+    w = wl.config_workload(args.config)
     times = []
     for i in range(args.warmup + args.steps):
         t, smp = oracle_sample(w)
@@ -185,9 +229,9 @@ def run_reference(args):
     return 0
 
 
-def rank_seed(rank: int) -> int:
+def rank_seed(rank: int, config: int = CONFIG_ID) -> int:
     """Seed of the independent layer a rank runs (rank 0: the standard workload)."""
-    return 1000 + CONFIG_ID + 7919 * rank
+    return 1000 + config + 7919 * rank
 
 
 def whole_job_value(world: int, steps: int, total_ms: float) -> float:
@@ -230,10 +274,11 @@ def run_ours(args):
         return max_over_ranks(x, world, "cuda")
 
     # Each rank: an independent layer (its own seeded inputs).
-    w = wl.config_workload(CONFIG_ID, seed=rank_seed(rank))
+    w = wl.config_workload(args.config, seed=rank_seed(rank, args.config))
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(x):
-        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).cuda().contiguous()
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(tdt).cuda().contiguous()
 
     Q, K, V = dev(w.Q), dev(w.K), dev(w.V)
     O = torch.empty_like(Q)
@@ -253,6 +298,8 @@ def run_ours(args):
     if st != ca.CA_OK:
         raise RuntimeError(f"device error after warm-up: {ca.status_string(st)}")
 
+    flush = needs_flush(w)
+    scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda") if flush else None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
@@ -260,6 +307,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         start.record(stream)
         for i in range(args.steps):
+            if flush:
+                scrub.zero_()
             ev[i][0].record(stream)
             layer.cluster(Q, K)
             ev[i][1].record(stream)
@@ -270,7 +319,9 @@ def run_ours(args):
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
-    total_ms = ranks_max(start.elapsed_time(end))
+    # with flushes, the steps are timed one by one (the flushes are not timed)
+    total_ms = ranks_max(sum(ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)) if flush
+                         else start.elapsed_time(end))
     clocks = clk.summary()
     stage = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
              for j, name in enumerate(("cluster", "route", "attend"))}
@@ -310,32 +361,73 @@ def run_ours(args):
     in_bytes = 3 * Q.numel() * Q.element_size()
     out_bytes = O.numel() * O.element_size()
 
+    # The same layer captured once in a CUDA graph and replayed.
+    graph_ms = None
+    try:
+        gstream = torch.cuda.Stream()
+        gstream.wait_stream(stream)
+        with torch.cuda.stream(gstream):
+            step()
+        gstream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gstream):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ranks_max(g0.elapsed_time(g1)) / args.steps
+        del graph
+    except Exception as e:  # capture is an extra figure; the timed line above stands
+        graph_ms = f"capture failed: {type(e).__name__}"
+
     pk = peaks()
     kept_f, smc_f = attention_flops(w)
     attn_s = stage["attend"] / 1e3
     achieved = (kept_f + smc_f) / attn_s / 1e12
+    if w.dtype == "bf16":
+        roof = {"kernel": "attention (ca_attend span: prep + attention)", "bound": "tensor",
+                "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_sus"],
+                "traffic": attention_traffic() if args.config == CONFIG_ID else None,
+                "traffic_unit": "bytes per launch (ncu dram__bytes_read + dram__bytes_write)",
+                "peak_source": f"bf16 dense sustained, {pk['source']}",
+                "algorithmic_flops": kept_f + smc_f}
+    else:
+        # fp32 inputs run the SIMT attention kernel on the FMA pipe: peak from
+        # 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
+        fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"kernel": "attention (ca_attend span: prep + attention)", "bound": "alu",
+                "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s", "frac": achieved / fp32_peak,
+                "traffic": None, "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                "algorithmic_flops": kept_f + smc_f}
     launches = args.steps * sum(ca.launch_count(shape, s) for s in (0, 1, 2))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16",
-        "dtype_detail": "clustering and routing f64; attention bf16 products with f32 accumulation",
+        "vs_baseline": None, "dtype": w.dtype,
+        "dtype_detail": ("clustering and routing f64; attention bf16 products with f32 accumulation"
+                         if w.dtype == "bf16" else "clustering and routing f64; attention f32"),
         "data": "synthetic", "config": workload_config(w),
         "latency_ms": ms_per_step, "stage_ms": stage, "dense_ms": dense_ms,
         "speedup_vs_dense": dense_ms / ms_per_step,
-        "roofline": {"kernel": "attention (ca_attend span: prep + attention)", "bound": "tensor",
-                     "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_sus"], "traffic": attention_traffic(),
-                     "traffic_unit": "bytes per launch (ncu dram__bytes_read + dram__bytes_write)",
-                     "peak_source": f"bf16 dense sustained, {pk['source']}",
-                     "algorithmic_flops": kept_f + smc_f},
+        "graph_ms_per_step": graph_ms,
+        "tflops": {"dense_equivalent": dense_flops(w) / (ms_per_step / 1e3) / 1e12,
+                   "algorithmic_attention": achieved},
+        "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": out_bytes, "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_cpu, smp = oracle_sample(w)
+        kept = {}
+        t_cpu, smp = oracle_sample(w, keep=kept)
+        line["error_vs_dense_fp64"] = error_vs_dense(w, O[0, kept["head"]].float().cpu().numpy(), kept)
         line["cpu_baseline"] = {"value": 1.0 / t_cpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"head 0 clustered and routed in full, attention of 48 of {w.C} query "
                                           f"clusters; extrapolated to {w.H} heads x {w.C} clusters "
@@ -354,6 +446,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", type=int, choices=[1, 2, 3, 4], default=CONFIG_ID,
+                    help="workload (default 2: the metric's N = 64k configuration)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
