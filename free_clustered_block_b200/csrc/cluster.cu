@@ -624,6 +624,209 @@ __global__ void __launch_bounds__(512) dir_kernel(
   }
 }
 
+// d = 128 (a 128-row sample at most): M alone is 128 KB, so one warp per node
+// would leave two nodes per SM. Here a 256-thread block owns one node at a
+// time and walks `npc` consecutive nodes of one tensor-head, staging M once.
+// Each of the three products of a power step is split over the 256 threads
+// as pairs of half sums (rows or columns 0-63 / 64-127), added in a fixed
+// order, so the result does not depend on scheduling.
+constexpr int kDirCThreads = 256;
+
+template <typename T>
+struct DirCCfg {
+  static constexpr int D = 128;
+  static constexpr int kRowStride = D + ((sizeof(T) == 2) ? 2 : 1);   // odd number of 32-bit words
+  static constexpr size_t kXBytes = (size_t)D * kRowStride * sizeof(T);
+  static constexpr size_t kSmem = (size_t)D * D * 8 + kXBytes;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
+    const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
+    int lvl_begin, int nodes_in_level, int npc, const double* __restrict__ M, const double* __restrict__ inv_s,
+    const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
+    int power_iters) {
+  using Cfg = DirCCfg<T>;
+  constexpr int D = 128, RS = Cfg::kRowStride;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* Ms = reinterpret_cast<double*>(smem_raw);             // D x D
+  T* Xs = reinterpret_cast<T*>(smem_raw + (size_t)D * D * 8);   // D rows x RS
+  __shared__ double red[2][D];
+  __shared__ double zs[D], ws[D], xbar[D], fj[D], vs[D];
+  __shared__ double qred[4][2];
+  __shared__ double vred[8];
+  __shared__ int srow[D];
+  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int ca = t & 127, ch = t >> 7;          // column / half split
+  const int rj = t >> 1, rh = t & 1;            // row / half split
+  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  {
+    const double2* src = reinterpret_cast<const double2*>(M + (size_t)th * D * D);
+    double2* dst = reinterpret_cast<double2*>(Ms);
+#pragma unroll 4
+    for (int e = t; e < D * D / 2; e += kDirCThreads) dst[e] = src[e];
+  }
+  // w = M z (z in zs) into ws; returns (z . w, xbar . w) to every thread
+  auto matvec = [&](double& zw, double& xw) {
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    const int b0 = ch * 64;
+#pragma unroll 4
+    for (int b = 0; b < 64; b += 4) {
+      a0 = fma(Ms[(b0 + b) * D + ca], zs[b0 + b], a0);
+      a1 = fma(Ms[(b0 + b + 1) * D + ca], zs[b0 + b + 1], a1);
+      a2 = fma(Ms[(b0 + b + 2) * D + ca], zs[b0 + b + 2], a2);
+      a3 = fma(Ms[(b0 + b + 3) * D + ca], zs[b0 + b + 3], a3);
+    }
+    red[ch][ca] = (a0 + a1) + (a2 + a3);
+    __syncthreads();
+    if (t < D) {
+      const double w = red[0][t] + red[1][t];
+      ws[t] = w;
+      double pz = zs[t] * w, px = xbar[t] * w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        pz += __shfl_xor_sync(0xffffffffu, pz, o);
+        px += __shfl_xor_sync(0xffffffffu, px, o);
+      }
+      if (lane == 0) { qred[warp][0] = pz; qred[warp][1] = px; }
+    }
+    __syncthreads();
+    zw = (qred[0][0] + qred[1][0]) + (qred[2][0] + qred[3][0]);
+    xw = (qred[0][1] + qred[1][1]) + (qred[2][1] + qred[3][1]);
+  };
+  const int first = blockIdx.x * npc, last = min(nodes_in_level, first + npc);
+  for (int local = first; local < last; ++local) {
+    const int node_id = lvl_begin + local;
+    const TreeNode nd = nodes[node_id];
+    const int m = min(D, nd.size);
+    const uint64_t key = node_stream(seed, (uint64_t)bh, (uint64_t)tensor, nd.heap);
+    const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
+    __syncthreads();   // the previous node is done with every shared array
+    if (t < D) {
+      int row = 0;
+      double sc = 0.0;
+      if (t < m) {
+        const int pos = (nd.size > m) ? (int)(((uint64_t)t * (uint64_t)nd.size + r) / (uint64_t)m) : t;
+        row = idx ? idx[(size_t)th * n + nd.off + pos] : nd.off + pos;
+        sc = (tensor == 0) ? inv_s[(size_t)bh * n + row] : 1.0;
+      }
+      srow[t] = row;
+      vs[t] = sc;
+    }
+    __syncthreads();
+    // stage the sample rows (rows >= m zero), 16-byte loads, 8 in flight
+    {
+      constexpr int VEC = 16 / (int)sizeof(T), CPR = D / VEC;   // chunks per row
+      constexpr int WPR = RS * (int)sizeof(T) / 4;              // row stride in 32-bit words
+      uint32_t* xw32 = reinterpret_cast<uint32_t*>(Xs);
+#pragma unroll
+      for (int u0 = 0; u0 < D * CPR; u0 += 8 * kDirCThreads) {
+        uint4 v4[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = u0 + u * kDirCThreads + t;
+          const int j = e / CPR, part = e % CPR;
+          v4[u] = make_uint4(0, 0, 0, 0);
+          if (e < D * CPR && j < m)
+            v4[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * D + part * VEC);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = u0 + u * kDirCThreads + t;
+          const int j = e / CPR, part = e % CPR;
+          if (e < D * CPR) {
+            uint32_t* dst = xw32 + (size_t)j * WPR + part * 4;
+            dst[0] = v4[u].x; dst[1] = v4[u].y; dst[2] = v4[u].z; dst[3] = v4[u].w;
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // sample mean
+    {
+      double a0 = 0.0, a1 = 0.0;
+      const int j0 = ch * 64;
+#pragma unroll 4
+      for (int j = 0; j < 64; j += 2) {
+        a0 = fma(vs[j0 + j], (double)to_f(Xs[(j0 + j) * RS + ca]), a0);
+        a1 = fma(vs[j0 + j + 1], (double)to_f(Xs[(j0 + j + 1) * RS + ca]), a1);
+      }
+      red[ch][ca] = a0 + a1;
+      __syncthreads();
+      if (t < D) xbar[t] = (red[0][t] + red[1][t]) / (double)m;
+    }
+    // warm start from the Box-Muller normal g
+    if (t < D) {
+      const uint64_t ua = splitmix64(key + 2ull * t + 1ull);
+      const uint64_t ub = splitmix64(key + 2ull * t + 2ull);
+      const double u1 = (double)((ua >> 11) + 1ull) * 0x1.0p-53;
+      const double u2 = (double)(ub >> 11) * 0x1.0p-53;
+      zs[t] = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+    }
+    __syncthreads();
+    double zw, xw;
+    matvec(zw, xw);
+    {
+      const double gi = (zw > 0.0) ? 1.0 / sqrt(zw) : 0.0;
+      if (t < D) {
+        const double gh = zs[t] * gi;
+        zs[t] = (nd.parent < 0) ? gh : 0.5 * (zvec[((size_t)th * NI + nd.parent) * D + t] + gh);
+      }
+    }
+    __syncthreads();
+    for (int it = 0; it < power_iters; ++it) {
+      matvec(zw, xw);
+      const double s = (zw > 0.0) ? 1.0 / sqrt(zw) : 0.0;
+      // v_j = s (scale_j X_j . w - xbar . w): two threads per row
+      double v = 0.0;
+      {
+        double d0 = 0.0, d1 = 0.0, d2 = 0.0, d3 = 0.0;
+        const T* xr = Xs + rj * RS + rh * 64;
+        const double* wr = ws + rh * 64;
+#pragma unroll 4
+        for (int c = 0; c < 64; c += 4) {
+          d0 = fma((double)to_f(xr[c]), wr[c], d0);
+          d1 = fma((double)to_f(xr[c + 1]), wr[c + 1], d1);
+          d2 = fma((double)to_f(xr[c + 2]), wr[c + 2], d2);
+          d3 = fma((double)to_f(xr[c + 3]), wr[c + 3], d3);
+        }
+        double d = (d0 + d1) + (d2 + d3);
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        v = (rj < m) ? s * fma(vs[rj], d, -xw) : 0.0;
+      }
+      if (rh == 0) fj[rj] = v * vs[rj];
+      double vsum = (rh == 0) ? v : 0.0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
+      if (lane == 0) vred[warp] = vsum;
+      __syncthreads();
+      vsum = ((vred[0] + vred[1]) + (vred[2] + vred[3])) + ((vred[4] + vred[5]) + (vred[6] + vred[7]));
+      // z'_a = (sum_j v_j scale_j X_ja - xbar_a sum_j v_j) / m: two threads per column
+      {
+        double a0 = 0.0, a1 = 0.0;
+        const int j0 = ch * 64;
+#pragma unroll 4
+        for (int j = 0; j < 64; j += 2) {
+          a0 = fma(fj[j0 + j], (double)to_f(Xs[(j0 + j) * RS + ca]), a0);
+          a1 = fma(fj[j0 + j + 1], (double)to_f(Xs[(j0 + j + 1) * RS + ca]), a1);
+        }
+        red[ch][ca] = a0 + a1;
+      }
+      __syncthreads();
+      if (t < D) zs[t] = ((red[0][t] + red[1][t]) - xbar[t] * vsum) / (double)m;
+      __syncthreads();
+    }
+    matvec(zw, xw);
+    const double qi = (zw > 0.0) ? 1.0 / sqrt(zw) : 0.0;
+    if (t < D) {
+      const size_t o = ((size_t)th * NI + node_id) * D + t;
+      zvec[o] = zs[t] * qi;
+      wvec[o] = ws[t] * qi;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // K2a: projection key_i = x_i . w_node for every position of the level's
 // internal nodes, stored as order-preserving uint64. A block covers
@@ -1068,14 +1271,22 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     const int dir_warps = DirCfg<T, D>::warps(m_cap);
     const size_t dir_smem = (size_t)D * D * 8 + (size_t)dir_warps * DirCfg<T, D>::warp_bytes(m_cap);
     cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
+    if (D == 128) cudaFuncSetAttribute(dirc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DirCCfg<T>::kSmem);
     cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
     cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
     for (int l = 0; l < plan.levels; ++l) {
       const int lb = plan.level_begin[l], le = plan.level_begin[l + 1], nl = le - lb;
       const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
       int* idx_out = idxbuf[(l + 1) & 1];
-      dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(
-          Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters, sample_factor);
+      if (D == 128 && sample_factor == 1) {
+        // about four blocks per SM over the whole level
+        const int npc = (int)(((long long)nl * TH + 4 * 148 - 1) / (4 * 148));
+        dirc_kernel<T><<<dim3((nl + npc - 1) / npc, TH), kDirCThreads, DirCCfg<T>::kSmem, st>>>(
+            Q, K, N_alloc, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters);
+      } else {
+        dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(
+            Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters, sample_factor);
+      }
       project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(Q, K, N_alloc, n, nodes, lb, le,
                                                                       inv_s, idx_in, NI, wvec, keys);
       if (plan.level_max_size[l] <= kSelCap)
