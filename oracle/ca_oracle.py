@@ -37,7 +37,8 @@ Readings where the paper leaves a step open (each is listed in the design doc):
    side of every split is the left child; the split count rule picks the
    smaller multiple of c on an exact tie;
  * selection: exact top-k (ties to the lower key-cluster index), not the
-   paper's approximate histogram;
+   paper's approximate histogram; adaptive selection as the exact greedy
+   prefix by estimated mass |b| e^{s_ab / sqrt(d)} (see adaptive_route);
  * compensation weight |c| is the number of real members of the cluster.
 
 Random numbers: SplitMix64 (Steele, Lea & Flood, "Fast splittable
@@ -142,6 +143,13 @@ def psd_root(M: np.ndarray) -> np.ndarray:
 def key_representation(K: np.ndarray, R_q: np.ndarray) -> np.ndarray:
     """Keys mapped to query space: y = R_q k (eq. 14)."""
     return np.asarray(K, dtype=np.float64) @ R_q.T
+
+
+def query_representation_adaptive(Q: np.ndarray, R_k: np.ndarray) -> np.ndarray:
+    """Query representation for adaptive selection: R_k q (eq. 15), under
+    which |R_k (q1 - q2)|^2 = (q1 - q2)^T K_c^T K_c (q1 - q2) / n; no
+    normalisation (Section 3.2.2 "Query clustering", first case)."""
+    return np.asarray(Q, dtype=np.float64) @ R_k.T
 
 
 def query_representation(Q: np.ndarray, R_k: np.ndarray) -> np.ndarray:
@@ -351,11 +359,12 @@ def _centroids(X: np.ndarray, leaves: Sequence[np.ndarray]) -> np.ndarray:
 
 def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int = 0,
                  power_iters: int = 8, sample_factor: int = 1,
-                 transform: bool = True) -> HeadClusters:
+                 transform: bool = True, query_form: str = "topk") -> HeadClusters:
     """Cluster the valid queries and keys of one head (rows [n, d]).
 
     Keys are split in the query-aware space R_q k; queries in the key-aware,
-    normalised space R_k q / |R_k q| (top-k form). ``transform=False`` splits
+    normalised space R_k q / |R_k q| (top-k form, eq. 16) or, with
+    ``query_form="adaptive"``, in R_k q (eq. 15). ``transform=False`` splits
     the raw vectors (R = I, no normalisation), the paper's ablation.
     """
     Q = np.asarray(Q, dtype=np.float64)
@@ -366,7 +375,8 @@ def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int
         R_q = psd_root(M_q)
         R_k = psd_root(M_k)
         Yk = key_representation(K, R_q)
-        Yq = query_representation(Q, R_k)
+        Yq = (query_representation(Q, R_k) if query_form == "topk"
+              else query_representation_adaptive(Q, R_k))
     else:
         R_q = R_k = np.eye(d)
         Yk, Yq = K, Q
@@ -418,9 +428,41 @@ def topk_route(scores: np.ndarray, k: int) -> np.ndarray:
     return kept
 
 
+def cluster_log_mass(scores: np.ndarray, count_k: np.ndarray, d: int) -> np.ndarray:
+    """Log of the estimated attention mass of key cluster b for query cluster
+    a: |b| e^{s_ab / sqrt(d)}, the weight the compensation gives an excluded
+    cluster (eq. 21-22), with s_ab the centroid score (eq. 18)."""
+    return (np.asarray(scores, np.float64) * (1.0 / math.sqrt(d))
+            + np.log(np.asarray(count_k, np.float64))[None, :])
+
+
+def adaptive_route(scores: np.ndarray, count_k: np.ndarray, d: int, recall: float,
+                   min_count: int = 16) -> List[np.ndarray]:
+    """Adaptive selection (Section 3.3.2 "Selection"): per query cluster, take
+    key clusters in decreasing estimated attention mass (ties to the lower
+    key-cluster index) until their mass reaches ``recall`` times the total,
+    and at least ``min_count`` of them (16 in the paper). Exact greedy
+    reading of the paper's histogram approximation: masses are
+    e^{w_b - max w} in fp64 with w = cluster_log_mass, summed in that order.
+    Returns one ascending int32 array per query cluster."""
+    W = cluster_log_mass(scores, count_k, d)
+    Cq, Ck = W.shape
+    idx = np.arange(Ck)
+    out = []
+    for a in range(Cq):
+        order = np.lexsort((idx, -W[a]))
+        mass = np.exp(W[a, order] - W[a, order[0]])
+        cum = np.cumsum(mass)
+        hit = cum >= recall * cum[-1]
+        k = (int(np.argmax(hit)) + 1 if hit.any() else Ck) if recall > 0 else 1
+        k = max(k, min(min_count, Ck))
+        out.append(np.sort(order[:k]).astype(np.int32))
+    return out
+
+
 def route_bits(kept: np.ndarray, Ck: int) -> np.ndarray:
     """Kept list as a bitmask [Cq, ceil(Ck/32)] uint32 (bit b%32 of word b//32)."""
-    Cq = kept.shape[0]
+    Cq = len(kept)
     W = -(-Ck // 32)
     bits = np.zeros((Cq, W), dtype=np.uint64)
     for a in range(Cq):

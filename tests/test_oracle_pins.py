@@ -460,3 +460,113 @@ def test_compensation_error_shrinks_as_clusters_tighten():
         errs.append(float(np.mean(e)))
     assert errs[0] > errs[1] > errs[2] > errs[3]
     assert errs[3] < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Adaptive selection (Section 3.3.2 "Selection") and the adaptive query
+# representation (eq. 15)
+# ---------------------------------------------------------------------------
+
+def _brute_adaptive(scores, count_k, d, recall, min_count):
+    """Direct evaluation of the definition: sort by mass with Python's sort,
+    add masses one at a time with math.fsum-free plain floats in that order."""
+    Cq, Ck = scores.shape
+    out = []
+    for a in range(Cq):
+        w = [float(scores[a, b]) / math.sqrt(d) + math.log(float(count_k[b])) for b in range(Ck)]
+        order = sorted(range(Ck), key=lambda b: (-w[b], b))
+        mass = [math.exp(w[b] - w[order[0]]) for b in order]
+        total = 0.0
+        for m in mass:
+            total += m
+        cum, k = 0.0, Ck
+        for i, m in enumerate(mass):
+            cum += m
+            if cum >= recall * total:
+                k = i + 1
+                break
+        if recall <= 0:
+            k = 1
+        k = max(k, min(min_count, Ck))
+        out.append(sorted(order[:k]))
+    return out
+
+
+@pytest.mark.parametrize("recall", [0.0, 0.3, 0.9, 0.999, 1.0])
+def test_adaptive_route_matches_brute_force(recall):
+    r = rng(31)
+    d = 16
+    scores = r.normal(size=(12, 40)) * 4.0
+    count_k = r.integers(1, 200, size=40)
+    got = orc.adaptive_route(scores, count_k, d, recall, min_count=5)
+    want = _brute_adaptive(scores, count_k, d, recall, 5)
+    assert [list(g) for g in got] == want
+
+
+def test_adaptive_route_at_zero_recall_is_top_k_by_mass():
+    # The paper: for top-k assignment the recall threshold is 0, so the count
+    # threshold alone decides; with equal counts the mass order is the score
+    # order and the result is exactly top-k.
+    r = rng(32)
+    scores = r.normal(size=(9, 30))
+    count_k = np.full(30, 64)
+    got = orc.adaptive_route(scores, count_k, 64, 0.0, min_count=7)
+    want = orc.topk_route(scores, 7)
+    assert all(np.array_equal(g, w) for g, w in zip(got, want))
+
+
+def test_adaptive_route_weights_cluster_size():
+    # Two clusters, the second with a lower centroid score but 1000 times the
+    # members: its estimated mass |b| e^{s/sqrt(d)} is larger, so it is taken
+    # first and alone reaches a 50% recall.
+    d = 4
+    scores = np.array([[2.0, 0.0]])
+    count_k = np.array([1, 1000])
+    got = orc.adaptive_route(scores, count_k, d, 0.5, min_count=1)
+    assert list(got[0]) == [1]
+
+
+def test_adaptive_route_is_minimal_and_reaches_recall():
+    r = rng(33)
+    d = 32
+    scores = r.normal(size=(20, 64)) * 6.0
+    count_k = r.integers(50, 130, size=64)
+    recall = 0.8
+    W = scores / math.sqrt(d) + np.log(count_k)[None, :]
+    for a, kept in enumerate(orc.adaptive_route(scores, count_k, d, recall, min_count=3)):
+        m = np.exp(W[a] - W[a].max())
+        total = m.sum()
+        assert m[kept].sum() >= recall * total * (1 - 1e-12)
+        if len(kept) > 3:
+            # dropping the lightest kept cluster falls below the recall
+            lightest = kept[np.argmin(m[kept])]
+            assert m[kept].sum() - m[lightest] < recall * total
+        # every kept cluster outweighs every excluded one
+        excl = np.setdiff1d(np.arange(64), kept)
+        assert m[kept].min() >= m[excl].max()
+
+
+def test_adaptive_query_representation_is_the_eq15_metric():
+    # |R_k (q1 - q2)|^2 = (q1 - q2)^T K_c^T K_c (q1 - q2) / n (eq. 15).
+    r = rng(34)
+    Q = r.normal(size=(200, 8)); K = r.normal(size=(200, 8)) + 0.5   # n tokens of each
+    _, M_k, _ = orc.metric_matrices(Q, K)
+    Kc = K - K.mean(axis=0)
+    Y = orc.query_representation_adaptive(Q, orc.psd_root(M_k))
+    for i, j in [(0, 1), (3, 17), (20, 49)]:
+        dq = Q[i] - Q[j]
+        want = float(np.sum((Kc @ dq) ** 2)) / K.shape[0]
+        got = float(np.sum((Y[i] - Y[j]) ** 2))
+        assert got == pytest.approx(want, rel=1e-10)
+
+
+def test_adaptive_route_breaks_mass_ties_to_the_lower_index():
+    # Equal scores and counts: every cluster has the same mass, so the first
+    # min_count clusters (lowest indices) are kept, and with 50% recall of 10
+    # equal masses, exactly the first 5.
+    scores = np.zeros((2, 10))
+    count_k = np.full(10, 32)
+    got = orc.adaptive_route(scores, count_k, 16, 0.0, min_count=3)
+    assert [list(g) for g in got] == [[0, 1, 2], [0, 1, 2]]
+    got = orc.adaptive_route(scores, count_k, 16, 0.5, min_count=1)
+    assert list(got[0]) == [0, 1, 2, 3, 4]
