@@ -282,6 +282,7 @@ struct TcParams {
   const int32_t* perm_q;      // [BH][C*c]
   const int32_t* count_k;     // [BH][C]
   const int32_t* kept_idx;    // [BH][C][k]
+  const int32_t* kept_count;  // [BH][C] kept per query cluster, or null (k each)
   const uint32_t* kept_bits;  // [BH][C][W]
   const float* logcnt;        // [BH][Cpad] natural log of counts
   __nv_bfloat16* O;           // [BH][N_alloc][D]
@@ -314,11 +315,16 @@ struct TcCfg {
   // TMEM: NB S buffers of KB columns (P_j as bf16 pairs over the front half
   // of its buffer), then O_0 and O_1 (fp32, D columns each)
   static constexpr int kNBufFit = (512 - 2 * D) / KB;
-  static constexpr int kNBuf = kNBufFit > 4 ? 4 : kNBufFit;
+  // S_{j+NB} is issued after PV_j; a centroid block takes two stages (kbar,
+  // then vbar), so the stage S_{j+NB} needs is free by then only while
+  // NB <= floor(stages / 2) + 1 (otherwise it waits on a PV not yet issued)
+  static constexpr int kNBufPipe = kStages / 2 + 1;
+  static constexpr int kNBuf = kNBufFit < kNBufPipe ? kNBufFit : kNBufPipe;
   static constexpr int kSPhase = (kNBuf % 2 == 0) ? kNBuf : 2 * kNBuf;   // blocks between uses of one s_full
   static constexpr uint32_t kSCol = 0;
   static constexpr uint32_t kOCol = kNBuf * KB;
   static_assert(kNBuf >= 2, "two S buffers at least");
+  static_assert(kNBuf <= kStages / 2 + 1 && kNBuf <= kStages, "S look-ahead must not outrun the stage ring");
   static_assert(kOCol + 2 * D <= kTmemCols, "S buffers and both O accumulators must fit in TMEM");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
@@ -369,14 +375,16 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int a = p.dense ? 0 : tile / p.tiles_per_cluster;          // query cluster
   const int sub_tile = p.dense ? 0 : tile % p.tiles_per_cluster;
   const int nsb = p.dense ? 1 : (p.c + KB - 1) / KB;               // key sub-blocks per cluster
-  const int J_kept = p.dense ? p.dense_key_blocks : p.k * nsb;
+  // kept key clusters of this query cluster (k, or its own count after adaptive selection)
+  const int kq = p.dense ? 0 : (p.kept_count ? min(max(p.kept_count[(size_t)bh * p.C + a], 0), p.k) : p.k);
+  const int J_kept = p.dense ? p.dense_key_blocks : kq * nsb;
   const int J_cent = (p.compensate && !p.dense) ? p.Cpad / KB : 0;
   const int J = J_kept + J_cent;
   const int n_items = J_kept + 2 * J_cent;
   const int32_t* kept_g = p.dense ? nullptr : p.kept_idx + ((size_t)bh * p.C + a) * p.k;
-  const bool kept_in_smem = !p.dense && p.k <= Cfg::kMaxKeptSmem;
+  const bool kept_in_smem = !p.dense && kq <= Cfg::kMaxKeptSmem;
   if (kept_in_smem) {
-    for (int i = threadIdx.x; i < p.k; i += Cfg::kThreads) {
+    for (int i = threadIdx.x; i < kq; i += Cfg::kThreads) {
       const int b = kept_g[i];
       kept_s[i] = b;
       kcnt_s[i] = p.count_k[(size_t)bh * p.C + b];
@@ -814,6 +822,7 @@ cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_
   p.dense_key_blocks = 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.perm_q = cl->perm_q; p.count_k = cl->count_k; p.kept_idx = rt->kept_idx; p.kept_bits = rt->kept_bits;
+  p.kept_count = rt->kept_count;
   p.logcnt = reinterpret_cast<const float*>(ws + L.logcnt);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.wait_limit = wait_limit();

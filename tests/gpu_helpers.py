@@ -11,6 +11,13 @@ def torch():
     return _t
 
 
+def check_device_error():
+    """Every bounded wait in the kernels reports a timeout through the
+    library's device error word; a GPU test must see it clear."""
+    st = ca.ca_get_device_error()
+    assert st == ca.CA_OK, f"device error: {ca.status_string(st)}"
+
+
 def dev_tensor(x: np.ndarray, dtype: str):
     """float32 numpy (bf16-exact for bf16 workloads) -> contiguous CUDA tensor."""
     t = torch()
@@ -28,7 +35,8 @@ def shape_of(w, n_valid=None):
 class Run:
     """Device buffers for one workload and the C-ABI calls on them."""
 
-    def __init__(self, w, k=None, compensate=None, seed=0, power_iters=8, transform=True):
+    def __init__(self, w, k=None, compensate=None, seed=0, power_iters=8, transform=True, selection="topk",
+                 recall=0.9, min_count=16):
         t = torch()
         self.w = w
         self.k = w.k if k is None else k
@@ -39,12 +47,14 @@ class Run:
         self.O = t.empty_like(self.Q)
         self.layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, self.k, dtype=w.dtype,
                                          compensate=self.compensate, power_iters=power_iters,
-                                         transform=transform, seed=seed)
+                                         transform=transform, seed=seed, selection=selection, recall=recall,
+                                         min_count=min_count)
         self.C = self.layer.C
 
     def cluster(self):
         self.layer.cluster(self.Q, self.K)
         t = torch(); t.cuda.synchronize()
+        check_device_error()
         b = self.layer.buf
         BH, C, c, d = self.w.B * self.w.H, self.C, self.w.c, self.w.d
         return dict(perm_q=b.perm_q.cpu().numpy().reshape(BH, C * c),
@@ -68,11 +78,17 @@ class Run:
     def route(self):
         self.layer.route()
         t = torch(); t.cuda.synchronize()
+        check_device_error()
         b = self.layer.buf
         BH, C = self.w.B * self.w.H, self.C
         W = (C + 31) // 32
         return (b.kept_idx.cpu().numpy().reshape(BH, C, self.k),
                 b.kept_bits.cpu().numpy().view(np.uint32).reshape(BH, C, W))
+
+    def route_counts(self):
+        """Per-query-cluster kept counts [BH, C] (adaptive selection)."""
+        b = self.layer.buf
+        return b.kept_count.cpu().numpy().reshape(self.w.B * self.w.H, self.C)
 
     def set_routes(self, kept_list):
         from oracle import ca_oracle as orc
@@ -85,6 +101,7 @@ class Run:
     def attend(self):
         self.layer.attend(self.Q, self.K, self.V, self.O)
         t = torch(); t.cuda.synchronize()
+        check_device_error()
         return self.O.float().cpu().numpy()
 
     def dense(self):
@@ -92,9 +109,11 @@ class Run:
         O = t.empty_like(self.Q)
         self.layer.dense(self.Q, self.K, self.V, O)
         t.cuda.synchronize()
+        check_device_error()
         return O.float().cpu().numpy()
 
     def forward(self):
         self.layer(self.Q, self.K, self.V, self.O)
         t = torch(); t.cuda.synchronize()
+        check_device_error()
         return self.O.float().cpu().numpy()

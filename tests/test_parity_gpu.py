@@ -42,6 +42,11 @@ def _cases():
                                                         seed=13, grid=(8, 9, 80)),
         "heavytail-bf16-d64-c256": lambda: wl.make_workload("heavytail", H=1, N=8192, d=64, c=256, k=4,
                                                             dtype="bf16", seed=14),
+        # 64-key blocks on the tensor cores, with compensation blocks
+        "heavytail-bf16-d64-c64": lambda: wl.make_workload("heavytail", H=1, N=8192, d=64, c=64, k=8,
+                                                           dtype="bf16", seed=15),
+        "lowrank-bf16-d128-c64": lambda: wl.make_workload("lowrank", H=1, N=2048, n_valid=2000, d=128, c=64,
+                                                          k=5, dtype="bf16", seed=16),
     }
 
 
