@@ -27,7 +27,7 @@ EXPORTED = [
     "ca_dense_workspace_bytes", "ca_forward_workspace_bytes", "ca_cluster", "ca_route", "ca_attend",
     "ca_dense_attend", "ca_forward", "ca_forward_host_workspace_bytes", "ca_forward_host",
     "ca_get_device_error", "ca_set_wait_limit", "ca_status_string", "ca_version", "ca_launch_count",
-    "ca_cluster_noalloc",
+    "ca_cluster_noalloc", "ca_route_adaptive",
 ]
 
 
@@ -49,7 +49,7 @@ class ca_shape(ctypes.Structure):
 
 class ca_cluster_params(ctypes.Structure):
     _fields_ = [("power_iters", ctypes.c_int), ("sample_factor", ctypes.c_int),
-                ("transform", ctypes.c_int), ("reserved", ctypes.c_int), ("seed", ctypes.c_uint64)]
+                ("transform", ctypes.c_int), ("query_form", ctypes.c_int), ("seed", ctypes.c_uint64)]
 
 
 class ca_clusters(ctypes.Structure):
@@ -58,7 +58,8 @@ class ca_clusters(ctypes.Structure):
 
 
 class ca_routes(ctypes.Structure):
-    _fields_ = [("k", ctypes.c_int), ("kept_idx", ctypes.c_void_p), ("kept_bits", ctypes.c_void_p)]
+    _fields_ = [("k", ctypes.c_int), ("kept_idx", ctypes.c_void_p), ("kept_bits", ctypes.c_void_p),
+                ("kept_count", ctypes.c_void_p)]
 
 
 _lib = None
@@ -93,6 +94,7 @@ def lib():
             "ca_version": (ctypes.c_char_p, []),
             "ca_launch_count": (i32, [P(ca_shape), i32]),
             "ca_cluster_noalloc": (i32, [vp, vp, P(ca_shape), P(ca_cluster_params), P(ca_clusters), vp]),
+            "ca_route_adaptive": (i32, [P(ca_shape), P(ca_clusters), ctypes.c_double, i32, P(ca_routes), vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -130,8 +132,10 @@ def make_shape(B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, dtype
 
 
 def make_params(power_iters: int = 8, sample_factor: int = 1, transform: int = 1,
-                seed: int = 0) -> ca_cluster_params:
-    return ca_cluster_params(power_iters, sample_factor, transform, 0, seed & ((1 << 64) - 1))
+                seed: int = 0, query_form: int = 0) -> ca_cluster_params:
+    """query_form 0: queries as R_k q / |R_k q| (top-k selection, eq. 16);
+    1: queries as R_k q (adaptive selection, eq. 15)."""
+    return ca_cluster_params(power_iters, sample_factor, transform, query_form, seed & ((1 << 64) - 1))
 
 
 def num_clusters(shape: ca_shape) -> int:
@@ -158,8 +162,8 @@ def clusters_struct(perm_q, perm_k, count_q, count_k, qbar, kbar) -> ca_clusters
     return ca_clusters(_ptr(perm_q), _ptr(perm_k), _ptr(count_q), _ptr(count_k), _ptr(qbar), _ptr(kbar))
 
 
-def routes_struct(k: int, kept_idx, kept_bits) -> ca_routes:
-    return ca_routes(k, _ptr(kept_idx), _ptr(kept_bits))
+def routes_struct(k: int, kept_idx, kept_bits, kept_count=None) -> ca_routes:
+    return ca_routes(k, _ptr(kept_idx), _ptr(kept_bits), _ptr(kept_count))
 
 
 def ca_cluster(Q, K, shape: ca_shape, params: Optional[ca_cluster_params], clusters: ca_clusters,
@@ -185,6 +189,15 @@ def ca_cluster_noalloc(Q, K, shape: ca_shape, params: Optional[ca_cluster_params
 def ca_route(shape: ca_shape, centroids: ca_clusters, routes: ca_routes, stream=None):
     _check(lib().ca_route(ctypes.byref(shape), ctypes.byref(centroids), ctypes.byref(routes),
                           _stream(stream)), "ca_route")
+
+
+def ca_route_adaptive(shape: ca_shape, centroids: ca_clusters, recall: float, min_count: int,
+                      routes: ca_routes, stream=None):
+    """Adaptive selection: per query cluster, key clusters by decreasing
+    estimated attention mass until `recall` of the total, at least
+    `min_count`; routes.kept_count receives the counts."""
+    _check(lib().ca_route_adaptive(ctypes.byref(shape), ctypes.byref(centroids), float(recall), int(min_count),
+                                   ctypes.byref(routes), _stream(stream)), "ca_route_adaptive")
 
 
 def ca_attend(Q, K, V, shape: ca_shape, clusters: ca_clusters, routes: ca_routes, compensate: bool, O,

@@ -48,6 +48,7 @@ ca_status check_params(const ca_shape* s, const ca_cluster_params* p) {
   const int a = p->sample_factor > 0 ? p->sample_factor : 1;
   if (dir_smem(s->d, a) > 227 * 1024) return CA_ERR_UNSUPPORTED;
   if (p->transform != 0 && p->transform != 1) return CA_ERR_INVALID_ARG;
+  if (p->query_form != 0 && p->query_form != 1) return CA_ERR_INVALID_ARG;
   return CA_OK;
 }
 
@@ -160,7 +161,24 @@ ca_status ca_route(const ca_shape* s, const ca_clusters* cen, const ca_routes* o
   if (out->k < 1 || out->k > C) return CA_ERR_INVALID_ARG;
   if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
   return cuda_status(launch_route(s, C, cen->qbar, cen->kbar, out->k, out->kept_idx, out->kept_bits,
-                                  static_cast<cudaStream_t>(stream)));
+                                  out->kept_count, static_cast<cudaStream_t>(stream)));
+}
+
+ca_status ca_route_adaptive(const ca_shape* s, const ca_clusters* cen, double recall, int min_count,
+                            const ca_routes* out, void* stream) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!cen || !cen->qbar || !cen->kbar || !cen->count_k || !out || !out->kept_idx || !out->kept_bits ||
+      !out->kept_count)
+    return CA_ERR_INVALID_ARG;
+  if (!aligned16(cen->qbar) || !aligned16(cen->kbar)) return CA_ERR_INVALID_ARG;
+  if (!(recall >= 0.0 && recall <= 1.0) || min_count < 1) return CA_ERR_INVALID_ARG;
+  const int C = (s->n_valid + s->c - 1) / s->c;
+  if (out->k < 1 || out->k > C) return CA_ERR_INVALID_ARG;
+  if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
+  return cuda_status(launch_route_adaptive(s, C, cen->qbar, cen->kbar, cen->count_k, recall, min_count, out->k,
+                                           out->kept_idx, out->kept_bits, out->kept_count,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* s, const ca_clusters* cl,
@@ -230,6 +248,7 @@ ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape
   cl.kbar = reinterpret_cast<double*>(ws + f.kbar);
   ca_routes rt;
   rt.k = k;
+  rt.kept_count = nullptr;
   rt.kept_idx = reinterpret_cast<int32_t*>(ws + f.kept_idx);
   rt.kept_bits = reinterpret_cast<uint32_t*>(ws + f.kept_bits);
   st = ca_cluster(Q, K, s, params, &cl, ws + f.scratch, f.cluster_bytes, stream);

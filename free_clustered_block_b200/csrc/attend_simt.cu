@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, int N_alloc, int n_valid,
     int c, int C, int k, const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
     const int32_t* __restrict__ kept_idx, const uint32_t* __restrict__ kept_bits,
-    const float* __restrict__ kbar32, const float* __restrict__ vbar32, const float* __restrict__ logcnt,
+    const int32_t* __restrict__ kept_count, const float* __restrict__ kbar32, const float* __restrict__ vbar32, const float* __restrict__ logcnt,
     int Cpad, int compensate, int mode, float scale, T* __restrict__ O) {
   constexpr int TPR = D / 16;
   constexpr int NT = kRows * TPR;
@@ -117,7 +117,9 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
   if (mode == 0) {
     const int32_t* kl = kept_idx + ((size_t)bh * C + a) * k;
     const int32_t* pk = perm_k + (size_t)bh * C * c;
-    for (int i = 0; i < k; ++i) {
+    // k each, or the query cluster's own count after adaptive selection
+    const int kq = kept_count ? min(max(kept_count[(size_t)bh * C + a], 0), k) : k;
+    for (int i = 0; i < kq; ++i) {
       const int b = kl[i];
       for (int t0 = 0; t0 < c; t0 += kTile) {
         __syncthreads();
@@ -189,7 +191,7 @@ cudaError_t run_simt(const void* Q, const void* K, const void* V, const ca_shape
   simt_attend_kernel<T, D><<<grid, kRows * (D / 16), 0, st>>>(
       (const T*)Q, (const T*)K, (const T*)V, s->N_alloc, s->n_valid, c, C, rt ? rt->k : 0,
       cl ? cl->perm_q : nullptr, cl ? cl->perm_k : nullptr, rt ? rt->kept_idx : nullptr,
-      rt ? rt->kept_bits : nullptr, kbar32, vbar32, logcnt, L ? L->Cpad : 0, compensate, mode, scale,
+      rt ? rt->kept_bits : nullptr, rt ? rt->kept_count : nullptr, kbar32, vbar32, logcnt, L ? L->Cpad : 0, compensate, mode, scale,
       (T*)O);
   return cudaGetLastError();
 }

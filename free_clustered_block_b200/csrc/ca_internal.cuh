@@ -142,7 +142,11 @@ cudaError_t launch_cluster(const void* Q, const void* K, const ca_shape* s,
                            const ca_cluster_params* p, const ca_clusters* out,
                            const TreePlan& plan, const ClusterWs& L, char* ws, cudaStream_t st);
 cudaError_t launch_route(const ca_shape* s, int C, const double* qbar, const double* kbar, int k,
-                         int32_t* kept_idx, uint32_t* kept_bits, cudaStream_t st);
+                         int32_t* kept_idx, uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st);
+size_t route_adaptive_smem(int C);
+cudaError_t launch_route_adaptive(const ca_shape* s, int C, const double* qbar, const double* kbar,
+                                  const int32_t* count_k, double recall, int min_count, int k, int32_t* kept_idx,
+                                  uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st);
 cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, const ca_shape* s,
                                const ca_clusters* cl, const AttendWs& L, char* ws, cudaStream_t st);
 cudaError_t launch_attend_simt(const void* Q, const void* K, const void* V, const ca_shape* s,

@@ -1251,6 +1251,9 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
   const int power_iters = p->power_iters > 0 ? p->power_iters : 8;
   const int sample_factor = p->sample_factor > 0 ? p->sample_factor : 1;
   const int transform = p->transform;
+  // queries are divided by |R_k q| only in the top-k form (eq. 16); the
+  // adaptive form (eq. 15) and the untransformed ablation use scale 1
+  const int normalize = transform && p->query_form == 0;
 
   if (plan.levels > 0) {
     plan_kernel<<<1, 1024, 0, st>>>(n, c, nodes, level_begin);
@@ -1260,12 +1263,12 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
                                                                                 metpart);
     metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
-    if (D == 64 && transform) {
+    if (D == 64 && normalize) {
       qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
     } else {
       const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
       cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
-      qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, transform, inv_s);
+      qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, normalize, inv_s);
     }
     const int m_cap = sample_factor * D;
     const int dir_warps = DirCfg<T, D>::warps(m_cap);

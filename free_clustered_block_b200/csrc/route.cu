@@ -32,7 +32,8 @@ template <int D, int QA>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* __restrict__ qbar,
                                                                  const double* __restrict__ kbar, int C, int k,
                                                                  int32_t* __restrict__ kept_idx,
-                                                                 uint32_t* __restrict__ kept_bits) {
+                                                                 uint32_t* __restrict__ kept_bits,
+                                                                 int32_t* __restrict__ kept_count) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* qs = reinterpret_cast<double*>(smem_raw);   // QA x D
   double* sc = qs + QA * D;                           // QA x C scores
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* _
     // membership, bitmask and ascending kept list
     int32_t* krow = kept_idx + ((size_t)bh * C + a0 + r) * k;
     uint32_t* brow = kept_bits + ((size_t)bh * C + a0 + r) * W;
+    if (kept_count && lane == 0) kept_count[(size_t)bh * C + a0 + r] = k;
     int base = 0, eqseen = 0;
     for (int i = 0; i < W; ++i) {
       const int b = i * 32 + lane;
@@ -177,24 +179,24 @@ size_t route_smem(int C) {
 
 template <int D, int QA>
 cudaError_t launch_qa(const ca_shape* s, int C, const double* qbar, const double* kbar, int k, int32_t* kept_idx,
-                      uint32_t* kept_bits, cudaStream_t st) {
+                      uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
   const size_t smem = route_smem<D, QA>(C);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((C + QA - 1) / QA, s->B * s->H);
-  route_kernel<D, QA><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, k, kept_idx, kept_bits);
+  route_kernel<D, QA><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, k, kept_idx, kept_bits, kept_count);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_d(const ca_shape* s, int C, const double* qbar, const double* kbar, int k, int32_t* kept_idx,
-                     uint32_t* kept_bits, cudaStream_t st) {
+                     uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
   // as many query clusters per block as the score rows allow in the budget
-  if (route_smem<D, 16>(C) <= kRouteSmemBudget) return launch_qa<D, 16>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
-  if (route_smem<D, 8>(C) <= kRouteSmemBudget) return launch_qa<D, 8>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
-  if (route_smem<D, 4>(C) <= kRouteSmemBudget) return launch_qa<D, 4>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
-  if (route_smem<D, 2>(C) <= kRouteSmemBudget) return launch_qa<D, 2>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
-  return launch_qa<D, 1>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+  if (route_smem<D, 16>(C) <= kRouteSmemBudget) return launch_qa<D, 16>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 8>(C) <= kRouteSmemBudget) return launch_qa<D, 8>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 4>(C) <= kRouteSmemBudget) return launch_qa<D, 4>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 2>(C) <= kRouteSmemBudget) return launch_qa<D, 2>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  return launch_qa<D, 1>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
 }
 
 }  // namespace
@@ -204,9 +206,159 @@ size_t route_smem_bytes(int C, int D) {
 }
 
 cudaError_t launch_route(const ca_shape* s, int C, const double* qbar, const double* kbar, int k,
-                         int32_t* kept_idx, uint32_t* kept_bits, cudaStream_t st) {
-  if (s->d == 64) return launch_d<64>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
-  return launch_d<128>(s, C, qbar, kbar, k, kept_idx, kept_bits, st);
+                         int32_t* kept_idx, uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
+  if (s->d == 64) return launch_d<64>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  return launch_d<128>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+}
+
+// ---------------------------------------------------------------------------
+// Adaptive selection (Section 3.3.2, second method): one block per query
+// cluster. w_b = s_ab / sqrt(d) + ln|b| is the log of the estimated attention
+// mass |b| e^{s_ab / sqrt(d)}; the key clusters are sorted by decreasing w
+// (ties to the lower index, bitonic network in shared memory), their masses
+// e^{w - w_max} summed in that order by one thread, and the shortest prefix
+// whose running sum reaches recall x total is kept (at least min(min_count,
+// C) clusters, at most the row capacity k).
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kAdaptThreads = 256;
+
+// bitonic width: the power of two >= C, at least 64
+int adaptive_cpad(int C) {
+  int p = 64;
+  while (p < C) p <<= 1;
+  return p;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAdaptThreads) route_adaptive_kernel(
+    const double* __restrict__ qbar, const double* __restrict__ kbar, const int32_t* __restrict__ count_k, int C,
+    int Cpad, double recall, int min_count, int k, int32_t* __restrict__ kept_idx,
+    uint32_t* __restrict__ kept_bits, int32_t* __restrict__ kept_count) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* w = reinterpret_cast<double*>(smem_raw);             // Cpad: log masses, then masses
+  int* id = reinterpret_cast<int*>(w + Cpad);                  // Cpad
+  uint32_t* bits = reinterpret_cast<uint32_t*>(id + Cpad);     // Cpad / 32
+  __shared__ double qa[D];
+  __shared__ int kcount;
+  const int a = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const double* kb = kbar + (size_t)bh * C * D;
+  for (int e = t; e < D; e += kAdaptThreads) qa[e] = qbar[((size_t)bh * C + a) * D + e];
+  for (int e = t; e < Cpad / 32; e += kAdaptThreads) bits[e] = 0u;
+  __syncthreads();
+  const double scale = 1.0 / sqrt((double)D);
+  for (int b = t; b < Cpad; b += kAdaptThreads) {
+    double v = -INFINITY;
+    if (b < C) {
+      const double2* kr = reinterpret_cast<const double2*>(kb + (size_t)b * D);
+      double s0 = 0.0, s1 = 0.0;
+#pragma unroll 8
+      for (int j = 0; j < D / 2; ++j) {
+        const double2 k2 = __ldg(kr + j);
+        s0 = fma(qa[2 * j], k2.x, s0);
+        s1 = fma(qa[2 * j + 1], k2.y, s1);
+      }
+      v = (s0 + s1) * scale + log((double)count_k[(size_t)bh * C + b]);
+    }
+    w[b] = v;
+    id[b] = b < C ? b : 0x7fffffff;
+  }
+  __syncthreads();
+  // bitonic sort: decreasing w, increasing index
+  for (int size = 2; size <= Cpad; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = t; i < Cpad; i += kAdaptThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const double wi = w[i], wj = w[j];
+          const int ii = id[i], ij = id[j];
+          const bool i_first = (wi > wj) || (wi == wj && ii < ij);
+          const bool up = ((i & size) == 0);
+          if (up ? !i_first : i_first) { w[i] = wj; w[j] = wi; id[i] = ij; id[j] = ii; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const double wmax = w[0];
+  __syncthreads();
+  for (int i = t; i < C; i += kAdaptThreads) w[i] = exp(w[i] - wmax);
+  __syncthreads();
+  if (t == 0) {
+    double total = 0.0;
+    for (int i = 0; i < C; ++i) total += w[i];
+    int kk = 1;
+    if (recall > 0.0) {
+      const double need = recall * total;
+      double cum = 0.0;
+      kk = C;
+      for (int i = 0; i < C; ++i) {
+        cum += w[i];
+        if (cum >= need) { kk = i + 1; break; }
+      }
+    }
+    kk = max(kk, min(min_count, C));
+    kcount = min(kk, k);
+  }
+  __syncthreads();
+  const int kk = kcount;
+  for (int i = t; i < kk; i += kAdaptThreads) atomicOr(&bits[id[i] >> 5], 1u << (id[i] & 31));
+  __syncthreads();
+  const int W = (C + 31) / 32;
+  for (int e = t; e < W; e += kAdaptThreads) kept_bits[((size_t)bh * C + a) * W + e] = bits[e];
+  if (t == 0) kept_count[(size_t)bh * C + a] = kk;
+  // ascending kept list: one warp scans the words' popcounts, 32 at a time
+  if (t < 32) {
+    int32_t* krow = kept_idx + ((size_t)bh * C + a) * k;
+    int base = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+      const int e = w0 + t;
+      const uint32_t m = e < W ? bits[e] : 0u;
+      const int cnt = __popc(m);
+      int inc = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (t >= o) inc += v;
+      }
+      int o = base + inc - cnt;
+      uint32_t mm = m;
+      while (mm) {
+        krow[o++] = e * 32 + (__ffs(mm) - 1);
+        mm &= mm - 1;
+      }
+      base += __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+}
+
+}  // namespace
+
+size_t route_adaptive_smem(int C) {
+  const int Cpad = adaptive_cpad(C);
+  return (size_t)Cpad * 12 + (size_t)(Cpad / 32) * 4;
+}
+
+cudaError_t launch_route_adaptive(const ca_shape* s, int C, const double* qbar, const double* kbar,
+                                  const int32_t* count_k, double recall, int min_count, int k, int32_t* kept_idx,
+                                  uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
+  const int Cpad = adaptive_cpad(C);
+  const size_t smem = route_adaptive_smem(C);
+  const dim3 grid(C, s->B * s->H);
+  cudaError_t e;
+  if (s->d == 64) {
+    e = cudaFuncSetAttribute(route_adaptive_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_adaptive_kernel<64><<<grid, kAdaptThreads, smem, st>>>(qbar, kbar, count_k, C, Cpad, recall, min_count, k,
+                                                                 kept_idx, kept_bits, kept_count);
+  } else {
+    e = cudaFuncSetAttribute(route_adaptive_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    route_adaptive_kernel<128><<<grid, kAdaptThreads, smem, st>>>(qbar, kbar, count_k, C, Cpad, recall, min_count,
+                                                                  k, kept_idx, kept_bits, kept_count);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace ca

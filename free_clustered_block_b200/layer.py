@@ -8,7 +8,7 @@ from __future__ import annotations
 from dataclasses import dataclass
 from typing import Optional
 
-from . import (CA_BF16, CA_FP32, ca_attend, ca_cluster, ca_dense_attend, ca_forward, ca_route,
+from . import (CA_BF16, CA_FP32, ca_attend, ca_cluster, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
                attend_workspace_bytes, cluster_workspace_bytes, clusters_struct, forward_workspace_bytes,
                make_params, make_shape, num_clusters, routes_struct)
 
@@ -23,6 +23,7 @@ class Buffers:
     kbar: object
     kept_idx: object
     kept_bits: object
+    kept_count: object
 
 
 class ClusterAttention:
@@ -33,12 +34,17 @@ class ClusterAttention:
 
     def __init__(self, B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, k: int,
                  dtype: str = "bf16", compensate: bool = True, power_iters: int = 8,
-                 sample_factor: int = 1, transform: bool = True, seed: int = 0, device="cuda"):
+                 sample_factor: int = 1, transform: bool = True, seed: int = 0, device="cuda",
+                 selection: str = "topk", recall: float = 0.9, min_count: int = 16):
         import torch
         self.torch = torch
         self.dtype_code = CA_BF16 if dtype == "bf16" else CA_FP32
         self.shape = make_shape(B, H, N_alloc, n_valid, d, c, self.dtype_code)
-        self.params = make_params(power_iters, sample_factor, int(transform), seed)
+        # adaptive selection pairs with the eq. 15 query representation
+        self.selection = selection
+        self.recall, self.min_count = recall, min_count
+        self.params = make_params(power_iters, sample_factor, int(transform), seed,
+                                  query_form=1 if selection == "adaptive" else 0)
         self.k = k
         self.compensate = compensate
         C = num_clusters(self.shape)
@@ -57,6 +63,7 @@ class ClusterAttention:
             kbar=torch.empty(BH * C * d, dtype=f64, device=device),
             kept_idx=torch.empty(BH * C * k, dtype=i32, device=device),
             kept_bits=torch.empty(BH * C * W, dtype=torch.int32, device=device),
+            kept_count=torch.empty(BH * C, dtype=i32, device=device),
         )
         nbytes = max(cluster_workspace_bytes(self.shape), attend_workspace_bytes(self.shape))
         self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
@@ -67,13 +74,18 @@ class ClusterAttention:
         return clusters_struct(b.perm_q, b.perm_k, b.count_q, b.count_k, b.qbar, b.kbar)
 
     def routes(self):
-        return routes_struct(self.k, self.buf.kept_idx, self.buf.kept_bits)
+        # top-k rows hold exactly k; adaptive rows hold their own count (capacity k)
+        count = self.buf.kept_count if self.selection == "adaptive" else None
+        return routes_struct(self.k, self.buf.kept_idx, self.buf.kept_bits, count)
 
     def cluster(self, Q, K, stream=None):
         ca_cluster(Q, K, self.shape, self.params, self.clusters(), self.workspace, stream)
 
     def route(self, stream=None):
-        ca_route(self.shape, self.clusters(), self.routes(), stream)
+        if self.selection == "adaptive":
+            ca_route_adaptive(self.shape, self.clusters(), self.recall, self.min_count, self.routes(), stream)
+        else:
+            ca_route(self.shape, self.clusters(), self.routes(), stream)
 
     def attend(self, Q, K, V, O, stream=None):
         ca_attend(Q, K, V, self.shape, self.clusters(), self.routes(), self.compensate, O, self.workspace,

@@ -63,12 +63,15 @@ typedef struct {
  *  sample_factor a, sample size min(a d, |S|) per split (0 -> default 1);
  *  transform     1 = interaction-aware transforms (Section 3.2.2), the default;
  *                0 = split the raw vectors (the paper's ablation);
+ *  query_form    0 = queries as R_k q / |R_k q| (eq. 16, for top-k selection),
+ *                    the default; 1 = queries as R_k q (eq. 15, for adaptive
+ *                    selection); ignored when transform is 0;
  *  seed          counter-based generator seed for samples and warm starts. */
 typedef struct {
   int power_iters;
   int sample_factor;
   int transform;
-  int reserved;
+  int query_form;
   uint64_t seed;
 } ca_cluster_params;
 
@@ -90,14 +93,20 @@ typedef struct {
 } ca_clusters;
 
 /* Routing result:
- *  kept_idx  int32 [B][H][C][k]: the k key clusters kept by each query
- *            cluster, ascending;
- *  kept_bits uint32 [B][H][C][ceil(C/32)]: the same set as a bitmask
- *            (bit b%32 of word b/32). */
+ *  kept_idx   int32 [B][H][C][k]: the key clusters kept by each query
+ *             cluster, ascending (row stride k);
+ *  kept_bits  uint32 [B][H][C][ceil(C/32)]: the same set as a bitmask
+ *             (bit b%32 of word b/32);
+ *  kept_count int32 [B][H][C] or NULL: how many entries of each kept_idx row
+ *             are used. NULL means every query cluster keeps exactly k (top-k
+ *             selection); ca_route writes k into it when given, and
+ *             ca_route_adaptive requires it (entries past the count are
+ *             unspecified). */
 typedef struct {
   int k;
   int32_t* kept_idx;
   uint32_t* kept_bits;
+  int32_t* kept_count;
 } ca_routes;
 
 /* Number of clusters C = ceil(n_valid / c); -1 if the shape is invalid. Host only. */
@@ -169,6 +178,22 @@ ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
                    const ca_routes* out, void* stream);
 
 /*
+ * ca_route_adaptive -- centroid scores and adaptive selection.
+ * Paper Section 3.3.2 "Selection", second method: per query cluster a, take
+ * key clusters in decreasing estimated attention mass |b| e^{s_ab / sqrt(d)}
+ * (the weight the compensation gives a cluster, eq. 21-22; ties to the lower
+ * key-cluster index) until their mass reaches `recall` times the total, and
+ * at least min(min_count, C) of them (the paper uses 16). Exact greedy
+ * selection in fp64 (masses e^{w - w_max}, summed in that order), not the
+ * paper's two-pass histogram. Reads centroids->qbar, kbar (16-byte aligned)
+ * and count_k. out->k is the capacity of a kept_idx row (k = C always
+ * suffices; a longer selection is cut at k); out->kept_count is required.
+ * recall in [0, 1]; min_count >= 1; C <= 8192.
+ */
+ca_status ca_route_adaptive(const ca_shape* shape, const ca_clusters* centroids, double recall,
+                            int min_count, const ca_routes* out, void* stream);
+
+/*
  * ca_attend -- block-sparse attention over the kept clusters with striped
  * mean-compensation (SMC) of the excluded ones.
  * Paper Section 1.2 (eq. 5-6) and Appendix A (eq. 21-22): for query i of
@@ -177,7 +202,9 @@ ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
  *         + sum_{b excluded} |b| e^{q_i.kbar_b/sqrt(d)} vbar_b ) / (same weights)
  * with |b| the member count of key cluster b and vbar_b its mean value.
  * compensate = 0 drops the second sum (plain block-sparse attention).
- * Reads clusters->perm_q/perm_k/count_k/kbar and routes->kept_idx/kept_bits;
+ * Reads clusters->perm_q/perm_k/count_k/kbar and routes->kept_idx/kept_bits
+ * (and routes->kept_count when it is not NULL: per-query-cluster counts, as
+ * written by ca_route_adaptive);
  * vbar is computed here. O: device [B][H][N_alloc][d], written in original
  * row order (padding rows 0). workspace >= ca_attend_workspace_bytes(shape).
  * bf16 with compensate != 0 supports C <= 8192 key clusters
