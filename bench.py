@@ -40,7 +40,7 @@ CONFIG_ID = 2
 # profiles/tc_attend_kernel_64_128_layer_B1_H8_N65536.md. It describes the
 # kernel source whose SHA-256 starts with `source_sha256`; for any other source
 # the bench reports null.
-ATTN_TRAFFIC = {"bytes": 205448192 + 52447232, "source_sha256": "1f30034b366e1e6c"}
+ATTN_TRAFFIC = {"bytes": 205589760 + 51571200, "source_sha256": "1a4712bdd0a67bd9"}
 
 
 def attention_traffic():
@@ -89,11 +89,20 @@ def dense_flops(w):
     return 4.0 * w.n_valid * w.n_valid * w.d * w.H * w.B
 
 
-def attention_flops(w):
+def attention_flops(w, kept_counts=None, count_q=None):
     """Algorithmic FLOPs of the attention step: kept blocks (QK^T and PV over
-    k*c keys per query) plus the compensation terms of the excluded clusters."""
-    kept = 4.0 * w.n_valid * (w.k * w.c) * w.d * w.H * w.B
-    smc = 4.0 * w.n_valid * (w.C - w.k) * w.d * w.H * w.B if w.compensate else 0.0
+    the kept clusters' c keys per query) plus the compensation terms of the
+    excluded clusters. With adaptive selection the per-query-cluster kept
+    counts (and the query-cluster sizes) give the sums."""
+    if kept_counts is None:
+        kept = 4.0 * w.n_valid * (w.k * w.c) * w.d * w.H * w.B
+        smc = 4.0 * w.n_valid * (w.C - w.k) * w.d * w.H * w.B if w.compensate else 0.0
+        return kept, smc
+    import numpy as np
+    kc = np.asarray(kept_counts, np.float64)
+    nq = np.asarray(count_q, np.float64)
+    kept = float(4.0 * (nq * kc * w.c).sum() * w.d)
+    smc = float(4.0 * (nq * (w.C - kc)).sum() * w.d) if w.compensate else 0.0
     return kept, smc
 
 
@@ -155,7 +164,7 @@ def blas_threads():
         return 1
 
 
-def oracle_sample(w, n_clusters=48, heads=(0,), keep=None):
+def oracle_sample(w, n_clusters=48, heads=(0,), keep=None, selection="topk", recall=0.9):
     """Time the oracle on a bounded sample and extrapolate to one whole layer.
     Per sampled head: full clustering of queries and keys, routing, and the
     attention of `n_clusters` query clusters (work per query cluster is the
@@ -167,8 +176,12 @@ def oracle_sample(w, n_clusters=48, heads=(0,), keep=None):
     for h in heads:
         Qf, Kf, Vf = (x[0, h, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         t0 = time.perf_counter()
-        hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h)
-        kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
+        if selection == "adaptive":
+            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, query_form="adaptive")
+            kept = orc.adaptive_route(orc.centroid_scores(hc.qbar, hc.kbar), hc.count_k, w.d, recall, 16)
+        else:
+            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h)
+            kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
         t1 = time.perf_counter()
         sample = list(range(0, w.C, max(1, w.C // n_clusters)))[:n_clusters]
         out = orc.compensated_attention(Qf, Kf, Vf, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, w.c,
@@ -282,8 +295,10 @@ def run_ours(args):
 
     Q, K, V = dev(w.Q), dev(w.K), dev(w.V)
     O = torch.empty_like(Q)
-    layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.k, dtype=w.dtype,
-                                compensate=w.compensate)
+    adaptive = args.selection == "adaptive"
+    layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.C if adaptive else w.k,
+                                dtype=w.dtype, compensate=w.compensate, selection=args.selection,
+                                recall=args.recall, min_count=16)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -319,6 +334,9 @@ def run_ours(args):
         end.record(stream)
         torch.cuda.synchronize()
         barrier()
+    st = ca.ca_get_device_error()
+    if st != ca.CA_OK:
+        raise RuntimeError(f"device error in the timed region: {ca.status_string(st)}")
     # with flushes, the steps are timed one by one (the flushes are not timed)
     total_ms = ranks_max(sum(ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)) if flush
                          else start.elapsed_time(end))
@@ -341,19 +359,32 @@ def run_ours(args):
     torch.cuda.synchronize()
     dense_ms = ranks_max(d0.elapsed_time(d1) / dense_iters)
 
-    # End to end through the C ABI with host buffers (pinned), copies inside the region.
+    # End to end with host buffers (pinned), copies inside the region: the
+    # single ca_forward_host call for top-k; the layer API (copy in, cluster,
+    # route, attend, copy out) for adaptive selection.
     shape = layer.shape
     hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
     hO = torch.empty_like(hQ).pin_memory()
-    wsh = torch.empty(ca.forward_host_workspace_bytes(shape, w.k), dtype=torch.uint8, device="cuda")
+    if adaptive:
+        dQ, dK, dV, dO = (torch.empty_like(x) for x in (Q, K, V, O))
+
+        def e2e_step():
+            dQ.copy_(hQ, non_blocking=True); dK.copy_(hK, non_blocking=True); dV.copy_(hV, non_blocking=True)
+            layer(dQ, dK, dV, dO)
+            hO.copy_(dO, non_blocking=True)
+    else:
+        wsh = torch.empty(ca.forward_host_workspace_bytes(shape, w.k), dtype=torch.uint8, device="cuda")
+
+        def e2e_step():
+            ca.ca_forward_host(hQ, hK, hV, shape, layer.params, w.k, w.compensate, hO, wsh)
     for _ in range(max(1, args.warmup)):
-        ca.ca_forward_host(hQ, hK, hV, shape, layer.params, w.k, w.compensate, hO, wsh)
+        e2e_step()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(args.steps):
-        ca.ca_forward_host(hQ, hK, hV, shape, layer.params, w.k, w.compensate, hO, wsh)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ranks_max(e0.elapsed_time(e1))
@@ -386,7 +417,11 @@ def run_ours(args):
         graph_ms = f"capture failed: {type(e).__name__}"
 
     pk = peaks()
-    kept_f, smc_f = attention_flops(w)
+    if adaptive:
+        kc = layer.buf.kept_count.cpu().numpy()
+        kept_f, smc_f = attention_flops(w, kc, layer.buf.count_q.cpu().numpy())
+    else:
+        kept_f, smc_f = attention_flops(w)
     attn_s = stage["attend"] / 1e3
     achieved = (kept_f + smc_f) / attn_s / 1e12
     if w.dtype == "bf16":
@@ -412,7 +447,10 @@ def run_ours(args):
         "vs_baseline": None, "dtype": w.dtype,
         "dtype_detail": ("clustering and routing f64; attention bf16 products with f32 accumulation"
                          if w.dtype == "bf16" else "clustering and routing f64; attention f32"),
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic",
+        "config": dict(workload_config(w), selection=args.selection,
+                       **({"recall": args.recall, "min_count": 16,
+                           "mean_kept": float(kc.mean())} if adaptive else {})),
         "latency_ms": ms_per_step, "stage_ms": stage, "dense_ms": dense_ms,
         "speedup_vs_dense": dense_ms / ms_per_step,
         "graph_ms_per_step": graph_ms,
@@ -426,7 +464,7 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         kept = {}
-        t_cpu, smp = oracle_sample(w, keep=kept)
+        t_cpu, smp = oracle_sample(w, keep=kept, selection=args.selection, recall=args.recall)
         line["error_vs_dense_fp64"] = error_vs_dense(w, O[0, kept["head"]].float().cpu().numpy(), kept)
         line["cpu_baseline"] = {"value": 1.0 / t_cpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"head 0 clustered and routed in full, attention of 48 of {w.C} query "
@@ -446,6 +484,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--selection", choices=["topk", "adaptive"], default="topk",
+                    help="key-cluster selection (adaptive: mass recall, capacity C per query cluster)")
+    ap.add_argument("--recall", type=float, default=0.9)
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4], default=CONFIG_ID,
                     help="workload (default 2: the metric's N = 64k configuration)")
     args = ap.parse_args()
