@@ -391,6 +391,34 @@ def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int
                         min_margin_q=rq.min_margin, min_margin_k=rk.min_margin)
 
 
+def random_leaves(n: int, c: int, *, seed: int, bh: int, tensor: int) -> List[np.ndarray]:
+    """Random clusters, the baseline of the paper's error analysis (Section
+    4, "random clustering and top-k" against the recursive split): token i
+    draws the counter-based key splitmix64(node_key(seed, bh, tensor, 0) ^ i)
+    (heap index 0 belongs to no node of the split tree); the tokens ordered
+    by (key, index) are cut into consecutive groups of c, the remainder group
+    last, members ascending."""
+    base = node_key(seed, bh, tensor, 0)
+    keys = np.array([splitmix64(base ^ i) for i in range(n)], dtype=np.uint64)
+    order = np.lexsort((np.arange(n), keys))
+    return [np.sort(order[a:a + c]) for a in range(0, n, c)]
+
+
+def cluster_head_random(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int = 0) -> HeadClusters:
+    """Random clusters of the valid queries and keys of one head, with the
+    same outputs as cluster_head (permutation, counts, centroids)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    n = Q.shape[0]
+    lq = random_leaves(n, c, seed=seed, bh=bh, tensor=0)
+    lk = random_leaves(n, c, seed=seed, bh=bh, tensor=1)
+    perm_q, count_q = _leaves_to_perm(lq, c)
+    perm_k, count_k = _leaves_to_perm(lk, c)
+    return HeadClusters(perm_q=perm_q, perm_k=perm_k, count_q=count_q, count_k=count_k,
+                        qbar=_centroids(Q, lq), kbar=_centroids(K, lk),
+                        min_margin_q=float("inf"), min_margin_k=float("inf"))
+
+
 def cluster_workload(Q: np.ndarray, K: np.ndarray, n_valid: int, c: int, *, seed: int = 0,
                      power_iters: int = 8, heads: Optional[Sequence[int]] = None,
                      transform: bool = True) -> List[HeadClusters]:

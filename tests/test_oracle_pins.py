@@ -570,3 +570,49 @@ def test_adaptive_route_breaks_mass_ties_to_the_lower_index():
     assert [list(g) for g in got] == [[0, 1, 2], [0, 1, 2]]
     got = orc.adaptive_route(scores, count_k, 16, 0.5, min_count=1)
     assert list(got[0]) == [0, 1, 2, 3, 4]
+
+
+# ---------------------------------------------------------------------------
+# Random-cluster baseline (the paper's error analysis compares the recursive
+# split with random clusters)
+# ---------------------------------------------------------------------------
+
+def test_random_leaves_partition_and_sizes():
+    n, c = 1000, 64
+    leaves = orc.random_leaves(n, c, seed=3, bh=1, tensor=0)
+    sizes = [len(l) for l in leaves]
+    assert sizes == [c] * (n // c) + [n % c]        # remainder last, as in the split tree
+    allm = np.concatenate(leaves)
+    assert np.array_equal(np.sort(allm), np.arange(n))
+    assert all(np.all(np.diff(l) > 0) for l in leaves)
+
+
+def test_random_leaves_follow_the_splitmix_keys():
+    # brute force: the first group holds the c tokens with the smallest keys
+    n, c = 300, 32
+    base = orc.node_key(9, 0, 1, 0)
+    keys = [orc.splitmix64(base ^ i) for i in range(n)]
+    first = sorted(sorted(range(n), key=lambda i: (keys[i], i))[:c])
+    assert list(orc.random_leaves(n, c, seed=9, bh=0, tensor=1)[0]) == first
+
+
+def test_tight_clusters_beat_random_ones_when_attention_is_sparse_and_with_compensation():
+    # The paper's error analysis (Section 1.2 / 3): when the sparsity
+    # assumption holds (well-separated mixture components, values independent
+    # of keys), tight clusters that capture the attention mass give the
+    # smaller error; and with centroid compensation tighter clusters give the
+    # smaller error in any case. Random clusters are the paper's baseline.
+    import workloads as wl
+    w = wl.make_workload("mixture", H=1, N=1024, d=32, c=32, k=4, dtype="fp32", seed=40)
+    Qf, Kf, Vf = (x[0, 0].astype(np.float64) for x in (w.Q, w.K, w.V))
+    dense = orc.dense_attention(Qf, Kf, Vf)
+    err = {}
+    for name, h in (("split", orc.cluster_head(Qf, Kf, w.c, seed=0)),
+                    ("random", orc.cluster_head_random(Qf, Kf, w.c, seed=0))):
+        kept = orc.topk_route(orc.centroid_scores(h.qbar, h.kbar), w.k)
+        for comp in (False, True):
+            O = orc.compensated_attention(Qf, Kf, Vf, h.perm_q, h.count_q, h.perm_k, h.count_k, kept, w.c,
+                                          compensate=comp)
+            err[name, comp] = np.linalg.norm(O - dense) / np.linalg.norm(dense)
+    assert err["split", False] < err["random", False]
+    assert err["split", True] < err["random", True]
