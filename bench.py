@@ -164,7 +164,7 @@ def blas_threads():
         return 1
 
 
-def oracle_sample(w, n_clusters=48, heads=(0,), keep=None, selection="topk", recall=0.9):
+def oracle_sample(w, n_clusters=48, heads=(0,), keep=None, selection="topk", recall=0.9, clustering="split"):
     """Time the oracle on a bounded sample and extrapolate to one whole layer.
     Per sampled head: full clustering of queries and keys, routing, and the
     attention of `n_clusters` query clusters (work per query cluster is the
@@ -176,7 +176,10 @@ def oracle_sample(w, n_clusters=48, heads=(0,), keep=None, selection="topk", rec
     for h in heads:
         Qf, Kf, Vf = (x[0, h, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         t0 = time.perf_counter()
-        if selection == "adaptive":
+        if clustering == "random":
+            hc = orc.cluster_head_random(Qf, Kf, w.c, seed=0, bh=h)
+            kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
+        elif selection == "adaptive":
             hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, query_form="adaptive")
             kept = orc.adaptive_route(orc.centroid_scores(hc.qbar, hc.kbar), hc.count_k, w.d, recall, 16)
         else:
@@ -287,7 +290,8 @@ def run_ours(args):
         return max_over_ranks(x, world, "cuda")
 
     # Each rank: an independent layer (its own seeded inputs).
-    w = wl.config_workload(args.config, seed=rank_seed(rank, args.config))
+    w = wl.config_workload(args.config, seed=rank_seed(rank, args.config),
+                           **({"compensate": False} if args.smc == "off" else {}))
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(x):
@@ -298,7 +302,7 @@ def run_ours(args):
     adaptive = args.selection == "adaptive"
     layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.C if adaptive else w.k,
                                 dtype=w.dtype, compensate=w.compensate, selection=args.selection,
-                                recall=args.recall, min_count=16)
+                                recall=args.recall, min_count=16, clustering=args.clustering)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -440,7 +444,13 @@ def run_ours(args):
                 "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s", "frac": achieved / fp32_peak,
                 "traffic": None, "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
                 "algorithmic_flops": kept_f + smc_f}
-    launches = args.steps * sum(ca.launch_count(shape, s) for s in (0, 1, 2))
+    per_step = [ca.launch_count(shape, s) for s in (0, 1, 2)]
+    if args.clustering == "random" and per_step[0] > 1:
+        # no metric, norm or direction kernels: plan, per level hash / select /
+        # count / scatter, centroids
+        levels = (per_step[0] - 6) // 5
+        per_step[0] = 2 + 4 * levels
+    launches = args.steps * sum(per_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -448,7 +458,7 @@ def run_ours(args):
         "dtype_detail": ("clustering and routing f64; attention bf16 products with f32 accumulation"
                          if w.dtype == "bf16" else "clustering and routing f64; attention f32"),
         "data": "synthetic",
-        "config": dict(workload_config(w), selection=args.selection,
+        "config": dict(workload_config(w), selection=args.selection, clustering=args.clustering,
                        **({"recall": args.recall, "min_count": 16,
                            "mean_kept": float(kc.mean())} if adaptive else {})),
         "latency_ms": ms_per_step, "stage_ms": stage, "dense_ms": dense_ms,
@@ -464,7 +474,8 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         kept = {}
-        t_cpu, smp = oracle_sample(w, keep=kept, selection=args.selection, recall=args.recall)
+        t_cpu, smp = oracle_sample(w, keep=kept, selection=args.selection, recall=args.recall,
+                                   clustering=args.clustering)
         line["error_vs_dense_fp64"] = error_vs_dense(w, O[0, kept["head"]].float().cpu().numpy(), kept)
         line["cpu_baseline"] = {"value": 1.0 / t_cpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"head 0 clustered and routed in full, attention of 48 of {w.C} query "
@@ -487,6 +498,9 @@ def main():
     ap.add_argument("--selection", choices=["topk", "adaptive"], default="topk",
                     help="key-cluster selection (adaptive: mass recall, capacity C per query cluster)")
     ap.add_argument("--recall", type=float, default=0.9)
+    ap.add_argument("--clustering", choices=["split", "random"], default="split",
+                    help="random: the random-cluster baseline of the paper's error analysis")
+    ap.add_argument("--smc", choices=["on", "off"], default="on", help="striped mean-compensation")
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4], default=CONFIG_ID,
                     help="workload (default 2: the metric's N = 64k configuration)")
     args = ap.parse_args()

@@ -49,6 +49,7 @@ ca_status check_params(const ca_shape* s, const ca_cluster_params* p) {
   if (dir_smem(s->d, a) > 227 * 1024) return CA_ERR_UNSUPPORTED;
   if (p->transform != 0 && p->transform != 1) return CA_ERR_INVALID_ARG;
   if (p->query_form != 0 && p->query_form != 1) return CA_ERR_INVALID_ARG;
+  if (p->method != 0 && p->method != 1) return CA_ERR_INVALID_ARG;
   return CA_OK;
 }
 
@@ -146,7 +147,7 @@ ca_status ca_cluster(const void* Q, const void* K, const ca_shape* s, const ca_c
   cluster_ws_layout(s, plan, &L);
   if (workspace_bytes < L.total) return CA_ERR_WORKSPACE;
   if (!workspace) return CA_ERR_INVALID_ARG;
-  ca_cluster_params p = {8, 1, 1, 0, 0ull};
+  ca_cluster_params p = {8, 1, 1, 0, 0ull, 0, 0};
   if (params) p = *params;
   return cuda_status(launch_cluster(Q, K, s, &p, out, plan, L, static_cast<char*>(workspace),
                                     static_cast<cudaStream_t>(stream)));

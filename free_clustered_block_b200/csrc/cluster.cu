@@ -955,6 +955,20 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   }
 }
 
+// Random-cluster baseline: the key of every position is the counter-based
+// hash of its token, the same at every level, so the splits cut the fixed
+// random order of the tokens into groups of c (remainder last). Positions
+// outside this level's nodes get a key too; nothing reads it.
+__global__ void __launch_bounds__(256) hash_keys_kernel(int n, const int* __restrict__ idx, uint64_t seed,
+                                                        uint64_t* __restrict__ keys) {
+  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int pos = blockIdx.x * 256 + threadIdx.x;
+  if (pos >= n) return;
+  const int row = idx ? idx[(size_t)th * n + pos] : pos;
+  keys[(size_t)th * n + pos] =
+      splitmix64(node_stream(seed, (uint64_t)bh, (uint64_t)tensor, 0ull) ^ (uint64_t)(uint32_t)row);
+}
+
 // ---------------------------------------------------------------------------
 // K2b: the t-th smallest key of a node (MSD radix select, 8-bit digits).
 // Nodes of at most kSelCap keys are read into shared memory once; larger
@@ -1255,20 +1269,23 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
   // adaptive form (eq. 15) and the untransformed ablation use scale 1
   const int normalize = transform && p->query_form == 0;
 
+  const bool random_clusters = p->method == 1;
   if (plan.levels > 0) {
     plan_kernel<<<1, 1024, 0, st>>>(n, c, nodes, level_begin);
-    colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
-    const size_t syrk_smem = SyrkCfg<D>::template smem<T>();
-    cudaFuncSetAttribute(syrk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
-    syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
-                                                                                metpart);
-    metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
-    if (D == 64 && normalize) {
-      qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
-    } else {
-      const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
-      cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
-      qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, normalize, inv_s);
+    if (!random_clusters) {
+      colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
+      const size_t syrk_smem = SyrkCfg<D>::template smem<T>();
+      cudaFuncSetAttribute(syrk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
+      syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
+                                                                                  metpart);
+      metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
+      if (D == 64 && normalize) {
+        qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
+      } else {
+        const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
+        cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
+        qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, normalize, inv_s);
+      }
     }
     const int m_cap = sample_factor * D;
     const int dir_warps = DirCfg<T, D>::warps(m_cap);
@@ -1281,7 +1298,9 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       const int lb = plan.level_begin[l], le = plan.level_begin[l + 1], nl = le - lb;
       const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
       int* idx_out = idxbuf[(l + 1) & 1];
-      if (D == 128 && sample_factor == 1) {
+      if (random_clusters) {
+        hash_keys_kernel<<<dim3((n + 255) / 256, TH), 256, 0, st>>>(n, idx_in, p->seed, keys);
+      } else if (D == 128 && sample_factor == 1) {
         // about four blocks per SM over the whole level
         const int npc = (int)(((long long)nl * TH + 4 * 148 - 1) / (4 * 148));
         dirc_kernel<T><<<dim3((nl + npc - 1) / npc, TH), kDirCThreads, DirCCfg<T>::kSmem, st>>>(
@@ -1290,8 +1309,9 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
         dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(
             Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters, sample_factor);
       }
-      project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(Q, K, N_alloc, n, nodes, lb, le,
-                                                                      inv_s, idx_in, NI, wvec, keys);
+      if (!random_clusters)
+        project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(
+            Q, K, N_alloc, n, nodes, lb, le, inv_s, idx_in, NI, wvec, keys);
       if (plan.level_max_size[l] <= kSelCap)
         select_kernel<256><<<dim3(nl, TH), 256, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
       else

@@ -35,7 +35,8 @@ class ClusterAttention:
     def __init__(self, B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, k: int,
                  dtype: str = "bf16", compensate: bool = True, power_iters: int = 8,
                  sample_factor: int = 1, transform: bool = True, seed: int = 0, device="cuda",
-                 selection: str = "topk", recall: float = 0.9, min_count: int = 16):
+                 selection: str = "topk", recall: float = 0.9, min_count: int = 16,
+                 clustering: str = "split"):
         import torch
         self.torch = torch
         self.dtype_code = CA_BF16 if dtype == "bf16" else CA_FP32
@@ -44,7 +45,8 @@ class ClusterAttention:
         self.selection = selection
         self.recall, self.min_count = recall, min_count
         self.params = make_params(power_iters, sample_factor, int(transform), seed,
-                                  query_form=1 if selection == "adaptive" else 0)
+                                  query_form=1 if selection == "adaptive" else 0,
+                                  method=1 if clustering == "random" else 0)
         self.k = k
         self.compensate = compensate
         C = num_clusters(self.shape)

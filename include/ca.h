@@ -66,13 +66,21 @@ typedef struct {
  *  query_form    0 = queries as R_k q / |R_k q| (eq. 16, for top-k selection),
  *                    the default; 1 = queries as R_k q (eq. 15, for adaptive
  *                    selection); ignored when transform is 0;
- *  seed          counter-based generator seed for samples and warm starts. */
+ *  seed          counter-based generator seed for samples and warm starts;
+ *  method        0 = recursive splitting (the method), the default;
+ *                1 = random clusters, the baseline of the paper's error
+ *                    analysis: token i of (b, h, tensor) gets the key
+ *                    SplitMix64(stream(seed, bh, tensor, 0) ^ i), and the
+ *                    tokens ordered by (key, i) form the clusters, c at a
+ *                    time, the remainder last (the other knobs are ignored). */
 typedef struct {
   int power_iters;
   int sample_factor;
   int transform;
   int query_form;
   uint64_t seed;
+  int method;
+  int reserved;   /* 0 */
 } ca_cluster_params;
 
 /* Clustering result, one entry per (b, h), C = ca_num_clusters(shape):

@@ -36,7 +36,7 @@ class Run:
     """Device buffers for one workload and the C-ABI calls on them."""
 
     def __init__(self, w, k=None, compensate=None, seed=0, power_iters=8, transform=True, selection="topk",
-                 recall=0.9, min_count=16):
+                 recall=0.9, min_count=16, clustering="split"):
         t = torch()
         self.w = w
         self.k = w.k if k is None else k
@@ -48,7 +48,7 @@ class Run:
         self.layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, self.k, dtype=w.dtype,
                                          compensate=self.compensate, power_iters=power_iters,
                                          transform=transform, seed=seed, selection=selection, recall=recall,
-                                         min_count=min_count)
+                                         min_count=min_count, clustering=clustering)
         self.C = self.layer.C
 
     def cluster(self):
