@@ -290,8 +290,17 @@ def run_ours(args):
         return max_over_ranks(x, world, "cuda")
 
     # Each rank: an independent layer (its own seeded inputs).
-    w = wl.config_workload(args.config, seed=rank_seed(rank, args.config),
-                           **({"compensate": False} if args.smc == "off" else {}))
+    if args.tokens:
+        # latency scaling: configuration 2's generator (H = 8, d = 64, c = 128)
+        # at another token count, keeping 1/8 of the clusters or a fixed 64
+        C = -(-args.tokens // 128)
+        kk = 64 if args.fixed_k else max(1, C // 8)
+        w = wl.make_workload("lowrank", B=1, H=8, N=args.tokens, d=64, c=128, k=min(kk, C), dtype="bf16",
+                             seed=rank_seed(rank, 2), compensate=args.smc == "on",
+                             name=f"cfg2gen-lowrank-N{args.tokens}-d64-bf16-k{min(kk, C)}", rank=16, noise=0.1)
+    else:
+        w = wl.config_workload(args.config, seed=rank_seed(rank, args.config),
+                               **({"compensate": False} if args.smc == "off" else {}))
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(x):
@@ -501,6 +510,9 @@ def main():
     ap.add_argument("--clustering", choices=["split", "random"], default="split",
                     help="random: the random-cluster baseline of the paper's error analysis")
     ap.add_argument("--smc", choices=["on", "off"], default="on", help="striped mean-compensation")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="latency scaling: configuration 2's generator at this token count")
+    ap.add_argument("--fixed-k", action="store_true", help="with --tokens: keep 64 clusters instead of 1/8")
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4], default=CONFIG_ID,
                     help="workload (default 2: the metric's N = 64k configuration)")
     args = ap.parse_args()
