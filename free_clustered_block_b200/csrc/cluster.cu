@@ -624,55 +624,58 @@ __global__ void __launch_bounds__(512) dir_kernel(
   }
 }
 
-// d = 128 (a 128-row sample at most): M alone is 128 KB, so one warp per node
-// would leave two nodes per SM. Here a 256-thread block owns one node at a
-// time and walks `npc` consecutive nodes of one tensor-head, staging M once.
-// Each of the three products of a power step is split over the 256 threads
-// as pairs of half sums (rows or columns 0-63 / 64-127), added in a fixed
-// order, so the result does not depend on scheduling.
-constexpr int kDirCThreads = 256;
-
-template <typename T>
+// One block of 2 d threads per node (a sample of at most d rows), walking
+// `npc` consecutive nodes of one tensor-head with M staged once. Used for
+// d = 128, where M alone is 128 KB and one warp per node would leave two
+// nodes per SM, and for d = 64 on the levels with few nodes, where one warp
+// per node is latency-bound. Each of the three products of a power step is
+// split over the threads as pairs of half sums (rows or columns 0..d/2-1 and
+// d/2..d-1), added in a fixed order, so the result does not depend on
+// scheduling.
+template <typename T, int D_>
 struct DirCCfg {
-  static constexpr int D = 128;
+  static constexpr int D = D_;
+  static constexpr int kThreads = 2 * D;
   static constexpr int kRowStride = D + ((sizeof(T) == 2) ? 2 : 1);   // odd number of 32-bit words
   static constexpr size_t kXBytes = (size_t)D * kRowStride * sizeof(T);
   static constexpr size_t kSmem = (size_t)D * D * 8 + kXBytes;
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
+template <typename T, int D_>
+__global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, int npc, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
     int power_iters) {
-  using Cfg = DirCCfg<T>;
-  constexpr int D = 128, RS = Cfg::kRowStride;
+  using Cfg = DirCCfg<T, D_>;
+  constexpr int D = D_, RS = Cfg::kRowStride;
+  constexpr int NT = Cfg::kThreads, HD = D / 2;   // threads, half length
+  constexpr int NWD = D / 32;                     // warps holding one value per column
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* Ms = reinterpret_cast<double*>(smem_raw);             // D x D
   T* Xs = reinterpret_cast<T*>(smem_raw + (size_t)D * D * 8);   // D rows x RS
   __shared__ double red[2][D];
   __shared__ double zs[D], ws[D], xbar[D], fj[D], vs[D];
-  __shared__ double qred[4][2];
-  __shared__ double vred[8];
+  __shared__ double qred[NWD][2];
+  __shared__ double vred[2 * NWD];
   __shared__ int srow[D];
   const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int ca = t & 127, ch = t >> 7;          // column / half split
+  const int ca = t & (D - 1), ch = t / D;       // column / half split
   const int rj = t >> 1, rh = t & 1;            // row / half split
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
   {
     const double2* src = reinterpret_cast<const double2*>(M + (size_t)th * D * D);
     double2* dst = reinterpret_cast<double2*>(Ms);
 #pragma unroll 4
-    for (int e = t; e < D * D / 2; e += kDirCThreads) dst[e] = src[e];
+    for (int e = t; e < D * D / 2; e += NT) dst[e] = src[e];
   }
   // w = M z (z in zs) into ws; returns (z . w, xbar . w) to every thread
   auto matvec = [&](double& zw, double& xw) {
     double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-    const int b0 = ch * 64;
+    const int b0 = ch * HD;
 #pragma unroll 4
-    for (int b = 0; b < 64; b += 4) {
+    for (int b = 0; b < HD; b += 4) {
       a0 = fma(Ms[(b0 + b) * D + ca], zs[b0 + b], a0);
       a1 = fma(Ms[(b0 + b + 1) * D + ca], zs[b0 + b + 1], a1);
       a2 = fma(Ms[(b0 + b + 2) * D + ca], zs[b0 + b + 2], a2);
@@ -692,8 +695,9 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
       if (lane == 0) { qred[warp][0] = pz; qred[warp][1] = px; }
     }
     __syncthreads();
-    zw = (qred[0][0] + qred[1][0]) + (qred[2][0] + qred[3][0]);
-    xw = (qred[0][1] + qred[1][1]) + (qred[2][1] + qred[3][1]);
+    zw = 0.0; xw = 0.0;
+#pragma unroll
+    for (int q = 0; q < NWD; ++q) { zw += qred[q][0]; xw += qred[q][1]; }
   };
   const int first = blockIdx.x * npc, last = min(nodes_in_level, first + npc);
   for (int local = first; local < last; ++local) {
@@ -721,11 +725,11 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
       constexpr int WPR = RS * (int)sizeof(T) / 4;              // row stride in 32-bit words
       uint32_t* xw32 = reinterpret_cast<uint32_t*>(Xs);
 #pragma unroll
-      for (int u0 = 0; u0 < D * CPR; u0 += 8 * kDirCThreads) {
+      for (int u0 = 0; u0 < D * CPR; u0 += 8 * NT) {
         uint4 v4[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int e = u0 + u * kDirCThreads + t;
+          const int e = u0 + u * NT + t;
           const int j = e / CPR, part = e % CPR;
           v4[u] = make_uint4(0, 0, 0, 0);
           if (e < D * CPR && j < m)
@@ -733,7 +737,7 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int e = u0 + u * kDirCThreads + t;
+          const int e = u0 + u * NT + t;
           const int j = e / CPR, part = e % CPR;
           if (e < D * CPR) {
             uint32_t* dst = xw32 + (size_t)j * WPR + part * 4;
@@ -746,9 +750,9 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
     // sample mean
     {
       double a0 = 0.0, a1 = 0.0;
-      const int j0 = ch * 64;
+      const int j0 = ch * HD;
 #pragma unroll 4
-      for (int j = 0; j < 64; j += 2) {
+      for (int j = 0; j < HD; j += 2) {
         a0 = fma(vs[j0 + j], (double)to_f(Xs[(j0 + j) * RS + ca]), a0);
         a1 = fma(vs[j0 + j + 1], (double)to_f(Xs[(j0 + j + 1) * RS + ca]), a1);
       }
@@ -782,10 +786,10 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
       double v = 0.0;
       {
         double d0 = 0.0, d1 = 0.0, d2 = 0.0, d3 = 0.0;
-        const T* xr = Xs + rj * RS + rh * 64;
-        const double* wr = ws + rh * 64;
+        const T* xr = Xs + rj * RS + rh * HD;
+        const double* wr = ws + rh * HD;
 #pragma unroll 4
-        for (int c = 0; c < 64; c += 4) {
+        for (int c = 0; c < HD; c += 4) {
           d0 = fma((double)to_f(xr[c]), wr[c], d0);
           d1 = fma((double)to_f(xr[c + 1]), wr[c + 1], d1);
           d2 = fma((double)to_f(xr[c + 2]), wr[c + 2], d2);
@@ -801,13 +805,15 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
       for (int o = 16; o > 0; o >>= 1) vsum += __shfl_xor_sync(0xffffffffu, vsum, o);
       if (lane == 0) vred[warp] = vsum;
       __syncthreads();
-      vsum = ((vred[0] + vred[1]) + (vred[2] + vred[3])) + ((vred[4] + vred[5]) + (vred[6] + vred[7]));
+      vsum = 0.0;
+#pragma unroll
+      for (int q = 0; q < 2 * NWD; ++q) vsum += vred[q];
       // z'_a = (sum_j v_j scale_j X_ja - xbar_a sum_j v_j) / m: two threads per column
       {
         double a0 = 0.0, a1 = 0.0;
-        const int j0 = ch * 64;
+        const int j0 = ch * HD;
 #pragma unroll 4
-        for (int j = 0; j < 64; j += 2) {
+        for (int j = 0; j < HD; j += 2) {
           a0 = fma(fj[j0 + j], (double)to_f(Xs[(j0 + j) * RS + ca]), a0);
           a1 = fma(fj[j0 + j + 1], (double)to_f(Xs[(j0 + j + 1) * RS + ca]), a1);
         }
@@ -836,6 +842,10 @@ __global__ void __launch_bounds__(kDirCThreads, 1) dirc_kernel(
 // one row (16 bytes per lane, coalesced); each group keeps kProjU rows in
 // flight.
 // ---------------------------------------------------------------------------
+// d = 64 levels with at most this many nodes (over all tensor-heads) use the
+// block-per-node power iteration
+constexpr long long kDirCMaxNodes64 = 148 * 4;
+
 constexpr int kProjSpan = 1024;
 constexpr int kProjNodes = 20;   // > kProjSpan / 65 + 2
 constexpr int kProjU = 4;
@@ -1291,7 +1301,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     const int dir_warps = DirCfg<T, D>::warps(m_cap);
     const size_t dir_smem = (size_t)D * D * 8 + (size_t)dir_warps * DirCfg<T, D>::warp_bytes(m_cap);
     cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
-    if (D == 128) cudaFuncSetAttribute(dirc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DirCCfg<T>::kSmem);
+    cudaFuncSetAttribute(dirc_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DirCCfg<T, D>::kSmem);
     cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
     cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
     for (int l = 0; l < plan.levels; ++l) {
@@ -1300,10 +1310,11 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       int* idx_out = idxbuf[(l + 1) & 1];
       if (random_clusters) {
         hash_keys_kernel<<<dim3((n + 255) / 256, TH), 256, 0, st>>>(n, idx_in, p->seed, keys);
-      } else if (D == 128 && sample_factor == 1) {
-        // about four blocks per SM over the whole level
+      } else if (sample_factor == 1 && (D == 128 || (long long)nl * TH <= kDirCMaxNodes64)) {
+        // a block per node: d = 128, or d = 64 levels with few nodes (about
+        // four blocks per SM over the whole level)
         const int npc = (int)(((long long)nl * TH + 4 * 148 - 1) / (4 * 148));
-        dirc_kernel<T><<<dim3((nl + npc - 1) / npc, TH), kDirCThreads, DirCCfg<T>::kSmem, st>>>(
+        dirc_kernel<T, D><<<dim3((nl + npc - 1) / npc, TH), DirCCfg<T, D>::kThreads, DirCCfg<T, D>::kSmem, st>>>(
             Q, K, N_alloc, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters);
       } else {
         dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(

@@ -26,7 +26,8 @@ namespace {
 
 constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr size_t kRouteSmemBudget = 120 * 1024;
+// one block per SM either way (its registers), so the score rows may use most of shared memory
+constexpr size_t kRouteSmemBudget = 200 * 1024;
 
 template <int D, int QA>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* __restrict__ qbar,
