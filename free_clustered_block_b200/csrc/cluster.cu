@@ -1015,20 +1015,33 @@ __global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__
     for (int i = threadIdx.x; i < 256; i += NT) hist[i] = 0;
     __syncthreads();
     const int cnt_total = global_mode ? size : ncand;
-    for (int i0 = 0; i0 < cnt_total; i0 += NT) {
-      const int i = i0 + threadIdx.x;
-      bool ok = false;
-      unsigned dg = 0;
-      if (i < cnt_total) {
-        const uint64_t k = global_mode ? base[i] : cand[i];
-        ok = (k & mask) == prefix;
-        dg = (unsigned)((k >> shift) & 0xFF);
-      }
-      // warp-aggregated histogram increment
+    // warp-aggregated histogram increment of one key
+    auto count = [&](bool ok, uint64_t k) {
+      const unsigned dg = (unsigned)((k >> shift) & 0xFF);
       const unsigned act = __ballot_sync(0xffffffffu, ok);
       if (ok) {
         const unsigned peers = __match_any_sync(act, dg);
         if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[dg], (unsigned)__popc(peers));
+      }
+    };
+    if (global_mode) {
+      // four keys per thread per step, their loads in flight together
+      for (int i0 = 0; i0 < cnt_total; i0 += NT * 4) {
+        uint64_t kk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * NT + threadIdx.x;
+          kk[u] = i < cnt_total ? base[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          count(i0 + u * NT + (int)threadIdx.x < cnt_total && (kk[u] & mask) == prefix, kk[u]);
+      }
+    } else {
+      for (int i0 = 0; i0 < cnt_total; i0 += NT) {
+        const int i = i0 + threadIdx.x;
+        const uint64_t k = i < cnt_total ? cand[i] : 0ull;
+        count(i < cnt_total && (k & mask) == prefix, k);
       }
     }
     __syncthreads();
@@ -1065,9 +1078,16 @@ __global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__
       if (threadIdx.x == 0) s_ncand = 0;
       __syncthreads();
       if (global_mode) {
-        for (int i = threadIdx.x; i < size; i += NT) {
-          const uint64_t k = base[i];
-          if ((k & mask) == prefix) cand[atomicAdd(&s_ncand, 1)] = k;
+        for (int i0 = 0; i0 < size; i0 += NT * 4) {
+          uint64_t kk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * NT + threadIdx.x;
+            kk[u] = i < size ? base[i] : ~prefix;   // ~prefix never matches (the mask is not empty)
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if ((kk[u] & mask) == prefix) cand[atomicAdd(&s_ncand, 1)] = kk[u];
         }
       } else {
         // in place: read all candidates first, then write the survivors
@@ -1323,8 +1343,9 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       if (!random_clusters)
         project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(
             Q, K, N_alloc, n, nodes, lb, le, inv_s, idx_in, NI, wvec, keys);
-      if (plan.level_max_size[l] <= kSelCap)
-        select_kernel<256><<<dim3(nl, TH), 256, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
+      if (plan.level_max_size[l] <= kSelCap)   // candidates buffer sized to the level's largest node
+        select_kernel<256><<<dim3(nl, TH), 256, (size_t)plan.level_max_size[l] * 8, st>>>(nodes, lb, nl, n, keys,
+                                                                                        sel);
       else
         select_kernel<1024><<<dim3(nl, TH), 1024, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
       const int pch = (plan.level_max_size[l] + kPartChunk - 1) / kPartChunk;
