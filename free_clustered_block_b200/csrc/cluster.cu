@@ -269,25 +269,33 @@ __global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* _
 }
 
 // M[th] for tensor-head th = 2 bh + tensor: queries (tensor 0) are split in
-// the key metric M_k, keys (tensor 1) in the query metric M_q.
+// the key metric M_k, keys (tensor 1) in the query metric M_q. One thread
+// per matrix element (grid.x covers D*D / 256), the chunk partials summed in
+// chunk order with four loads in flight.
 template <int D>
 __global__ void __launch_bounds__(256) metric_reduce_kernel(const double* __restrict__ part, int nch,
                                                             int n, int transform,
                                                             double* __restrict__ M) {
-  const int th = blockIdx.x, bh = th >> 1, tensor = th & 1;
+  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const int src = 1 - tensor;  // z index: 0 = Q^T Q, 1 = K_c^T K_c
   const double* p = part + ((size_t)bh * 2 + src) * nch * D * D;
-  for (int e = threadIdx.x; e < D * D; e += 256) {
-    double v;
-    if (transform) {
-      v = 0.0;
-      for (int ch = 0; ch < nch; ++ch) v += p[(size_t)ch * D * D + e];
-      v /= (double)n;
-    } else {
-      v = (e / D == e % D) ? 1.0 : 0.0;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e >= D * D) return;
+  double v;
+  if (transform) {
+    v = 0.0;
+    int ch = 0;
+    for (; ch + 4 <= nch; ch += 4) {
+      const double a0 = p[(size_t)ch * D * D + e], a1 = p[(size_t)(ch + 1) * D * D + e];
+      const double a2 = p[(size_t)(ch + 2) * D * D + e], a3 = p[(size_t)(ch + 3) * D * D + e];
+      v += a0; v += a1; v += a2; v += a3;
     }
-    M[(size_t)th * D * D + e] = v;
+    for (; ch < nch; ++ch) v += p[(size_t)ch * D * D + e];
+    v /= (double)n;
+  } else {
+    v = (e / D == e % D) ? 1.0 : 0.0;
   }
+  M[(size_t)th * D * D + e] = v;
 }
 
 // ---------------------------------------------------------------------------
@@ -1308,7 +1316,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       cudaFuncSetAttribute(syrk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
       syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
                                                                                   metpart);
-      metric_reduce_kernel<D><<<TH, 256, 0, st>>>(metpart, nch, n, transform, M);
+      metric_reduce_kernel<D><<<dim3(D * D / 256, TH), 256, 0, st>>>(metpart, nch, n, transform, M);
       if (D == 64 && normalize) {
         qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
       } else {
