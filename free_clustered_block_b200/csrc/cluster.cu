@@ -872,6 +872,7 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   __shared__ double ws[kProjNodes][D];
   __shared__ int n_off[kProjNodes], n_end[kProjNodes], n_id[kProjNodes];
   __shared__ unsigned char slot_of[kProjSpan];
+  __shared__ int rows_s[kProjSpan];      // source row of each position
   __shared__ int s_cnt;
   const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
@@ -910,12 +911,24 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   }
   __syncthreads();
   const int cnt = s_cnt;
-  for (int p = threadIdx.x; p < kProjSpan; p += 256) {
-    const int pos = base + p;
-    unsigned char sl = 255;
-    for (int q = 0; q < cnt; ++q)
-      if (pos >= n_off[q] && pos < n_end[q]) sl = (unsigned char)q;
-    slot_of[p] = sl;
+  // node slot of each position of the span and, for the positions inside a
+  // node of this level (only those: elsewhere the index buffer holds nothing
+  // meaningful), the source row, all of a thread's index loads in flight
+  {
+    unsigned char sl[kProjSpan / 256];
+    int rv[kProjSpan / 256];
+#pragma unroll
+    for (int u = 0; u < kProjSpan / 256; ++u) {
+      const int pos = base + u * 256 + threadIdx.x;
+      sl[u] = 255;
+      for (int q = 0; q < cnt; ++q)
+        if (pos >= n_off[q] && pos < n_end[q]) sl[u] = (unsigned char)q;
+      slot_of[u * 256 + threadIdx.x] = sl[u];
+      rv[u] = 0;
+      if (sl[u] != 255) rv[u] = idx ? idx[(size_t)th * n + pos] : pos;
+    }
+#pragma unroll
+    for (int u = 0; u < kProjSpan / 256; ++u) rows_s[u * 256 + threadIdx.x] = rv[u];
   }
   for (int e = threadIdx.x; e < cnt * D; e += 256)
     ws[e / D][e % D] = wvec[((size_t)th * NI + n_id[e / D]) * D + (e % D)];
@@ -937,7 +950,7 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
       const int pos = base + rr;
       slot[u] = (rr < kProjSpan && pos < n) ? slot_of[rr] : 255;
       row[u] = 0;
-      if (slot[u] != 255) row[u] = idx ? idx[(size_t)th * n + pos] : pos;
+      if (slot[u] != 255) row[u] = rows_s[rr];
     }
 #pragma unroll
     for (int u = 0; u < kProjU; ++u) {
