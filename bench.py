@@ -40,7 +40,7 @@ CONFIG_ID = 2
 # profiles/tc_attend_kernel_64_128_layer_B1_H8_N65536.md. It describes the
 # kernel source whose SHA-256 starts with `source_sha256`; for any other source
 # the bench reports null.
-ATTN_TRAFFIC = {"bytes": 205589760 + 51571200, "source_sha256": "1a4712bdd0a67bd9"}
+ATTN_TRAFFIC = {"bytes": 205780992 + 52542720, "source_sha256": "7644549fa28628af"}
 
 
 def attention_traffic():

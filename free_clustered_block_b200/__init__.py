@@ -26,7 +26,7 @@ EXPORTED = [
     "ca_num_clusters", "ca_check_shape", "ca_cluster_workspace_bytes", "ca_attend_workspace_bytes",
     "ca_dense_workspace_bytes", "ca_forward_workspace_bytes", "ca_cluster", "ca_route", "ca_attend",
     "ca_dense_attend", "ca_forward", "ca_forward_host_workspace_bytes", "ca_forward_host",
-    "ca_get_device_error", "ca_set_wait_limit", "ca_status_string", "ca_version", "ca_launch_count",
+    "ca_get_device_error", "ca_set_wait_limit", "ca_check_bounded_wait", "ca_status_string", "ca_version", "ca_launch_count",
     "ca_cluster_noalloc", "ca_route_adaptive",
 ]
 
@@ -91,6 +91,7 @@ def lib():
             "ca_forward_host": (i32, [vp, vp, vp, P(ca_shape), P(ca_cluster_params), i32, i32, vp, vp, sz, vp]),
             "ca_get_device_error": (i32, [vp]),
             "ca_set_wait_limit": (None, [u64]),
+            "ca_check_bounded_wait": (i32, [u64, i32, vp]),
             "ca_status_string": (ctypes.c_char_p, [i32]),
             "ca_version": (ctypes.c_char_p, []),
             "ca_launch_count": (i32, [P(ca_shape), i32]),
@@ -241,8 +242,12 @@ def ca_get_device_error(stream=None) -> int:
     return lib().ca_get_device_error(_stream(stream))
 
 
-def ca_set_wait_limit(spins: int):
-    lib().ca_set_wait_limit(spins)
+def ca_set_wait_limit(limit_ns: int):
+    lib().ca_set_wait_limit(limit_ns)
+
+
+def ca_check_bounded_wait(limit_ns: int, arrive: bool, stream=None) -> int:
+    return lib().ca_check_bounded_wait(limit_ns, 1 if arrive else 0, _stream(stream))
 
 
 def launch_count(shape: ca_shape, stage: int) -> int:

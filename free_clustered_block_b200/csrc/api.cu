@@ -309,6 +309,11 @@ ca_status ca_get_device_error(void* stream) {
 
 void ca_set_wait_limit(uint64_t spins) { set_wait_limit(spins); }
 
+ca_status ca_check_bounded_wait(uint64_t limit_ns, int arrive, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return CA_ERR_INVALID_ARG;
+  return cuda_status(launch_bounded_wait_check(limit_ns, arrive ? 1 : 0, static_cast<cudaStream_t>(stream)));
+}
+
 int ca_launch_count(const ca_shape* s, int stage) {
   if (check_shape(s) != CA_OK) return -1;
   const int pad = s->N_alloc > s->n_valid ? 1 : 0;

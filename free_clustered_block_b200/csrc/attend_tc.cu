@@ -830,6 +830,30 @@ cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_
   return dispatch(D, KB, maps, p, grid, st);
 }
 
+// One CTA waits, through the same bounded wait as the attention kernel, on an
+// mbarrier that completes only if `arrive` is set: with arrive = 0 nothing
+// ever flips it, the wait runs out after limit_ns and raises CA_ERR_TIMEOUT in
+// the device error word. Touches no global data besides that word.
+__global__ void bounded_wait_check_kernel(uint64_t limit_ns, int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (arrive) mbar_arrive(&bar);
+    wait_bar(&bar, 0, limit_ns, &abort_flag);
+  }
+}
+
+cudaError_t launch_bounded_wait_check(uint64_t limit_ns, int arrive, cudaStream_t st) {
+  bounded_wait_check_kernel<<<1, 32, 0, st>>>(limit_ns, arrive);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const ca_shape* s, void* O,
                             cudaStream_t st) {
   const int BH = s->B * s->H, D = s->d;

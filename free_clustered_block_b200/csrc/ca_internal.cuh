@@ -133,6 +133,7 @@ bool attend_ws_layout(const ca_shape* s, AttendWs* ws);
 // The error word lives in attend_tc.cu; other units reach it through these.
 uint64_t wait_limit();                            // iteration cap of bounded waits
 cudaError_t device_error_read_clear(unsigned* out, cudaStream_t st);
+cudaError_t launch_bounded_wait_check(uint64_t limit_ns, int arrive, cudaStream_t st);
 void set_wait_limit(uint64_t spins);
 
 // ---------------------------------------------------------------------------

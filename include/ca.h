@@ -267,6 +267,16 @@ ca_status ca_get_device_error(void* stream);
  * default of 1 s. Host only; affects later launches. */
 void ca_set_wait_limit(uint64_t limit_ns);
 
+/* Failure-detection check: launch one CTA on `stream` that waits, through the
+ * same bounded mbarrier wait as the attention kernel, on a barrier that
+ * completes only when `arrive` is non-zero. With arrive = 0 nothing completes
+ * it: the wait gives up after limit_ns nanoseconds and sets CA_ERR_TIMEOUT in
+ * the device error word (read it with ca_get_device_error); with arrive != 0
+ * the word stays CA_OK. Reads and writes no caller memory. Returns
+ * CA_ERR_INVALID_ARG for limit_ns = 0 or above 10 s, CA_ERR_CUDA if the launch
+ * fails. */
+ca_status ca_check_bounded_wait(uint64_t limit_ns, int arrive, void* stream);
+
 /* Number of kernel launches one call makes for this shape (host only):
  * stage 0 = ca_cluster, 1 = ca_route, 2 = ca_attend, 3 = ca_dense_attend;
  * -1 for an invalid shape or stage. */
