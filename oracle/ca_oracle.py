@@ -20,6 +20,10 @@ What is computed, per head (Section 3.1 "Overview"; later revision Section 4):
     the first principal component warm-started from the parent's estimate and
     a random normal vector, project, put the multiple of c closest to |S|/2
     below the split; repeat until all sets but at most one hold c vectors;
+    or diagonalized recursive splitting (Section 3.2.1 "Diagonalized
+    recursive splitting"): rotate once into the principal-component basis of
+    the full set, then split every set on the coordinate of highest variance
+    in its sample;
  5. centroid scores q_bar . k_bar (eq. 18) and top-k selection per query
     cluster (Section 3.3.2 "Selection");
  6. block-sparse attention over the kept clusters with striped
@@ -39,7 +43,12 @@ Readings where the paper leaves a step open (each is listed in the design doc):
  * selection: exact top-k (ties to the lower key-cluster index), not the
    paper's approximate histogram; adaptive selection as the exact greedy
    prefix by estimated mass |b| e^{s_ab / sqrt(d)} (see adaptive_route);
- * compensation weight |c| is the number of real members of the cluster.
+ * compensation weight |c| is the number of real members of the cluster;
+ * diagonalized splitting: the basis diagonalises the (centred) covariance
+   of the representations over all valid rows; basis vectors are ordered by
+   descending eigenvalue and signed so that their largest-magnitude entry is
+   positive; the per-set sample is the basic splitting's, and the highest
+   sample variance picks the coordinate (lowest index on a tie).
 
 Random numbers: SplitMix64 (Steele, Lea & Flood, "Fast splittable
 pseudorandom number generators", OOPSLA 2014) on a per-node counter, turned
@@ -59,6 +68,7 @@ __all__ = [
     "metric_matrices", "psd_root", "key_representation", "query_representation",
     "split_count", "plan_tree", "num_clusters",
     "PddpResult", "pddp_partition", "pddp_partition_metric_form",
+    "pca_basis", "diagonal_partition",
     "HeadClusters", "cluster_head", "cluster_workload",
     "centroid_scores", "topk_route", "route_bits",
     "compensated_attention", "dense_attention",
@@ -326,6 +336,79 @@ def pddp_partition_metric_form(X: np.ndarray, M: np.ndarray, c: int, *, seed: in
 
 
 # ---------------------------------------------------------------------------
+# Diagonalized recursive splitting.
+# ---------------------------------------------------------------------------
+
+def pca_basis(Y: np.ndarray) -> tuple:
+    """Principal-component basis of the representations Y (rows, the full
+    set) from the eigendecomposition of their covariance (Section 3.2.1
+    "Diagonalized recursive splitting"; later revision Section 4.1.1).
+
+    Returns (U, lam): the columns of U are unit eigenvectors ordered by
+    descending eigenvalue lam (ties keep the solver's order); each column's
+    entry of largest magnitude (the first such entry on an exact tie) is made
+    positive, which fixes which side of a split is "below".
+    """
+    Y = np.asarray(Y, dtype=np.float64)
+    n = Y.shape[0]
+    Yc = Y - Y.mean(axis=0)
+    cov = Yc.T @ Yc / n
+    lam, U = np.linalg.eigh(cov)
+    order = np.argsort(-lam, kind="stable")
+    lam, U = lam[order], U[:, order].copy()
+    for j in range(U.shape[1]):
+        i = int(np.argmax(np.abs(U[:, j])))
+        if U[i, j] < 0:
+            U[:, j] = -U[:, j]
+    return U, lam
+
+
+def diagonal_partition(Y: np.ndarray, c: int, *, seed: int, bh: int, tensor: int,
+                       sample_factor: int = 1, record: bool = False) -> PddpResult:
+    """Diagonalized recursive splitting of the rows of Y (already transformed).
+
+    The rows are rotated once into the principal-component basis of the full
+    set, Z = Y U (pca_basis). At every set S: take the same sample of
+    min(a d, |S|) members as the basic splitting (a = sample_factor), find
+    the coordinate whose variance over the sample is highest (the lowest
+    coordinate index on an exact tie) and split S on that coordinate with the
+    multiple of c closest to |S|/2 below, equal values ordered by token
+    index; recurse until sets hold at most c vectors.
+    """
+    Y = np.asarray(Y, dtype=np.float64)
+    n, d = Y.shape
+    U, _ = pca_basis(Y)
+    Z = Y @ U
+    res = PddpResult(leaves=[])
+    m_cap = sample_factor * d
+
+    def rec(members: np.ndarray, heap: int):
+        size = members.shape[0]
+        if size <= c:
+            res.leaves.append(members)
+            return
+        key = node_key(seed, bh, tensor, heap)
+        m = min(m_cap, size)
+        Zs = Z[members[_sample_positions(size, m, key)]]
+        var = ((Zs - Zs.mean(axis=0)) ** 2).mean(axis=0)
+        j = int(np.argmax(var))                   # first maximum on ties
+        proj = Z[members, j] + 0.0
+        t = split_count(size, c)
+        order = np.lexsort((members, proj))
+        srt = proj[order]
+        spread = float(srt[-1] - srt[0])
+        margin = float(srt[t] - srt[t - 1]) / spread if spread > 0 else 0.0
+        res.min_margin = min(res.min_margin, margin)
+        if record:
+            res.splits.append((heap, size, t, float(srt[t - 1]), float(srt[t]), j))
+        rec(np.sort(members[order[:t]]), 2 * heap)
+        rec(np.sort(members[order[t:]]), 2 * heap + 1)
+
+    rec(np.arange(n), 1)
+    return res
+
+
+# ---------------------------------------------------------------------------
 # Clustering of one head: transforms + PDDP + centroids.
 # ---------------------------------------------------------------------------
 
@@ -359,13 +442,16 @@ def _centroids(X: np.ndarray, leaves: Sequence[np.ndarray]) -> np.ndarray:
 
 def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int = 0,
                  power_iters: int = 8, sample_factor: int = 1,
-                 transform: bool = True, query_form: str = "topk") -> HeadClusters:
+                 transform: bool = True, query_form: str = "topk",
+                 splitting: str = "basic") -> HeadClusters:
     """Cluster the valid queries and keys of one head (rows [n, d]).
 
     Keys are split in the query-aware space R_q k; queries in the key-aware,
     normalised space R_k q / |R_k q| (top-k form, eq. 16) or, with
     ``query_form="adaptive"``, in R_k q (eq. 15). ``transform=False`` splits
     the raw vectors (R = I, no normalisation), the paper's ablation.
+    ``splitting`` is "basic" (power iteration per set) or "diagonal"
+    (one principal-component rotation, coordinate splits).
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -380,10 +466,14 @@ def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int
     else:
         R_q = R_k = np.eye(d)
         Yk, Yq = K, Q
-    rq = pddp_partition(Yq, R_k, c, seed=seed, bh=bh, tensor=0,
-                        power_iters=power_iters, sample_factor=sample_factor)
-    rk = pddp_partition(Yk, R_q, c, seed=seed, bh=bh, tensor=1,
-                        power_iters=power_iters, sample_factor=sample_factor)
+    if splitting == "diagonal":
+        rq = diagonal_partition(Yq, c, seed=seed, bh=bh, tensor=0, sample_factor=sample_factor)
+        rk = diagonal_partition(Yk, c, seed=seed, bh=bh, tensor=1, sample_factor=sample_factor)
+    else:
+        rq = pddp_partition(Yq, R_k, c, seed=seed, bh=bh, tensor=0,
+                            power_iters=power_iters, sample_factor=sample_factor)
+        rk = pddp_partition(Yk, R_q, c, seed=seed, bh=bh, tensor=1,
+                            power_iters=power_iters, sample_factor=sample_factor)
     perm_q, count_q = _leaves_to_perm(rq.leaves, c)
     perm_k, count_k = _leaves_to_perm(rk.leaves, c)
     return HeadClusters(perm_q=perm_q, perm_k=perm_k, count_q=count_q, count_k=count_k,
@@ -421,7 +511,8 @@ def cluster_head_random(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, 
 
 def cluster_workload(Q: np.ndarray, K: np.ndarray, n_valid: int, c: int, *, seed: int = 0,
                      power_iters: int = 8, heads: Optional[Sequence[int]] = None,
-                     transform: bool = True) -> List[HeadClusters]:
+                     transform: bool = True, splitting: str = "basic",
+                     query_form: str = "topk") -> List[HeadClusters]:
     """Cluster every (b, h) of [B, H, N_alloc, d] inputs; rows >= n_valid are padding."""
     B, H = Q.shape[:2]
     out = []
@@ -431,7 +522,8 @@ def cluster_workload(Q: np.ndarray, K: np.ndarray, n_valid: int, c: int, *, seed
             if heads is not None and bh not in heads:
                 continue
             out.append(cluster_head(Q[b, h, :n_valid], K[b, h, :n_valid], c, seed=seed,
-                                    bh=bh, power_iters=power_iters, transform=transform))
+                                    bh=bh, power_iters=power_iters, transform=transform,
+                                    splitting=splitting, query_form=query_form))
     return out
 
 

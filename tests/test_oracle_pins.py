@@ -616,3 +616,147 @@ def test_tight_clusters_beat_random_ones_when_attention_is_sparse_and_with_compe
             err[name, comp] = np.linalg.norm(O - dense) / np.linalg.norm(dense)
     assert err["split", False] < err["random", False]
     assert err["split", True] < err["random", True]
+
+
+# ---------------------------------------------------------------------------
+# Diagonalized recursive splitting (Section 3.2.1 "Diagonalized recursive
+# splitting"; later revision Section 4.1.1).
+# ---------------------------------------------------------------------------
+
+def test_pca_basis_matches_svd_of_centred_rows():
+    """The basis diagonalises the covariance: compare with the right singular
+    vectors of the centred rows (a different library routine), eigenvalue =
+    singular value^2 / n, same order, same sign rule."""
+    rng = np.random.default_rng(101)
+    A = rng.standard_normal((6, 6))
+    Y = rng.standard_normal((400, 6)) @ A + rng.standard_normal(6) * 3.0
+    U, lam = orc.pca_basis(Y)
+    Yc = Y - Y.mean(axis=0)
+    _, sv, Vt = np.linalg.svd(Yc, full_matrices=False)
+    np.testing.assert_allclose(lam, sv ** 2 / Y.shape[0], rtol=1e-12)
+    assert np.all(np.diff(lam) <= 0)
+    for j in range(6):
+        v = Vt[j]
+        i = int(np.argmax(np.abs(v)))
+        v = v if v[i] > 0 else -v
+        np.testing.assert_allclose(U[:, j], v, atol=1e-10)
+        assert U[np.argmax(np.abs(U[:, j])), j] > 0
+
+
+def test_diagonal_split_of_line_data_follows_the_signed_principal_direction():
+    """Points along a known direction u (largest entry positive) plus small
+    noise: the first split puts the t points with the smallest u . y below it,
+    whatever their token order."""
+    rng = np.random.default_rng(102)
+    d, n, c = 8, 200, 16
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    if u[np.argmax(np.abs(u))] < 0:
+        u = -u
+    s = rng.standard_normal(n) * 10.0
+    Y = s[:, None] * u[None, :] + rng.standard_normal((n, d)) * 1e-3
+    r = orc.diagonal_partition(Y, c, seed=0, bh=0, tensor=0, record=True)
+    heap, size, t, lo_max, up_min, j = r.splits[0]
+    assert heap == 1 and size == n and j == 0      # the leading coordinate
+    t_want = orc.split_count(n, c)
+    assert t == t_want and t != n - t
+    below = np.sort(np.argsort(Y @ u, kind="stable")[:t])
+    # leaves of the left subtree are exactly the t smallest along +u
+    left = np.sort(np.concatenate([lv for lv in r.leaves if np.isin(lv, below).all()]))
+    np.testing.assert_array_equal(left, below)
+
+
+def test_diagonal_root_split_uses_leading_component_when_sample_is_whole_set():
+    """With |S| <= d the sample is the whole set, whose variance along basis
+    vector j is eigenvalue j: the root splits on the leading principal
+    component (a flipped eigenvalue order would pick the smallest)."""
+    rng = np.random.default_rng(103)
+    d, n, c = 32, 32, 4
+    Y = rng.standard_normal((n, d)) * np.linspace(3.0, 0.1, d)
+    r = orc.diagonal_partition(Y, c, seed=5, bh=1, tensor=1, record=True)
+    _, _, t, _, _, j = r.splits[0]
+    assert j == 0
+    Yc = Y - Y.mean(axis=0)
+    _, _, Vt = np.linalg.svd(Yc, full_matrices=False)
+    v = Vt[0] if Vt[0][np.argmax(np.abs(Vt[0]))] > 0 else -Vt[0]
+    proj = Y @ v
+    below = set(np.lexsort((np.arange(n), proj))[:t].tolist())
+    first_leaves = []
+    acc = 0
+    for lv in r.leaves:
+        if acc >= t:
+            break
+        first_leaves.extend(lv.tolist())
+        acc += len(lv)
+    assert set(first_leaves) == below
+
+
+def test_diagonal_partition_invariant_to_coordinate_permutation():
+    """Permuting the coordinates of every row permutes the basis vectors'
+    entries (largest entry and its sign kept): the same partition."""
+    rng = np.random.default_rng(104)
+    d, n, c = 12, 900, 32
+    A = rng.standard_normal((d, d))
+    Y = rng.standard_normal((n, d)) @ A
+    pi = rng.permutation(d)
+    r1 = orc.diagonal_partition(Y, c, seed=3, bh=0, tensor=0)
+    r2 = orc.diagonal_partition(Y[:, pi], c, seed=3, bh=0, tensor=0)
+    assert r1.min_margin > 1e-9
+    assert len(r1.leaves) == len(r2.leaves)
+    for a, b in zip(r1.leaves, r2.leaves):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_diagonal_partition_of_sign_symmetric_data_is_coordinate_splitting():
+    """Rows made of every sign pattern of a few base rows have an exactly
+    diagonal covariance, so the basis is the coordinate axes sorted by
+    variance (the sign rule makes each axis +e_i) and every split is a split
+    on the raw coordinate of highest sample variance: checked against that
+    direct procedure."""
+    rng = np.random.default_rng(105)
+    d, c = 3, 8
+    base = rng.uniform(0.5, 1.5, size=(13, d)) * np.array([2.0, 1.0, 3.0])
+    signs = np.array([[1 if (m >> b) & 1 else -1 for b in range(d)] for m in range(2 ** d)])
+    Y = (base[:, None, :] * signs[None, :, :]).reshape(-1, d)
+    n = Y.shape[0]
+    r = orc.diagonal_partition(Y, c, seed=9, bh=2, tensor=1, sample_factor=4)
+
+    want = []
+
+    def rec(members, heap):
+        if members.shape[0] <= c:
+            want.append(members)
+            return
+        size = members.shape[0]
+        key = orc.node_key(9, 2, 1, heap)
+        m = min(4 * d, size)
+        if size <= m:
+            pos = np.arange(size)
+        else:
+            off = orc.sample_offset(key, size)
+            pos = (np.arange(m) * size + off) // m
+        S = Y[members[pos]]
+        j = int(np.argmax(S.var(axis=0)))
+        t = orc.split_count(size, c)
+        order = np.lexsort((members, Y[members, j]))
+        rec(np.sort(members[order[:t]]), 2 * heap)
+        rec(np.sort(members[order[t:]]), 2 * heap + 1)
+
+    rec(np.arange(n), 1)
+    assert len(r.leaves) == len(want)
+    for a, b in zip(r.leaves, want):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_diagonal_cluster_head_partitions_both_tensors():
+    rng = np.random.default_rng(106)
+    n, d, c = 1000, 16, 64
+    Q = rng.standard_normal((n, d))
+    K = rng.standard_normal((n, d)) + 0.5
+    for transform in (True, False):
+        for form in ("topk", "adaptive"):
+            h = orc.cluster_head(Q, K, c, seed=1, transform=transform, query_form=form,
+                                 splitting="diagonal")
+            for perm, cnt in ((h.perm_q, h.count_q), (h.perm_k, h.count_k)):
+                assert sorted(perm[perm >= 0].tolist()) == list(range(n))
+                assert cnt.sum() == n and (cnt[:-1] == c).all()
