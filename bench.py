@@ -180,10 +180,12 @@ def oracle_sample(w, n_clusters=48, heads=(0,), keep=None, selection="topk", rec
             hc = orc.cluster_head_random(Qf, Kf, w.c, seed=0, bh=h)
             kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
         elif selection == "adaptive":
-            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, query_form="adaptive")
+            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, query_form="adaptive",
+                                  splitting="diagonal" if clustering == "diagonal" else "basic")
             kept = orc.adaptive_route(orc.centroid_scores(hc.qbar, hc.kbar), hc.count_k, w.d, recall, 16)
         else:
-            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h)
+            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h,
+                                  splitting="diagonal" if clustering == "diagonal" else "basic")
             kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
         t1 = time.perf_counter()
         sample = list(range(0, w.C, max(1, w.C // n_clusters)))[:n_clusters]
@@ -459,6 +461,9 @@ def run_ours(args):
         # count / scatter, centroids
         levels = (per_step[0] - 6) // 5
         per_step[0] = 2 + 4 * levels
+    if args.clustering == "diagonal" and per_step[0] > 1:
+        # weighted query column sums and Gram, covariance reduce, basis
+        per_step[0] += 4
     launches = args.steps * sum(per_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -507,8 +512,9 @@ def main():
     ap.add_argument("--selection", choices=["topk", "adaptive"], default="topk",
                     help="key-cluster selection (adaptive: mass recall, capacity C per query cluster)")
     ap.add_argument("--recall", type=float, default=0.9)
-    ap.add_argument("--clustering", choices=["split", "random"], default="split",
-                    help="random: the random-cluster baseline of the paper's error analysis")
+    ap.add_argument("--clustering", choices=["split", "diagonal", "random"], default="split",
+                    help="diagonal: diagonalized recursive splitting; random: the random-cluster "
+                         "baseline of the paper's error analysis")
     ap.add_argument("--smc", choices=["on", "off"], default="on", help="striped mean-compensation")
     ap.add_argument("--tokens", type=int, default=0,
                     help="latency scaling: configuration 2's generator at this token count")

@@ -137,7 +137,8 @@ def make_params(power_iters: int = 8, sample_factor: int = 1, transform: int = 1
                 seed: int = 0, query_form: int = 0, method: int = 0) -> ca_cluster_params:
     """query_form 0: queries as R_k q / |R_k q| (top-k selection, eq. 16);
     1: queries as R_k q (adaptive selection, eq. 15). method 0: recursive
-    splitting; 1: random clusters (the error-analysis baseline)."""
+    splitting; 1: random clusters (the error-analysis baseline); 2:
+    diagonalized recursive splitting."""
     return ca_cluster_params(power_iters, sample_factor, transform, query_form, seed & ((1 << 64) - 1), method, 0)
 
 

@@ -49,7 +49,8 @@ ca_status check_params(const ca_shape* s, const ca_cluster_params* p) {
   if (dir_smem(s->d, a) > 227 * 1024) return CA_ERR_UNSUPPORTED;
   if (p->transform != 0 && p->transform != 1) return CA_ERR_INVALID_ARG;
   if (p->query_form != 0 && p->query_form != 1) return CA_ERR_INVALID_ARG;
-  if (p->method != 0 && p->method != 1) return CA_ERR_INVALID_ARG;
+  if (p->method < 0 || p->method > 2) return CA_ERR_INVALID_ARG;
+  if (p->method == 2 && a != 1) return CA_ERR_UNSUPPORTED;
   return CA_OK;
 }
 

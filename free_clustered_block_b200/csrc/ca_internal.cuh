@@ -112,7 +112,7 @@ inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 struct ClusterWs {
   size_t nodes, level_begin, M, kmean, colsum_part, met_part, inv_s, idx0, idx1, keys, zvec, wvec,
-      sel, chunk_cnt, total;
+      sel, chunk_cnt, cov, basis, basis_scratch, total;
   int nch = 0;       // metric row chunks
   int pch_max = 0;   // partition chunks per node, max over levels
   int TH = 0, BH = 0;
@@ -120,6 +120,16 @@ struct ClusterWs {
 constexpr int kMetricChunk = 2048;     // rows per metric partial
 constexpr int kPartChunk = 2048;       // positions per partition chunk
 bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, ClusterWs* ws);
+
+// Diagonalized splitting (diag.cu): covariances from the Gram partials, the
+// principal-component directions W per tensor-head, and the per-level choice
+// of the highest-variance coordinate.
+cudaError_t launch_diag_basis(int D, int TH, int BH, int nch, int n, const double* part, const double* M,
+                              double* C, double* scratch, double* W, cudaStream_t st);
+template <typename T, int D>
+cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const TreeNode* nodes, int lvl_begin,
+                            int nodes_in_level, int TH, const double* W, const double* inv_s, const int* idx,
+                            int NI, double* wvec, uint64_t seed, cudaStream_t st);
 
 struct AttendWs {
   size_t qp, kp, vp, kbar_hi, kbar_lo, vbar_hi, vbar_lo, vbar32, kbar32, logcnt, total;

@@ -105,16 +105,24 @@ __global__ void __launch_bounds__(1024) plan_kernel(int n, int c, TreeNode* node
 // ---------------------------------------------------------------------------
 // S1: column sums of K (for the key mean), per row chunk.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
+// With kW the rows are scaled by w[bh n + row] first (the queries' 1 / |R_k q|
+// for the covariance of their representations).
+template <typename T, int D, bool kW = false>
 __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, int N_alloc, int n,
-                                                     double* __restrict__ part) {
+                                                     double* __restrict__ part,
+                                                     const double* __restrict__ w = nullptr) {
   constexpr int RG = 256 / D;
   const int bh = blockIdx.y, ch = blockIdx.x, nch = gridDim.x;
   const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
   const int col = threadIdx.x % D, rg = threadIdx.x / D;
   const T* base = K + (size_t)bh * N_alloc * D;
   double acc = 0.0;
-  for (int r = r0 + rg; r < r1; r += RG) acc += (double)to_f(base[(size_t)r * D + col]);
+  if constexpr (kW) {
+    for (int r = r0 + rg; r < r1; r += RG)
+      acc = fma((double)to_f(base[(size_t)r * D + col]), w[(size_t)bh * n + r], acc);
+  } else {
+    for (int r = r0 + rg; r < r1; r += RG) acc += (double)to_f(base[(size_t)r * D + col]);
+  }
   __shared__ double red[256];
   red[threadIdx.x] = acc;
   __syncthreads();
@@ -165,10 +173,14 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
-template <typename T, int D>
+// kW: one launch over the queries only (grid.z = 1), rows scaled by
+// w[bh n + row] and centred by the weighted mean taken from colpart; the
+// result goes to the queries' slot (z = 0) of part. This is the covariance of
+// the query representations before the transform (diagonalized splitting).
+template <typename T, int D, bool kW = false>
 __global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* __restrict__ K, int N_alloc,
                                              int n, int nch, const double* __restrict__ colpart,
-                                             double* __restrict__ part) {
+                                             double* __restrict__ part, const double* __restrict__ w = nullptr) {
   using Cfg = SyrkCfg<D>;
   constexpr int R = Cfg::R, NTH = Cfg::kThreads, ROWS = Cfg::kRows;
   constexpr int VEC = 16 / sizeof(T);                 // elements per 16-byte chunk
@@ -189,7 +201,7 @@ __global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* _
   if (r0 < r1) issue(r0);
   for (int c = threadIdx.x; c < D; c += NTH) {
     double m = 0.0;
-    if (z == 1) {
+    if (kW || z == 1) {
       for (int i = 0; i < nch; ++i) m += colpart[((size_t)bh * nch + i) * D + c];
       m /= (double)n;
     }
@@ -212,7 +224,11 @@ __global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* _
     const int rows = min(ROWS, r1 - rt);
     for (int e = threadIdx.x; e < ROWS * D; e += NTH) {
       const int rr = e / D, cc = e % D;
-      xs[rr * D + syrk_pos(cc)] = rr < rows ? (double)to_f(raw[e]) - mean[cc] : 0.0;
+      if constexpr (kW)
+        xs[rr * D + syrk_pos(cc)] =
+            rr < rows ? (double)to_f(raw[e]) * w[(size_t)bh * n + rt + rr] - mean[cc] : 0.0;
+      else
+        xs[rr * D + syrk_pos(cc)] = rr < rows ? (double)to_f(raw[e]) - mean[cc] : 0.0;
     }
     __syncthreads();
     if (rt + ROWS < r1) issue(rt + ROWS);
@@ -1321,6 +1337,8 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
   const int normalize = transform && p->query_form == 0;
 
   const bool random_clusters = p->method == 1;
+  const bool diagonal = p->method == 2;
+  double* basis = reinterpret_cast<double*>(ws + L.basis);
   if (plan.levels > 0) {
     plan_kernel<<<1, 1024, 0, st>>>(n, c, nodes, level_begin);
     if (!random_clusters) {
@@ -1337,6 +1355,20 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
         cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
         qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, normalize, inv_s);
       }
+      if (diagonal) {
+        // covariance of the scaled query rows (weights 1 / |R_k q| in the
+        // top-k form, 1 otherwise): weighted column sums into the key sums'
+        // buffer and the centred weighted Gram into the queries' slot of the
+        // partials, both free once M and the query scales exist
+        colsum_kernel<T, D, true><<<dim3(nch, BH), 256, 0, st>>>(Q, N_alloc, n, colpart, inv_s);
+        cudaFuncSetAttribute(syrk_kernel<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
+        syrk_kernel<T, D, true><<<dim3(nch, BH, 1), SyrkCfg<D>::kThreads, syrk_smem, st>>>(
+            Q, K, N_alloc, n, nch, colpart, metpart, inv_s);
+        const cudaError_t e = launch_diag_basis(D, TH, BH, nch, n, metpart, M,
+                                                reinterpret_cast<double*>(ws + L.cov),
+                                                reinterpret_cast<double*>(ws + L.basis_scratch), basis, st);
+        if (e != cudaSuccess) return e;
+      }
     }
     const int m_cap = sample_factor * D;
     const int dir_warps = DirCfg<T, D>::warps(m_cap);
@@ -1351,6 +1383,10 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       int* idx_out = idxbuf[(l + 1) & 1];
       if (random_clusters) {
         hash_keys_kernel<<<dim3((n + 255) / 256, TH), 256, 0, st>>>(n, idx_in, p->seed, keys);
+      } else if (diagonal) {
+        const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, TH, basis, inv_s, idx_in,
+                                                    NI, wvec, p->seed, st);
+        if (e != cudaSuccess) return e;
       } else if (sample_factor == 1 && (D == 128 || (long long)nl * TH <= kDirCMaxNodes64)) {
         // a block per node: d = 128, or d = 64 levels with few nodes (about
         // four blocks per SM over the whole level)
@@ -1436,6 +1472,9 @@ bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, ClusterWs* w) {
   w->wvec = take(TH * NI * d * 8);
   w->sel = take(TH * NI * 16);
   w->chunk_cnt = take(TH * chunk_cnt * 8);
+  w->cov = take(TH * d * d * 8);
+  w->basis = take(TH * d * d * 8);
+  w->basis_scratch = take(TH * 2 * d * d * 8);
   w->total = o;
   return true;
 }

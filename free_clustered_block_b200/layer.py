@@ -13,6 +13,9 @@ from . import (CA_BF16, CA_FP32, ca_attend, ca_cluster, ca_dense_attend, ca_forw
                make_params, make_shape, num_clusters, routes_struct)
 
 
+CLUSTERING_METHODS = {"split": 0, "random": 1, "diagonal": 2}
+
+
 @dataclass
 class Buffers:
     perm_q: object
@@ -28,6 +31,10 @@ class Buffers:
 
 class ClusterAttention:
     """One layer's shape, knobs and device buffers.
+
+    clustering: "split" (basic recursive splitting, power iteration per set),
+    "diagonal" (diagonalized recursive splitting) or "random" (random
+    clusters, the error-analysis baseline).
 
     Q, K, V, O: torch CUDA tensors [B, H, N_alloc, d], bf16 or fp32, contiguous.
     """
@@ -46,7 +53,7 @@ class ClusterAttention:
         self.recall, self.min_count = recall, min_count
         self.params = make_params(power_iters, sample_factor, int(transform), seed,
                                   query_form=1 if selection == "adaptive" else 0,
-                                  method=1 if clustering == "random" else 0)
+                                  method=CLUSTERING_METHODS[clustering])
         self.k = k
         self.compensate = compensate
         C = num_clusters(self.shape)

@@ -58,7 +58,8 @@ typedef struct {
   int dtype;         /* ca_dtype of Q, K, V and O */
 } ca_shape;
 
-/* Clustering knobs (paper Section 3.2.1 "Basic recursive splitting"):
+/* Clustering knobs (paper Section 3.2.1, "Basic recursive splitting" and
+ * "Diagonalized recursive splitting"):
  *  power_iters   p, power-iteration steps per split (0 -> default 8);
  *  sample_factor a, sample size min(a d, |S|) per split (0 -> default 1);
  *  transform     1 = interaction-aware transforms (Section 3.2.2), the default;
@@ -72,7 +73,16 @@ typedef struct {
  *                    analysis: token i of (b, h, tensor) gets the key
  *                    SplitMix64(stream(seed, bh, tensor, 0) ^ i), and the
  *                    tokens ordered by (key, i) form the clusters, c at a
- *                    time, the remainder last (the other knobs are ignored). */
+ *                    time, the remainder last (the other knobs are ignored);
+ *                2 = diagonalized recursive splitting: the representations
+ *                    are rotated once into the principal-component basis of
+ *                    the full set (eigenvectors of their covariance by
+ *                    descending eigenvalue, each signed so that its
+ *                    largest-magnitude entry is positive) and every set is
+ *                    split on the coordinate with the highest variance over
+ *                    the basic splitting's sample (lowest index on a tie);
+ *                    power_iters is ignored; sample_factor must be 0 or 1
+ *                    (CA_ERR_UNSUPPORTED otherwise). */
 typedef struct {
   int power_iters;
   int sample_factor;
