@@ -68,7 +68,7 @@ constexpr double kJacobiEps = 2.220446049250313e-16;   // 2^-52
 
 template <int D>
 struct BasisCfg {
-  static constexpr int kThreads = D == 64 ? 256 : 512;
+  static constexpr int kThreads = 512;   // 16 warps: each step's latency spread over more schedulers
   static constexpr int P = D / 2;                       // pairs per step
   static constexpr int kPacked = D * (D + 1) / 2;
   static constexpr int kBlocks = P * (P + 1) / 2;       // pair blocks (k <= l)
@@ -119,15 +119,19 @@ __device__ void jacobi_eigen(double* A, double* Vt, const uint32_t* blk, const i
         if (e >= NB) break;
         const uint32_t kl = blk[e];
         const int k = (int)(kl >> 16), l = (int)(kl & 0xFFFFu);
-        const double ck = cs[k], sk = sn[k], cl = cs[l], sl = sn[l];
-        if (sk == 0.0 && sl == 0.0) continue;
+        const double ck = cs[k], sk = sn[k], cl = cs[l], sl = sn[l];   // (1, 0): identity, exactly
+        // d = 128: late sweeps skip most rotations, so skipping idle blocks pays; at d = 64
+        // the branch-free loop is faster
+        if constexpr (D == 128) {
+          if (sk == 0.0 && sl == 0.0) continue;
+        }
         const int pk = pp[k], qk = qq[k];
         if (k == l) {
           const int ip = off[pk] + pk, iq = off[qk] + qk, io = packed_off(off, pk, qk);
           const double aa = A[ip], ee = A[iq], bb = A[io];
           A[ip] = ck * ck * aa - 2.0 * ck * sk * bb + sk * sk * ee;
           A[iq] = sk * sk * aa + 2.0 * ck * sk * bb + ck * ck * ee;
-          A[io] = 0.0;
+          A[io] = sk == 0.0 ? bb : 0.0;
         } else {
           const int pl = pp[l], ql = qq[l];
           const int i00 = packed_off(off, pk, pl), i01 = packed_off(off, pk, ql);
@@ -144,7 +148,9 @@ __device__ void jacobi_eigen(double* A, double* Vt, const uint32_t* blk, const i
         const int e = t + u * NT;
         const int k = e / D, i = e % D;
         const double c = cs[k], s = sn[k];
-        if (s == 0.0) continue;
+        if constexpr (D == 128) {
+          if (s == 0.0) continue;
+        }
         const int p = pp[k], q = qq[k];
         const double vp = Vt[p * D + i], vq = Vt[q * D + i];
         Vt[p * D + i] = c * vp - s * vq;
