@@ -46,9 +46,11 @@ Readings where the paper leaves a step open (each is listed in the design doc):
  * compensation weight |c| is the number of real members of the cluster;
  * diagonalized splitting: the basis diagonalises the (centred) covariance
    of the representations over all valid rows; basis vectors are ordered by
-   descending eigenvalue and signed so that their largest-magnitude entry is
-   positive; the per-set sample is the basic splitting's, and the highest
-   sample variance picks the coordinate (lowest index on a tie).
+   descending eigenvalue and signed so that the raw-space direction R u_j
+   has its largest-magnitude entry positive (a sign that does not depend on
+   which root of the metric forms the representation); the per-set sample is
+   the basic splitting's, and the highest sample variance picks the
+   coordinate (lowest index on a tie).
 
 Random numbers: SplitMix64 (Steele, Lea & Flood, "Fast splittable
 pseudorandom number generators", OOPSLA 2014) on a per-node counter, turned
@@ -339,15 +341,18 @@ def pddp_partition_metric_form(X: np.ndarray, M: np.ndarray, c: int, *, seed: in
 # Diagonalized recursive splitting.
 # ---------------------------------------------------------------------------
 
-def pca_basis(Y: np.ndarray) -> tuple:
+def pca_basis(Y: np.ndarray, factor: Optional[np.ndarray] = None) -> tuple:
     """Principal-component basis of the representations Y (rows, the full
     set) from the eigendecomposition of their covariance (Section 3.2.1
     "Diagonalized recursive splitting"; later revision Section 4.1.1).
 
-    Returns (U, lam): the columns of U are unit eigenvectors ordered by
-    descending eigenvalue lam (ties keep the solver's order); each column's
-    entry of largest magnitude (the first such entry on an exact tie) is made
-    positive, which fixes which side of a split is "below".
+    Y holds the rows x F of the raw rows x (F = ``factor``, the identity when
+    None). Returns (U, lam): the columns of U are unit eigenvectors ordered by
+    descending eigenvalue lam (ties keep the solver's order), each signed so
+    that the raw-space direction w_j = F u_j (coordinate j of a row is
+    x . w_j) has its entry of largest magnitude (the first on an exact tie)
+    positive; this fixes which side of a split is "below", and w_j is the
+    same for every factor F with F F^T equal to the metric.
     """
     Y = np.asarray(Y, dtype=np.float64)
     n = Y.shape[0]
@@ -356,16 +361,19 @@ def pca_basis(Y: np.ndarray) -> tuple:
     lam, U = np.linalg.eigh(cov)
     order = np.argsort(-lam, kind="stable")
     lam, U = lam[order], U[:, order].copy()
+    Wd = U if factor is None else np.asarray(factor, dtype=np.float64) @ U
     for j in range(U.shape[1]):
-        i = int(np.argmax(np.abs(U[:, j])))
-        if U[i, j] < 0:
+        i = int(np.argmax(np.abs(Wd[:, j])))
+        if Wd[i, j] < 0:
             U[:, j] = -U[:, j]
     return U, lam
 
 
 def diagonal_partition(Y: np.ndarray, c: int, *, seed: int, bh: int, tensor: int,
-                       sample_factor: int = 1, record: bool = False) -> PddpResult:
-    """Diagonalized recursive splitting of the rows of Y (already transformed).
+                       sample_factor: int = 1, record: bool = False,
+                       factor: Optional[np.ndarray] = None) -> PddpResult:
+    """Diagonalized recursive splitting of the rows of Y (already transformed,
+    Y = X F with ``factor`` F; the identity when None).
 
     The rows are rotated once into the principal-component basis of the full
     set, Z = Y U (pca_basis). At every set S: take the same sample of
@@ -377,7 +385,7 @@ def diagonal_partition(Y: np.ndarray, c: int, *, seed: int, bh: int, tensor: int
     """
     Y = np.asarray(Y, dtype=np.float64)
     n, d = Y.shape
-    U, _ = pca_basis(Y)
+    U, _ = pca_basis(Y, factor)
     Z = Y @ U
     res = PddpResult(leaves=[])
     m_cap = sample_factor * d
@@ -467,8 +475,9 @@ def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int
         R_q = R_k = np.eye(d)
         Yk, Yq = K, Q
     if splitting == "diagonal":
-        rq = diagonal_partition(Yq, c, seed=seed, bh=bh, tensor=0, sample_factor=sample_factor)
-        rk = diagonal_partition(Yk, c, seed=seed, bh=bh, tensor=1, sample_factor=sample_factor)
+        # Y = X R with R symmetric (query rows also scaled by 1 / |R_k q|)
+        rq = diagonal_partition(Yq, c, seed=seed, bh=bh, tensor=0, sample_factor=sample_factor, factor=R_k)
+        rk = diagonal_partition(Yk, c, seed=seed, bh=bh, tensor=1, sample_factor=sample_factor, factor=R_q)
     else:
         rq = pddp_partition(Yq, R_k, c, seed=seed, bh=bh, tensor=0,
                             power_iters=power_iters, sample_factor=sample_factor)

@@ -760,3 +760,29 @@ def test_diagonal_cluster_head_partitions_both_tensors():
             for perm, cnt in ((h.perm_q, h.count_q), (h.perm_k, h.count_k)):
                 assert sorted(perm[perm >= 0].tolist()) == list(range(n))
                 assert cnt.sum() == n and (cnt[:-1] == c).all()
+
+
+def test_diagonal_partition_does_not_depend_on_the_metric_factor():
+    """Any factor F with F F^T = M gives the representation X F a rotation of
+    X R (R the symmetric root), whose principal coordinates are the same up
+    to sign; the sign rule is stated on the raw-space direction F u_j, so
+    the partition with the symmetric root and with the Cholesky factor (a
+    different library routine) is the same."""
+    rng = np.random.default_rng(107)
+    n, d, c = 1500, 12, 64
+    X = rng.standard_normal((n, d)) @ rng.standard_normal((d, d)) + 0.3
+    Qm = rng.standard_normal((3 * n, d)) @ rng.standard_normal((d, d))
+    M = Qm.T @ Qm / Qm.shape[0]
+    R = orc.psd_root(M)
+    L = np.linalg.cholesky(M)
+    np.testing.assert_allclose(L @ L.T, R @ R, rtol=1e-10, atol=1e-10)
+    for seed in range(4):
+        r1 = orc.diagonal_partition(X @ R, c, seed=seed, bh=0, tensor=1, factor=R)
+        r2 = orc.diagonal_partition(X @ L, c, seed=seed, bh=0, tensor=1, factor=L)
+        assert r1.min_margin > 1e-9
+        for a, b in zip(r1.leaves, r2.leaves):
+            np.testing.assert_array_equal(a, b)
+    # the raw-space directions themselves agree, signs included
+    U_r, _ = orc.pca_basis(X @ R, R)
+    U_l, _ = orc.pca_basis(X @ L, L)
+    np.testing.assert_allclose(R @ U_r, L @ U_l, atol=1e-8)
