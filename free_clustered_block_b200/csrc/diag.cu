@@ -9,17 +9,17 @@
 // metric, eq. 13-14; queries in the top-k form also scaled by 1 / |R_k q|,
 // eq. 16), the covariance of the representations is R C R, where C is the
 // covariance of the (scaled) raw rows. Its unit eigenvectors u_j, ordered by
-// descending eigenvalue and signed so that their largest-magnitude entry is
-// positive, give coordinate j of a row as y . u_j = x . w_j with
-// w_j = R u_j. The rotation is therefore never materialised: the per-set
+// descending eigenvalue, give coordinate j of a row as y . u_j = x . w_j with
+// w_j = R u_j, each signed so that w_j's entry of largest magnitude is
+// positive. The rotation is therefore never materialised: the per-set
 // kernel evaluates the sample's coordinates through the w_j, picks the
 // coordinate of highest sample variance, and hands w_j to the projection
 // kernel shared with the basic splitting (which multiplies the query scale).
 //
 // Kernels:
 //   cov_reduce_kernel   chunk partials -> C per tensor-head (fp64)
-//   diag_basis_kernel   one CTA per tensor-head: Jacobi eigensolver for the
-//                       root of the metric, R C R, Jacobi again, W = (R U)^T
+//   diag_basis_kernel   one CTA per tensor-head: pivoted Cholesky factor F of
+//                       the metric, F^T C F, Jacobi eigensolver, W = (F U')^T
 //   diag_dir_kernel     per set: sample coordinates, variances, argmax, w_j*
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -165,8 +165,15 @@ __device__ void jacobi_eigen(double* A, double* Vt, const uint32_t* blk, const i
 // One CTA per tensor-head th. M[th]: the metric whose root transforms this
 // tensor (the identity without the transform); C[th]: covariance of the
 // (scaled) raw rows. Writes W[th] transposed (D x D, W[th][k][j] = entry k of
-// w_j, j in order of descending eigenvalue) and uses scratch[th] (2 D x D)
-// for R and C R.
+// w_j, j in order of descending eigenvalue) and uses scratch[th] (2 D x D).
+//
+// Any factor F with F F^T = M serves in place of the symmetric root R: F = R O
+// for an orthogonal O, so F^T C F = O^T (R C R) O has eigenvectors O^T u_j and
+// F O^T u_j = R u_j. F comes from a pivoted Cholesky factorisation (Higham,
+// "Accuracy and Stability of Numerical Algorithms", Section 10.3: pivot on the
+// largest remaining diagonal entry, stop when it falls to D eps max(diag M)),
+// D steps instead of a second Jacobi solve. The sign of each w_j is then set
+// on w_j itself, which does not depend on the factor.
 template <int D>
 __global__ void __launch_bounds__(BasisCfg<D>::kThreads, 1) diag_basis_kernel(const double* __restrict__ M,
                                                                              const double* __restrict__ C,
@@ -179,42 +186,72 @@ __global__ void __launch_bounds__(BasisCfg<D>::kThreads, 1) diag_basis_kernel(co
   double* Vt = A + Cfg::kPacked;                                     // D x D
   uint32_t* blk = reinterpret_cast<uint32_t*>(Vt + D * D);           // pair blocks (k, l), k <= l
   __shared__ double cs[P], sn[P], lam[D], sgn[D];
-  __shared__ int pp[P], qq[P], rnk[D], off[D];
-  const int th = blockIdx.x, t = threadIdx.x;
+  __shared__ int pp[P], qq[P], rnk[D], off[D], used[D];
+  __shared__ double piv_d, piv_inv, tol_s;
+  __shared__ int piv_s, stop_s;
+  const int th = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const double* Mg = M + (size_t)th * D * D;
   const double* Cg = C + (size_t)th * D * D;
-  double* Rg = scratch + (size_t)th * 2 * D * D;
-  double* Tg = Rg + D * D;
+  double* Fg = scratch + (size_t)th * 2 * D * D;   // F transposed: Fg[k][i] = F[i][k]
+  double* Tg = Fg + D * D;
   double* Wg = W + (size_t)th * D * D;
 
-  if (t < D) off[t] = packed<D>(t, t) - t;
+  if (t < D) { off[t] = packed<D>(t, t) - t; used[t] = 0; }
   if (t < P) {
     const int base = t * P - t * (t - 1) / 2;
     for (int l = t; l < P; ++l) blk[base + (l - t)] = ((uint32_t)t << 16) | (uint32_t)l;
   }
+  if (t == 0) stop_s = 0;
   for (int e = t; e < D * D; e += NT) {
     const int i = e / D, j = e % D;
     if (j >= i) A[packed<D>(i, j)] = Mg[e];
-    Vt[e] = (i == j) ? 1.0 : 0.0;
+    Vt[e] = 0.0;
   }
   __syncthreads();
-  // 1. M = V diag(lambda) V^T; R = V diag(sqrt(max(lambda, 0))) V^T
-  jacobi_eigen<D, NT>(A, Vt, blk, off, cs, sn, pp, qq);
-  if (t < D) lam[t] = sqrt(fmax(A[packed<D>(t, t)], 0.0));
-  __syncthreads();
+  // 1. M = F F^T, F[i][k] in Vt (row-major); columns after a stop stay zero
+  for (int k = 0; k < D; ++k) {
+    if (warp == 0) {
+      double best = -1.0;
+      int bi = D;
+      for (int i = lane; i < D; i += 32)
+        if (!used[i]) {
+          const double v = A[off[i] + i];
+          if (v > best) { best = v; bi = i; }
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+      }
+      if (lane == 0) {
+        if (k == 0) tol_s = best * (double)D * kJacobiEps;
+        if (bi >= D || !(best > tol_s)) {
+          stop_s = 1;
+        } else {
+          const double dk = sqrt(best);
+          piv_s = bi; piv_d = dk; piv_inv = 1.0 / dk; used[bi] = 1;
+        }
+      }
+    }
+    __syncthreads();
+    if (stop_s) break;
+    const int p = piv_s;
+    const double dk = piv_d, inv = piv_inv;
+    for (int i = t; i < D; i += NT)
+      Vt[i * D + k] = (i == p) ? dk : (used[i] ? 0.0 : A[packed_off(off, i, p)] * inv);
+    __syncthreads();
+    for (int e = t; e < D * D; e += NT) {   // Schur complement on the rows not yet pivoted
+      const int i = e / D, j = e % D;
+      if (j >= i && !used[i] && !used[j]) A[off[i] + j] -= Vt[i * D + k] * Vt[j * D + k];
+    }
+    __syncthreads();
+  }
   for (int e = t; e < D * D; e += NT) {
-    const int i = e / D, j = e % D;
-    if (j < i) continue;
-    double acc = 0.0;
-#pragma unroll 4
-    for (int k = 0; k < D; ++k) acc = fma(Vt[k * D + i] * lam[k], Vt[k * D + j], acc);
-    Rg[i * D + j] = acc;
-    Rg[j * D + i] = acc;
+    const int i = e / D, k = e % D;
+    Fg[k * D + i] = Vt[e];
   }
-  __syncthreads();
-  for (int e = t; e < D * D; e += NT) Vt[e] = Rg[e];   // Vt now holds R
-  __syncthreads();
-  // 2. C R, then the upper triangle of R (C R)
+  // 2. C F, then the upper triangle of F^T (C F)
   for (int e = t; e < D * D; e += NT) {
     const int i = e / D, j = e % D;
     double acc = 0.0;
@@ -228,38 +265,42 @@ __global__ void __launch_bounds__(BasisCfg<D>::kThreads, 1) diag_basis_kernel(co
     if (j < i) continue;
     double acc = 0.0;
 #pragma unroll 4
-    for (int k = 0; k < D; ++k) acc = fma(Vt[i * D + k], Tg[k * D + j], acc);
+    for (int k = 0; k < D; ++k) acc = fma(Vt[k * D + i], Tg[k * D + j], acc);
     A[packed<D>(i, j)] = acc;
   }
   __syncthreads();
   for (int e = t; e < D * D; e += NT) Vt[e] = (e / D == e % D) ? 1.0 : 0.0;
   __syncthreads();
-  // 3. R C R = U diag(mu) U^T
+  // 3. F^T C F = U' diag(mu) U'^T
   jacobi_eigen<D, NT>(A, Vt, blk, off, cs, sn, pp, qq);
-  if (t < D) lam[t] = A[packed<D>(t, t)];
+  if (t < D) lam[t] = A[off[t] + t];
   __syncthreads();
   if (t < D) {
     const double mu = lam[t];
     int r = 0;
     for (int i = 0; i < D; ++i) r += (lam[i] > mu) || (lam[i] == mu && i < t);
     rnk[t] = r;
-    double best = -1.0;
-    int bi = 0;
-    for (int i = 0; i < D; ++i) {
-      const double a = fabs(Vt[t * D + i]);
-      if (a > best) { best = a; bi = i; }
-    }
-    sgn[t] = Vt[t * D + bi] < 0.0 ? -1.0 : 1.0;
   }
   __syncthreads();
-  // 4. w_j = R u_j, stored as column rank(j)
+  // 4. w_j = F u'_j into column rank(j), then each column signed by its largest-magnitude entry
   for (int e = t; e < D * D; e += NT) {
     const int j = e / D, c = e % D;
     double acc = 0.0;
 #pragma unroll 4
-    for (int k = 0; k < D; ++k) acc = fma(Rg[k * D + c], Vt[j * D + k], acc);
-    Wg[(size_t)c * D + rnk[j]] = sgn[j] * acc;
+    for (int k = 0; k < D; ++k) acc = fma(Fg[k * D + c], Vt[j * D + k], acc);
+    Wg[(size_t)c * D + rnk[j]] = acc;
   }
+  __syncthreads();
+  if (t < D) {
+    double best = -1.0, v = 0.0;
+    for (int c = 0; c < D; ++c) {
+      const double x = Wg[(size_t)c * D + t];
+      if (fabs(x) > best) { best = fabs(x); v = x; }
+    }
+    sgn[t] = v < 0.0 ? -1.0 : 1.0;
+  }
+  __syncthreads();
+  for (int e = t; e < D * D; e += NT) Wg[e] *= sgn[e % D];
 }
 
 // ---------------------------------------------------------------------------

@@ -76,9 +76,10 @@ typedef struct {
  *                    time, the remainder last (the other knobs are ignored);
  *                2 = diagonalized recursive splitting: the representations
  *                    are rotated once into the principal-component basis of
- *                    the full set (eigenvectors of their covariance by
- *                    descending eigenvalue, each signed so that its
- *                    largest-magnitude entry is positive) and every set is
+ *                    the full set (eigenvectors u_j of their covariance by
+ *                    descending eigenvalue, each signed so that the
+ *                    raw-space direction R u_j has its largest-magnitude
+ *                    entry positive) and every set is
  *                    split on the coordinate with the highest variance over
  *                    the basic splitting's sample (lowest index on a tie);
  *                    power_iters is ignored; sample_factor must be 0 or 1
