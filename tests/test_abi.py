@@ -86,6 +86,16 @@ def test_calls_are_rejected_before_launch(lib):
     p = ca.make_params(power_iters=-1)
     assert lib.ca_cluster(_fake(A), _fake(A), ctypes.byref(s), ctypes.byref(p), ctypes.byref(cl), _fake(A),
                           need, None) == ca.CA_ERR_INVALID_ARG
+    # method out of range; diagonalized splitting takes only the sample factor a = 1
+    for bad, want in ((ca.make_params(method=3), ca.CA_ERR_INVALID_ARG),
+                      (ca.make_params(method=-1), ca.CA_ERR_INVALID_ARG),
+                      (ca.make_params(method=2, sample_factor=2), ca.CA_ERR_UNSUPPORTED),
+                      (ca.make_params(query_form=2), ca.CA_ERR_INVALID_ARG)):
+        assert lib.ca_cluster(_fake(A), _fake(A), ctypes.byref(s), ctypes.byref(bad), ctypes.byref(cl),
+                              _fake(A), need, None) == want
+    # the bounded-wait check rejects a zero or over-long limit before launching
+    assert lib.ca_check_bounded_wait(0, 0, None) == ca.CA_ERR_INVALID_ARG
+    assert lib.ca_check_bounded_wait(20_000_000_000, 0, None) == ca.CA_ERR_INVALID_ARG
     # k out of range
     for k in (0, 17):
         r = ca.ca_routes(k, A, A)
