@@ -220,15 +220,30 @@ def error_vs_dense(w, O_gpu_head, kept, n_clusters=8):
     return res
 
 
+def build_workload(args, rank: int):
+    """The layer a rank runs: a configuration's workload, or (--tokens) the
+    latency-scaling workload: configuration 2's generator (H = 8, d = 64,
+    c = 128) at another token count, keeping 1/8 of the clusters or a fixed 64."""
+    import workloads as wl
+    if args.tokens:
+        C = -(-args.tokens // 128)
+        kk = 64 if args.fixed_k else max(1, C // 8)
+        return wl.make_workload("lowrank", B=1, H=8, N=args.tokens, d=64, c=128, k=min(kk, C), dtype="bf16",
+                                seed=rank_seed(rank, 2), compensate=args.smc == "on",
+                                name=f"cfg2gen-lowrank-N{args.tokens}-d64-bf16-k{min(kk, C)}", rank=16,
+                                noise=0.1)
+    return wl.config_workload(args.config, seed=rank_seed(rank, args.config),
+                              **({"compensate": False} if args.smc == "off" else {}))
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import workloads as wl
-    w = wl.config_workload(args.config)
+    w = build_workload(args, 0)
     times = []
     for i in range(args.warmup + args.steps):
-        t, smp = oracle_sample(w)
+        t, smp = oracle_sample(w, selection=args.selection, recall=args.recall, clustering=args.clustering)
         if i >= args.warmup:
             times.append(t)
     t = statistics.mean(times)
@@ -237,7 +252,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": dict(workload_config(w), selection=args.selection, clustering=args.clustering,
+                       **({"recall": args.recall, "min_count": 16} if args.selection == "adaptive" else {})),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"per step: head 0 clustered and routed in full, attention of 48 of "
                                    f"{w.C} query clusters; extrapolated to {w.H} heads x {w.C} clusters"},
@@ -292,17 +308,7 @@ def run_ours(args):
         return max_over_ranks(x, world, "cuda")
 
     # Each rank: an independent layer (its own seeded inputs).
-    if args.tokens:
-        # latency scaling: configuration 2's generator (H = 8, d = 64, c = 128)
-        # at another token count, keeping 1/8 of the clusters or a fixed 64
-        C = -(-args.tokens // 128)
-        kk = 64 if args.fixed_k else max(1, C // 8)
-        w = wl.make_workload("lowrank", B=1, H=8, N=args.tokens, d=64, c=128, k=min(kk, C), dtype="bf16",
-                             seed=rank_seed(rank, 2), compensate=args.smc == "on",
-                             name=f"cfg2gen-lowrank-N{args.tokens}-d64-bf16-k{min(kk, C)}", rank=16, noise=0.1)
-    else:
-        w = wl.config_workload(args.config, seed=rank_seed(rank, args.config),
-                               **({"compensate": False} if args.smc == "off" else {}))
+    w = build_workload(args, rank)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(x):
