@@ -451,7 +451,7 @@ def _centroids(X: np.ndarray, leaves: Sequence[np.ndarray]) -> np.ndarray:
 def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int = 0,
                  power_iters: int = 8, sample_factor: int = 1,
                  transform: bool = True, query_form: str = "topk",
-                 splitting: str = "basic") -> HeadClusters:
+                 splitting: str = "basic", c_k: Optional[int] = None) -> HeadClusters:
     """Cluster the valid queries and keys of one head (rows [n, d]).
 
     Keys are split in the query-aware space R_q k; queries in the key-aware,
@@ -459,8 +459,12 @@ def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int
     ``query_form="adaptive"``, in R_k q (eq. 15). ``transform=False`` splits
     the raw vectors (R = I, no normalisation), the paper's ablation.
     ``splitting`` is "basic" (power iteration per set) or "diagonal"
-    (one principal-component rotation, coordinate splits).
+    (one principal-component rotation, coordinate splits). ``c`` is the
+    query cluster size; ``c_k`` the key cluster size (``c`` when None), the
+    paper evaluating 64 for queries and 128 for keys (Section 3.1): each
+    tensor's tree follows its own size.
     """
+    ck = c if c_k is None else c_k
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     d = Q.shape[1]
@@ -477,14 +481,14 @@ def cluster_head(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int
     if splitting == "diagonal":
         # Y = X R with R symmetric (query rows also scaled by 1 / |R_k q|)
         rq = diagonal_partition(Yq, c, seed=seed, bh=bh, tensor=0, sample_factor=sample_factor, factor=R_k)
-        rk = diagonal_partition(Yk, c, seed=seed, bh=bh, tensor=1, sample_factor=sample_factor, factor=R_q)
+        rk = diagonal_partition(Yk, ck, seed=seed, bh=bh, tensor=1, sample_factor=sample_factor, factor=R_q)
     else:
         rq = pddp_partition(Yq, R_k, c, seed=seed, bh=bh, tensor=0,
                             power_iters=power_iters, sample_factor=sample_factor)
-        rk = pddp_partition(Yk, R_q, c, seed=seed, bh=bh, tensor=1,
+        rk = pddp_partition(Yk, R_q, ck, seed=seed, bh=bh, tensor=1,
                             power_iters=power_iters, sample_factor=sample_factor)
     perm_q, count_q = _leaves_to_perm(rq.leaves, c)
-    perm_k, count_k = _leaves_to_perm(rk.leaves, c)
+    perm_k, count_k = _leaves_to_perm(rk.leaves, ck)
     return HeadClusters(perm_q=perm_q, perm_k=perm_k, count_q=count_q, count_k=count_k,
                         qbar=_centroids(Q, rq.leaves), kbar=_centroids(K, rk.leaves),
                         min_margin_q=rq.min_margin, min_margin_k=rk.min_margin)
@@ -503,16 +507,19 @@ def random_leaves(n: int, c: int, *, seed: int, bh: int, tensor: int) -> List[np
     return [np.sort(order[a:a + c]) for a in range(0, n, c)]
 
 
-def cluster_head_random(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int = 0) -> HeadClusters:
+def cluster_head_random(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, bh: int = 0,
+                        c_k: Optional[int] = None) -> HeadClusters:
     """Random clusters of the valid queries and keys of one head, with the
-    same outputs as cluster_head (permutation, counts, centroids)."""
+    same outputs as cluster_head (permutation, counts, centroids); keys in
+    groups of ``c_k`` (``c`` when None)."""
+    ck = c if c_k is None else c_k
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     n = Q.shape[0]
     lq = random_leaves(n, c, seed=seed, bh=bh, tensor=0)
-    lk = random_leaves(n, c, seed=seed, bh=bh, tensor=1)
+    lk = random_leaves(n, ck, seed=seed, bh=bh, tensor=1)
     perm_q, count_q = _leaves_to_perm(lq, c)
-    perm_k, count_k = _leaves_to_perm(lk, c)
+    perm_k, count_k = _leaves_to_perm(lk, ck)
     return HeadClusters(perm_q=perm_q, perm_k=perm_k, count_q=count_q, count_k=count_k,
                         qbar=_centroids(Q, lq), kbar=_centroids(K, lk),
                         min_margin_q=float("inf"), min_margin_k=float("inf"))
@@ -521,7 +528,7 @@ def cluster_head_random(Q: np.ndarray, K: np.ndarray, c: int, *, seed: int = 0, 
 def cluster_workload(Q: np.ndarray, K: np.ndarray, n_valid: int, c: int, *, seed: int = 0,
                      power_iters: int = 8, heads: Optional[Sequence[int]] = None,
                      transform: bool = True, splitting: str = "basic",
-                     query_form: str = "topk") -> List[HeadClusters]:
+                     query_form: str = "topk", c_k: Optional[int] = None) -> List[HeadClusters]:
     """Cluster every (b, h) of [B, H, N_alloc, d] inputs; rows >= n_valid are padding."""
     B, H = Q.shape[:2]
     out = []
@@ -532,7 +539,7 @@ def cluster_workload(Q: np.ndarray, K: np.ndarray, n_valid: int, c: int, *, seed
                 continue
             out.append(cluster_head(Q[b, h, :n_valid], K[b, h, :n_valid], c, seed=seed,
                                     bh=bh, power_iters=power_iters, transform=transform,
-                                    splitting=splitting, query_form=query_form))
+                                    splitting=splitting, query_form=query_form, c_k=c_k))
     return out
 
 
@@ -610,7 +617,7 @@ def _members(perm: np.ndarray, count: np.ndarray, c: int, a: int) -> np.ndarray:
 
 def compensated_attention(Q, K, V, perm_q, count_q, perm_k, count_k, kept, c: int, *,
                           compensate: bool = True, clusters: Optional[Sequence[int]] = None,
-                          n_out: Optional[int] = None) -> np.ndarray:
+                          n_out: Optional[int] = None, c_k: Optional[int] = None) -> np.ndarray:
     """Block-sparse attention over the kept key clusters, with striped
     mean-compensation of every excluded key cluster (eq. 21-22).
 
@@ -618,6 +625,7 @@ def compensated_attention(Q, K, V, perm_q, count_q, perm_k, count_k, kept, c: in
       o_i = (sum_{b kept} sum_{j in b} e^{l_ij} v_j
              + sum_{b excluded} |b| e^{q_i . k_bar_b / sqrt(d)} v_bar_b) / (same weights)
     with l_ij = q_i . k_j / sqrt(d); ``compensate=False`` drops the second sum.
+    ``c`` is the slot size of perm_q, ``c_k`` that of perm_k (``c`` when None).
     Returns O [n_out, d] in original token order (rows of clusters not
     evaluated are left at 0).
     """
@@ -626,7 +634,7 @@ def compensated_attention(Q, K, V, perm_q, count_q, perm_k, count_k, kept, c: in
     scale = 1.0 / math.sqrt(d)
     Cq = count_q.shape[0]
     Ck = count_k.shape[0]
-    kmem = [_members(perm_k, count_k, c, b) for b in range(Ck)]
+    kmem = [_members(perm_k, count_k, c if c_k is None else c_k, b) for b in range(Ck)]
     kbar = np.stack([K[m].mean(axis=0) for m in kmem])
     vbar = np.stack([V[m].mean(axis=0) for m in kmem])
     logcnt = np.log(count_k.astype(np.float64))
@@ -679,10 +687,11 @@ class ForwardResult:
 def forward_head(Q, K, V, c: int, k: int, *, seed: int = 0, bh: int = 0,
                  power_iters: int = 8, compensate: bool = True,
                  clusters_subset: Optional[Sequence[int]] = None,
-                 transform: bool = True) -> ForwardResult:
-    """cluster -> route -> attend for one head's valid rows [n, d]."""
-    hc = cluster_head(Q, K, c, seed=seed, bh=bh, power_iters=power_iters, transform=transform)
+                 transform: bool = True, c_k: Optional[int] = None) -> ForwardResult:
+    """cluster -> route -> attend for one head's valid rows [n, d]; ``c`` is
+    the query cluster size, ``c_k`` the key cluster size (``c`` when None)."""
+    hc = cluster_head(Q, K, c, seed=seed, bh=bh, power_iters=power_iters, transform=transform, c_k=c_k)
     kept = topk_route(centroid_scores(hc.qbar, hc.kbar), k)
     O = compensated_attention(Q, K, V, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, c,
-                              compensate=compensate, clusters=clusters_subset)
+                              compensate=compensate, clusters=clusters_subset, c_k=c_k)
     return ForwardResult(clusters=hc, kept=kept, O=O)

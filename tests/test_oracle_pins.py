@@ -786,3 +786,66 @@ def test_diagonal_partition_does_not_depend_on_the_metric_factor():
     U_r, _ = orc.pca_basis(X @ R, R)
     U_l, _ = orc.pca_basis(X @ L, L)
     np.testing.assert_allclose(R @ U_r, L @ U_l, atol=1e-8)
+
+
+# ---------------------------------------------------------------------------
+# Unequal query and key cluster sizes (the paper evaluates 64 for queries and
+# 128 for keys, Section 3.1).
+# ---------------------------------------------------------------------------
+
+def test_unequal_cluster_sizes_follow_each_tensors_tree():
+    r = rng(108)
+    n, d = 1000, 16
+    Q = r.standard_normal((n, d)); K = r.standard_normal((n, d))
+    hc = orc.cluster_head(Q, K, 64, seed=2, c_k=128)
+    assert hc.count_q.tolist() == [64] * 15 + [40]
+    assert hc.count_k.tolist() == [128] * 7 + [104]
+    assert hc.perm_q.shape[0] == 16 * 64 and hc.perm_k.shape[0] == 8 * 128
+    for perm in (hc.perm_q, hc.perm_k):
+        assert sorted(perm[perm >= 0].tolist()) == list(range(n))
+    # equal sizes through c_k give the default call exactly
+    a = orc.cluster_head(Q, K, 64, seed=2)
+    b = orc.cluster_head(Q, K, 64, seed=2, c_k=64)
+    np.testing.assert_array_equal(a.perm_k, b.perm_k)
+    np.testing.assert_array_equal(a.perm_q, b.perm_q)
+
+
+@pytest.mark.parametrize("compensate", [True, False])
+def test_unequal_sizes_keeping_every_key_cluster_is_dense(compensate):
+    r = rng(109)
+    n, d = 700, 16
+    Q = r.standard_normal((n, d)); K = r.standard_normal((n, d)); V = r.standard_normal((n, d))
+    hc = orc.cluster_head(Q, K, 64, seed=3, c_k=128)
+    S = orc.centroid_scores(hc.qbar, hc.kbar)
+    assert S.shape == (11, 6)
+    kept = orc.topk_route(S, 6)
+    O = orc.compensated_attention(Q, K, V, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, 64,
+                                  compensate=compensate, c_k=128)
+    assert np.abs(O - orc.dense_attention(Q, K, V)).max() < 1e-12
+
+
+def test_unequal_sizes_cluster_constant_keys_make_compensation_exact():
+    # 8 key components x 128 identical keys (and values), queries free: with
+    # c_k = 128 the key clusters are the components, so every excluded key
+    # cluster is represented exactly by |b| e^{q . k_bar / sqrt(d)} v_bar, for
+    # every k, while the queries are split at c_q = 64.
+    r = rng(110)
+    d = 16
+    mu_k = r.standard_normal((8, d)); mu_v = r.standard_normal((8, d))
+    z = np.repeat(np.arange(8), 128); z = z[r.permutation(z.size)]
+    K, V = mu_k[z], mu_v[z]
+    Q = r.standard_normal((z.size, d))
+    hc = orc.cluster_head(Q, K, 64, seed=4, c_k=128)
+    for b in range(8):
+        assert len(set(z[hc.perm_k[b * 128:(b + 1) * 128]])) == 1
+    assert hc.count_q.tolist() == [64] * 16
+    dense = orc.dense_attention(Q, K, V)
+    S = orc.centroid_scores(hc.qbar, hc.kbar)
+    for k in (1, 3, 8):
+        kept = orc.topk_route(S, k)
+        O = orc.compensated_attention(Q, K, V, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, 64, c_k=128)
+        assert np.abs(O - dense).max() < 1e-12
+        # the key slots read with the query size would be wrong
+        if k < 8:
+            bad = orc.compensated_attention(Q, K, V, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, 64)
+            assert np.abs(bad - dense).max() > 1e-3
