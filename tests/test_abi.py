@@ -114,3 +114,11 @@ def test_calls_are_rejected_before_launch(lib):
     s96 = ca.make_shape(1, 1, 1024, 1024, 96, 64, ca.CA_FP32)
     assert lib.ca_dense_attend(_fake(A), _fake(A), _fake(A), ctypes.byref(s96), _fake(A), None, 0,
                                None) == ca.CA_ERR_UNSUPPORTED
+
+
+def test_noalloc_scratch_covers_its_stated_examples(lib):
+    # the allocation-free clustering entry promises room for two 65,536-token
+    # heads at d = 64 or one 75,600-token head at d = 128 in its 16 MiB
+    for args in ((1, 2, 65536, 65536, 64, 128), (1, 1, 76800, 75600, 128, 128)):
+        s = ca.make_shape(*args, ca.CA_BF16)
+        assert 0 < ca.cluster_workspace_bytes(s) <= 16 << 20
