@@ -30,7 +30,7 @@ What is computed, per head (Section 3.1 "Overview"; later revision Section 4):
     mean-compensation of every excluded cluster (eq. 21-22, Appendix A);
  7. dense attention softmax(Q K^T / sqrt(d)) V (eq. 1).
 
-Readings where the paper leaves a step open (each is listed in the design doc):
+Readings where the paper leaves a step open:
  * sample: a systematic sample p_j = floor((j |S| + r) / m), j < m, with the
    offset r drawn by the counter-based generator below; all of S if |S| <= m;
  * power iteration count p = 8 (not stated in the paper);
