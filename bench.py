@@ -367,7 +367,7 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     value = whole_job_value(world, args.steps, total_ms)
 
-    # Dense attention (this build's own kernel) on the same inputs, for the speedup.
+    # Dense attention (this library's own kernel) on the same inputs, for the speedup.
     Od = torch.empty_like(Q)
     layer.dense(Q, K, V, Od)
     torch.cuda.synchronize()

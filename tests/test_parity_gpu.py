@@ -1,6 +1,6 @@
 """GPU path vs the fp64 oracle, element by element, through the C ABI.
 
-Bar (from the task definition of this path):
+Bar:
  * cluster sizes and the partition: bit-exact;
  * routing masks: bit-exact given the oracle's centroids;
  * attention output given the oracle's permutation, mask and centroids:
