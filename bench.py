@@ -35,23 +35,32 @@ UNIT = "layer-fwd/s"
 CONFIG_ID = 2
 
 
-# DRAM traffic (read + write bytes) of one attention-kernel launch on this
-# workload, from the ncu capture summarised in
-# profiles/tc_attend_kernel_64_128_layer_B1_H8_N65536.md. It describes the
-# kernel source whose SHA-256 starts with `source_sha256`; for any other source
-# the bench reports null.
-ATTN_TRAFFIC = {"bytes": 205780992 + 52542720, "source_sha256": "7644549fa28628af"}
+# Figures taken from single-kernel ncu captures of the attention kernel
+# (`ncu --set full --clock-control none -k regex:tc_attend -s 1 -c 1` around
+# `python bench.py --steps 1 --warmup 3 --no-cpu-baseline [--config N]`):
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) and tensor-pipe
+# activity of one launch. Each entry holds for the attention source whose
+# SHA-256 starts with `sha` and the workload it names; for any other source
+# or workload the bench reports null.
+ATTN_CAPTURES = []
 
 
-def attention_traffic():
+def _attn_source_sha():
     import hashlib
     src = os.path.join(ROOT, "free_clustered_block_b200", "csrc", "attend_tc.cu")
     try:
         with open(src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()
+            return hashlib.sha256(f.read()).hexdigest()
     except OSError:
-        return None
-    return ATTN_TRAFFIC["bytes"] if h.startswith(ATTN_TRAFFIC["source_sha256"]) else None
+        return ""
+
+
+def attention_capture(workload_name):
+    h = _attn_source_sha()
+    for c in ATTN_CAPTURES:
+        if h.startswith(c["sha"]) and c["workload"] == workload_name:
+            return c
+    return None
 
 
 def peaks():
@@ -107,18 +116,48 @@ def attention_flops(w, kept_counts=None, count_q=None):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks and throttle reasons sampled while the timed region runs: a
+    thread reads them through NVML every 10 ms (read-only queries); without
+    NVML, nvidia-smi every 200 ms."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.thread = None
+        self.samples = []
+
+    def _nvml_loop(self, nvml, handle):
+        while not self.stop:
+            try:
+                sm = nvml.nvmlDeviceGetClockInfo(handle, nvml.NVML_CLOCK_SM)
+                mx = nvml.nvmlDeviceGetMaxClockInfo(handle, nvml.NVML_CLOCK_SM)
+                rs = nvml.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((float(sm), float(mx), int(rs)))
+            except Exception:
+                pass
+            time.sleep(0.01)
 
     def __enter__(self):
+        import threading
+        self.stop = False
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+            import pynvml as nvml
+            nvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.gpu]) if vis and vis.split(",")[0].isdigit() else self.gpu
+            handle = nvml.nvmlDeviceGetHandleByIndex(idx)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nvml, handle), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
+        fields = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
                                           "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except OSError:
@@ -126,7 +165,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        self.lines = []
+        self.stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -134,25 +175,28 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for l in out.splitlines():
+                parts = [p.strip() for p in l.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, mx = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                rs = 0
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        rs |= self.REASONS[nm]
+                self.samples.append((sm, mx, rs))
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            parts = [p.strip() for p in l.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted(nm for nm, bit in self.REASONS.items() if any(r & bit for _, _, r in self.samples))
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples), "sm_max_mhz": self.samples[-1][1],
+                "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml every 10 ms" if self.thread is not None else "nvidia-smi every 200 ms"}
 
 
 def blas_threads():
@@ -254,7 +298,8 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(workload_config(w), selection=args.selection, clustering=args.clustering,
                        **({"recall": args.recall, "min_count": 16} if args.selection == "adaptive" else {})),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": affinity_cores(), "blas_threads": blas_threads(),
+                         "kind": "oracle",
                          "sample": f"per step: head 0 clustered and routed in full, attention of 48 of "
                                    f"{w.C} query clusters; extrapolated to {w.H} heads x {w.C} clusters"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -284,13 +329,200 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def cluster_levels(ca, shape):
+    """Levels of the split tree (the clustering launches 6 + 5 per level)."""
+    n = ca.launch_count(shape, 0)
+    return max(0, (n - 6) // 5)
+
+
+def cluster_row_bytes(w, levels):
+    """Algorithmic HBM bytes of the clustering stage: at every level of the
+    split tree both tensors' rows are read once for the projections
+    (2 x B x H x n x d x element size per level)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    return float(levels) * 2 * w.B * w.H * w.n_valid * w.d * esz
+
+
+def affinity_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def make_layer(ca, w, args):
+    adaptive = args.selection == "adaptive"
+    return ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.C if adaptive else w.k,
+                               dtype=w.dtype, compensate=w.compensate, selection=args.selection,
+                               recall=args.recall, min_count=16, clustering=args.clustering)
+
+
+def time_layer(ca, torch, w, layer, Q, K, V, O, steps, warmup, barrier, local, sample_clocks=True):
+    """Warm up, then time `steps` layer forwards with CUDA events on the
+    launching stream: per step the clustering, the routing, the attention's
+    preparation and the attention kernel (ca_attend_prepared) separately.
+    Returns (total ms, per-stage mean ms, clock summary)."""
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.cluster(Q, K)
+        layer.route()
+        layer.attend_prepare(Q, K, V)
+        layer.attend_prepared(Q, K, V, O)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    st = ca.ca_get_device_error()
+    if st != ca.CA_OK:
+        raise RuntimeError(f"device error after warm-up: {ca.status_string(st)}")
+    flush = needs_flush(w)
+    scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda") if flush else None
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local) if sample_clocks else None
+    if clk:
+        clk.__enter__()
+    try:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(steps):
+            if flush:
+                scrub.zero_()
+            ev[i][0].record(stream)
+            layer.cluster(Q, K)
+            ev[i][1].record(stream)
+            layer.route()
+            ev[i][2].record(stream)
+            layer.attend_prepare(Q, K, V)
+            ev[i][3].record(stream)
+            layer.attend_prepared(Q, K, V, O)
+            ev[i][4].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    finally:
+        if clk:
+            clk.__exit__(None, None, None)
+    st = ca.ca_get_device_error()
+    if st != ca.CA_OK:
+        raise RuntimeError(f"device error in the timed region: {ca.status_string(st)}")
+    # with flushes, the steps are timed one by one (the flushes are not timed)
+    total_ms = (sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(steps)) if flush
+                else start.elapsed_time(end))
+    names = ("cluster", "route", "attend_prep", "attend_kernel")
+    stage = {nm: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps))
+             for j, nm in enumerate(names)}
+    stage["attend"] = stage["attend_prep"] + stage["attend_kernel"]
+    return total_ms, stage, (clk.summary() if clk else None)
+
+
+def time_dense(torch, layer, Q, K, V, iters):
+    stream = torch.cuda.current_stream()
+    Od = torch.empty_like(Q)
+    layer.dense(Q, K, V, Od)
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(iters):
+        layer.dense(Q, K, V, Od)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    return d0.elapsed_time(d1) / iters
+
+
+def rooflines(ca, w, layer, stage, dense_ms, adaptive):
+    """Attention kernel (tensor pipe, its own event time, burst peak: the
+    timed region is short), dense kernel (same), clustering stage (HBM)."""
+    pk = peaks()
+    if adaptive:
+        kc = layer.buf.kept_count.cpu().numpy()
+        kept_f, smc_f = attention_flops(w, kc, layer.buf.count_q.cpu().numpy())
+    else:
+        kept_f, smc_f = attention_flops(w)
+    attn_s = stage["attend_kernel"] / 1e3
+    achieved = (kept_f + smc_f) / attn_s / 1e12
+    cap = attention_capture(w.name)
+    if w.dtype == "bf16":
+        roof = {"kernel": f"tc_attend_kernel<{w.d}> (ca_attend_prepared: the attention kernel"
+                          f"{' + padding-row zeroing' if w.N_alloc > w.n_valid else ''})",
+                "bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16"],
+                "peak_source": f"bf16 dense burst (cuBLAS), {pk['source']}",
+                "traffic": cap["traffic"] if cap else None,
+                "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                "tensor_pipe_pct": cap["tensor_pipe_pct"] if cap else None,
+                "algorithmic_flops": kept_f + smc_f, "kernel_ms": stage["attend_kernel"]}
+        dflops = dense_flops(w)
+        dense_roof = {"kernel": f"tc_attend_kernel<{w.d}> dense mode", "bound": "tensor",
+                      "achieved": dflops / (dense_ms / 1e3) / 1e12, "peak": pk["bf16"], "unit": "TFLOP/s",
+                      "frac": dflops / (dense_ms / 1e3) / 1e12 / pk["bf16"],
+                      "peak_source": f"bf16 dense burst (cuBLAS), {pk['source']}"}
+    else:
+        # fp32 inputs run the SIMT attention kernel on the FMA pipe: peak from
+        # 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
+        fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"kernel": "simt_attend_kernel (ca_attend_prepared)", "bound": "alu", "achieved": achieved,
+                "peak": fp32_peak, "unit": "TFLOP/s", "frac": achieved / fp32_peak, "traffic": None,
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                "algorithmic_flops": kept_f + smc_f, "kernel_ms": stage["attend_kernel"]}
+        dense_roof = None
+    levels = cluster_levels(ca, layer.shape)
+    cbytes = cluster_row_bytes(w, levels)
+    gbs = cbytes / (stage["cluster"] / 1e3) / 1e9
+    cluster_roof = {"stage": "clustering (ca_cluster)", "bound": "hbm", "levels": levels,
+                    "algorithmic_bytes": cbytes, "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                    "frac": gbs / pk["hbm"],
+                    "definition": "per level, both tensors' rows read once: levels x 2 x B x H x n x d x bytes"}
+    return roof, dense_roof, cluster_roof, (kept_f, smc_f)
+
+
+def run_sweep(args):
+    """Configuration 5: latency and error against dense attention over cluster
+    size, keep fraction and compensation (one JSON line per point)."""
+    import numpy as np
+    import torch
+    import free_clustered_block_b200 as ca
+    import workloads as wl
+    torch.cuda.set_device(0)
+    no_barrier = (lambda: None)
+    for d in (64, 128):
+        for c in (64, 128, 256):
+            for keep in (1 / 32, 1 / 8, 1 / 4, 1.0):
+                for smc in (True, False):
+                    w = wl.config_workload(5, d=d, c=c, keep=keep, compensate=smc)
+                    Q, K, V = (torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+                               .cuda().contiguous() for x in (w.Q, w.K, w.V))
+                    O = torch.empty_like(Q)
+                    layer = make_layer(ca, w, args)
+                    total_ms, stage, _ = time_layer(ca, torch, w, layer, Q, K, V, O, args.steps, args.warmup,
+                                                    no_barrier, 0, sample_clocks=False)
+                    ms = total_ms / args.steps
+                    dense_ms = time_dense(torch, layer, Q, K, V, 3)
+                    roof, dense_roof, cluster_roof, _ = rooflines(ca, w, layer, stage, dense_ms, False)
+                    line = {"sweep": "config 5", "config": workload_config(w), "keep": keep,
+                            "latency_ms": ms, "stage_ms": stage, "dense_ms": dense_ms,
+                            "speedup_vs_dense": dense_ms / ms,
+                            "attention_frac": roof["frac"], "dense_frac": dense_roof["frac"],
+                            "cluster_hbm_frac": cluster_roof["frac"]}
+                    if not args.no_cpu_baseline:
+                        kept = {}
+                        oracle_sample(w, n_clusters=8, keep=kept)
+                        line["error_vs_dense_fp64"] = error_vs_dense(w, O[0, kept["head"]].float().cpu().numpy(),
+                                                                     kept)
+                    print(json.dumps(line), flush=True)
+                    del layer, Q, K, V, O
+                    torch.cuda.empty_cache()
+    return 0
+
+
 def run_ours(args):
     import numpy as np
     import torch
     import torch.distributed as dist
 
     import free_clustered_block_b200 as ca
-    import workloads as wl
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -317,68 +549,16 @@ def run_ours(args):
     Q, K, V = dev(w.Q), dev(w.K), dev(w.V)
     O = torch.empty_like(Q)
     adaptive = args.selection == "adaptive"
-    layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.C if adaptive else w.k,
-                                dtype=w.dtype, compensate=w.compensate, selection=args.selection,
-                                recall=args.recall, min_count=16, clustering=args.clustering)
+    layer = make_layer(ca, w, args)
     stream = torch.cuda.current_stream()
 
-    def step():
-        layer.cluster(Q, K)
-        layer.route()
-        layer.attend(Q, K, V, O)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    st = ca.ca_get_device_error()
-    if st != ca.CA_OK:
-        raise RuntimeError(f"device error after warm-up: {ca.status_string(st)}")
-
-    flush = needs_flush(w)
-    scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device="cuda") if flush else None
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        start.record(stream)
-        for i in range(args.steps):
-            if flush:
-                scrub.zero_()
-            ev[i][0].record(stream)
-            layer.cluster(Q, K)
-            ev[i][1].record(stream)
-            layer.route()
-            ev[i][2].record(stream)
-            layer.attend(Q, K, V, O)
-            ev[i][3].record(stream)
-        end.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    st = ca.ca_get_device_error()
-    if st != ca.CA_OK:
-        raise RuntimeError(f"device error in the timed region: {ca.status_string(st)}")
-    # with flushes, the steps are timed one by one (the flushes are not timed)
-    total_ms = ranks_max(sum(ev[i][0].elapsed_time(ev[i][3]) for i in range(args.steps)) if flush
-                         else start.elapsed_time(end))
-    clocks = clk.summary()
-    stage = {name: statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps))
-             for j, name in enumerate(("cluster", "route", "attend"))}
+    local_ms, stage, clocks = time_layer(ca, torch, w, layer, Q, K, V, O, args.steps, args.warmup, barrier, local)
+    total_ms = ranks_max(local_ms)
     ms_per_step = total_ms / args.steps
     value = whole_job_value(world, args.steps, total_ms)
 
     # Dense attention (this library's own kernel) on the same inputs, for the speedup.
-    Od = torch.empty_like(Q)
-    layer.dense(Q, K, V, Od)
-    torch.cuda.synchronize()
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dense_iters = max(1, min(args.steps, 3))
-    d0.record(stream)
-    for _ in range(dense_iters):
-        layer.dense(Q, K, V, Od)
-    d1.record(stream)
-    torch.cuda.synchronize()
-    dense_ms = ranks_max(d0.elapsed_time(d1) / dense_iters)
+    dense_ms = ranks_max(time_dense(torch, layer, Q, K, V, max(1, min(args.steps, 3))))
 
     # End to end with host buffers (pinned), copies inside the region: the
     # single ca_forward_host call for top-k; the layer API (copy in, cluster,
@@ -419,11 +599,11 @@ def run_ours(args):
         gstream = torch.cuda.Stream()
         gstream.wait_stream(stream)
         with torch.cuda.stream(gstream):
-            step()
+            layer(Q, K, V, O)
         gstream.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=gstream):
-            step()
+            layer(Q, K, V, O)
         graph.replay()
         torch.cuda.synchronize()
         g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -437,30 +617,8 @@ def run_ours(args):
     except Exception as e:  # capture is an extra figure; the timed line above stands
         graph_ms = f"capture failed: {type(e).__name__}"
 
-    pk = peaks()
-    if adaptive:
-        kc = layer.buf.kept_count.cpu().numpy()
-        kept_f, smc_f = attention_flops(w, kc, layer.buf.count_q.cpu().numpy())
-    else:
-        kept_f, smc_f = attention_flops(w)
-    attn_s = stage["attend"] / 1e3
-    achieved = (kept_f + smc_f) / attn_s / 1e12
-    if w.dtype == "bf16":
-        roof = {"kernel": "attention (ca_attend span: prep + attention)", "bound": "tensor",
-                "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_sus"],
-                "traffic": attention_traffic() if args.config == CONFIG_ID else None,
-                "traffic_unit": "bytes per launch (ncu dram__bytes_read + dram__bytes_write)",
-                "peak_source": f"bf16 dense sustained, {pk['source']}",
-                "algorithmic_flops": kept_f + smc_f}
-    else:
-        # fp32 inputs run the SIMT attention kernel on the FMA pipe: peak from
-        # 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
-        fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
-        roof = {"kernel": "attention (ca_attend span: prep + attention)", "bound": "alu",
-                "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s", "frac": achieved / fp32_peak,
-                "traffic": None, "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
-                "algorithmic_flops": kept_f + smc_f}
+    roof, dense_roof, cluster_roof, (kept_f, smc_f) = rooflines(ca, w, layer, stage, dense_ms, adaptive)
+    kc = layer.buf.kept_count.cpu().numpy() if adaptive else None
     per_step = [ca.launch_count(shape, s) for s in (0, 1, 2)]
     if args.clustering == "random" and per_step[0] > 1:
         # no metric, norm or direction kernels: plan, per level hash / select /
@@ -485,8 +643,10 @@ def run_ours(args):
         "speedup_vs_dense": dense_ms / ms_per_step,
         "graph_ms_per_step": graph_ms,
         "tflops": {"dense_equivalent": dense_flops(w) / (ms_per_step / 1e3) / 1e12,
-                   "algorithmic_attention": achieved},
+                   "algorithmic_attention": roof["achieved"]},
         "roofline": roof,
+        "dense_roofline": dense_roof,
+        "cluster_roofline": cluster_roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": out_bytes, "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": launches,
@@ -497,7 +657,8 @@ def run_ours(args):
         t_cpu, smp = oracle_sample(w, keep=kept, selection=args.selection, recall=args.recall,
                                    clustering=args.clustering)
         line["error_vs_dense_fp64"] = error_vs_dense(w, O[0, kept["head"]].float().cpu().numpy(), kept)
-        line["cpu_baseline"] = {"value": 1.0 / t_cpu, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": 1.0 / t_cpu, "unit": UNIT, "cores": affinity_cores(),
+                                "blas_threads": blas_threads(), "kind": "oracle",
                                 "sample": f"head 0 clustered and routed in full, attention of 48 of {w.C} query "
                                           f"clusters; extrapolated to {w.H} heads x {w.C} clusters "
                                           f"({t_cpu:.1f} s per layer)"}
@@ -525,11 +686,14 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="latency scaling: configuration 2's generator at this token count")
     ap.add_argument("--fixed-k", action="store_true", help="with --tokens: keep 64 clusters instead of 1/8")
-    ap.add_argument("--config", type=int, choices=[1, 2, 3, 4], default=CONFIG_ID,
-                    help="workload (default 2: the metric's N = 64k configuration)")
+    ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=CONFIG_ID,
+                    help="workload (default 2: the metric's N = 64k configuration); 5: the sweep over cluster "
+                         "size, keep fraction and compensation at N = 32,768, one JSON line per point")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.config == 5:
+        return run_sweep(args)
     return run_ours(args)
 
 

@@ -27,7 +27,8 @@ EXPORTED = [
     "ca_dense_workspace_bytes", "ca_forward_workspace_bytes", "ca_cluster", "ca_route", "ca_attend",
     "ca_dense_attend", "ca_forward", "ca_forward_host_workspace_bytes", "ca_forward_host",
     "ca_get_device_error", "ca_set_wait_limit", "ca_check_bounded_wait", "ca_status_string", "ca_version", "ca_launch_count",
-    "ca_cluster_noalloc", "ca_route_adaptive",
+    "ca_cluster_noalloc", "ca_route_adaptive", "ca_check_exp2_poly",
+    "ca_attend_prepare", "ca_attend_prepared",
 ]
 
 
@@ -90,13 +91,17 @@ def lib():
             "ca_forward_host_workspace_bytes": (sz, [P(ca_shape), i32]),
             "ca_forward_host": (i32, [vp, vp, vp, P(ca_shape), P(ca_cluster_params), i32, i32, vp, vp, sz, vp]),
             "ca_get_device_error": (i32, [vp]),
-            "ca_set_wait_limit": (None, [u64]),
+            "ca_set_wait_limit": (i32, [u64]),
             "ca_check_bounded_wait": (i32, [u64, i32, vp]),
             "ca_status_string": (ctypes.c_char_p, [i32]),
             "ca_version": (ctypes.c_char_p, []),
             "ca_launch_count": (i32, [P(ca_shape), i32]),
             "ca_cluster_noalloc": (i32, [vp, vp, P(ca_shape), P(ca_cluster_params), P(ca_clusters), vp]),
             "ca_route_adaptive": (i32, [P(ca_shape), P(ca_clusters), ctypes.c_double, i32, P(ca_routes), vp]),
+            "ca_check_exp2_poly": (i32, [vp, vp, i32, vp]),
+            "ca_attend_prepare": (i32, [vp, vp, vp, P(ca_shape), P(ca_clusters), vp, sz, vp]),
+            "ca_attend_prepared": (i32, [vp, vp, vp, P(ca_shape), P(ca_clusters), P(ca_routes), i32, vp, vp, sz,
+                                         vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -213,6 +218,24 @@ def ca_attend(Q, K, V, shape: ca_shape, clusters: ca_clusters, routes: ca_routes
     _check(st, "ca_attend")
 
 
+def ca_attend_prepare(Q, K, V, shape: ca_shape, clusters: ca_clusters, workspace, stream=None):
+    """First half of ca_attend: value centroids and the cluster-ordered copies into the workspace."""
+    st = lib().ca_attend_prepare(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), ctypes.byref(clusters),
+                                 _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(st, "ca_attend_prepare")
+
+
+def ca_attend_prepared(Q, K, V, shape: ca_shape, clusters: ca_clusters, routes: ca_routes, compensate: bool, O,
+                       workspace, stream=None):
+    """Second half of ca_attend: the attention kernel, from a prepared workspace."""
+    st = lib().ca_attend_prepared(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), ctypes.byref(clusters),
+                                  ctypes.byref(routes), int(bool(compensate)), _ptr(O), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                  _stream(stream))
+    _check(st, "ca_attend_prepared")
+
+
 def ca_dense_attend(Q, K, V, shape: ca_shape, O, workspace=None, stream=None):
     st = lib().ca_dense_attend(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shape), _ptr(O), _ptr(workspace),
                                0 if workspace is None else workspace.numel() * workspace.element_size(),
@@ -244,11 +267,16 @@ def ca_get_device_error(stream=None) -> int:
 
 
 def ca_set_wait_limit(limit_ns: int):
-    lib().ca_set_wait_limit(limit_ns)
+    _check(lib().ca_set_wait_limit(limit_ns), "ca_set_wait_limit")
 
 
 def ca_check_bounded_wait(limit_ns: int, arrive: bool, stream=None) -> int:
     return lib().ca_check_bounded_wait(limit_ns, 1 if arrive else 0, _stream(stream))
+
+
+def ca_check_exp2_poly(x, y, stream=None):
+    """y[i] = the attention kernel's FMA-pipe evaluation of 2^x[i] (device fp32 tensors)."""
+    _check(lib().ca_check_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)), "ca_check_exp2_poly")
 
 
 def launch_count(shape: ca_shape, stage: int) -> int:

@@ -8,8 +8,6 @@
 
 namespace ca {
 size_t route_smem_bytes(int C, int D);
-cudaError_t device_error_read_clear(unsigned* out, cudaStream_t st);
-void set_wait_limit(uint64_t spins);
 }  // namespace ca
 
 using namespace ca;
@@ -17,7 +15,8 @@ using namespace ca;
 namespace {
 
 constexpr int kMaxRouteC = 8192;
-constexpr int kMaxCompensatedC = 8192;
+// Longest accepted limit of a bounded device-side wait.
+constexpr uint64_t kMaxWaitLimitNs = 10000000000ull;   // 10 s
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -183,32 +182,70 @@ ca_status ca_route_adaptive(const ca_shape* s, const ca_clusters* cen, double re
                                            static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+
+// Checks shared by ca_attend and its two halves.
+ca_status check_attend(const void* Q, const void* K, const void* V, const ca_shape* s, const ca_clusters* cl,
+                       const ca_routes* rt, const void* O, size_t workspace_bytes, const void* workspace,
+                       AttendWs* L) {
+  ca_status st = check_shape(s);
+  if (st != CA_OK) return st;
+  if (!Q || !K || !V || !cl || !cl->perm_q || !cl->perm_k || !cl->count_k || !cl->kbar) return CA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return CA_ERR_INVALID_ARG;
+  if (rt) {
+    if (!O || !rt->kept_idx || !rt->kept_bits || !aligned16(O)) return CA_ERR_INVALID_ARG;
+    const int C = (s->n_valid + s->c - 1) / s->c;
+    if (rt->k < 1 || rt->k > C) return CA_ERR_INVALID_ARG;
+  }
+  attend_ws_layout(s, L);
+  if (workspace_bytes < L->total) return CA_ERR_WORKSPACE;
+  if (!workspace) return CA_ERR_INVALID_ARG;
+  return CA_OK;
+}
+
+cudaError_t attend_blocks(const void* Q, const void* K, const void* V, const ca_shape* s, const ca_clusters* cl,
+                          const ca_routes* rt, int compensate, void* O, const AttendWs& L, char* ws,
+                          cudaStream_t cs) {
+  cudaError_t e = (s->dtype == CA_BF16) ? launch_attend_tc(s, cl, rt, compensate, O, L, ws, cs)
+                                        : launch_attend_simt(Q, K, V, s, cl, rt, compensate, O, L, ws, cs);
+  if (e == cudaSuccess) e = launch_zero_pad_rows(O, s, cs);
+  return e;
+}
+
+}  // namespace
+
 ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* s, const ca_clusters* cl,
                     const ca_routes* rt, int compensate, void* O, void* workspace, size_t workspace_bytes,
                     void* stream) {
-  ca_status st = check_shape(s);
-  if (st != CA_OK) return st;
-  if (!Q || !K || !V || !O || !cl || !rt || !cl->perm_q || !cl->perm_k || !cl->count_k || !cl->kbar ||
-      !rt->kept_idx || !rt->kept_bits)
-    return CA_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return CA_ERR_INVALID_ARG;
-  const int C = (s->n_valid + s->c - 1) / s->c;
-  if (rt->k < 1 || rt->k > C) return CA_ERR_INVALID_ARG;
-  // the bf16 kernel keeps one compensation bias per key cluster on chip
-  if (compensate && s->dtype == CA_BF16 && C > kMaxCompensatedC) return CA_ERR_UNSUPPORTED;
+  if (!rt) return CA_ERR_INVALID_ARG;
   AttendWs L;
-  attend_ws_layout(s, &L);
-  if (workspace_bytes < L.total) return CA_ERR_WORKSPACE;
-  if (!workspace) return CA_ERR_INVALID_ARG;
+  ca_status st = check_attend(Q, K, V, s, cl, rt, O, workspace_bytes, workspace, &L);
+  if (st != CA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   cudaError_t e = launch_attend_prep(Q, K, V, s, cl, L, ws, cs);
-  if (e == cudaSuccess) {
-    if (s->dtype == CA_BF16) e = launch_attend_tc(s, cl, rt, compensate, O, L, ws, cs);
-    else e = launch_attend_simt(Q, K, V, s, cl, rt, compensate, O, L, ws, cs);
-  }
-  if (e == cudaSuccess) e = launch_zero_pad_rows(O, s, cs);
+  if (e == cudaSuccess) e = attend_blocks(Q, K, V, s, cl, rt, compensate, O, L, ws, cs);
   return cuda_status(e);
+}
+
+ca_status ca_attend_prepare(const void* Q, const void* K, const void* V, const ca_shape* s,
+                            const ca_clusters* cl, void* workspace, size_t workspace_bytes, void* stream) {
+  AttendWs L;
+  ca_status st = check_attend(Q, K, V, s, cl, nullptr, nullptr, workspace_bytes, workspace, &L);
+  if (st != CA_OK) return st;
+  return cuda_status(launch_attend_prep(Q, K, V, s, cl, L, static_cast<char*>(workspace),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+ca_status ca_attend_prepared(const void* Q, const void* K, const void* V, const ca_shape* s,
+                             const ca_clusters* cl, const ca_routes* rt, int compensate, void* O,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (!rt) return CA_ERR_INVALID_ARG;
+  AttendWs L;
+  ca_status st = check_attend(Q, K, V, s, cl, rt, O, workspace_bytes, workspace, &L);
+  if (st != CA_OK) return st;
+  return cuda_status(attend_blocks(Q, K, V, s, cl, rt, compensate, O, L, static_cast<char*>(workspace),
+                                   static_cast<cudaStream_t>(stream)));
 }
 
 ca_status ca_dense_attend(const void* Q, const void* K, const void* V, const ca_shape* s, void* O,
@@ -308,11 +345,22 @@ ca_status ca_get_device_error(void* stream) {
   return word ? static_cast<ca_status>(word) : CA_OK;
 }
 
-void ca_set_wait_limit(uint64_t spins) { set_wait_limit(spins); }
+ca_status ca_set_wait_limit(uint64_t limit_ns) {
+  if (limit_ns > kMaxWaitLimitNs) return CA_ERR_INVALID_ARG;
+  set_wait_limit(limit_ns);
+  return CA_OK;
+}
 
 ca_status ca_check_bounded_wait(uint64_t limit_ns, int arrive, void* stream) {
-  if (limit_ns == 0 || limit_ns > 10000000000ull) return CA_ERR_INVALID_ARG;
+  if (limit_ns == 0 || limit_ns > kMaxWaitLimitNs) return CA_ERR_INVALID_ARG;
   return cuda_status(launch_bounded_wait_check(limit_ns, arrive ? 1 : 0, static_cast<cudaStream_t>(stream)));
+}
+
+ca_status ca_check_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0) return CA_ERR_INVALID_ARG;
+  if (n == 0) return CA_OK;   // nothing is read or written
+  if (!x || !y) return CA_ERR_INVALID_ARG;
+  return cuda_status(launch_exp2_poly_check(x, y, n, static_cast<cudaStream_t>(stream)));
 }
 
 int ca_launch_count(const ca_shape* s, int stage) {

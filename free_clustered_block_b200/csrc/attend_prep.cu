@@ -20,21 +20,25 @@ template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v
 }
 
 // One block per key cluster: vbar (fp64 mean of the members' values), and the
-// fp32 / bf16 hi-lo forms of kbar and vbar; log count.
+// fp32 / bf16 hi-lo forms of kbar and vbar; log count. The hi-lo forms are
+// laid out in blocks of 64 centroids as the tensor-core kernel loads them:
+// block cb holds the hi parts of centroids 64 cb .. 64 cb + 63 in rows 0-63
+// and their lo parts in rows 64-127 ([BH][Cpad / 64][128][D]).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) centroid_prep_kernel(
     const T* __restrict__ V, int N_alloc, int c, int C, int Cpad, const int32_t* __restrict__ perm_k,
     const int32_t* __restrict__ count_k, const double* __restrict__ kbar, float* __restrict__ kbar32,
-    float* __restrict__ vbar32, __nv_bfloat16* __restrict__ kbar_hi, __nv_bfloat16* __restrict__ kbar_lo,
-    __nv_bfloat16* __restrict__ vbar_hi, __nv_bfloat16* __restrict__ vbar_lo, float* __restrict__ logcnt) {
+    float* __restrict__ vbar32, __nv_bfloat16* __restrict__ kbar_hl, __nv_bfloat16* __restrict__ vbar_hl,
+    float* __restrict__ logcnt) {
   constexpr int RG = 256 / D;
   const int b = blockIdx.x, bh = blockIdx.y;
   const int col = threadIdx.x % D, rg = threadIdx.x / D;
-  const size_t o_pad = ((size_t)bh * Cpad + b) * D + col;
+  const size_t o_hi = (((size_t)bh * (Cpad / 64) + b / 64) * 128 + (b % 64)) * D + col;
+  const size_t o_lo = o_hi + (size_t)64 * D;
   if (b >= C) {   // padding centroids of the tensor-core tiles
     if (rg == 0) {
       const __nv_bfloat16 z = __float2bfloat16(0.f);
-      kbar_hi[o_pad] = z; kbar_lo[o_pad] = z; vbar_hi[o_pad] = z; vbar_lo[o_pad] = z;
+      kbar_hl[o_hi] = z; kbar_hl[o_lo] = z; vbar_hl[o_hi] = z; vbar_hl[o_lo] = z;
       if (col == 0) logcnt[(size_t)bh * Cpad + b] = -INFINITY;
     }
     return;
@@ -57,8 +61,8 @@ __global__ void __launch_bounds__(256) centroid_prep_kernel(
     kbar32[o32] = (float)kb;
     const __nv_bfloat16 khi = __double2bfloat16(kb);
     const __nv_bfloat16 vhi = __double2bfloat16(vb);
-    kbar_hi[o_pad] = khi; kbar_lo[o_pad] = __double2bfloat16(kb - (double)__bfloat162float(khi));
-    vbar_hi[o_pad] = vhi; vbar_lo[o_pad] = __double2bfloat16(vb - (double)__bfloat162float(vhi));
+    kbar_hl[o_hi] = khi; kbar_hl[o_lo] = __double2bfloat16(kb - (double)__bfloat162float(khi));
+    vbar_hl[o_hi] = vhi; vbar_hl[o_lo] = __double2bfloat16(vb - (double)__bfloat162float(vhi));
     if (col == 0) logcnt[(size_t)bh * Cpad + b] = logf((float)cnt);
   }
 }
@@ -109,10 +113,8 @@ bool attend_ws_layout(const ca_shape* s, AttendWs* w) {
   w->qp = take(tc ? rows : 0);
   w->kp = take(tc ? rows : 0);
   w->vp = take(tc ? rows : 0);
-  w->kbar_hi = take(BH * Cpad * d * 2);
-  w->kbar_lo = take(BH * Cpad * d * 2);
-  w->vbar_hi = take(BH * Cpad * d * 2);
-  w->vbar_lo = take(BH * Cpad * d * 2);
+  w->kbar_hl = take(BH * Cpad * 2 * d * 2);
+  w->vbar_hl = take(BH * Cpad * 2 * d * 2);
   w->vbar32 = take(BH * C * d * 4);
   w->kbar32 = take(BH * C * d * 4);
   w->logcnt = take(BH * Cpad * 4);
@@ -125,22 +127,18 @@ cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, cons
   const int BH = s->B * s->H, C = L.C, Cpad = L.Cpad, c = s->c;
   float* kbar32 = reinterpret_cast<float*>(ws + L.kbar32);
   float* vbar32 = reinterpret_cast<float*>(ws + L.vbar32);
-  __nv_bfloat16* khi = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_hi);
-  __nv_bfloat16* klo = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_lo);
-  __nv_bfloat16* vhi = reinterpret_cast<__nv_bfloat16*>(ws + L.vbar_hi);
-  __nv_bfloat16* vlo = reinterpret_cast<__nv_bfloat16*>(ws + L.vbar_lo);
+  __nv_bfloat16* khl = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_hl);
+  __nv_bfloat16* vhl = reinterpret_cast<__nv_bfloat16*>(ws + L.vbar_hl);
   float* logcnt = reinterpret_cast<float*>(ws + L.logcnt);
   const dim3 g(Cpad, BH);
   if (s->dtype == CA_BF16) {
     using T = __nv_bfloat16;
     if (s->d == 64)
       centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
-                                                     cl->count_k, cl->kbar, kbar32, vbar32, khi, klo, vhi,
-                                                     vlo, logcnt);
+                                                     cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
     else
       centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
-                                                      cl->count_k, cl->kbar, kbar32, vbar32, khi, klo,
-                                                      vhi, vlo, logcnt);
+                                                      cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
     const int slots = C * c;
     const size_t vecs = (size_t)slots * (s->d * 2 / 16);
     const dim3 gp((unsigned)((vecs + 255) / 256), BH, 3);
@@ -157,12 +155,10 @@ cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, cons
     using T = float;
     if (s->d == 64)
       centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
-                                                     cl->count_k, cl->kbar, kbar32, vbar32, khi, klo, vhi,
-                                                     vlo, logcnt);
+                                                     cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
     else
       centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
-                                                      cl->count_k, cl->kbar, kbar32, vbar32, khi, klo,
-                                                      vhi, vlo, logcnt);
+                                                      cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
   }
   return cudaGetLastError();
 }

@@ -7,42 +7,57 @@
 // q . kbar_b / sqrt(d) + ln|b| and value vbar_b). The dense form (eq. 1) is
 // the same kernel with every key block kept and no compensation.
 //
-// One CTA handles one 128-row query tile of one head and holds an SM (512
-// TMEM columns: three S buffers and O):
-//   warp 0      TMA producer (one thread): Q tile once, then a ring of
-//               stages holding (K, V) of a kept key block, (kbar_hi,
-//               kbar_lo) or (vbar_hi, vbar_lo) of a centroid block;
-//   warp 1      MMA issuer (the converged warp, one elected lane issuing):
-//               S_j = Q K_j^T into TMEM buffer j % 3 and O += P_j V_j with
-//               P_j read from TMEM. S_{j+2} is issued right behind PV_j: its
-//               buffer was last read by PV_{j-1}, so the tensor pipe gets both
-//               without waiting for PV_j, and the softmax of S_{j+1} overlaps;
-//   warps 2..9  softmax, two threads per query row (one per half of the key
-//               block): read S_j from TMEM, apply the key mask /
-//               compensation bias, exchange the row max through shared
-//               memory, keep a running max (rescaling O only when the max
-//               grows by more than 2^8), write P_j as bf16 over the front of
-//               S_j, accumulate the row sums in registers, and finally write
-//               O / l to the query's original row.
-// Centroids are split into bf16 hi + lo parts and enter as two MMAs each.
+// One CTA holds an SM and works on TWO 128-row query tiles at once, so the
+// tensor core computes one tile's products while the other tile's softmax
+// runs (512 TMEM columns: S_0, S_1 of 128 columns, O_0, O_1 of d columns):
+//   warps 0-3   softmax of tile 0, one thread per query row: read the row of
+//               S_j from TMEM into registers, mask / bias it, take the row
+//               maximum, write P_j = 2^(S_j - m) as bf16 over the front of
+//               S_j, keep the row sum; rescale the row of O only when the
+//               running maximum grows by more than 2^8; finally O / l to the
+//               query's original row;
+//   warps 4-7   the same for tile 1;
+//   warp 8      TMA producer (one thread): both Q tiles once, then a ring of
+//               K slots and a ring of V slots, each slot one 128-row tile;
+//   warp 9      MMA issuer (the warp polls, one leader lane issues each
+//               group of products from precomputed descriptors):
+//               S_t = Q_t K_j^T and O_t += P_t V_j, each tile advancing on
+//               its own as soon as the operands are ready. At d = 128, S_t of
+//               block j+1 overwrites P_t of block j, so it waits for
+//               O_t += P_t V_j; at d = 64, P_t has its own TMEM columns.
+//   warps 10-11 idle.
+// A key block is 128 key slots: one or half of a kept key cluster (c = 128,
+// 256), two kept clusters of 64 (c = 64), or 128 consecutive keys (dense).
+// A compensation block is 64 key-cluster centroids: bf16 hi parts in rows
+// 0-63 of the slot and lo parts in rows 64-127, so that two N = 64 products
+// carry the fp64 centroid (~16 significant bits) into the fp32 accumulator.
+// When both tiles of a CTA attend the same key blocks (the two halves of a
+// 256-query cluster, or dense attention) each K and V tile is loaded once
+// and serves both.
 // Every wait is bounded: on a timeout the CTA sets the library's device error
 // word (CA_ERR_TIMEOUT), drains what it issued, frees TMEM and returns.
 #include <cuda.h>
+
+#include <atomic>
 
 #include "ca_internal.cuh"
 
 namespace ca {
 
+// One word per device, shared by every stream and caller of the library.
 __device__ unsigned int g_device_error = 0;
-static uint64_t g_wait_limit = 0;
 // Bounded waits are timed with the global nanosecond timer.
-constexpr uint64_t kDefaultWaitLimit = 1000000000ull;   // 1 s
+constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;   // 1 s
+static std::atomic<uint64_t> g_wait_limit_ns{0};
 // Drains (letting copies and MMAs already issued finish before the CTA
 // leaves) use their own bound, independent of the adjustable wait limit.
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
-uint64_t wait_limit() { return g_wait_limit ? g_wait_limit : kDefaultWaitLimit; }
-void set_wait_limit(uint64_t spins) { g_wait_limit = spins; }
+uint64_t wait_limit() {
+  const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return v ? v : kDefaultWaitLimitNs;
+}
+void set_wait_limit(uint64_t limit_ns) { g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed); }
 
 cudaError_t device_error_read_clear(unsigned* out, cudaStream_t st) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_device_error, sizeof(unsigned), 0,
@@ -82,6 +97,17 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe, for loops that poll several barriers (try_wait may
+// suspend the thread until the one barrier it names completes).
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
@@ -99,22 +125,32 @@ __device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, uint64
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 // tcgen05.mma (A and B from shared memory, or A from TMEM) and commit, issued
-// by one elected lane of a converged warp: the whole warp computes the
-// (warp-uniform) operands, so issue needs no divergent single-lane code.
-__device__ __forceinline__ void mma_ss_elect(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// by the calling thread alone: the MMA warp's leader lane issues whole groups
+// of products this way, with no per-product election.
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u)
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
-__device__ __forceinline__ void mma_ts_elect(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n .reg .pred p, e;\n setp.ne.b32 p, %4, 0;\n elect.sync _|e, 0xffffffff;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n}\n" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u)
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+__device__ __forceinline__ void tc_commit(uint64_t* b) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+               : "memory");
+}
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(e));
+  return e != 0;
+}
+// Commit issued by one elected lane of a converged warp.
 __device__ __forceinline__ void tc_commit_elect(uint64_t* b) {
   asm volatile(
       "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
@@ -181,16 +217,18 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// 2^t0, 2^t1 (t <= 8) on the FMA pipe, to take part of the load off the
-// MUFU ex2 unit: t = n + f with n = round(t) (adding and subtracting 1.5 * 2^23
-// leaves the rounded integer in the low mantissa bits), 2^f on [-1/2, 1/2] by
-// a cubic fitted to the least maximum relative error on that interval
-// (< 8e-5, far below the bf16 rounding of P), and n added into the exponent
-// field with one integer multiply-add. t is clamped at -126 (2^-126 is as good
-// as 0 in a bf16 P).
+// 2^t0, 2^t1 on the FMA pipe, to take part of the load off the MUFU ex2
+// unit. t = n + f with n = round(t): adding 1.5 * 2^23 leaves the rounded
+// integer in the low mantissa bits of y, and subtracting it back gives n
+// exactly, so f = t - n lies in [-1/2, 1/2]. 2^f is the cubic of least
+// maximum relative error on that interval, found by the Remez exchange
+// algorithm (exp2_poly_fit.py beside this file; 7.5e-5 relative). n enters
+// the exponent field with one integer multiply-add (y's low bits times 2^23).
+// t is clamped at -126 first: 2^-126 is as good as 0 for a bf16 P.
 __device__ __forceinline__ void exp2_poly2(float t0, float t1, float& r0, float& r1) {
   constexpr float kRound = 12582912.f;   // 1.5 * 2^23
-  constexpr float c0 = 0.9999281168f, c1 = 0.6932609677f, c2 = 0.2426105440f, c3 = 0.0551713221f;
+  constexpr float c0 = 9.9992805719e-01f, c1 = 6.9326096773e-01f, c2 = 2.4261112511e-01f,
+                  c3 = 5.5171668530e-02f;
   const uint64_t t2 = f2_pack(fmaxf(t0, -126.f), fmaxf(t1, -126.f));
   const uint64_t y2 = add2(t2, f2_pack(kRound, kRound));
   const uint64_t n2 = add2(y2, f2_pack(-kRound, -kRound));
@@ -201,16 +239,12 @@ __device__ __forceinline__ void exp2_poly2(float t0, float t1, float& r0, float&
   float y0, y1, q0, q1;
   f2_unpack(y2, y0, y1);
   f2_unpack(q2, q0, q1);
-  // low mantissa bits of y hold n (two's complement); times 2^23 moves them to the exponent
   r0 = __int_as_float(__float_as_int(y0) * 8388608 + __float_as_int(q0));
   r1 = __int_as_float(__float_as_int(y1) * 8388608 + __float_as_int(q1));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (canonical layouts of the
@@ -243,7 +277,9 @@ __device__ __forceinline__ void raise_timeout(volatile int* abort_flag) {
   *abort_flag = 1;
 }
 // Bounded wait (limit in ns); false on timeout or when another role aborted.
-__device__ __noinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, uint64_t limit_ns,
+// Every helper here is inlined: ptxas cannot allocate the registers of the
+// kernel's setmaxnreg regions when they contain a call.
+__device__ __forceinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, uint64_t limit_ns,
                                            volatile int* abort_flag) {
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
@@ -254,152 +290,275 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* b, uint32_t parity, uint64_
     }
   }
 }
-// The first probe is inline: a barrier that has already flipped costs no call.
+// A barrier that has already flipped is taken on the first probe.
 __device__ __forceinline__ bool wait_bar(uint64_t* b, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
   if (mbar_try(b, parity)) return true;
   return wait_bar_slow(b, parity, limit_ns, abort_flag);
 }
 // Bounded wait used while draining: ignores the abort flag, fixed limit.
-__device__ __noinline__ void drain_bar(uint64_t* b, uint32_t parity) {
+__device__ __forceinline__ void drain_bar(uint64_t* b, uint32_t parity) {
   const uint64_t t0 = now_ns();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try(b, parity)) return;
     if ((i & 31) == 31 && now_ns() - t0 > kDrainLimitNs) return;
   }
 }
+// Progress watchdog of a polling loop: call on every turn without progress;
+// returns false (after raising the timeout) once no progress was made for
+// limit_ns, or when another role aborted.
+struct Watchdog {
+  uint64_t t0 = 0;
+  uint32_t idle = 0;
+  __device__ __forceinline__ void progressed() { idle = 0; }
+  __device__ __forceinline__ bool ok(uint64_t limit_ns, volatile int* abort_flag) {
+    if (idle == 0) t0 = now_ns();
+    __nanosleep(32);   // leave the issue slots to the softmax warps meanwhile
+    if ((++idle & 31) != 0) return true;
+    if (*abort_flag) return false;
+    if (now_ns() - t0 > limit_ns) { raise_timeout(abort_flag); return false; }
+    return true;
+  }
+};
 
 // ---------------------------------------------------------------------------
-// Kernel parameters
+// Kernel parameters and per-tile bookkeeping
 // ---------------------------------------------------------------------------
 struct TcParams {
   int C, c, k, Cpad, n_valid, N_alloc;
-  int tiles_per_cluster;      // c / 128 (>= 1)
-  int rows_per_tile;          // min(c, 128)
+  int tiles_per_cluster;      // c / 128 (1 when c = 64)
+  int rows_per_tile;          // min(c, 128): query rows of a tile that belong to its cluster
+  int n_tiles;                // sparse: query tiles over all heads
   int compensate;
+  int J_cent;                 // compensation blocks per tile: ceil(C / 64) with compensation, else 0
   int dense;                  // 1: identity order, every key block kept
-  int dense_key_blocks;       // ceil(n_valid / KB) in dense mode
+  int dense_tiles;            // dense: query tiles per head
+  int dense_key_blocks;       // dense: ceil(n_valid / 128)
   float scale_log2;           // log2(e) / sqrt(d)
   const int32_t* perm_q;      // [BH][C*c]
   const int32_t* count_k;     // [BH][C]
   const int32_t* kept_idx;    // [BH][C][k]
   const int32_t* kept_count;  // [BH][C] kept per query cluster, or null (k each)
   const uint32_t* kept_bits;  // [BH][C][W]
-  const float* logcnt;        // [BH][Cpad] natural log of counts
+  const float* logcnt;        // [BH][Cpad] natural log of counts (-inf past C)
   __nv_bfloat16* O;           // [BH][N_alloc][D]
   uint64_t wait_limit;
 };
 
-template <int D, int KB>
-struct TcCfg {
-  static constexpr int kSub = D / 64;                                  // 64-column sub-tiles per row
-  static constexpr int kQBytes = 128 * D * 2;
-  static constexpr int kTileBytes = KB * D * 2;                        // one K (or V) block
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kMaxKeptSmem = 1024;                            // kept list staged in shared memory
-  static constexpr int kMaxBias = 8192;                                // centroid columns (C <= 8192)
-  static constexpr int kFixedBytes = 256 + kMaxBias * 4 + 2 * 2 * 128 * 4 + 2 * kMaxKeptSmem * 4 + 1024;
-  static constexpr int kStagesFit = (200 * 1024 - kQBytes - kFixedBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 4 ? 4 : (kStagesFit < 2 ? 2 : kStagesFit);
-  static constexpr int kBarOff = kQBytes + kStages * kStageBytes;
-  static constexpr int kBiasOff = kBarOff + 256;                       // compensation bias per centroid column
-  static constexpr int kXchOff = kBiasOff + kMaxBias * 4;              // (m, l) exchange [2 groups][2][128]
-  static constexpr int kKeptOff = kXchOff + 2 * 2 * 128 * 4;
-  // + alignment slack; at least 116 KB so that one CTA (and its 512 TMEM
-  // columns) holds an SM
-  static constexpr int kSmemCalc = kKeptOff + 2 * kMaxKeptSmem * 4 + 1024;
-  static constexpr int kSmem = kSmemCalc > 116 * 1024 ? kSmemCalc : 116 * 1024;
-  static constexpr int kGroupThreads = 128;                            // one softmax group: a thread per row
-  static constexpr int kSoftmaxThreads = 2 * kGroupThreads;
-  static constexpr int kThreads = 128 + kSoftmaxThreads;               // warps 0-3: producer, MMA, 2 idle
-  static constexpr uint32_t kTmemCols = 512;
-  // TMEM: NB S buffers of KB columns (P_j as bf16 pairs over the front half
-  // of its buffer), then O_0 and O_1 (fp32, D columns each)
-  static constexpr int kNBufFit = (512 - 2 * D) / KB;
-  // S_{j+NB} is issued after PV_j; a centroid block takes two stages (kbar,
-  // then vbar), so the stage S_{j+NB} needs is free by then only while
-  // NB <= floor(stages / 2) + 1 (otherwise it waits on a PV not yet issued)
-  static constexpr int kNBufPipe = kStages / 2 + 1;
-  static constexpr int kNBuf = kNBufFit < kNBufPipe ? kNBufFit : kNBufPipe;
-  static constexpr int kSPhase = (kNBuf % 2 == 0) ? kNBuf : 2 * kNBuf;   // blocks between uses of one s_full
-  static constexpr uint32_t kSCol = 0;
-  static constexpr uint32_t kOCol = kNBuf * KB;
-  static_assert(kNBuf >= 2, "two S buffers at least");
-  static_assert(kNBuf <= kStages / 2 + 1 && kNBuf <= kStages, "S look-ahead must not outrun the stage ring");
-  static_assert(kOCol + 2 * D <= kTmemCols, "S buffers and both O accumulators must fit in TMEM");
-  static_assert(kSmem <= 227 * 1024, "shared memory");
+struct Tile {
+  int bh, a, sub;
+  int kq;        // kept key clusters
+  int J_kept;    // kept key blocks
+  int J;         // all blocks (kept, then compensation); 0 for a missing tile
+  int qrow;      // first Q row of the tile (permuted rows; head rows in dense mode)
 };
 
-// Pairs of P columns (bit q % 8) whose exponentials run on the FMA pipe
-// instead of the MUFU unit.
-#ifndef CA_TC_POLY_PAIRS
-#define CA_TC_POLY_PAIRS 0x00
+__device__ __forceinline__ Tile make_tile(const TcParams& p, int t) {
+  Tile T;
+  T.bh = 0; T.a = 0; T.sub = 0; T.kq = 0; T.J_kept = 0; T.J = 0; T.qrow = 0;
+  if (p.dense) {
+    const int ti = blockIdx.x * 2 + t;
+    T.bh = blockIdx.y;
+    if (ti < p.dense_tiles) {
+      T.qrow = ti * 128;
+      T.J_kept = p.dense_key_blocks;
+      T.J = T.J_kept;
+    }
+    return T;
+  }
+  const int ti = blockIdx.x * 2 + t;
+  if (ti >= p.n_tiles) return T;
+  const int per_head = p.C * p.tiles_per_cluster;
+  T.bh = ti / per_head;
+  const int rem = ti % per_head;
+  T.a = rem / p.tiles_per_cluster;
+  T.sub = rem % p.tiles_per_cluster;
+  T.kq = p.kept_count ? min(max(p.kept_count[(size_t)T.bh * p.C + T.a], 0), p.k) : p.k;
+  T.J_kept = p.c >= 128 ? T.kq * (p.c / 128) : (T.kq + 1) / 2;
+  T.J = T.J_kept + p.J_cent;
+  T.qrow = (T.bh * p.C + T.a) * p.c + T.sub * 128;
+  return T;
+}
+
+// Position of item i of the interleaved (tile, block) order: (0,0), (1,0),
+// (0,1), (1,1), ... while both tiles have blocks, then the longer tile's rest.
+__device__ __forceinline__ void item_at(int i, int J0, int J1, int& t, int& j) {
+  const int m = J0 < J1 ? J0 : J1;
+  if (i < 2 * m) { t = i & 1; j = i >> 1; }
+  else { t = J0 > J1 ? 0 : 1; j = m + (i - 2 * m); }
+}
+
+template <int D>
+struct TcCfg {
+  static constexpr int kSub = D / 64;                  // 64-column (128-byte) sub-tiles per row
+  static constexpr int kTileBytes = 128 * D * 2;       // a Q tile, or one ring slot (128 rows)
+  static constexpr int kSubBytes = 128 * 128;          // one sub-tile of a 128-row tile
+  static constexpr int kKS = D == 64 ? 5 : 2;          // K ring slots
+  static constexpr int kVS = D == 64 ? 5 : 2;          // V ring slots
+  static constexpr int kMaxKept = 512;                 // kept list staged in shared memory
+  static constexpr int kKOff = 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kKS * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVS * kTileBytes;
+  static constexpr int kBiasOff = kBarOff + 512;       // per softmax warp: 64 compensation biases
+  static constexpr int kKeptOff = kBiasOff + 8 * 64 * 4;
+  static constexpr int kSmem = kKeptOff + 2 * 2 * kMaxKept * 4 + 1024;   // + alignment slack
+  static constexpr int kThreads = 384;
+  // Registers per thread: the launch gives every thread kRegLaunch (the most
+  // 384 threads can hold); then the producer / MMA warpgroup gives registers
+  // back (setmaxnreg.dec) and the two softmax warpgroups take them
+  // (setmaxnreg.inc), which holds one row of S in registers. The shares must
+  // add up to exactly the launch's total, or the increase would wait forever;
+  // the host refuses to launch a build whose register count is not kRegLaunch.
+  static constexpr int kRegLaunch = 168;
+  static constexpr int kRegSoftmax = 208;
+  static constexpr int kRegOther = 88;
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM: S_t at t * 128. At d = 64, P_t has its own 64 columns (so S_t of
+  // the next block can be computed while P_t is still being read) and O_t
+  // follows; at d = 128 the O accumulators need the room, so P_t is written
+  // over the front of S_t and S_t of the next block waits for O_t += P_t V.
+  static constexpr bool kAliasP = D == 128;
+  static constexpr uint32_t kPCol = kAliasP ? 0 : 256;       // P_t at kPCol + t * kPStride
+  static constexpr uint32_t kPStride = kAliasP ? 128 : 64;
+  static constexpr uint32_t kOCol = kAliasP ? 256 : 384;     // O_t at kOCol + t * D
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kOCol + 2 * D <= kTmemCols, "TMEM");
+  static_assert(kAliasP || kPCol + 2 * 64 <= kOCol, "TMEM: P columns");
+  static_assert(kRegLaunch * kThreads == 65536 / (kThreads * 8) * 8 * kThreads, "launch register count");
+  static_assert(256 * kRegSoftmax + 128 * kRegOther == kThreads * kRegLaunch, "register split");
+};
+
+// Pairs of P columns (bit q % 8 of the mask) whose exponentials run on the
+// FMA pipe (exp2_poly2) instead of the MUFU unit. Measured on B200 (the
+// attention of the N = 65,536 d = 64 layer): with three pairs in eight on the
+// FMA pipe the kernel took 2.05 ms, with none 1.94 ms, so at d = 64 all
+// exponentials stay on the MUFU unit; at d = 128 one pair in eight moves.
+#ifndef CA_TC_POLY64
+#define CA_TC_POLY64 0x00
 #endif
-constexpr unsigned kPolyPairs = CA_TC_POLY_PAIRS;
+#ifndef CA_TC_POLY128
+#define CA_TC_POLY128 0x01
+#endif
 
-// Items in load order: kept key sub-blocks (K,V), then per centroid block
-// (kbar hi, lo) and (vbar hi, vbar lo).
-struct Item { int kind; int row; };   // kind 0 KV, 1 KBAR, 2 VBAR
+// One block of one row, from the NC values of S already in registers: mask
+// or bias them, update the running maximum (lazily), and turn them into
+// P = 2^(S - m) as bf16 pairs (pk) plus the row sum. Returns whether the
+// maximum moved (O must then be scaled by `factor`).
+template <int NC, unsigned kPoly>
+__device__ __forceinline__ bool softmax_block(float (&v)[NC], uint32_t (&pk)[NC / 2], float sc, const float* bias,
+                                              int v0, int v1, float& m_ref, float& l, float& factor) {
+  const bool special = bias != nullptr || v0 < 64 || (NC > 64 && v1 < 64);
+  if (special) {
+    if (bias) {
+#pragma unroll
+      for (int q = 0; q < NC; ++q) v[q] = fmaf(v[q], sc, bias[q]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < NC; ++q) v[q] = ((q < 64) ? (q < v0) : (q - 64 < v1)) ? v[q] * sc : -INFINITY;
+    }
+  }
+  float m4[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) m4[q] = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < NC; q += 2) m4[(q >> 1) & 3] = max3(m4[(q >> 1) & 3], v[q], v[q + 1]);
+  float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+  if (!special) mx *= sc;   // log2 units (masked / biased values already are)
+  const bool need = mx > m_ref + 8.f;
+  factor = 1.f;
+  if (need) {
+    factor = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+    m_ref = mx;
+    l *= factor;
+  }
+  const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref;
+  const float xs = special ? 1.f : sc;
+  const uint64_t xs2 = f2_pack(xs, xs), nb2 = f2_pack(nb, nb);
+  uint64_t ls2[2] = {0ull, 0ull};
+#pragma unroll
+  for (int q = 0; q < NC / 2; ++q) {
+    float t0, t1, p0, p1;
+    f2_unpack(fma2(f2_pack(v[2 * q], v[2 * q + 1]), xs2, nb2), t0, t1);
+    if ((kPoly >> (q & 7)) & 1u) exp2_poly2(t0, t1, p0, p1);
+    else { p0 = ex2(t0); p1 = ex2(t1); }
+    ls2[q & 1] = add2(ls2[q & 1], f2_pack(p0, p1));
+    pk[q] = pack_bf16(p0, p1);
+  }
+  float a0, a1;
+  f2_unpack(add2(ls2[0], ls2[1]), a0, a1);
+  l += a0 + a1;
+  return need;
+}
 
-template <int D, int KB>
-__global__ void __launch_bounds__(TcCfg<D, KB>::kThreads, 1)
+template <int D>
+__global__ void __launch_bounds__(TcCfg<D>::kThreads, 1)
 tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_khi,
-                 const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_vhi,
-                 const __grid_constant__ CUtensorMap tm_vlo, const TcParams p) {
-  using Cfg = TcCfg<D, KB>;
-  constexpr int NS = Cfg::kStages;
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
+                 const __grid_constant__ CUtensorMap tm_vc, const TcParams p) {
+  using Cfg = TcCfg<D>;
+  constexpr int KS = Cfg::kKS, VS = Cfg::kVS;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                          ~static_cast<uintptr_t>(1023));
-  unsigned char* sQ = smem;
-  unsigned char* sStage = smem + Cfg::kQBytes;
+  unsigned char* sQ = smem;                        // [2] Q tiles
+  unsigned char* sK = smem + Cfg::kKOff;           // [KS] K slots
+  unsigned char* sV = smem + Cfg::kVOff;           // [VS] V slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOff);
-  uint64_t* full = bars;              // [NS] stage loaded
-  uint64_t* empty = bars + NS;        // [NS] stage released
-  uint64_t* q_full = bars + 2 * NS;   // Q tile loaded
-  constexpr int NB = Cfg::kNBuf;
-  uint64_t* s_full = q_full + 1;      // [NB][2] S_j computed in buffer j % NB, for group j % 2
-  uint64_t* p_full = s_full + 2 * NB; // [NB] P_j written in buffer j % NB
-  uint64_t* pv_done = p_full + NB;    // [NB] O_{j%2} += P_j V_j completed (j % NB)
-  uint64_t* drain = pv_done + NB;
+  uint64_t* q_full = bars;                 // [2]
+  uint64_t* kfull = q_full + 2;            // [KS]
+  uint64_t* kempty = kfull + KS;           // [KS]
+  uint64_t* vfull = kempty + KS;           // [VS]
+  uint64_t* vempty = vfull + VS;           // [VS]
+  uint64_t* s_full = vempty + VS;          // [2] S_t computed
+  uint64_t* s_free = s_full + 2;           // [2] S_t read into registers (128 arrivals; separate P only)
+  uint64_t* p_full = s_free + 2;           // [2] P_t written (128 arrivals)
+  uint64_t* pv_done = p_full + 2;          // [2] O_t += P_t V completed
+  uint64_t* drain = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* bias_all = reinterpret_cast<float*>(smem + Cfg::kBiasOff);
-  float* xch = reinterpret_cast<float*>(smem + Cfg::kXchOff);
-  int32_t* kept_s = reinterpret_cast<int32_t*>(smem + Cfg::kKeptOff);        // kept key clusters
-  int32_t* kcnt_s = kept_s + Cfg::kMaxKeptSmem;                               // their member counts
+  float* bias_w = reinterpret_cast<float*>(smem + Cfg::kBiasOff);   // [8 warps][64]
+  int32_t* kept_s = reinterpret_cast<int32_t*>(smem + Cfg::kKeptOff);   // [2][kMaxKept]
+  int32_t* kcnt_s = kept_s + 2 * Cfg::kMaxKept;                         // [2][kMaxKept]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int tile = blockIdx.x;
-  const int a = p.dense ? 0 : tile / p.tiles_per_cluster;          // query cluster
-  const int sub_tile = p.dense ? 0 : tile % p.tiles_per_cluster;
-  const int nsb = p.dense ? 1 : (p.c + KB - 1) / KB;               // key sub-blocks per cluster
-  // kept key clusters of this query cluster (k, or its own count after adaptive selection)
-  const int kq = p.dense ? 0 : (p.kept_count ? min(max(p.kept_count[(size_t)bh * p.C + a], 0), p.k) : p.k);
-  const int J_kept = p.dense ? p.dense_key_blocks : kq * nsb;
-  const int J_cent = (p.compensate && !p.dense) ? p.Cpad / KB : 0;
-  const int J = J_kept + J_cent;
-  const int n_items = J_kept + 2 * J_cent;
-  const int32_t* kept_g = p.dense ? nullptr : p.kept_idx + ((size_t)bh * p.C + a) * p.k;
-  const bool kept_in_smem = !p.dense && kq <= Cfg::kMaxKeptSmem;
-  if (kept_in_smem) {
-    for (int i = threadIdx.x; i < kq; i += Cfg::kThreads) {
-      const int b = kept_g[i];
+  const Tile T0 = make_tile(p, 0), T1 = make_tile(p, 1);
+  // both tiles attend the same key blocks: dense attention, or the two
+  // halves of one 256-query cluster
+  const bool shared_kv = T1.J > 0 && (p.dense || (p.c == 256 && T0.bh == T1.bh && T0.a == T1.a));
+  // kept lists (and the kept clusters' sizes) in shared memory when they fit
+  const bool kept_sm0 = !p.dense && T0.kq <= Cfg::kMaxKept;
+  const bool kept_sm1 = !p.dense && T1.kq <= Cfg::kMaxKept;
+  const int32_t* kept_g0 = p.dense ? nullptr : p.kept_idx + ((size_t)T0.bh * p.C + T0.a) * p.k;
+  const int32_t* kept_g1 = p.dense ? nullptr : p.kept_idx + ((size_t)T1.bh * p.C + T1.a) * p.k;
+  if (kept_sm0 && T0.J > 0) {
+    for (int i = threadIdx.x; i < T0.kq; i += Cfg::kThreads) {
+      const int b = kept_g0[i];
       kept_s[i] = b;
-      kcnt_s[i] = p.count_k[(size_t)bh * p.C + b];
+      kcnt_s[i] = p.count_k[(size_t)T0.bh * p.C + b];
     }
   }
-  const int32_t* kept = kept_in_smem ? kept_s : kept_g;
+  if (kept_sm1 && T1.J > 0) {
+    for (int i = threadIdx.x; i < T1.kq; i += Cfg::kThreads) {
+      const int b = kept_g1[i];
+      kept_s[Cfg::kMaxKept + i] = b;
+      kcnt_s[Cfg::kMaxKept + i] = p.count_k[(size_t)T1.bh * p.C + b];
+    }
+  }
+  auto kept_at = [&](int t, int i) -> int {
+    const bool sm = t ? kept_sm1 : kept_sm0;
+    return sm ? kept_s[t * Cfg::kMaxKept + i] : (t ? kept_g1 : kept_g0)[i];
+  };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    mbar_init(q_full, 1);
-    for (int b = 0; b < NB; ++b) {
-      mbar_init(&s_full[2 * b], 1);
-      mbar_init(&s_full[2 * b + 1], 1);
-      mbar_init(&p_full[b], Cfg::kGroupThreads);
-      mbar_init(&pv_done[b], 1);
+    // with shared K/V tiles a slot is free once both tiles' products read it
+    const uint32_t users = shared_kv ? 2u : 1u;
+    for (int s = 0; s < KS; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], users); }
+    for (int s = 0; s < VS; ++s) { mbar_init(&vfull[s], 1); mbar_init(&vempty[s], users); }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&pv_done[t], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -415,313 +574,334 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint64_t limit = p.wait_limit;
-
-  auto item_of = [&](int i) -> Item {
-    Item it;
-    if (i < J_kept) {
-      it.kind = 0;
-      if (p.dense) it.row = i * KB;
-      else {
-        const int b = kept[i / nsb];
-        it.row = (bh * p.C + b) * p.c + (i % nsb) * KB;
-      }
-    } else {
-      const int t = i - J_kept;
-      it.kind = 1 + (t & 1);
-      it.row = bh * p.Cpad + (t >> 1) * KB;
-    }
-    return it;
+  const int NI = T0.J + T1.J;                   // (tile, block) items
+  const int NR = shared_kv ? T0.J : NI;         // ring items (one per item, or one per block when shared)
+  const int nsb = p.c >= 128 ? p.c / 128 : 1;   // key blocks per kept cluster (c >= 128)
+  // Ring index of block j of tile t: the producer fills the rings in the
+  // interleaved order (0,0), (1,0), (0,1), (1,1), ... (or one entry per block
+  // when the tiles share K/V); each tile consumes its own entries in order.
+  const int m01 = T0.J < T1.J ? T0.J : T1.J;
+  auto ring_of = [&](int t, int j) -> int {
+    if (shared_kv) return j;
+    return j < m01 ? 2 * j + t : 2 * m01 + (j - m01);
   };
 
-  if (warp == 0) {
+  if (warp >= 8) {
+   // producer / MMA warpgroup: gives registers to the softmax warpgroups
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Cfg::kRegOther));
+   if (warp == 8) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      int issued = 0;
       bool ok = true;
-      mbar_expect_tx(q_full, Cfg::kQBytes);
-      for (int s = 0; s < Cfg::kSub; ++s) {
-        if (p.dense) tma_3d(sQ + s * 128 * 128, &tm_q, q_full, s * 64, tile * 128, bh);
-        else tma_2d(sQ + s * 128 * 128, &tm_q, q_full, s * 64, (bh * p.C + a) * p.c + sub_tile * 128);
-      }
-      for (int i = 0; i < n_items && ok; ++i) {
-        const int s = i % NS, r = i / NS;
-        const Item it = item_of(i);
-        if (!wait_bar(&empty[s], (r & 1) ^ 1, limit, abort_flag)) { ok = false; break; }
-        unsigned char* dst = sStage + s * Cfg::kStageBytes;
-        mbar_expect_tx(&full[s], Cfg::kStageBytes);
-        const CUtensorMap* m0 = it.kind == 0 ? &tm_k : (it.kind == 1 ? &tm_khi : &tm_vhi);
-        const CUtensorMap* m1 = it.kind == 0 ? &tm_v : (it.kind == 1 ? &tm_klo : &tm_vlo);
+      for (int t = 0; t < 2; ++t) {
+        const Tile& Tt = t ? T1 : T0;
+        if (Tt.J == 0) continue;
+        mbar_expect_tx(&q_full[t], Cfg::kTileBytes);
         for (int sb = 0; sb < Cfg::kSub; ++sb) {
+          unsigned char* dst = sQ + t * Cfg::kTileBytes + sb * Cfg::kSubBytes;
+          if (p.dense) tma_3d(dst, &tm_q, &q_full[t], sb * 64, Tt.qrow, Tt.bh);
+          else tma_2d(dst, &tm_q, &q_full[t], sb * 64, Tt.qrow);
+        }
+      }
+      // Load the K (is_v = 0) or V tile of ring item r into `dst`.
+      auto load_item = [&](int r, bool is_v, unsigned char* dst, uint64_t* bar) {
+        int t = 0, j = r;
+        if (!shared_kv) item_at(r, T0.J, T1.J, t, j);
+        const Tile& Tt = t ? T1 : T0;
+        mbar_expect_tx(bar, Cfg::kTileBytes);
+        const CUtensorMap* mk = is_v ? &tm_v : &tm_k;
+        const CUtensorMap* mc = is_v ? &tm_vc : &tm_kc;
+        for (int sb = 0; sb < Cfg::kSub; ++sb) {
+          unsigned char* d = dst + sb * Cfg::kSubBytes;
           if (p.dense) {
-            tma_3d(dst + sb * KB * 128, m0, &full[s], sb * 64, it.row, bh);
-            tma_3d(dst + Cfg::kTileBytes + sb * KB * 128, m1, &full[s], sb * 64, it.row, bh);
+            tma_3d(d, mk, bar, sb * 64, j * 128, Tt.bh);
+          } else if (j < Tt.J_kept) {
+            if (p.c >= 128) {
+              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.C + kept_at(t, j / nsb)) * p.c + (j % nsb) * 128);
+            } else {
+              // two key clusters of 64; an odd count repeats the first (its
+              // columns are masked, and its values stay finite)
+              const int b0 = kept_at(t, 2 * j);
+              const int b1 = (2 * j + 1 < Tt.kq) ? kept_at(t, 2 * j + 1) : b0;
+              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.C + b0) * 64);
+              tma_2d(d + 64 * 128, mk, bar, sb * 64, (Tt.bh * p.C + b1) * 64);
+            }
           } else {
-            tma_2d(dst + sb * KB * 128, m0, &full[s], sb * 64, it.row);
-            tma_2d(dst + Cfg::kTileBytes + sb * KB * 128, m1, &full[s], sb * 64, it.row);
+            const int cb = j - Tt.J_kept;
+            tma_2d(d, mc, bar, sb * 64, (Tt.bh * (p.Cpad / 64) + cb) * 128);
           }
         }
-        issued = i + 1;
+      };
+      int kn = 0, vn = 0;
+      Watchdog wd;
+      while (vn < NR) {
+        bool prog = false;
+        if (kn < NR && mbar_test(&kempty[kn % KS], ((kn / KS) & 1) ^ 1)) {
+          load_item(kn, false, sK + (kn % KS) * Cfg::kTileBytes, &kfull[kn % KS]);
+          ++kn;
+          prog = true;
+        }
+        if (vn < kn && mbar_test(&vempty[vn % VS], ((vn / VS) & 1) ^ 1)) {
+          load_item(vn, true, sV + (vn % VS) * Cfg::kTileBytes, &vfull[vn % VS]);
+          ++vn;
+          prog = true;
+        }
+        if (prog) wd.progressed();
+        else if (!wd.ok(limit, abort_flag)) { ok = false; break; }
       }
       if (!ok) {
         // Let every copy already issued land before the CTA leaves.
-        drain_bar(q_full, 0);
-        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i) drain_bar(&full[i % NS], (i / NS) & 1);
+        if (T0.J > 0) drain_bar(&q_full[0], 0);
+        if (T1.J > 0) drain_bar(&q_full[1], 0);
+        for (int i = (kn > KS ? kn - KS : 0); i < kn; ++i) drain_bar(&kfull[i % KS], (i / KS) & 1);
+        for (int i = (vn > VS ? vn - VS : 0); i < vn; ++i) drain_bar(&vfull[i % VS], (i / VS) & 1);
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 9) {
     // ------------------------------------------------------------- MMA issuer
-    // The whole warp runs this loop (so descriptors are warp-uniform); one
-    // elected lane issues each tcgen05 instruction and every commit.
-    constexpr uint32_t id_qk = idesc_bf16(128, KB, 0);
+    // The whole warp runs this loop (so decisions are warp-uniform); the
+    // leader lane issues the products. Each tile advances on its own: its next PV_t as soon as P_t and the V tile
+    // are there, its next S_t as soon as the K tile is there and S_t (or, at
+    // d = 128, P_t under it) has been consumed.
+    constexpr uint32_t id_qk128 = idesc_bf16(128, 128, 0);
+    constexpr uint32_t id_qk64 = idesc_bf16(128, 64, 0);
     constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
-    const uint32_t q_base = su32(sQ);
-    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, limit, abort_flag));
-    };
-    bool ok = wwait(q_full, 0);
-    // item index of block j's QK and PV operands
-    auto qk_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept); };
-    auto pv_item = [&](int j) { return j < J_kept ? j : J_kept + 2 * (j - J_kept) + 1; };
-    auto issue_qk = [&](int j) -> bool {
-      const int i = qk_item(j);
-      const int s = i % NS, r = i / NS;
-      if (!wwait(&full[s], r & 1)) return false;
-      tc_fence_after();
-      const uint32_t kb = su32(sStage + s * Cfg::kStageBytes);
-      const uint32_t d_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
-      const int nmat = (j < J_kept) ? 1 : 2;   // centroids: hi then lo
-      for (int mtx = 0; mtx < nmat; ++mtx) {
-        const uint32_t bbase = kb + mtx * Cfg::kTileBytes;
+    bool ok = true;
+    if (T0.J > 0) ok = __all_sync(0xffffffffu, wait_bar(&q_full[0], 0, limit, abort_flag));
+    if (ok && T1.J > 0) ok = __all_sync(0xffffffffu, wait_bar(&q_full[1], 0, limit, abort_flag));
+    int qn0 = 0, qn1 = 0, pn0 = 0, pn1 = 0;
+    Watchdog wd;
+    // Descriptor templates: the start address sits in the low 14 bits (in
+    // 16-byte units), so a tile or a K step is a small constant added to the
+    // low word; every product's descriptors cost one add each.
+    const uint64_t qd0 = sdesc(su32(sQ), 16, 1024);
+    const uint64_t kd0 = sdesc(su32(sK), 16, 1024);
+    const uint64_t vd0 = sdesc(su32(sV), Cfg::kSubBytes, 1024);
+    const bool leader = elect_one();
+    // S_t = Q_t K_j^T into TMEM (leader lane), then the commits
+    auto issue_qk = [&](int t, int j, int r) {
+      if (leader) {
+        const uint64_t qd = qd0 + (uint64_t)((t * Cfg::kTileBytes) >> 4);
+        const uint64_t kd = kd0 + (uint64_t)(((r % KS) * Cfg::kTileBytes) >> 4);
+        const uint32_t s_tmem = tmem + (uint32_t)(t * 128);
+        if (j < (t ? T1.J_kept : T0.J_kept)) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk & 3) * 32);   // 16 bf16 along K inside the 128B row
-          const uint64_t ad = sdesc(q_base + (kk >> 2) * 128 * 128 + off, 16, 1024);
-          const uint64_t bd = sdesc(bbase + (kk >> 2) * KB * 128 + off, 16, 1024);
-          mma_ss_elect(d_tmem, ad, bd, id_qk, (mtx > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * Cfg::kSubBytes + (kk & 3) * 32) >> 4);
+            mma_ss(s_tmem, qd + off, kd + off, id_qk128, kk > 0 ? 1u : 0u);
+          }
+        } else {
+          // centroid hi parts (rows 0-63), then lo parts (rows 64-127)
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = (uint64_t)(((kk >> 2) * Cfg::kSubBytes + (kk & 3) * 32) >> 4);
+              mma_ss(s_tmem, qd + off, kd + off + (uint64_t)((half * 64 * 128) >> 4), id_qk64,
+                     (half > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+        }
+        tc_commit(&s_full[t]);
+        tc_commit(&kempty[r % KS]);
+      }
+      __syncwarp();
+    };
+    // O_t += P_t V_j (leader lane), then the commits
+    auto issue_pv = [&](int t, int j, int r) {
+      if (leader) {
+        const uint64_t vd = vd0 + (uint64_t)(((r % VS) * Cfg::kTileBytes) >> 4);
+        const uint32_t p_tmem = tmem + Cfg::kPCol + (uint32_t)(t * Cfg::kPStride);
+        const uint32_t o_tmem = tmem + Cfg::kOCol + (uint32_t)(t * D);
+        if (j < (t ? T1.J_kept : T0.J_kept)) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)((half * 64 * 128 + kk * 16 * 128) >> 4), id_pv,
+                     (j > 0 || half > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(&pv_done[t]);
+        tc_commit(&vempty[r % VS]);
+      }
+      __syncwarp();
+    };
+    while (ok && (pn0 < T0.J || pn1 < T1.J)) {
+      bool prog = false;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int J = t ? T1.J : T0.J;
+        int& qn = t ? qn1 : qn0;
+        int& pn = t ? pn1 : pn0;
+        if (pn < qn) {
+          const int r = ring_of(t, pn);
+          const bool rdy = mbar_test(&p_full[t], pn & 1) && mbar_test(&vfull[r % VS], (r / VS) & 1);
+          if (__all_sync(0xffffffffu, rdy)) {
+            tc_fence_after();
+            issue_pv(t, pn, r);
+            ++pn;
+            prog = true;
+          }
+        }
+        if (qn < J) {
+          const int r = ring_of(t, qn);
+          // S_t of block qn overwrites what block qn - 1 left there: its S
+          // must have been read (separate P), or its PV completed (P under S)
+          uint64_t* freed = Cfg::kAliasP ? &pv_done[t] : &s_free[t];
+          const bool rdy = (qn == 0 || (Cfg::kAliasP ? pn >= qn : true)) &&
+                           (qn == 0 || mbar_test(freed, (qn - 1) & 1)) && mbar_test(&kfull[r % KS], (r / KS) & 1);
+          if (__all_sync(0xffffffffu, rdy)) {
+            tc_fence_after();
+            issue_qk(t, qn, r);
+            ++qn;
+            prog = true;
+          }
         }
       }
-      tc_commit_elect(&s_full[(j % NB) * 2 + (j & 1)]);
-      if (j >= J_kept) tc_commit_elect(&empty[s]);   // kbar stage is free once S is computed
-      return true;
-    };
-    // S_0 .. S_{NB-1} ahead; S_{j+NB} reuses buffer j % NB once PV_j (its
-    // last reader) has completed. Blocks alternate between the two softmax
-    // groups, so the other group works on S_{j+1} meanwhile.
-    for (int j = 0; j < NB && j < J && ok; ++j) ok = issue_qk(j);
-    for (int j = 0; j < J && ok; ++j) {
-      if (!wwait(&p_full[j % NB], (j / NB) & 1)) { ok = false; break; }
-      tc_fence_after();
-      const int i = pv_item(j);
-      const int s = i % NS, r = i / NS;
-      if (j >= J_kept) {
-        if (!wwait(&full[s], r & 1)) { ok = false; break; }
-        tc_fence_after();
-      }
-      const uint32_t vb = su32(sStage + s * Cfg::kStageBytes) + (j < J_kept ? Cfg::kTileBytes : 0);
-      const uint32_t p_tmem = tmem + Cfg::kSCol + (uint32_t)((j % NB) * KB);
-      const uint32_t o_tmem = tmem + Cfg::kOCol + (uint32_t)((j & 1) * D);   // O of the block's group
-      const int nmat = (j < J_kept) ? 1 : 2;
-      for (int mtx = 0; mtx < nmat; ++mtx) {
-        const uint32_t bbase = vb + mtx * Cfg::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < KB / 16; ++kk) {
-          const uint64_t bd = sdesc(bbase + kk * 16 * 128, KB * 128, 1024);
-          mma_ts_elect(o_tmem, p_tmem + kk * 8, bd, id_pv, (j >= 2 || mtx > 0 || kk > 0) ? 1u : 0u);
-        }
-      }
-      tc_commit_elect(&pv_done[j % NB]);
-      tc_commit_elect(&empty[s]);
-      if (j + NB < J) {
-        if (!wwait(&pv_done[j % NB], (j / NB) & 1)) { ok = false; break; }
-        tc_fence_after();
-        if (!issue_qk(j + NB)) { ok = false; break; }
-      }
+      if (prog) wd.progressed();
+      else if (!wd.ok(limit, abort_flag)) ok = false;
     }
     // Drain: every MMA issued so far has completed once `drain` flips.
     tc_commit_elect(drain);
     if (lane == 0) drain_bar(drain, 0);
     __syncwarp();
-  } else if (warp >= 4) {
+   }
+  } else {
     // ------------------------------------------------------------- softmax
-    // Group g (warps 4-7 or 8-11) takes the blocks j with j % 2 == g, one
-    // thread per query row, and accumulates them in its own O_g.
-    const int g = (warp - 4) >> 2;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Cfg::kRegSoftmax));
+    constexpr unsigned kPoly = D == 64 ? (unsigned)CA_TC_POLY64 : (unsigned)CA_TC_POLY128;
+    const int t = warp >> 2;
+    const Tile Tt = make_tile(p, t);
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;           // row of the query tile
-    const int sth = threadIdx.x - 128;        // 0..255 over both groups
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t s_addr = lane_addr + (uint32_t)(t * 128);
+    const uint32_t p_addr = lane_addr + Cfg::kPCol + (uint32_t)(t * Cfg::kPStride);
+    const uint32_t o_addr = lane_addr + Cfg::kOCol + (uint32_t)(t * D);
     const float sc = p.scale_log2;
-    // compensation bias of every centroid column (log2 units; -inf where the
-    // key cluster is kept or is padding), once per CTA
-    if (J_cent > 0) {
-      const uint32_t* kb_row = p.kept_bits + ((size_t)bh * p.C + a) * ((p.C + 31) / 32);
-      const float log2e = 1.4426950408889634f;
-      for (int e = sth; e < J_cent * KB; e += Cfg::kSoftmaxThreads) {
-        float bv = -INFINITY;
-        if (e < p.C && !((kb_row[e >> 5] >> (e & 31)) & 1u)) bv = p.logcnt[(size_t)bh * p.Cpad + e] * log2e;
-        bias_all[e] = bv;
-      }
-    }
-    named_sync(1, Cfg::kSoftmaxThreads);
-    float m_used = -INFINITY, lreg = 0.f;
+    float* bias = bias_w + warp * 64;
+    const uint32_t* kb_row =
+        p.dense ? nullptr : p.kept_bits + ((size_t)Tt.bh * p.C + Tt.a) * ((p.C + 31) / 32);
+    // the tile's kept clusters' sizes: staged in shared memory, or read through the kept list
+    const bool ksm = !p.dense && Tt.kq <= Cfg::kMaxKept;
+    const int32_t* kcnt_t = kcnt_s + t * Cfg::kMaxKept;
+    const int32_t* kept_t = p.dense ? nullptr : p.kept_idx + ((size_t)Tt.bh * p.C + Tt.a) * p.k;
+    const int32_t* cnt_h = p.count_k + (size_t)Tt.bh * p.C;
+    auto cnt_of = [&](int i) -> int { return ksm ? kcnt_t[i] : cnt_h[kept_t[i]]; };
+    float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = g; j < J; j += 2) {
-      const bool cent = j >= J_kept;
-      int valid = KB;   // real keys in a kept block
-      if (!cent) {
-        if (p.dense) valid = min(KB, p.n_valid - j * KB);
-        else {
-          const int cnt = kept_in_smem ? kcnt_s[j / nsb] : p.count_k[(size_t)bh * p.C + kept[j / nsb]];
-          valid = min(KB, cnt - (j % nsb) * KB);
-        }
-      }
-      const float* bias = bias_all + (cent ? (j - J_kept) * KB : 0);
-      const uint32_t sbuf = lane_addr + Cfg::kSCol + (uint32_t)((j % NB) * KB);
-      ok = __all_sync(0xffffffffu, wait_bar(&s_full[(j % NB) * 2 + g], (j / Cfg::kSPhase) & 1, limit, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      // pass 1: the row maximum, 64 columns per TMEM round trip. Partial and
-      // centroid blocks (rare) get their mask / bias here and are written
-      // back, so that pass 2 has a single path.
-      const bool special = cent || valid < KB;
-      float m8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-#pragma unroll 1
-      for (int c0 = 0; c0 < KB; c0 += 64) {
-        float v[64];
-        CA_TMEM_LD32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
-        CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(v + 32));
-        tmem_wait_ld();
-        if (special) {
-          if (cent) {
-#pragma unroll
-            for (int q = 0; q < 64; ++q) v[q] = fmaf(v[q], sc, bias[c0 + q]);
-          } else {
-#pragma unroll
-            for (int q = 0; q < 64; ++q) v[q] = (c0 + q < valid) ? v[q] : -INFINITY;
-          }
-          CA_TMEM_ST32(sbuf + (uint32_t)c0, reinterpret_cast<uint32_t*>(v));
-          CA_TMEM_ST32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(v + 32));
-        }
-#pragma unroll
-        for (int q = 0; q < 64; q += 2) m8[(q >> 1) & 7] = max3(m8[(q >> 1) & 7], v[q], v[q + 1]);
-      }
-      if (special) tmem_wait_st();
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      if (!cent) mx *= sc;                   // log2 units (centroid values already are)
-      // lazy rescale: move the reference max only when it grows by > 8 (x 256)
-      float factor = 1.f;
-      const bool need = mx > m_used + 8.f;
-      if (need) {
-        factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - mx);
-        m_used = mx;
-        lreg *= factor;
-      }
-      // O_g already holds blocks j-2, j-4, ...: rescale it (whole warp, as
-      // TMEM loads and stores are warp-wide) once PV_{j-2} has completed.
-      if (j >= 2 && __any_sync(0xffffffffu, need)) {
-        ok = __all_sync(0xffffffffu, wait_bar(&pv_done[(j - 2) % NB], ((j - 2) / NB) & 1, limit, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t oaddr = lane_addr + Cfg::kOCol + (uint32_t)(g * D);
+    // P_t and O_t of the previous block are free once its PV completed
+    // (with P under S this is implied by S_t having been computed)
+    auto wait_prev_pv = [&](int j) -> bool {
+      if (Cfg::kAliasP || j == 0) return true;
+      const bool r = __all_sync(0xffffffffu, wait_bar(&pv_done[t], (j - 1) & 1, limit, abort_flag));
+      if (r) tc_fence_after();
+      return r;
+    };
+    // O_t holds blocks 0..j-1: scale it when the reference maximum moved
+    auto rescale_o = [&](int j, bool need, float factor) {
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t ov[32];
-          CA_TMEM_LD32(oaddr + (uint32_t)c0, ov);
+          CA_TMEM_LD32(o_addr + (uint32_t)c0, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * factor);
-          CA_TMEM_ST32(oaddr + (uint32_t)c0, ov);
+          CA_TMEM_ST32(o_addr + (uint32_t)c0, ov);
         }
       }
-      const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
-      // pass 2: P = 2^(x - m) as bf16 pairs over the front half of the buffer
-      // (the pairs of columns c0.. land on columns c0/2.., already read)
-      const float xs = cent ? 1.f : sc;
-      const uint64_t xs2 = f2_pack(xs, xs), nb2 = f2_pack(nb, nb);
-      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};   // packed partial row sums
-      // 32 columns per step, two steps per loop turn; the next step's TMEM
-      // load is in flight while a step computes
-      auto p_step = [&](const float* v, int c0) {
-        uint32_t pk[16];
+    };
+    for (int j = 0; j < Tt.J; ++j) {
+      const bool cent = j >= Tt.J_kept;
+      int v0 = 64, v1 = 64;   // real keys in the two 64-column halves of a kept block
+      if (cent) {
+        // compensation bias of this block's 64 centroids (log2 units; -inf
+        // where the key cluster is kept or is padding), staged per warp
+        const float log2e = 1.4426950408889634f;
+        __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          float t0, t1, p0, p1;
-          f2_unpack(fma2(f2_pack(v[2 * q], v[2 * q + 1]), xs2, nb2), t0, t1);
-          if ((kPolyPairs >> (q & 7)) & 1) exp2_poly2(t0, t1, p0, p1);
-          else { p0 = ex2(t0); p1 = ex2(t1); }
-          ls2[q & 3] = add2(ls2[q & 3], f2_pack(p0, p1));
-          pk[q] = pack_bf16(p0, p1);
+        for (int h = 0; h < 2; ++h) {
+          const int e = h * 32 + lane;
+          const int b = (j - Tt.J_kept) * 64 + e;
+          float bv = -INFINITY;
+          if (b < p.C && !((kb_row[b >> 5] >> (b & 31)) & 1u)) bv = p.logcnt[(size_t)Tt.bh * p.Cpad + b] * log2e;
+          bias[e] = bv;
         }
-        CA_TMEM_ST16(sbuf + (uint32_t)(c0 / 2), pk);
-      };
-      float va[32], vb[32];
-      CA_TMEM_LD32(sbuf, reinterpret_cast<uint32_t*>(va));
-#pragma unroll 1
-      for (int c0 = 0; c0 < KB; c0 += 64) {
-        tmem_wait_ld();
-        CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 32), reinterpret_cast<uint32_t*>(vb));
-        p_step(va, c0);
-        tmem_wait_ld();
-        if (c0 + 64 < KB) CA_TMEM_LD32(sbuf + (uint32_t)(c0 + 64), reinterpret_cast<uint32_t*>(va));
-        p_step(vb, c0 + 32);
+        __syncwarp();
+      } else if (p.dense) {
+        const int rem = p.n_valid - j * 128;
+        v0 = min(max(rem, 0), 64);
+        v1 = min(max(rem - 64, 0), 64);
+      } else if (p.c >= 128) {
+        const int rem = cnt_of(j / nsb) - (j % nsb) * 128;
+        v0 = min(max(rem, 0), 64);
+        v1 = min(max(rem - 64, 0), 64);
+      } else {
+        v0 = cnt_of(2 * j);
+        v1 = (2 * j + 1 < Tt.kq) ? cnt_of(2 * j + 1) : 0;
       }
-      {
-        float a0, a1;
-        f2_unpack(add2(add2(ls2[0], ls2[1]), add2(ls2[2], ls2[3])), a0, a1);
-        lreg += a0 + a1;
+      ok = __all_sync(0xffffffffu, wait_bar(&s_full[t], j & 1, limit, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float factor;
+      bool need;
+      if (cent) {
+        float v[64];
+        uint32_t pk[32];
+        CA_TMEM_LD32(s_addr, reinterpret_cast<uint32_t*>(v));
+        CA_TMEM_LD32(s_addr + 32u, reinterpret_cast<uint32_t*>(v + 32));
+        tmem_wait_ld();
+        if (!Cfg::kAliasP) { tc_fence_before(); mbar_arrive(&s_free[t]); }
+        need = softmax_block<64, kPoly>(v, pk, sc, bias, 64, 0, m_ref, l, factor);
+        if (!(ok = wait_prev_pv(j))) break;
+        CA_TMEM_ST32(p_addr, pk);
+      } else {
+        float v[128];
+        uint32_t pk[64];
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) CA_TMEM_LD32(s_addr + (uint32_t)c0, reinterpret_cast<uint32_t*>(v + c0));
+        tmem_wait_ld();
+        if (!Cfg::kAliasP) { tc_fence_before(); mbar_arrive(&s_free[t]); }
+        need = softmax_block<128, kPoly>(v, pk, sc, nullptr, v0, v1, m_ref, l, factor);
+        if (!(ok = wait_prev_pv(j))) break;
+        CA_TMEM_ST32(p_addr, pk);
+        CA_TMEM_ST32(p_addr + 32u, (pk + 32));
       }
+      rescale_o(j, need, factor);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j % NB]);
+      mbar_arrive(&p_full[t]);
     }
-    // epilogue: merge the two groups' (m, l, O) and write O / l to the
-    // query's original row; group g writes columns [g D/2, (g+1) D/2)
-    const int jl0 = (J >= 1) ? ((J - 1) & ~1) : -1;          // last block of group 0
-    const int jl1 = (J >= 2) ? (((J - 2) & ~1) + 1) : -1;    // last block of group 1
-    const int jl = g ? jl1 : jl0;
-    if (ok && jl >= 0)
-      ok = __all_sync(0xffffffffu, wait_bar(&pv_done[jl % NB], (jl / NB) & 1, limit, abort_flag));
-    xch[(g * 2 + 0) * 128 + row] = jl >= 0 ? m_used : -INFINITY;
-    xch[(g * 2 + 1) * 128 + row] = jl >= 0 ? lreg : 0.f;
-    named_sync(1, Cfg::kSoftmaxThreads);
-    if (ok) {
-      tc_fence_after();
-      const float m0 = xch[0 * 128 + row], l0 = xch[1 * 128 + row];
-      const float m1 = xch[2 * 128 + row], l1 = xch[3 * 128 + row];
-      const float M = fmaxf(m0, m1);
-      const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
-      const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
-      const float l = l0 * f0 + l1 * f1;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float w0 = f0 * inv, w1 = f1 * inv;
-      int orow;
-      if (p.dense) orow = tile * 128 + row < p.n_valid ? tile * 128 + row : -1;
-      else orow = row < p.rows_per_tile ? p.perm_q[(size_t)bh * p.C * p.c + (size_t)a * p.c + sub_tile * 128 + row]
-                                        : -1;
-      constexpr int OH = D / 2;
-      __nv_bfloat16* dst = p.O + ((size_t)bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D + g * OH;
+    // epilogue: O / l to the query's original row
+    if (ok && Tt.J > 0) {
+      ok = __all_sync(0xffffffffu, wait_bar(&pv_done[t], (Tt.J - 1) & 1, limit, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        int orow;
+        if (p.dense) orow = Tt.qrow + row < p.n_valid ? Tt.qrow + row : -1;
+        else orow = (Tt.sub * 128 + row < p.c && row < p.rows_per_tile) ? p.perm_q[(size_t)Tt.qrow + row] : -1;
+        __nv_bfloat16* dst = p.O + ((size_t)Tt.bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D;
 #pragma unroll
-      for (int c0 = 0; c0 < OH; c0 += 32) {
-        uint32_t o0[32], o1[32];
-        // an accumulator whose group had no block was never written
-        if (jl0 >= 0) CA_TMEM_LD32(lane_addr + Cfg::kOCol + (uint32_t)(g * OH + c0), o0);
-        if (jl1 >= 0) CA_TMEM_LD32(lane_addr + Cfg::kOCol + (uint32_t)(D + g * OH + c0), o1);
-        tmem_wait_ld();
-        if (orow >= 0) {
-          uint4 w[4];
-          uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          CA_TMEM_LD32(o_addr + (uint32_t)c0, o);
+          tmem_wait_ld();
+          if (orow >= 0) {
+            uint4 w[4];
+            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            float x0 = 0.f, x1 = 0.f;
-            if (jl0 >= 0) { x0 = __uint_as_float(o0[2 * q]) * w0; x1 = __uint_as_float(o0[2 * q + 1]) * w0; }
-            if (jl1 >= 0) { x0 = fmaf(__uint_as_float(o1[2 * q]), w1, x0); x1 = fmaf(__uint_as_float(o1[2 * q + 1]), w1, x1); }
-            wp[q] = pack_bf16(x0, x1);
+            for (int q = 0; q < 16; ++q) wp[q] = pack_bf16(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv);
+            uint4* gp = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) gp[q] = w[q];
           }
-          uint4* gp = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) gp[q] = w[q];
         }
       }
     }
@@ -733,6 +913,17 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(Cfg::kTmemCols));
   }
+}
+
+// Evaluates exp2_poly2 on n inputs (pairs), for checking it against exp2f.
+__global__ void exp2_poly_check_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float t0 = x[i], t1 = i + 1 < n ? x[i + 1] : 0.f;
+  float r0, r1;
+  exp2_poly2(t0, t1, r0, r1);
+  y[i] = r0;
+  if (i + 1 < n) y[i + 1] = r1;
 }
 
 // ---------------------------------------------------------------------------
@@ -779,23 +970,23 @@ bool make_map_3d(CUtensorMap* m, const void* base, int BH, int N_alloc, int n_va
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int KB>
-cudaError_t launch_tc(const CUtensorMap maps[7], const TcParams& p, dim3 grid, cudaStream_t st) {
-  using Cfg = TcCfg<D, KB>;
-  cudaError_t e = cudaFuncSetAttribute(tc_attend_kernel<D, KB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Cfg::kSmem);
+template <int D>
+cudaError_t launch_tc(const CUtensorMap maps[5], const TcParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = TcCfg<D>;
+  // The register split inside the kernel assumes exactly kRegLaunch registers
+  // per thread at launch; any other count could leave setmaxnreg.inc waiting.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, tc_attend_kernel<D>);
   if (e != cudaSuccess) return e;
-  tc_attend_kernel<D, KB><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                                   maps[5], maps[6], p);
+  if (fa.numRegs != Cfg::kRegLaunch) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(tc_attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  if (e != cudaSuccess) return e;
+  tc_attend_kernel<D><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
   return cudaGetLastError();
 }
 
-// Key-block width: 128 keys, or 64 when the cluster size is 64.
-int key_block(int D, int c) { return c >= 128 ? 128 : 64; (void)D; }
-
-cudaError_t dispatch(int D, int KB, const CUtensorMap maps[7], const TcParams& p, dim3 grid, cudaStream_t st) {
-  if (D == 64) return KB == 128 ? launch_tc<64, 128>(maps, p, grid, st) : launch_tc<64, 64>(maps, p, grid, st);
-  return KB == 128 ? launch_tc<128, 128>(maps, p, grid, st) : launch_tc<128, 64>(maps, p, grid, st);
+cudaError_t dispatch(int D, const CUtensorMap maps[5], const TcParams& p, dim3 grid, cudaStream_t st) {
+  return D == 64 ? launch_tc<64>(maps, p, grid, st) : launch_tc<128>(maps, p, grid, st);
 }
 
 }  // namespace
@@ -803,31 +994,31 @@ cudaError_t dispatch(int D, int KB, const CUtensorMap maps[7], const TcParams& p
 cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_routes* rt, int compensate,
                              void* O, const AttendWs& L, char* ws, cudaStream_t st) {
   const int BH = s->B * s->H, D = s->d, c = s->c, C = L.C;
-  const int KB = key_block(D, c);
   const uint64_t slots = (uint64_t)BH * C * c;
-  CUtensorMap maps[7];
-  bool ok = make_map_2d(&maps[0], ws + L.qp, slots, D, 128) && make_map_2d(&maps[1], ws + L.kp, slots, D, KB) &&
-            make_map_2d(&maps[2], ws + L.vp, slots, D, KB) &&
-            make_map_2d(&maps[3], ws + L.kbar_hi, (uint64_t)BH * L.Cpad, D, KB) &&
-            make_map_2d(&maps[4], ws + L.kbar_lo, (uint64_t)BH * L.Cpad, D, KB) &&
-            make_map_2d(&maps[5], ws + L.vbar_hi, (uint64_t)BH * L.Cpad, D, KB) &&
-            make_map_2d(&maps[6], ws + L.vbar_lo, (uint64_t)BH * L.Cpad, D, KB);
+  const uint64_t cent_rows = (uint64_t)BH * L.Cpad * 2;   // hi and lo rows of every 64-centroid block
+  CUtensorMap maps[5];
+  bool ok = make_map_2d(&maps[0], ws + L.qp, slots, D, 128) &&
+            make_map_2d(&maps[1], ws + L.kp, slots, D, c >= 128 ? 128 : 64) &&
+            make_map_2d(&maps[2], ws + L.vp, slots, D, c >= 128 ? 128 : 64) &&
+            make_map_2d(&maps[3], ws + L.kbar_hl, cent_rows, D, 128) &&
+            make_map_2d(&maps[4], ws + L.vbar_hl, cent_rows, D, 128);
   if (!ok) return cudaErrorInvalidValue;
-  TcParams p;
+  TcParams p{};
   p.C = C; p.c = c; p.k = rt->k; p.Cpad = L.Cpad; p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
   p.tiles_per_cluster = c >= 128 ? c / 128 : 1;
   p.rows_per_tile = c >= 128 ? 128 : c;
+  p.n_tiles = BH * C * p.tiles_per_cluster;
   p.compensate = compensate;
+  p.J_cent = compensate ? (C + 63) / 64 : 0;
   p.dense = 0;
-  p.dense_key_blocks = 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.perm_q = cl->perm_q; p.count_k = cl->count_k; p.kept_idx = rt->kept_idx; p.kept_bits = rt->kept_bits;
   p.kept_count = rt->kept_count;
   p.logcnt = reinterpret_cast<const float*>(ws + L.logcnt);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.wait_limit = wait_limit();
-  const dim3 grid(C * p.tiles_per_cluster, BH);
-  return dispatch(D, KB, maps, p, grid, st);
+  const dim3 grid((unsigned)((p.n_tiles + 1) / 2));
+  return dispatch(D, maps, p, grid, st);
 }
 
 // One CTA waits, through the same bounded wait as the attention kernel, on an
@@ -854,27 +1045,33 @@ cudaError_t launch_bounded_wait_check(uint64_t limit_ns, int arrive, cudaStream_
   return cudaGetLastError();
 }
 
+cudaError_t launch_exp2_poly_check(const float* x, float* y, int n, cudaStream_t st) {
+  const int pairs = (n + 1) / 2;
+  exp2_poly_check_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const ca_shape* s, void* O,
                             cudaStream_t st) {
   const int BH = s->B * s->H, D = s->d;
-  const int KB = key_block(D, 128);
-  CUtensorMap maps[7];
+  CUtensorMap maps[5];
   bool ok = make_map_3d(&maps[0], Q, BH, s->N_alloc, s->n_valid, D, 128) &&
-            make_map_3d(&maps[1], K, BH, s->N_alloc, s->n_valid, D, KB) &&
-            make_map_3d(&maps[2], V, BH, s->N_alloc, s->n_valid, D, KB);
+            make_map_3d(&maps[1], K, BH, s->N_alloc, s->n_valid, D, 128) &&
+            make_map_3d(&maps[2], V, BH, s->N_alloc, s->n_valid, D, 128);
   if (!ok) return cudaErrorInvalidValue;
-  maps[3] = maps[1]; maps[4] = maps[1]; maps[5] = maps[2]; maps[6] = maps[2];
+  maps[3] = maps[1]; maps[4] = maps[2];
   TcParams p{};
   p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
   p.tiles_per_cluster = 1; p.rows_per_tile = 128;
-  p.compensate = 0; p.dense = 1;
-  p.dense_key_blocks = (s->n_valid + KB - 1) / KB;
-  p.c = KB;
+  p.compensate = 0; p.J_cent = 0; p.dense = 1;
+  p.dense_tiles = (s->n_valid + 127) / 128;
+  p.dense_key_blocks = (s->n_valid + 127) / 128;
+  p.c = 128;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.wait_limit = wait_limit();
-  const dim3 grid((s->n_valid + 127) / 128, BH);
-  return dispatch(D, KB, maps, p, grid, st);
+  const dim3 grid((unsigned)((p.dense_tiles + 1) / 2), BH);
+  return dispatch(D, maps, p, grid, st);
 }
 
 }  // namespace ca

@@ -132,7 +132,7 @@ cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const Tr
                             int NI, double* wvec, uint64_t seed, cudaStream_t st);
 
 struct AttendWs {
-  size_t qp, kp, vp, kbar_hi, kbar_lo, vbar_hi, vbar_lo, vbar32, kbar32, logcnt, total;
+  size_t qp, kp, vp, kbar_hl, vbar_hl, vbar32, kbar32, logcnt, total;
   int C = 0, Cpad = 0;
 };
 bool attend_ws_layout(const ca_shape* s, AttendWs* ws);
@@ -141,10 +141,11 @@ bool attend_ws_layout(const ca_shape* s, AttendWs* ws);
 // Device error word and bounded waits.
 // ---------------------------------------------------------------------------
 // The error word lives in attend_tc.cu; other units reach it through these.
-uint64_t wait_limit();                            // iteration cap of bounded waits
+uint64_t wait_limit();                            // time limit (ns) of bounded waits
 cudaError_t device_error_read_clear(unsigned* out, cudaStream_t st);
 cudaError_t launch_bounded_wait_check(uint64_t limit_ns, int arrive, cudaStream_t st);
-void set_wait_limit(uint64_t spins);
+cudaError_t launch_exp2_poly_check(const float* x, float* y, int n, cudaStream_t st);
+void set_wait_limit(uint64_t limit_ns);
 
 // ---------------------------------------------------------------------------
 // Launchers (each returns cudaGetLastError() of its launches).

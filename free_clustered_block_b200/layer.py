@@ -8,7 +8,7 @@ from __future__ import annotations
 from dataclasses import dataclass
 from typing import Optional
 
-from . import (CA_BF16, CA_FP32, ca_attend, ca_cluster, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
+from . import (CA_BF16, CA_FP32, ca_attend, ca_attend_prepare, ca_attend_prepared, ca_cluster, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
                attend_workspace_bytes, cluster_workspace_bytes, clusters_struct, forward_workspace_bytes,
                make_params, make_shape, num_clusters, routes_struct)
 
@@ -99,6 +99,15 @@ class ClusterAttention:
     def attend(self, Q, K, V, O, stream=None):
         ca_attend(Q, K, V, self.shape, self.clusters(), self.routes(), self.compensate, O, self.workspace,
                   stream)
+
+    def attend_prepare(self, Q, K, V, stream=None):
+        """ca_attend's first half (value centroids, cluster-ordered copies)."""
+        ca_attend_prepare(Q, K, V, self.shape, self.clusters(), self.workspace, stream)
+
+    def attend_prepared(self, Q, K, V, O, stream=None):
+        """ca_attend's second half: the attention kernel on the prepared workspace."""
+        ca_attend_prepared(Q, K, V, self.shape, self.clusters(), self.routes(), self.compensate, O, self.workspace,
+                           stream)
 
     def __call__(self, Q, K, V, O=None, stream=None):
         if O is None:

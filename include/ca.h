@@ -175,7 +175,9 @@ ca_status ca_cluster(const void* Q, const void* K, const ca_shape* shape,
  * 65,536-token heads at d = 64 fit, eight do not). Nothing here calls
  * cudaMalloc, cudaFree or any allocating routine. The first call on a device
  * looks up the array's device address (with that device current), so make
- * that first call before any stream capture. All calls share the one array:
+ * that first call before any stream capture; the address is looked up again
+ * when the current context is no longer the one it was found in (after
+ * cudaDeviceReset, for example). All calls share the one array:
  * calls whose work overlaps on the GPU (different streams, or several host
  * threads) race on it and must be serialised by the caller.
  */
@@ -226,12 +228,29 @@ ca_status ca_route_adaptive(const ca_shape* shape, const ca_clusters* centroids,
  * written by ca_route_adaptive);
  * vbar is computed here. O: device [B][H][N_alloc][d], written in original
  * row order (padding rows 0). workspace >= ca_attend_workspace_bytes(shape).
- * bf16 with compensate != 0 supports C <= 8192 key clusters
- * (CA_ERR_UNSUPPORTED beyond).
  */
 ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* shape,
                     const ca_clusters* clusters, const ca_routes* routes, int compensate,
                     void* O, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ca_attend_prepare / ca_attend_prepared -- ca_attend in two halves, for
+ * callers that time or schedule the attention kernel on its own.
+ * ca_attend_prepare writes into the workspace what the attention reads: the
+ * value centroids vbar, the centroid forms the kernels load (bf16 hi/lo
+ * parts, fp32 copies, log counts) and, for bf16, the cluster-ordered copies
+ * of Q, K and V. ca_attend_prepared then runs the attention (and zeroes O's
+ * padding rows) from that workspace; it must follow a ca_attend_prepare on
+ * the same stream with the same Q, K, V, clusters and workspace, and reads
+ * Q, K, V again only for fp32 inputs. Same arguments, layouts and errors as
+ * ca_attend (ca_attend_prepare takes no routes and no O).
+ */
+ca_status ca_attend_prepare(const void* Q, const void* K, const void* V, const ca_shape* shape,
+                            const ca_clusters* clusters, void* workspace, size_t workspace_bytes,
+                            void* stream);
+ca_status ca_attend_prepared(const void* Q, const void* K, const void* V, const ca_shape* shape,
+                             const ca_clusters* clusters, const ca_routes* routes, int compensate,
+                             void* O, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * ca_dense_attend -- plain softmax(Q K^T / sqrt(d)) V over the n_valid keys
@@ -269,14 +288,20 @@ ca_status ca_forward_host(const void* Q_host, const void* K_host, const void* V_
  * ca_get_device_error -- synchronise `stream` and report (then clear) the
  * device-side error word of the current device: CA_ERR_TIMEOUT if a bounded
  * wait inside a kernel gave up, CA_ERR_CUDA if the stream holds a CUDA error,
- * CA_OK otherwise.
+ * CA_OK otherwise. The error word is ONE word per device, shared by every
+ * stream and every caller of the library in the process: a timeout raised by
+ * work on one stream is reported to whichever caller reads the word first
+ * (and that read clears it), so callers that share a device and need to
+ * attribute errors must serialise their calls and their reads.
  */
 ca_status ca_get_device_error(void* stream);
 
 /* Test hook: the time limit, in nanoseconds, of every bounded device-side
  * wait (mbarrier waits on TMA copies and tensor-core work); 0 restores the
- * default of 1 s. Host only; affects later launches. */
-void ca_set_wait_limit(uint64_t limit_ns);
+ * default of 1 s. Limits above 10 s are rejected with CA_ERR_INVALID_ARG
+ * (a longer bound would let a lost arrival hold the GPU). Host only, atomic;
+ * affects later launches. */
+ca_status ca_set_wait_limit(uint64_t limit_ns);
 
 /* Failure-detection check: launch one CTA on `stream` that waits, through the
  * same bounded mbarrier wait as the attention kernel, on a barrier that
@@ -287,6 +312,14 @@ void ca_set_wait_limit(uint64_t limit_ns);
  * CA_ERR_INVALID_ARG for limit_ns = 0 or above 10 s, CA_ERR_CUDA if the launch
  * fails. */
 ca_status ca_check_bounded_wait(uint64_t limit_ns, int arrive, void* stream);
+
+/* Check of the attention kernel's FMA-pipe exponential: writes to y[i] the
+ * kernel's own evaluation of 2^x[i] (round-to-nearest split t = n + f, a
+ * Remez cubic for 2^f on [-1/2, 1/2], n added to the exponent; inputs below
+ * -126 are clamped there). x, y: device fp32 arrays of n elements. Async on
+ * `stream`. n = 0 does nothing; CA_ERR_INVALID_ARG for n < 0, or for null
+ * pointers with n > 0. */
+ca_status ca_check_exp2_poly(const float* x, float* y, int n, void* stream);
 
 /* Number of kernel launches one call makes for this shape (host only):
  * stage 0 = ca_cluster, 1 = ca_route, 2 = ca_attend, 3 = ca_dense_attend;

@@ -23,7 +23,7 @@ def lib():
 def declared_symbols():
     text = open(os.path.join(ROOT, "include", "ca.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ca_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ca_[a-z_0-9]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -122,3 +122,11 @@ def test_noalloc_scratch_covers_its_stated_examples(lib):
     for args in ((1, 2, 65536, 65536, 64, 128), (1, 1, 76800, 75600, 128, 128)):
         s = ca.make_shape(*args, ca.CA_BF16)
         assert 0 < ca.cluster_workspace_bytes(s) <= 16 << 20
+
+
+def test_wait_limit_setter_rejects_limits_above_ten_seconds(lib):
+    assert lib.ca_set_wait_limit(10_000_000_001) == ca.CA_ERR_INVALID_ARG
+    assert lib.ca_set_wait_limit(2**64 - 1) == ca.CA_ERR_INVALID_ARG
+    assert lib.ca_set_wait_limit(5_000_000) == ca.CA_OK
+    assert lib.ca_set_wait_limit(0) == ca.CA_OK          # back to the default
+    assert lib.ca_check_exp2_poly(None, None, 4, None) == ca.CA_ERR_INVALID_ARG
