@@ -42,7 +42,10 @@ CONFIG_ID = 2
 # activity of one launch. Each entry holds for the attention source whose
 # SHA-256 starts with `sha` and the workload it names; for any other source
 # or workload the bench reports null.
-ATTN_CAPTURES = []
+ATTN_CAPTURES = [
+    {"sha": "f2f522f50ab311e0", "workload": "cfg2-lowrank-N65536-d64-bf16",
+     "traffic": 205490688 + 51618304, "tensor_pipe_pct": 30.08},
+]
 
 
 def _attn_source_sha():
