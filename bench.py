@@ -6,9 +6,14 @@
 One step is one forward of one attention layer on the tabular-shaped
 workload (B=1, H=8, N=65,536 tokens, d=64, bf16, cluster size 128, 64 of 512
 key clusters kept per query cluster, compensation on), inputs resident in HBM.
-Under torchrun each rank runs its own independent layer (weak scaling, no
-collective on the data path); the reported value is layer forwards per second
-over all ranks, timed with CUDA events as the max over ranks.
+Under torchrun the layer's heads are split over the ranks (each head is
+clustered and attended on its own, so no collective runs on the data path;
+strong scaling); --shard layers gives each rank an independent layer
+instead (weak scaling). The reported value is layer forwards per second over
+all ranks, timed with CUDA events as the max over ranks.
+
+--config 5 runs the sweep over cluster size, keep fraction and compensation
+at N = 32,768 (d = 64 and 128), one JSON line per point.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (one head's clustering and routing, a sample of its query clusters'
@@ -353,11 +358,25 @@ def affinity_cores():
         return os.cpu_count() or 1
 
 
-def make_layer(ca, w, args):
+def make_layer(ca, w, args, head_base=0):
     adaptive = args.selection == "adaptive"
     return ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.C if adaptive else w.k,
                                dtype=w.dtype, compensate=w.compensate, selection=args.selection,
-                               recall=args.recall, min_count=16, clustering=args.clustering)
+                               recall=args.recall, min_count=16, clustering=args.clustering,
+                               head_base=head_base)
+
+
+def head_share(w, world, rank):
+    """This rank's slice of one layer's heads: the workload restricted to the
+    flattened heads [b0, b1) (B = 1, H = b1 - b0) and b0, the global index of
+    its first head."""
+    import dataclasses
+    from free_clustered_block_b200 import heads
+    b0, b1 = heads.rank_slice(w.B * w.H, world, rank)
+    cut = lambda x: x.reshape(w.B * w.H, w.N_alloc, w.d)[b0:b1][None]
+    ws = dataclasses.replace(w, B=1, H=b1 - b0, Q=cut(w.Q), K=cut(w.K), V=cut(w.V),
+                             name=f"{w.name}-heads{b0}-{b1}")
+    return ws, b0
 
 
 def time_layer(ca, torch, w, layer, Q, K, V, O, steps, warmup, barrier, local, sample_clocks=True):
@@ -542,8 +561,18 @@ def run_ours(args):
     def ranks_max(x):
         return max_over_ranks(x, world, "cuda")
 
-    # Each rank: an independent layer (its own seeded inputs).
-    w = build_workload(args, rank)
+    # One layer split by heads across the ranks (the default for N > 1: no
+    # collective on the data path), or (--shard layers) an independent layer
+    # per rank.
+    shard_heads = world > 1 and args.shard == "heads"
+    head_base = 0
+    if shard_heads:
+        w_layer = build_workload(args, 0)
+        w, head_base = head_share(w_layer, world, rank)
+    else:
+        w = w_layer = build_workload(args, rank)
+    if w.H == 0:
+        raise RuntimeError("more ranks than heads: every rank needs at least one head")
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(x):
@@ -552,13 +581,15 @@ def run_ours(args):
     Q, K, V = dev(w.Q), dev(w.K), dev(w.V)
     O = torch.empty_like(Q)
     adaptive = args.selection == "adaptive"
-    layer = make_layer(ca, w, args)
+    layer = make_layer(ca, w, args, head_base)
     stream = torch.cuda.current_stream()
+    # layer forwards completed by all ranks together per step
+    layers_per_step = 1 if shard_heads else world
 
     local_ms, stage, clocks = time_layer(ca, torch, w, layer, Q, K, V, O, args.steps, args.warmup, barrier, local)
     total_ms = ranks_max(local_ms)
     ms_per_step = total_ms / args.steps
-    value = whole_job_value(world, args.steps, total_ms)
+    value = whole_job_value(layers_per_step, args.steps, total_ms)
 
     # Dense attention (this library's own kernel) on the same inputs, for the speedup.
     dense_ms = ranks_max(time_dense(torch, layer, Q, K, V, max(1, min(args.steps, 3))))
@@ -592,7 +623,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ranks_max(e0.elapsed_time(e1))
-    e2e_value = whole_job_value(world, args.steps, e2e_ms)
+    e2e_value = whole_job_value(layers_per_step, args.steps, e2e_ms)
     in_bytes = 3 * Q.numel() * Q.element_size()
     out_bytes = O.numel() * O.element_size()
 
@@ -634,18 +665,22 @@ def run_ours(args):
     launches = args.steps * sum(per_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if shard_heads else "weak",
         "vs_baseline": None, "dtype": w.dtype,
         "dtype_detail": ("clustering and routing f64; attention bf16 products with f32 accumulation"
                          if w.dtype == "bf16" else "clustering and routing f64; attention f32"),
         "data": "synthetic",
-        "config": dict(workload_config(w), selection=args.selection, clustering=args.clustering,
+        "config": dict(workload_config(w_layer), selection=args.selection, clustering=args.clustering,
+                       parallelism=(f"heads split over {world} GPUs ({w.H} per GPU, head_base {head_base} on "
+                                    f"rank {rank})" if shard_heads else
+                                    (f"an independent layer per GPU ({world} GPUs)" if world > 1 else "one GPU")),
                        **({"recall": args.recall, "min_count": 16,
                            "mean_kept": float(kc.mean())} if adaptive else {})),
         "latency_ms": ms_per_step, "stage_ms": stage, "dense_ms": dense_ms,
         "speedup_vs_dense": dense_ms / ms_per_step,
         "graph_ms_per_step": graph_ms,
-        "tflops": {"dense_equivalent": dense_flops(w) / (ms_per_step / 1e3) / 1e12,
+        "tflops": {"dense_equivalent": layers_per_step * dense_flops(w_layer) / (ms_per_step / 1e3) / 1e12,
                    "algorithmic_attention": roof["achieved"]},
         "roofline": roof,
         "dense_roofline": dense_roof,
@@ -689,6 +724,9 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="latency scaling: configuration 2's generator at this token count")
     ap.add_argument("--fixed-k", action="store_true", help="with --tokens: keep 64 clusters instead of 1/8")
+    ap.add_argument("--shard", choices=["heads", "layers"], default="heads",
+                    help="with N > 1 GPUs: split one layer's heads over the GPUs (default) or run an independent "
+                         "layer per GPU")
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=CONFIG_ID,
                     help="workload (default 2: the metric's N = 64k configuration); 5: the sweep over cluster "
                          "size, keep fraction and compensation at N = 32,768, one JSON line per point")

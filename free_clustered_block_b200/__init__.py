@@ -51,7 +51,7 @@ class ca_shape(ctypes.Structure):
 class ca_cluster_params(ctypes.Structure):
     _fields_ = [("power_iters", ctypes.c_int), ("sample_factor", ctypes.c_int),
                 ("transform", ctypes.c_int), ("query_form", ctypes.c_int), ("seed", ctypes.c_uint64),
-                ("method", ctypes.c_int), ("reserved", ctypes.c_int)]
+                ("method", ctypes.c_int), ("head_base", ctypes.c_int)]
 
 
 class ca_clusters(ctypes.Structure):
@@ -139,12 +139,14 @@ def make_shape(B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, dtype
 
 
 def make_params(power_iters: int = 8, sample_factor: int = 1, transform: int = 1,
-                seed: int = 0, query_form: int = 0, method: int = 0) -> ca_cluster_params:
+                seed: int = 0, query_form: int = 0, method: int = 0, head_base: int = 0) -> ca_cluster_params:
     """query_form 0: queries as R_k q / |R_k q| (top-k selection, eq. 16);
     1: queries as R_k q (adaptive selection, eq. 15). method 0: recursive
     splitting; 1: random clusters (the error-analysis baseline); 2:
-    diagonalized recursive splitting."""
-    return ca_cluster_params(power_iters, sample_factor, transform, query_form, seed & ((1 << 64) - 1), method, 0)
+    diagonalized recursive splitting. head_base: global index of the call's
+    first (b, h) pair, for a call on a slice of a layer's heads."""
+    return ca_cluster_params(power_iters, sample_factor, transform, query_form, seed & ((1 << 64) - 1), method,
+                             head_base)
 
 
 def num_clusters(shape: ca_shape) -> int:

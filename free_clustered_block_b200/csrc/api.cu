@@ -50,6 +50,7 @@ ca_status check_params(const ca_shape* s, const ca_cluster_params* p) {
   if (p->query_form != 0 && p->query_form != 1) return CA_ERR_INVALID_ARG;
   if (p->method < 0 || p->method > 2) return CA_ERR_INVALID_ARG;
   if (p->method == 2 && a != 1) return CA_ERR_UNSUPPORTED;
+  if (p->head_base < 0) return CA_ERR_INVALID_ARG;
   return CA_OK;
 }
 

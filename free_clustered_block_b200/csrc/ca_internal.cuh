@@ -129,7 +129,7 @@ cudaError_t launch_diag_basis(int D, int TH, int BH, int nch, int n, const doubl
 template <typename T, int D>
 cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const TreeNode* nodes, int lvl_begin,
                             int nodes_in_level, int TH, const double* W, const double* inv_s, const int* idx,
-                            int NI, double* wvec, uint64_t seed, cudaStream_t st);
+                            int NI, double* wvec, uint64_t seed, int head_base, cudaStream_t st);
 
 struct AttendWs {
   size_t qp, kp, vp, kbar_hl, vbar_hl, vbar32, kbar32, logcnt, total;

@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(512) dir_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
-    int power_iters, int sample_factor) {
+    int head_base, int power_iters, int sample_factor) {
   using Cfg = DirCfg<T, D>;
   constexpr int CPL = D / 32;                      // coordinates per lane: a = lane + 32 c
   constexpr int RS = Cfg::kRowStride;
@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(512) dir_kernel(
   const int node_id = lvl_begin + local;
   const TreeNode nd = nodes[node_id];
   const int m = min(m_cap, nd.size);
-  const uint64_t key = node_stream(seed, (uint64_t)bh, (uint64_t)tensor, nd.heap);
+  const uint64_t key = node_stream(seed, (uint64_t)(head_base + bh), (uint64_t)tensor, nd.heap);
   const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
   const int* idx_th = idx ? idx + (size_t)th * n : nullptr;
@@ -670,7 +670,7 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, int npc, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
-    int power_iters) {
+    int head_base, int power_iters) {
   using Cfg = DirCCfg<T, D_>;
   constexpr int D = D_, RS = Cfg::kRowStride;
   constexpr int NT = Cfg::kThreads, HD = D / 2;   // threads, half length
@@ -728,7 +728,7 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
     const int node_id = lvl_begin + local;
     const TreeNode nd = nodes[node_id];
     const int m = min(D, nd.size);
-    const uint64_t key = node_stream(seed, (uint64_t)bh, (uint64_t)tensor, nd.heap);
+    const uint64_t key = node_stream(seed, (uint64_t)(head_base + bh), (uint64_t)tensor, nd.heap);
     const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
     __syncthreads();   // the previous node is done with every shared array
     if (t < D) {
@@ -1007,13 +1007,13 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
 // random order of the tokens into groups of c (remainder last). Positions
 // outside this level's nodes get a key too; nothing reads it.
 __global__ void __launch_bounds__(256) hash_keys_kernel(int n, const int* __restrict__ idx, uint64_t seed,
-                                                        uint64_t* __restrict__ keys) {
+                                                        int head_base, uint64_t* __restrict__ keys) {
   const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
   const int pos = blockIdx.x * 256 + threadIdx.x;
   if (pos >= n) return;
   const int row = idx ? idx[(size_t)th * n + pos] : pos;
   keys[(size_t)th * n + pos] =
-      splitmix64(node_stream(seed, (uint64_t)bh, (uint64_t)tensor, 0ull) ^ (uint64_t)(uint32_t)row);
+      splitmix64(node_stream(seed, (uint64_t)(head_base + bh), (uint64_t)tensor, 0ull) ^ (uint64_t)(uint32_t)row);
 }
 
 // ---------------------------------------------------------------------------
@@ -1382,20 +1382,22 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
       int* idx_out = idxbuf[(l + 1) & 1];
       if (random_clusters) {
-        hash_keys_kernel<<<dim3((n + 255) / 256, TH), 256, 0, st>>>(n, idx_in, p->seed, keys);
+        hash_keys_kernel<<<dim3((n + 255) / 256, TH), 256, 0, st>>>(n, idx_in, p->seed, p->head_base, keys);
       } else if (diagonal) {
         const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, TH, basis, inv_s, idx_in,
-                                                    NI, wvec, p->seed, st);
+                                                    NI, wvec, p->seed, p->head_base, st);
         if (e != cudaSuccess) return e;
       } else if (sample_factor == 1 && (D == 128 || (long long)nl * TH <= kDirCMaxNodes64)) {
         // a block per node: d = 128, or d = 64 levels with few nodes (about
         // four blocks per SM over the whole level)
         const int npc = (int)(((long long)nl * TH + 4 * 148 - 1) / (4 * 148));
         dirc_kernel<T, D><<<dim3((nl + npc - 1) / npc, TH), DirCCfg<T, D>::kThreads, DirCCfg<T, D>::kSmem, st>>>(
-            Q, K, N_alloc, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters);
+            Q, K, N_alloc, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base,
+            power_iters);
       } else {
         dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(
-            Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, power_iters, sample_factor);
+            Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base, power_iters,
+            sample_factor);
       }
       if (!random_clusters)
         project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(

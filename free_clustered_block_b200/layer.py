@@ -37,13 +37,17 @@ class ClusterAttention:
     clusters, the error-analysis baseline).
 
     Q, K, V, O: torch CUDA tensors [B, H, N_alloc, d], bf16 or fp32, contiguous.
+
+    head_base: global index of the first (b, h) pair these tensors hold, when
+    they are a slice of a larger layer's heads (one GPU's share of a layer
+    split across GPUs); the clusters are then those the whole layer would get.
     """
 
     def __init__(self, B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, k: int,
                  dtype: str = "bf16", compensate: bool = True, power_iters: int = 8,
                  sample_factor: int = 1, transform: bool = True, seed: int = 0, device="cuda",
                  selection: str = "topk", recall: float = 0.9, min_count: int = 16,
-                 clustering: str = "split"):
+                 clustering: str = "split", head_base: int = 0):
         import torch
         self.torch = torch
         self.dtype_code = CA_BF16 if dtype == "bf16" else CA_FP32
@@ -53,7 +57,7 @@ class ClusterAttention:
         self.recall, self.min_count = recall, min_count
         self.params = make_params(power_iters, sample_factor, int(transform), seed,
                                   query_form=1 if selection == "adaptive" else 0,
-                                  method=CLUSTERING_METHODS[clustering])
+                                  method=CLUSTERING_METHODS[clustering], head_base=head_base)
         self.k = k
         self.compensate = compensate
         C = num_clusters(self.shape)

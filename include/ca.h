@@ -83,7 +83,14 @@ typedef struct {
  *                    split on the coordinate with the highest variance over
  *                    the basic splitting's sample (lowest index on a tie);
  *                    power_iters is ignored; sample_factor must be 0 or 1
- *                    (CA_ERR_UNSUPPORTED otherwise). */
+ *                    (CA_ERR_UNSUPPORTED otherwise);
+ *  head_base     global index of this call's first (b, h) pair, >= 0 (0 for a
+ *                whole layer): the random streams of head (b, h) are keyed by
+ *                head_base + b*H + h, so a call on a slice of a layer's heads
+ *                (pointers offset to the slice, H the slice's head count)
+ *                reproduces exactly the clusters the whole-layer call makes
+ *                for those heads. This is how one layer's heads are split
+ *                across GPUs. */
 typedef struct {
   int power_iters;
   int sample_factor;
@@ -91,7 +98,7 @@ typedef struct {
   int query_form;
   uint64_t seed;
   int method;
-  int reserved;   /* 0 */
+  int head_base;
 } ca_cluster_params;
 
 /* Clustering result, one entry per (b, h), C = ca_num_clusters(shape):

@@ -61,3 +61,56 @@ def test_single_rank_helpers():
     assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
     assert bench.whole_job_value(1, 10, 100.0) == pytest.approx(100.0)
     assert bench.rank_seed(0) == 1002
+
+
+def _heads_rank_main(rank, world, port, n_heads, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from free_clustered_block_b200 import heads, make_params
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        b, e = heads.rank_slice(n_heads, world, rank)
+        params = make_params(head_base=b)
+        # what every rank runs, gathered on every rank
+        mine = torch.tensor([b, e, params.head_base], dtype=torch.int64)
+        allv = [torch.zeros(3, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(allv, mine)
+        q.put((rank, [tuple(int(x) for x in t) for t in allv]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("n_heads", [8, 40, 5])
+def test_two_gloo_ranks_split_a_layer_by_heads(n_heads):
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_heads_rank_main, args=(r, world, port, n_heads, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert res[0][1] == res[1][1]                   # both ranks see the same plan
+    plan = res[0][1]
+    covered = [h for (b, e, hb) in plan for h in range(b, e)]
+    assert covered == list(range(n_heads))          # every head exactly once, in order
+    for (b, e, hb) in plan:
+        assert hb == b                              # random streams keyed by the global head index
+    sizes = [e - b for (b, e, _) in plan]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_head_slices_edge_cases():
+    import sys
+    sys.path.insert(0, ROOT)
+    from free_clustered_block_b200 import heads
+    assert heads.head_slices(3, 8) == [(0, 1), (1, 2), (2, 3)] + [(3, 3)] * 5
+    assert heads.head_slices(0, 2) == [(0, 0), (0, 0)]
+    assert heads.head_slices(40, 8) == [(5 * r, 5 * r + 5) for r in range(8)]
+    with pytest.raises(ValueError):
+        heads.rank_slice(4, 2, 2)
