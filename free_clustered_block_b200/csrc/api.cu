@@ -298,8 +298,40 @@ ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape
   return ca_attend(Q, K, V, s, &cl, &rt, compensate, O, ws + f.scratch, f.attend_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// ca_forward_host pipelines groups of heads: the host-to-device copies of one
+// group overlap the forward of the previous one and the device-to-host copy
+// of the one before. Groups are contiguous ranges of the flattened heads,
+// sizes differing by at most one (the first groups take one more).
+constexpr int kHostGroups = 4;
+
+int host_groups(const ca_shape* s) {
+  const int BH = s->B * s->H;
+  return BH < kHostGroups ? BH : kHostGroups;
+}
+
+// Shape of group g: B = 1, H = the group's head count; first flattened head in *first.
+ca_shape group_shape(const ca_shape* s, int g, int G, int* first) {
+  const int BH = s->B * s->H, base = BH / G, extra = BH % G;
+  *first = g * base + (g < extra ? g : extra);
+  ca_shape gs = *s;
+  gs.B = 1;
+  gs.H = base + (g < extra ? 1 : 0);
+  return gs;
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t ca_forward_host_workspace_bytes(const ca_shape* s, int k) {
-  const size_t base = ca_forward_workspace_bytes(s, k);
+  if (check_shape(s) != CA_OK) return 0;
+  int first = 0;
+  const ca_shape g0 = group_shape(s, 0, host_groups(s), &first);   // the largest group
+  const size_t base = ca_forward_workspace_bytes(&g0, k);
   if (!base) return 0;
   const size_t esz = s->dtype == CA_BF16 ? 2 : 4;
   const size_t t = (size_t)s->B * s->H * s->N_alloc * s->d * esz;
@@ -312,27 +344,78 @@ ca_status ca_forward_host(const void* Qh, const void* Kh, const void* Vh, const 
   ca_status st = check_shape(s);
   if (st != CA_OK) return st;
   if (!Qh || !Kh || !Vh || !Oh) return CA_ERR_INVALID_ARG;
+  if ((st = check_params(s, params)) != CA_OK) return st;
   const size_t need = ca_forward_host_workspace_bytes(s, k);
   if (!need) return CA_ERR_INVALID_ARG;
   if (workspace_bytes < need) return CA_ERR_WORKSPACE;
   if (!workspace) return CA_ERR_INVALID_ARG;
+  const int G = host_groups(s);
   const size_t esz = s->dtype == CA_BF16 ? 2 : 4;
-  const size_t t = (size_t)s->B * s->H * s->N_alloc * s->d * esz;
+  const size_t head_bytes = (size_t)s->N_alloc * s->d * esz;
+  const size_t t = (size_t)s->B * s->H * head_bytes;
   char* ws = static_cast<char*>(workspace);
-  const size_t base = ca_forward_workspace_bytes(s, k);
+  int first = 0;
+  const ca_shape g0 = group_shape(s, 0, G, &first);
+  const size_t base = ca_forward_workspace_bytes(&g0, k);
   char* dQ = ws + base;
   char* dK = dQ + align_up(t);
   char* dV = dK + align_up(t);
   char* dO = dV + align_up(t);
+  ca_cluster_params p = {8, 1, 1, 0, 0ull, 0, 0};
+  if (params) p = *params;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemcpyAsync(dQ, Qh, t, cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dK, Kh, t, cudaMemcpyHostToDevice, cs);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dV, Vh, t, cudaMemcpyHostToDevice, cs);
-  if (e != cudaSuccess) return cuda_status(e);
-  st = ca_forward(dQ, dK, dV, s, params, k, compensate, dO, ws, base, stream);
+  // helper streams for the two copy directions, and their events
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_in[kHostGroups] = {}, ev_out[kHostGroups] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+  for (int g = 0; g < G && e == cudaSuccess; ++g) {
+    e = cudaEventCreateWithFlags(&ev_in[g], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[g], cudaEventDisableTiming);
+  }
+  // the inputs must not be overwritten before earlier work on `stream` is done with them
+  cudaEvent_t ev_start = nullptr;
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, cs);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_start, 0);
+  for (int g = 0; g < G && e == cudaSuccess; ++g) {
+    int b0 = 0;
+    const ca_shape gs = group_shape(s, g, G, &b0);
+    const size_t off = (size_t)b0 * head_bytes, bytes = (size_t)gs.H * head_bytes;
+    e = cudaMemcpyAsync(dQ + off, static_cast<const char*>(Qh) + off, bytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dK + off, static_cast<const char*>(Kh) + off, bytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dV + off, static_cast<const char*>(Vh) + off, bytes, cudaMemcpyHostToDevice, s_in);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[g], s_in);
+  }
+  for (int g = 0; g < G && e == cudaSuccess && st == CA_OK; ++g) {
+    int b0 = 0;
+    const ca_shape gs = group_shape(s, g, G, &b0);
+    const size_t off = (size_t)b0 * head_bytes, bytes = (size_t)gs.H * head_bytes;
+    e = cudaStreamWaitEvent(cs, ev_in[g], 0);
+    if (e != cudaSuccess) break;
+    ca_cluster_params pg = p;
+    pg.head_base = p.head_base + b0;
+    st = ca_forward(dQ + off, dK + off, dV + off, &gs, &pg, k, compensate, dO + off, ws, base, stream);
+    if (st != CA_OK) break;
+    e = cudaEventRecord(ev_out[g], cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_out[g], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(Oh) + off, dO + off, bytes, cudaMemcpyDeviceToHost, s_out);
+  }
+  // wait for everything issued on the three streams, then release the helpers
+  if (s_in) { const cudaError_t e2 = cudaStreamSynchronize(s_in); if (e == cudaSuccess) e = e2; }
+  { const cudaError_t e2 = cudaStreamSynchronize(cs); if (e == cudaSuccess) e = e2; }
+  if (s_out) { const cudaError_t e2 = cudaStreamSynchronize(s_out); if (e == cudaSuccess) e = e2; }
+  for (int g = 0; g < G; ++g) {
+    if (ev_in[g]) cudaEventDestroy(ev_in[g]);
+    if (ev_out[g]) cudaEventDestroy(ev_out[g]);
+  }
+  if (ev_start) cudaEventDestroy(ev_start);
+  if (s_in) cudaStreamDestroy(s_in);
+  if (s_out) cudaStreamDestroy(s_out);
   if (st != CA_OK) return st;
-  e = cudaMemcpyAsync(Oh, dO, t, cudaMemcpyDeviceToHost, cs);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   return cuda_status(e);
 }
 

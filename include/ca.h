@@ -280,10 +280,16 @@ ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * ca_forward_host -- ca_forward on HOST buffers: copies Q, K, V (host, ideally
- * pinned) into device staging carved from the workspace, runs the forward,
- * copies O back to host, all on `stream`, and synchronises the stream before
- * returning. workspace >= ca_forward_host_workspace_bytes(shape, k).
+ * ca_forward_host -- ca_forward on HOST buffers: copies Q, K, V (host; pinned
+ * memory lets the copies overlap the work) into device staging carved from
+ * the workspace, runs the forward, copies O back to host, and synchronises
+ * before returning. The heads are processed in up to four groups (contiguous
+ * ranges of the flattened heads, keyed by their global index as with
+ * head_base, so the result equals the whole-layer ca_forward): the copy of a
+ * group's inputs overlaps the forward of the previous group, and the copy of
+ * a group's output the forward of the next. The forward runs on `stream`;
+ * the copies on two short-lived helper streams that start after the work
+ * already queued on `stream`. workspace >= ca_forward_host_workspace_bytes(shape, k).
  */
 size_t ca_forward_host_workspace_bytes(const ca_shape* shape, int k);
 ca_status ca_forward_host(const void* Q_host, const void* K_host, const void* V_host,
