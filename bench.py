@@ -93,12 +93,24 @@ def needs_flush(w):
     return input_bytes(w) < 2 * L2_BYTES
 
 
+def key_size(w):
+    """Key cluster size of a workload (the query cluster size c unless set)."""
+    return getattr(w, "c_k", 0) or w.c
+
+
+def key_clusters(w):
+    return -(-w.n_valid // key_size(w))
+
+
 def workload_config(w):
     mb = input_bytes(w) / 3 / 1e6
     l2 = (f"L2 flushed (512 MB write) before every timed step: Q, K, V are 3 x {mb:.1f} MB" if needs_flush(w)
           else f"inputs larger than L2: Q, K, V are 3 x {mb:.0f} MB per layer (L2 126 MB)")
-    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N_alloc, "n_valid": w.n_valid, "d": w.d, "c": w.c,
-            "k": w.k, "clusters": w.C, "compensate": bool(w.compensate), "input_dtype": w.dtype, "l2": l2}
+    out = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N_alloc, "n_valid": w.n_valid, "d": w.d, "c": w.c,
+           "k": w.k, "clusters": w.C, "compensate": bool(w.compensate), "input_dtype": w.dtype, "l2": l2}
+    if key_size(w) != w.c:
+        out.update(c_k=key_size(w), key_clusters=key_clusters(w))
+    return out
 
 
 def dense_flops(w):
@@ -111,15 +123,16 @@ def attention_flops(w, kept_counts=None, count_q=None):
     the kept clusters' c keys per query) plus the compensation terms of the
     excluded clusters. With adaptive selection the per-query-cluster kept
     counts (and the query-cluster sizes) give the sums."""
+    ck, Ck = key_size(w), key_clusters(w)
     if kept_counts is None:
-        kept = 4.0 * w.n_valid * (w.k * w.c) * w.d * w.H * w.B
-        smc = 4.0 * w.n_valid * (w.C - w.k) * w.d * w.H * w.B if w.compensate else 0.0
+        kept = 4.0 * w.n_valid * (w.k * ck) * w.d * w.H * w.B
+        smc = 4.0 * w.n_valid * (Ck - w.k) * w.d * w.H * w.B if w.compensate else 0.0
         return kept, smc
     import numpy as np
     kc = np.asarray(kept_counts, np.float64)
     nq = np.asarray(count_q, np.float64)
-    kept = float(4.0 * (nq * kc * w.c).sum() * w.d)
-    smc = float(4.0 * (nq * (w.C - kc)).sum() * w.d) if w.compensate else 0.0
+    kept = float(4.0 * (nq * kc * ck).sum() * w.d)
+    smc = float(4.0 * (nq * (Ck - kc)).sum() * w.d) if w.compensate else 0.0
     return kept, smc
 
 
@@ -229,20 +242,20 @@ def oracle_sample(w, n_clusters=48, heads=(0,), keep=None, selection="topk", rec
         Qf, Kf, Vf = (x[0, h, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         t0 = time.perf_counter()
         if clustering == "random":
-            hc = orc.cluster_head_random(Qf, Kf, w.c, seed=0, bh=h)
+            hc = orc.cluster_head_random(Qf, Kf, w.c, seed=0, bh=h, c_k=key_size(w))
             kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
         elif selection == "adaptive":
-            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, query_form="adaptive",
+            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, query_form="adaptive", c_k=key_size(w),
                                   splitting="diagonal" if clustering == "diagonal" else "basic")
             kept = orc.adaptive_route(orc.centroid_scores(hc.qbar, hc.kbar), hc.count_k, w.d, recall, 16)
         else:
-            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h,
+            hc = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=h, c_k=key_size(w),
                                   splitting="diagonal" if clustering == "diagonal" else "basic")
             kept = orc.topk_route(orc.centroid_scores(hc.qbar, hc.kbar), w.k)
         t1 = time.perf_counter()
         sample = list(range(0, w.C, max(1, w.C // n_clusters)))[:n_clusters]
         out = orc.compensated_attention(Qf, Kf, Vf, hc.perm_q, hc.count_q, hc.perm_k, hc.count_k, kept, w.c,
-                                        compensate=w.compensate, clusters=sample)
+                                        compensate=w.compensate, clusters=sample, c_k=key_size(w))
         t2 = time.perf_counter()
         t_head.append((t1 - t0) + (t2 - t1) * w.C / len(sample))
         if keep is not None and h == heads[0]:
@@ -284,8 +297,25 @@ def build_workload(args, rank: int):
                                 seed=rank_seed(rank, 2), compensate=args.smc == "on",
                                 name=f"cfg2gen-lowrank-N{args.tokens}-d64-bf16-k{min(kk, C)}", rank=16,
                                 noise=0.1)
-    return wl.config_workload(args.config, seed=rank_seed(rank, args.config),
-                              **({"compensate": False} if args.smc == "off" else {}))
+    w = wl.config_workload(args.config, seed=rank_seed(rank, args.config),
+                           **({"compensate": False} if args.smc == "off" else {}))
+    return with_cluster_sizes(w, args)
+
+
+def with_cluster_sizes(w, args):
+    """--cq / --ck: other query / key cluster sizes on the same inputs, keeping
+    the configuration's fraction of key clusters."""
+    if not (getattr(args, "cq", 0) or getattr(args, "ck", 0)):
+        return w
+    import dataclasses
+    cq = args.cq or w.c
+    ck = args.ck or w.c
+    keep = w.k / w.C
+    Ck = -(-w.n_valid // ck)
+    k = max(1, min(Ck, math.ceil(keep * Ck - 1e-9)))
+    w2 = dataclasses.replace(w, c=cq, k=k, name=f"{w.name}-cq{cq}-ck{ck}")
+    object.__setattr__(w2, "c_k", ck)
+    return w2
 
 
 def run_reference(args):
@@ -360,10 +390,10 @@ def affinity_cores():
 
 def make_layer(ca, w, args, head_base=0):
     adaptive = args.selection == "adaptive"
-    return ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, w.C if adaptive else w.k,
+    return ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, key_clusters(w) if adaptive else w.k,
                                dtype=w.dtype, compensate=w.compensate, selection=args.selection,
                                recall=args.recall, min_count=16, clustering=args.clustering,
-                               head_base=head_base)
+                               head_base=head_base, c_k=getattr(w, "c_k", 0))
 
 
 def head_share(w, world, rank):
@@ -724,6 +754,11 @@ def main():
     ap.add_argument("--tokens", type=int, default=0,
                     help="latency scaling: configuration 2's generator at this token count")
     ap.add_argument("--fixed-k", action="store_true", help="with --tokens: keep 64 clusters instead of 1/8")
+    ap.add_argument("--cq", type=int, default=0, choices=[0, 64, 128, 256],
+                    help="query cluster size (default: the configuration's)")
+    ap.add_argument("--ck", type=int, default=0, choices=[0, 64, 128, 256],
+                    help="key cluster size (default: the query cluster size); --cq 64 --ck 128 is the paper's "
+                         "evaluated block shape")
     ap.add_argument("--shard", choices=["heads", "layers"], default="heads",
                     help="with N > 1 GPUs: split one layer's heads over the GPUs (default) or run an independent "
                          "layer per GPU")

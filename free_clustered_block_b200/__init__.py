@@ -28,7 +28,7 @@ EXPORTED = [
     "ca_dense_attend", "ca_forward", "ca_forward_host_workspace_bytes", "ca_forward_host",
     "ca_get_device_error", "ca_set_wait_limit", "ca_check_bounded_wait", "ca_status_string", "ca_version", "ca_launch_count",
     "ca_cluster_noalloc", "ca_route_adaptive", "ca_check_exp2_poly",
-    "ca_attend_prepare", "ca_attend_prepared",
+    "ca_attend_prepare", "ca_attend_prepared", "ca_num_key_clusters",
 ]
 
 
@@ -45,7 +45,7 @@ class CAError(RuntimeError):
 class ca_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N_alloc", ctypes.c_int),
                 ("n_valid", ctypes.c_int), ("d", ctypes.c_int), ("c", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("c_k", ctypes.c_int)]
 
 
 class ca_cluster_params(ctypes.Structure):
@@ -78,6 +78,7 @@ def lib():
         vp, sz, i32, u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint64
         sig = {
             "ca_num_clusters": (i32, [P(ca_shape)]),
+            "ca_num_key_clusters": (i32, [P(ca_shape)]),
             "ca_check_shape": (i32, [P(ca_shape)]),
             "ca_cluster_workspace_bytes": (sz, [P(ca_shape)]),
             "ca_attend_workspace_bytes": (sz, [P(ca_shape)]),
@@ -134,8 +135,9 @@ def _stream(stream) -> Optional[int]:
     return getattr(stream, "cuda_stream", stream)
 
 
-def make_shape(B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, dtype: int) -> ca_shape:
-    return ca_shape(B, H, N_alloc, n_valid, d, c, dtype)
+def make_shape(B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, dtype: int, c_k: int = 0) -> ca_shape:
+    """c: query cluster size; c_k: key cluster size (0: the same as c)."""
+    return ca_shape(B, H, N_alloc, n_valid, d, c, dtype, c_k)
 
 
 def make_params(power_iters: int = 8, sample_factor: int = 1, transform: int = 1,
@@ -150,7 +152,13 @@ def make_params(power_iters: int = 8, sample_factor: int = 1, transform: int = 1
 
 
 def num_clusters(shape: ca_shape) -> int:
+    """Query clusters C."""
     return lib().ca_num_clusters(ctypes.byref(shape))
+
+
+def num_key_clusters(shape: ca_shape) -> int:
+    """Key clusters C_k."""
+    return lib().ca_num_key_clusters(ctypes.byref(shape))
 
 
 def cluster_workspace_bytes(shape: ca_shape) -> int:

@@ -26,14 +26,19 @@ ca_status check_shape(const ca_shape* s) {
   if (s->dtype != CA_BF16 && s->dtype != CA_FP32) return CA_ERR_INVALID_ARG;
   if (s->d != 64 && s->d != 128) return CA_ERR_UNSUPPORTED;
   if (s->c != 64 && s->c != 128 && s->c != 256) return CA_ERR_UNSUPPORTED;
+  if (s->c_k != 0 && s->c_k != 64 && s->c_k != 128 && s->c_k != 256) return CA_ERR_UNSUPPORTED;
   // every per-head index fits in int32; whole tensors fit in size_t
   const long long C = ((long long)s->n_valid + s->c - 1) / s->c;
-  if ((long long)s->N_alloc > (1ll << 30) || C * s->c > (1ll << 30)) return CA_ERR_UNSUPPORTED;
+  const long long ck = s->c_k ? s->c_k : s->c;
+  const long long Ck = ((long long)s->n_valid + ck - 1) / ck;
+  if ((long long)s->N_alloc > (1ll << 30) || C * s->c > (1ll << 30) || Ck * ck > (1ll << 30))
+    return CA_ERR_UNSUPPORTED;
   if ((long long)s->B * s->H > 65535) return CA_ERR_UNSUPPORTED;   // grid.y
   return CA_OK;
 }
 
 bool plan_for(const ca_shape* s, TreePlan* plan) { return host_plan(s->n_valid, s->c, plan); }
+bool plan_for_keys(const ca_shape* s, TreePlan* plan) { return host_plan(s->n_valid, key_c(s), plan); }
 
 size_t dir_smem(int d, int a) {
   // one warp's share of the per-node kernel (fp32 sample rows, the larger case) plus M
@@ -68,23 +73,24 @@ struct ForwardWs {
 };
 
 bool forward_layout(const ca_shape* s, int k, ForwardWs* f) {
-  TreePlan plan;
-  if (!plan_for(s, &plan)) return false;
+  TreePlan plan, plan_k;
+  if (!plan_for(s, &plan) || !plan_for_keys(s, &plan_k)) return false;
   ClusterWs cw;
   AttendWs aw;
-  cluster_ws_layout(s, plan, &cw);
+  cluster_ws_layout(s, plan, plan_k, &cw);
   attend_ws_layout(s, &aw);
   const size_t BH = (size_t)s->B * s->H, C = plan.C, c = s->c, d = s->d;
+  const size_t Ck = plan_k.C, ck = key_c(s);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
   f->perm_q = take(BH * C * c * 4);
-  f->perm_k = take(BH * C * c * 4);
+  f->perm_k = take(BH * Ck * ck * 4);
   f->count_q = take(BH * C * 4);
-  f->count_k = take(BH * C * 4);
+  f->count_k = take(BH * Ck * 4);
   f->qbar = take(BH * C * d * 8);
-  f->kbar = take(BH * C * d * 8);
+  f->kbar = take(BH * Ck * d * 8);
   f->kept_idx = take(BH * C * (size_t)k * 4);
-  f->kept_bits = take(BH * C * ((C + 31) / 32) * 4);
+  f->kept_bits = take(BH * C * ((Ck + 31) / 32) * 4);
   f->cluster_bytes = cw.total;
   f->attend_bytes = aw.total;
   f->scratch = take(cw.total > aw.total ? cw.total : aw.total);
@@ -98,17 +104,22 @@ extern "C" {
 
 int ca_num_clusters(const ca_shape* s) {
   if (check_shape(s) != CA_OK) return -1;
-  return (s->n_valid + s->c - 1) / s->c;
+  return num_q_clusters(s);
+}
+
+int ca_num_key_clusters(const ca_shape* s) {
+  if (check_shape(s) != CA_OK) return -1;
+  return num_k_clusters(s);
 }
 
 ca_status ca_check_shape(const ca_shape* s) { return check_shape(s); }
 
 size_t ca_cluster_workspace_bytes(const ca_shape* s) {
   if (check_shape(s) != CA_OK) return 0;
-  TreePlan plan;
-  if (!plan_for(s, &plan)) return 0;
+  TreePlan plan, plan_k;
+  if (!plan_for(s, &plan) || !plan_for_keys(s, &plan_k)) return 0;
   ClusterWs w;
-  cluster_ws_layout(s, plan, &w);
+  cluster_ws_layout(s, plan, plan_k, &w);
   return w.total;
 }
 
@@ -126,8 +137,7 @@ size_t ca_dense_workspace_bytes(const ca_shape* s) {
 
 size_t ca_forward_workspace_bytes(const ca_shape* s, int k) {
   if (check_shape(s) != CA_OK) return 0;
-  const int C = (s->n_valid + s->c - 1) / s->c;
-  if (k < 1 || k > C) return 0;
+  if (k < 1 || k > num_k_clusters(s)) return 0;
   ForwardWs f;
   if (!forward_layout(s, k, &f)) return 0;
   return f.total;
@@ -142,15 +152,15 @@ ca_status ca_cluster(const void* Q, const void* K, const ca_shape* s, const ca_c
     return CA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K)) return CA_ERR_INVALID_ARG;
   if ((st = check_params(s, params)) != CA_OK) return st;
-  TreePlan plan;
-  if (!plan_for(s, &plan)) return CA_ERR_UNSUPPORTED;
+  TreePlan plan, plan_k;
+  if (!plan_for(s, &plan) || !plan_for_keys(s, &plan_k)) return CA_ERR_UNSUPPORTED;
   ClusterWs L;
-  cluster_ws_layout(s, plan, &L);
+  cluster_ws_layout(s, plan, plan_k, &L);
   if (workspace_bytes < L.total) return CA_ERR_WORKSPACE;
   if (!workspace) return CA_ERR_INVALID_ARG;
   ca_cluster_params p = {8, 1, 1, 0, 0ull, 0, 0};
   if (params) p = *params;
-  return cuda_status(launch_cluster(Q, K, s, &p, out, plan, L, static_cast<char*>(workspace),
+  return cuda_status(launch_cluster(Q, K, s, &p, out, plan, plan_k, L, static_cast<char*>(workspace),
                                     static_cast<cudaStream_t>(stream)));
 }
 
@@ -159,10 +169,10 @@ ca_status ca_route(const ca_shape* s, const ca_clusters* cen, const ca_routes* o
   if (st != CA_OK) return st;
   if (!cen || !cen->qbar || !cen->kbar || !out || !out->kept_idx || !out->kept_bits) return CA_ERR_INVALID_ARG;
   if (!aligned16(cen->qbar) || !aligned16(cen->kbar)) return CA_ERR_INVALID_ARG;
-  const int C = (s->n_valid + s->c - 1) / s->c;
-  if (out->k < 1 || out->k > C) return CA_ERR_INVALID_ARG;
-  if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
-  return cuda_status(launch_route(s, C, cen->qbar, cen->kbar, out->k, out->kept_idx, out->kept_bits,
+  const int C = num_q_clusters(s), Ck = num_k_clusters(s);
+  if (out->k < 1 || out->k > Ck) return CA_ERR_INVALID_ARG;
+  if (C > kMaxRouteC || Ck > kMaxRouteC) return CA_ERR_UNSUPPORTED;
+  return cuda_status(launch_route(s, C, Ck, cen->qbar, cen->kbar, out->k, out->kept_idx, out->kept_bits,
                                   out->kept_count, static_cast<cudaStream_t>(stream)));
 }
 
@@ -175,10 +185,10 @@ ca_status ca_route_adaptive(const ca_shape* s, const ca_clusters* cen, double re
     return CA_ERR_INVALID_ARG;
   if (!aligned16(cen->qbar) || !aligned16(cen->kbar)) return CA_ERR_INVALID_ARG;
   if (!(recall >= 0.0 && recall <= 1.0) || min_count < 1) return CA_ERR_INVALID_ARG;
-  const int C = (s->n_valid + s->c - 1) / s->c;
-  if (out->k < 1 || out->k > C) return CA_ERR_INVALID_ARG;
-  if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
-  return cuda_status(launch_route_adaptive(s, C, cen->qbar, cen->kbar, cen->count_k, recall, min_count, out->k,
+  const int C = num_q_clusters(s), Ck = num_k_clusters(s);
+  if (out->k < 1 || out->k > Ck) return CA_ERR_INVALID_ARG;
+  if (C > kMaxRouteC || Ck > kMaxRouteC) return CA_ERR_UNSUPPORTED;
+  return cuda_status(launch_route_adaptive(s, C, Ck, cen->qbar, cen->kbar, cen->count_k, recall, min_count, out->k,
                                            out->kept_idx, out->kept_bits, out->kept_count,
                                            static_cast<cudaStream_t>(stream)));
 }
@@ -195,8 +205,7 @@ ca_status check_attend(const void* Q, const void* K, const void* V, const ca_sha
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return CA_ERR_INVALID_ARG;
   if (rt) {
     if (!O || !rt->kept_idx || !rt->kept_bits || !aligned16(O)) return CA_ERR_INVALID_ARG;
-    const int C = (s->n_valid + s->c - 1) / s->c;
-    if (rt->k < 1 || rt->k > C) return CA_ERR_INVALID_ARG;
+    if (rt->k < 1 || rt->k > num_k_clusters(s)) return CA_ERR_INVALID_ARG;
   }
   attend_ws_layout(s, L);
   if (workspace_bytes < L->total) return CA_ERR_WORKSPACE;
@@ -271,9 +280,8 @@ ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape
   if (!Q || !K || !V || !O) return CA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return CA_ERR_INVALID_ARG;
   if ((st = check_params(s, params)) != CA_OK) return st;
-  const int C = (s->n_valid + s->c - 1) / s->c;
-  if (k < 1 || k > C) return CA_ERR_INVALID_ARG;
-  if (C > kMaxRouteC) return CA_ERR_UNSUPPORTED;
+  if (k < 1 || k > num_k_clusters(s)) return CA_ERR_INVALID_ARG;
+  if (num_q_clusters(s) > kMaxRouteC || num_k_clusters(s) > kMaxRouteC) return CA_ERR_UNSUPPORTED;
   ForwardWs f;
   if (!forward_layout(s, k, &f)) return CA_ERR_UNSUPPORTED;
   if (workspace_bytes < f.total) return CA_ERR_WORKSPACE;
@@ -452,11 +460,15 @@ int ca_launch_count(const ca_shape* s, int stage) {
   const int pad = s->N_alloc > s->n_valid ? 1 : 0;
   switch (stage) {
     case 0: {
-      TreePlan plan;
-      if (!plan_for(s, &plan)) return -1;
+      TreePlan plan, plan_k;
+      if (!plan_for(s, &plan) || !plan_for_keys(s, &plan_k)) return -1;
       // plan, colsum, syrk, metric reduce, query norms; per level: direction,
       // projection, select, partition count, partition scatter; centroids.
-      return plan.levels > 0 ? 5 + 5 * plan.levels + 1 : 1;
+      // With unequal sizes each tensor walks its own tree (a plan and a
+      // centroid launch each).
+      if (key_c(s) == s->c) return plan.levels > 0 ? 5 + 5 * plan.levels + 1 : 1;
+      const bool any = plan.levels > 0 || plan_k.levels > 0;
+      return (any ? 2 + 4 : 0) + 5 * (plan.levels + plan_k.levels) + 2;
     }
     case 1: return 1;
     case 2: return (s->dtype == CA_BF16 ? 2 : 1) + 1 + pad;   // prep (+ permute), attention, pad rows

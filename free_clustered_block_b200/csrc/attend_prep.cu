@@ -68,15 +68,18 @@ __global__ void __launch_bounds__(256) centroid_prep_kernel(
 }
 
 // Cluster-ordered copy: dst[bh][slot] = src[bh][perm[slot]] (zero for pad
-// slots). One 16-byte vector per thread; blockIdx.z selects Q / K / V.
+// slots). One 16-byte vector per thread; blockIdx.z selects Q / K / V. The
+// queries have slots_q slots per head (query clusters of c), keys and values
+// slots_k (key clusters of c_k).
 template <int D>
 __global__ void __launch_bounds__(256) permute_rows_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-    const __nv_bfloat16* __restrict__ V, int N_alloc, int slots, const int32_t* __restrict__ perm_q,
+    const __nv_bfloat16* __restrict__ V, int N_alloc, int slots_q, int slots_k, const int32_t* __restrict__ perm_q,
     const int32_t* __restrict__ perm_k, __nv_bfloat16* __restrict__ Qp, __nv_bfloat16* __restrict__ Kp,
     __nv_bfloat16* __restrict__ Vp) {
   constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
   const int bh = blockIdx.y, z = blockIdx.z;
+  const int slots = z == 0 ? slots_q : slots_k;
   const __nv_bfloat16* src = (z == 0 ? Q : (z == 1 ? K : V)) + (size_t)bh * N_alloc * D;
   __nv_bfloat16* dst = (z == 0 ? Qp : (z == 1 ? Kp : Vp)) + (size_t)bh * slots * D;
   const int32_t* perm = (z == 0 ? perm_q : perm_k) + (size_t)bh * slots;
@@ -102,21 +105,21 @@ __global__ void zero_rows_kernel(uint4* __restrict__ O, size_t row_vecs, size_t 
 }  // namespace
 
 bool attend_ws_layout(const ca_shape* s, AttendWs* w) {
-  const size_t BH = (size_t)s->B * s->H, d = s->d, c = s->c;
-  const size_t C = (s->n_valid + c - 1) / c;
-  const size_t Cpad = (C + 127) / 128 * 128;
-  w->C = (int)C; w->Cpad = (int)Cpad;
+  const size_t BH = (size_t)s->B * s->H, d = s->d, c = s->c, ck = key_c(s);
+  const size_t C = num_q_clusters(s), Ck = num_k_clusters(s);
+  const size_t Cpad = (Ck + 127) / 128 * 128;
+  w->C = (int)C; w->Ck = (int)Ck; w->Cpad = (int)Cpad;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
   const bool tc = (s->dtype == CA_BF16);
-  const size_t rows = BH * C * c * d * 2;
-  w->qp = take(tc ? rows : 0);
-  w->kp = take(tc ? rows : 0);
-  w->vp = take(tc ? rows : 0);
+  const size_t rows_q = BH * C * c * d * 2, rows_k = BH * Ck * ck * d * 2;
+  w->qp = take(tc ? rows_q : 0);
+  w->kp = take(tc ? rows_k : 0);
+  w->vp = take(tc ? rows_k : 0);
   w->kbar_hl = take(BH * Cpad * 2 * d * 2);
   w->vbar_hl = take(BH * Cpad * 2 * d * 2);
-  w->vbar32 = take(BH * C * d * 4);
-  w->kbar32 = take(BH * C * d * 4);
+  w->vbar32 = take(BH * Ck * d * 4);
+  w->kbar32 = take(BH * Ck * d * 4);
   w->logcnt = take(BH * Cpad * 4);
   w->total = o;
   return true;
@@ -124,7 +127,8 @@ bool attend_ws_layout(const ca_shape* s, AttendWs* w) {
 
 cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, const ca_shape* s,
                                const ca_clusters* cl, const AttendWs& L, char* ws, cudaStream_t st) {
-  const int BH = s->B * s->H, C = L.C, Cpad = L.Cpad, c = s->c;
+  // key centroids: C key clusters of c = c_k slots
+  const int BH = s->B * s->H, C = L.Ck, Cpad = L.Cpad, c = key_c(s);
   float* kbar32 = reinterpret_cast<float*>(ws + L.kbar32);
   float* vbar32 = reinterpret_cast<float*>(ws + L.vbar32);
   __nv_bfloat16* khl = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_hl);
@@ -139,18 +143,19 @@ cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, cons
     else
       centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
                                                       cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
-    const int slots = C * c;
+    const int slots_q = L.C * s->c, slots_k = C * c;
+    const int slots = slots_q > slots_k ? slots_q : slots_k;
     const size_t vecs = (size_t)slots * (s->d * 2 / 16);
     const dim3 gp((unsigned)((vecs + 255) / 256), BH, 3);
     T* Qp = reinterpret_cast<T*>(ws + L.qp);
     T* Kp = reinterpret_cast<T*>(ws + L.kp);
     T* Vp = reinterpret_cast<T*>(ws + L.vp);
     if (s->d == 64)
-      permute_rows_kernel<64><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc, slots,
-                                                  cl->perm_q, cl->perm_k, Qp, Kp, Vp);
+      permute_rows_kernel<64><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc, slots_q,
+                                                  slots_k, cl->perm_q, cl->perm_k, Qp, Kp, Vp);
     else
       permute_rows_kernel<128><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc,
-                                                   slots, cl->perm_q, cl->perm_k, Qp, Kp, Vp);
+                                                   slots_q, slots_k, cl->perm_q, cl->perm_k, Qp, Kp, Vp);
   } else {
     using T = float;
     if (s->d == 64)

@@ -72,7 +72,7 @@ __device__ __forceinline__ void simt_tile(SimtState<D>& st, const float* Ks, con
 template <typename T, int D>
 __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, int N_alloc, int n_valid,
-    int c, int C, int k, const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
+    int c, int C, int ck, int Ck, int k, const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
     const int32_t* __restrict__ kept_idx, const uint32_t* __restrict__ kept_bits,
     const int32_t* __restrict__ kept_count, const float* __restrict__ kbar32, const float* __restrict__ vbar32, const float* __restrict__ logcnt,
     int Cpad, int compensate, int mode, float scale, T* __restrict__ O) {
@@ -116,15 +116,15 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
   };
   if (mode == 0) {
     const int32_t* kl = kept_idx + ((size_t)bh * C + a) * k;
-    const int32_t* pk = perm_k + (size_t)bh * C * c;
+    const int32_t* pk = perm_k + (size_t)bh * Ck * ck;
     // k each, or the query cluster's own count after adaptive selection
     const int kq = kept_count ? min(max(kept_count[(size_t)bh * C + a], 0), k) : k;
     for (int i = 0; i < kq; ++i) {
       const int b = kl[i];
-      for (int t0 = 0; t0 < c; t0 += kTile) {
+      for (int t0 = 0; t0 < ck; t0 += kTile) {
         __syncthreads();
         if (threadIdx.x < kTile) {
-          const int kr = pk[b * c + t0 + threadIdx.x];
+          const int kr = pk[b * ck + t0 + threadIdx.x];
           krow[threadIdx.x] = kr;
           bias[threadIdx.x] = kr >= 0 ? 0.f : -INFINITY;
         }
@@ -135,19 +135,19 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
       }
     }
     if (compensate) {
-      const uint32_t* kb = kept_bits + ((size_t)bh * C + a) * ((C + 31) / 32);
-      for (int b0 = 0; b0 < C; b0 += kTile) {
+      const uint32_t* kb = kept_bits + ((size_t)bh * C + a) * ((Ck + 31) / 32);
+      for (int b0 = 0; b0 < Ck; b0 += kTile) {
         __syncthreads();
         if (threadIdx.x < kTile) {
           const int b = b0 + threadIdx.x;
           float bs = -INFINITY;
-          if (b < C && !((kb[b >> 5] >> (b & 31)) & 1u)) bs = logcnt[(size_t)bh * Cpad + b];
+          if (b < Ck && !((kb[b >> 5] >> (b & 31)) & 1u)) bs = logcnt[(size_t)bh * Cpad + b];
           bias[threadIdx.x] = bs;
         }
         for (int e = threadIdx.x; e < kTile * D; e += NT) {
           const int j = e / D, col = e % D, b = b0 + j;
-          Ks[e] = b < C ? kbar32[((size_t)bh * C + b) * D + col] : 0.f;
-          Vs[e] = b < C ? vbar32[((size_t)bh * C + b) * D + col] : 0.f;
+          Ks[e] = b < Ck ? kbar32[((size_t)bh * Ck + b) * D + col] : 0.f;
+          Vs[e] = b < Ck ? vbar32[((size_t)bh * Ck + b) * D + col] : 0.f;
         }
         __syncthreads();
         simt_tile<D>(st, Ks, Vs, bias, scale, p);
@@ -179,8 +179,8 @@ template <typename T, int D>
 cudaError_t run_simt(const void* Q, const void* K, const void* V, const ca_shape* s, const ca_clusters* cl,
                      const ca_routes* rt, int compensate, void* O, const AttendWs* L, char* ws, int mode,
                      cudaStream_t st) {
-  const int BH = s->B * s->H, c = s->c;
-  const int C = (s->n_valid + c - 1) / c;
+  const int BH = s->B * s->H, c = s->c, ck = key_c(s);
+  const int C = num_q_clusters(s), Ck = num_k_clusters(s);
   const float scale = 1.0f / sqrtf((float)D);
   dim3 grid;
   if (mode == 0) grid = dim3(C * (c / kRows), BH);
@@ -189,7 +189,7 @@ cudaError_t run_simt(const void* Q, const void* K, const void* V, const ca_shape
   const float* vbar32 = L ? reinterpret_cast<const float*>(ws + L->vbar32) : nullptr;
   const float* logcnt = L ? reinterpret_cast<const float*>(ws + L->logcnt) : nullptr;
   simt_attend_kernel<T, D><<<grid, kRows * (D / 16), 0, st>>>(
-      (const T*)Q, (const T*)K, (const T*)V, s->N_alloc, s->n_valid, c, C, rt ? rt->k : 0,
+      (const T*)Q, (const T*)K, (const T*)V, s->N_alloc, s->n_valid, c, C, ck, Ck, rt ? rt->k : 0,
       cl ? cl->perm_q : nullptr, cl ? cl->perm_k : nullptr, rt ? rt->kept_idx : nullptr,
       rt ? rt->kept_bits : nullptr, rt ? rt->kept_count : nullptr, kbar32, vbar32, logcnt, L ? L->Cpad : 0, compensate, mode, scale,
       (T*)O);

@@ -324,7 +324,9 @@ struct Watchdog {
 // Kernel parameters and per-tile bookkeeping
 // ---------------------------------------------------------------------------
 struct TcParams {
-  int C, c, k, Cpad, n_valid, N_alloc;
+  int C, c;                   // query clusters and their size
+  int Ck, ck;                 // key clusters and their size
+  int k, Cpad, n_valid, N_alloc;
   int tiles_per_cluster;      // c / 128 (1 when c = 64)
   int rows_per_tile;          // min(c, 128): query rows of a tile that belong to its cluster
   int n_tiles;                // sparse: query tiles over all heads
@@ -373,7 +375,7 @@ __device__ __forceinline__ Tile make_tile(const TcParams& p, int t) {
   T.a = rem / p.tiles_per_cluster;
   T.sub = rem % p.tiles_per_cluster;
   T.kq = p.kept_count ? min(max(p.kept_count[(size_t)T.bh * p.C + T.a], 0), p.k) : p.k;
-  T.J_kept = p.c >= 128 ? T.kq * (p.c / 128) : (T.kq + 1) / 2;
+  T.J_kept = p.ck >= 128 ? T.kq * (p.ck / 128) : (T.kq + 1) / 2;
   T.J = T.J_kept + p.J_cent;
   T.qrow = (T.bh * p.C + T.a) * p.c + T.sub * 128;
   return T;
@@ -533,14 +535,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int i = threadIdx.x; i < T0.kq; i += Cfg::kThreads) {
       const int b = kept_g0[i];
       kept_s[i] = b;
-      kcnt_s[i] = p.count_k[(size_t)T0.bh * p.C + b];
+      kcnt_s[i] = p.count_k[(size_t)T0.bh * p.Ck + b];
     }
   }
   if (kept_sm1 && T1.J > 0) {
     for (int i = threadIdx.x; i < T1.kq; i += Cfg::kThreads) {
       const int b = kept_g1[i];
       kept_s[Cfg::kMaxKept + i] = b;
-      kcnt_s[Cfg::kMaxKept + i] = p.count_k[(size_t)T1.bh * p.C + b];
+      kcnt_s[Cfg::kMaxKept + i] = p.count_k[(size_t)T1.bh * p.Ck + b];
     }
   }
   auto kept_at = [&](int t, int i) -> int {
@@ -576,7 +578,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint64_t limit = p.wait_limit;
   const int NI = T0.J + T1.J;                   // (tile, block) items
   const int NR = shared_kv ? T0.J : NI;         // ring items (one per item, or one per block when shared)
-  const int nsb = p.c >= 128 ? p.c / 128 : 1;   // key blocks per kept cluster (c >= 128)
+  const int nsb = p.ck >= 128 ? p.ck / 128 : 1;   // key blocks per kept cluster (c_k >= 128)
   // Ring index of block j of tile t: the producer fills the rings in the
   // interleaved order (0,0), (1,0), (0,1), (1,1), ... (or one entry per block
   // when the tiles share K/V); each tile consumes its own entries in order.
@@ -616,15 +618,15 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (p.dense) {
             tma_3d(d, mk, bar, sb * 64, j * 128, Tt.bh);
           } else if (j < Tt.J_kept) {
-            if (p.c >= 128) {
-              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.C + kept_at(t, j / nsb)) * p.c + (j % nsb) * 128);
+            if (p.ck >= 128) {
+              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.Ck + kept_at(t, j / nsb)) * p.ck + (j % nsb) * 128);
             } else {
               // two key clusters of 64; an odd count repeats the first (its
               // columns are masked, and its values stay finite)
               const int b0 = kept_at(t, 2 * j);
               const int b1 = (2 * j + 1 < Tt.kq) ? kept_at(t, 2 * j + 1) : b0;
-              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.C + b0) * 64);
-              tma_2d(d + 64 * 128, mk, bar, sb * 64, (Tt.bh * p.C + b1) * 64);
+              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.Ck + b0) * 64);
+              tma_2d(d + 64 * 128, mk, bar, sb * 64, (Tt.bh * p.Ck + b1) * 64);
             }
           } else {
             const int cb = j - Tt.J_kept;
@@ -786,12 +788,12 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float sc = p.scale_log2;
     float* bias = bias_w + warp * 64;
     const uint32_t* kb_row =
-        p.dense ? nullptr : p.kept_bits + ((size_t)Tt.bh * p.C + Tt.a) * ((p.C + 31) / 32);
+        p.dense ? nullptr : p.kept_bits + ((size_t)Tt.bh * p.C + Tt.a) * ((p.Ck + 31) / 32);
     // the tile's kept clusters' sizes: staged in shared memory, or read through the kept list
     const bool ksm = !p.dense && Tt.kq <= Cfg::kMaxKept;
     const int32_t* kcnt_t = kcnt_s + t * Cfg::kMaxKept;
     const int32_t* kept_t = p.dense ? nullptr : p.kept_idx + ((size_t)Tt.bh * p.C + Tt.a) * p.k;
-    const int32_t* cnt_h = p.count_k + (size_t)Tt.bh * p.C;
+    const int32_t* cnt_h = p.count_k + (size_t)Tt.bh * p.Ck;
     auto cnt_of = [&](int i) -> int { return ksm ? kcnt_t[i] : cnt_h[kept_t[i]]; };
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
@@ -830,7 +832,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const int e = h * 32 + lane;
           const int b = (j - Tt.J_kept) * 64 + e;
           float bv = -INFINITY;
-          if (b < p.C && !((kb_row[b >> 5] >> (b & 31)) & 1u)) bv = p.logcnt[(size_t)Tt.bh * p.Cpad + b] * log2e;
+          if (b < p.Ck && !((kb_row[b >> 5] >> (b & 31)) & 1u)) bv = p.logcnt[(size_t)Tt.bh * p.Cpad + b] * log2e;
           bias[e] = bv;
         }
         __syncwarp();
@@ -838,7 +840,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int rem = p.n_valid - j * 128;
         v0 = min(max(rem, 0), 64);
         v1 = min(max(rem - 64, 0), 64);
-      } else if (p.c >= 128) {
+      } else if (p.ck >= 128) {
         const int rem = cnt_of(j / nsb) - (j % nsb) * 128;
         v0 = min(max(rem, 0), 64);
         v1 = min(max(rem - 64, 0), 64);
@@ -993,23 +995,24 @@ cudaError_t dispatch(int D, const CUtensorMap maps[5], const TcParams& p, dim3 g
 
 cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_routes* rt, int compensate,
                              void* O, const AttendWs& L, char* ws, cudaStream_t st) {
-  const int BH = s->B * s->H, D = s->d, c = s->c, C = L.C;
-  const uint64_t slots = (uint64_t)BH * C * c;
+  const int BH = s->B * s->H, D = s->d, c = s->c, C = L.C, ck = key_c(s), Ck = L.Ck;
+  const uint64_t slots_q = (uint64_t)BH * C * c, slots_k = (uint64_t)BH * Ck * ck;
   const uint64_t cent_rows = (uint64_t)BH * L.Cpad * 2;   // hi and lo rows of every 64-centroid block
   CUtensorMap maps[5];
-  bool ok = make_map_2d(&maps[0], ws + L.qp, slots, D, 128) &&
-            make_map_2d(&maps[1], ws + L.kp, slots, D, c >= 128 ? 128 : 64) &&
-            make_map_2d(&maps[2], ws + L.vp, slots, D, c >= 128 ? 128 : 64) &&
+  bool ok = make_map_2d(&maps[0], ws + L.qp, slots_q, D, 128) &&
+            make_map_2d(&maps[1], ws + L.kp, slots_k, D, ck >= 128 ? 128 : 64) &&
+            make_map_2d(&maps[2], ws + L.vp, slots_k, D, ck >= 128 ? 128 : 64) &&
             make_map_2d(&maps[3], ws + L.kbar_hl, cent_rows, D, 128) &&
             make_map_2d(&maps[4], ws + L.vbar_hl, cent_rows, D, 128);
   if (!ok) return cudaErrorInvalidValue;
   TcParams p{};
-  p.C = C; p.c = c; p.k = rt->k; p.Cpad = L.Cpad; p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
+  p.C = C; p.c = c; p.Ck = Ck; p.ck = ck;
+  p.k = rt->k; p.Cpad = L.Cpad; p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
   p.tiles_per_cluster = c >= 128 ? c / 128 : 1;
   p.rows_per_tile = c >= 128 ? 128 : c;
   p.n_tiles = BH * C * p.tiles_per_cluster;
   p.compensate = compensate;
-  p.J_cent = compensate ? (C + 63) / 64 : 0;
+  p.J_cent = compensate ? (Ck + 63) / 64 : 0;
   p.dense = 0;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.perm_q = cl->perm_q; p.count_k = cl->count_k; p.kept_idx = rt->kept_idx; p.kept_bits = rt->kept_bits;
@@ -1066,7 +1069,7 @@ cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const c
   p.compensate = 0; p.J_cent = 0; p.dense = 1;
   p.dense_tiles = (s->n_valid + 127) / 128;
   p.dense_key_blocks = (s->n_valid + 127) / 128;
-  p.c = 128;
+  p.c = 128; p.ck = 128;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   p.O = static_cast<__nv_bfloat16*>(O);
   p.wait_limit = wait_limit();

@@ -105,21 +105,28 @@ __device__ __forceinline__ uint64_t ordered_key(double v) {
   return (b & 0x8000000000000000ull) ? ~b : (b | 0x8000000000000000ull);
 }
 
+// Key cluster size and the cluster counts of a (validated) shape.
+inline int key_c(const ca_shape* s) { return s->c_k ? s->c_k : s->c; }
+inline int num_q_clusters(const ca_shape* s) { return (s->n_valid + s->c - 1) / s->c; }
+inline int num_k_clusters(const ca_shape* s) { return (s->n_valid + key_c(s) - 1) / key_c(s); }
+
 // ---------------------------------------------------------------------------
 // Workspace layouts (byte offsets; every region 256-byte aligned).
 // ---------------------------------------------------------------------------
 inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 
 struct ClusterWs {
-  size_t nodes, level_begin, M, kmean, colsum_part, met_part, inv_s, idx0, idx1, keys, zvec, wvec,
-      sel, chunk_cnt, cov, basis, basis_scratch, total;
+  size_t nodes, level_begin, nodes_k, level_begin_k, M, kmean, colsum_part, met_part, inv_s, idx0, idx1, keys,
+      zvec, wvec, sel, chunk_cnt, cov, basis, basis_scratch, total;
   int nch = 0;       // metric row chunks
   int pch_max = 0;   // partition chunks per node, max over levels
   int TH = 0, BH = 0;
+  int NI = 0;        // internal nodes per tensor-head, the larger of the two trees
 };
 constexpr int kMetricChunk = 2048;     // rows per metric partial
 constexpr int kPartChunk = 2048;       // positions per partition chunk
-bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, ClusterWs* ws);
+// plan_k: the key tree when the key cluster size differs (else plan again)
+bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, const TreePlan& plan_k, ClusterWs* ws);
 
 // Diagonalized splitting (diag.cu): covariances from the Gram partials, the
 // principal-component directions W per tensor-head, and the per-level choice
@@ -129,11 +136,13 @@ cudaError_t launch_diag_basis(int D, int TH, int BH, int nch, int n, const doubl
 template <typename T, int D>
 cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const TreeNode* nodes, int lvl_begin,
                             int nodes_in_level, int TH, const double* W, const double* inv_s, const int* idx,
-                            int NI, double* wvec, uint64_t seed, int head_base, cudaStream_t st);
+                            int NI, double* wvec, uint64_t seed, int head_base, int tsel, cudaStream_t st);
 
 struct AttendWs {
   size_t qp, kp, vp, kbar_hl, vbar_hl, vbar32, kbar32, logcnt, total;
-  int C = 0, Cpad = 0;
+  int C = 0;      // query clusters
+  int Ck = 0;     // key clusters
+  int Cpad = 0;   // key clusters rounded up to 128 (compensation tiles)
 };
 bool attend_ws_layout(const ca_shape* s, AttendWs* ws);
 
@@ -152,11 +161,12 @@ void set_wait_limit(uint64_t limit_ns);
 // ---------------------------------------------------------------------------
 cudaError_t launch_cluster(const void* Q, const void* K, const ca_shape* s,
                            const ca_cluster_params* p, const ca_clusters* out,
-                           const TreePlan& plan, const ClusterWs& L, char* ws, cudaStream_t st);
-cudaError_t launch_route(const ca_shape* s, int C, const double* qbar, const double* kbar, int k,
+                           const TreePlan& plan, const TreePlan& plan_k, const ClusterWs& L, char* ws,
+                           cudaStream_t st);
+cudaError_t launch_route(const ca_shape* s, int Cq, int Ck, const double* qbar, const double* kbar, int k,
                          int32_t* kept_idx, uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st);
 size_t route_adaptive_smem(int C);
-cudaError_t launch_route_adaptive(const ca_shape* s, int C, const double* qbar, const double* kbar,
+cudaError_t launch_route_adaptive(const ca_shape* s, int Cq, int Ck, const double* qbar, const double* kbar,
                                   const int32_t* count_k, double recall, int min_count, int k, int32_t* kept_idx,
                                   uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st);
 cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, const ca_shape* s,

@@ -22,6 +22,12 @@ template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v
   return __bfloat162float(v);
 }
 
+// Tensor-head of a block: th = 2 bh + tensor. With tsel < 0 the grid row y
+// enumerates every tensor-head (both tensors, one tree); with tsel = 0 or 1
+// it enumerates the heads of that tensor alone (each tensor walks its own
+// tree when the query and key cluster sizes differ).
+__device__ __forceinline__ int tensor_head(int y, int tsel) { return tsel < 0 ? y : 2 * y + tsel; }
+
 // Warp sum of a double, fixed butterfly order (deterministic).
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -461,13 +467,13 @@ __global__ void __launch_bounds__(512) dir_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
-    int head_base, int power_iters, int sample_factor) {
+    int head_base, int power_iters, int sample_factor, int tsel) {
   using Cfg = DirCfg<T, D>;
   constexpr int CPL = D / 32;                      // coordinates per lane: a = lane + 32 c
   constexpr int RS = Cfg::kRowStride;
   const int m_cap = sample_factor * D;
   const int nwarps = blockDim.x >> 5;
-  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int th = tensor_head(blockIdx.y, tsel), bh = th >> 1, tensor = th & 1;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* Ms = reinterpret_cast<double*>(smem_raw);                          // D*D
@@ -670,7 +676,7 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, int npc, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
-    int head_base, int power_iters) {
+    int head_base, int power_iters, int tsel) {
   using Cfg = DirCCfg<T, D_>;
   constexpr int D = D_, RS = Cfg::kRowStride;
   constexpr int NT = Cfg::kThreads, HD = D / 2;   // threads, half length
@@ -683,7 +689,7 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
   __shared__ double qred[NWD][2];
   __shared__ double vred[2 * NWD];
   __shared__ int srow[D];
-  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int th = tensor_head(blockIdx.y, tsel), bh = th >> 1, tensor = th & 1;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int ca = t & (D - 1), ch = t / D;       // column / half split
   const int rj = t >> 1, rh = t & 1;            // row / half split
@@ -880,7 +886,7 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
                                                       int lb, int le, const double* __restrict__ inv_s,
                                                       const int* __restrict__ idx, int NI,
                                                       const double* __restrict__ wvec,
-                                                      uint64_t* __restrict__ keys) {
+                                                      uint64_t* __restrict__ keys, int tsel) {
   constexpr int EPL = 16 / sizeof(T);        // elements per lane (16 bytes)
   constexpr int G = D / EPL;                 // lanes per row
   constexpr int RPW = 32 / G;                // rows per warp step
@@ -890,7 +896,7 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   __shared__ unsigned char slot_of[kProjSpan];
   __shared__ int rows_s[kProjSpan];      // source row of each position
   __shared__ int s_cnt;
-  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int th = tensor_head(blockIdx.y, tsel), bh = th >> 1, tensor = th & 1;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
   const int base = blockIdx.x * kProjSpan;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1007,8 +1013,8 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
 // random order of the tokens into groups of c (remainder last). Positions
 // outside this level's nodes get a key too; nothing reads it.
 __global__ void __launch_bounds__(256) hash_keys_kernel(int n, const int* __restrict__ idx, uint64_t seed,
-                                                        int head_base, uint64_t* __restrict__ keys) {
-  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+                                                        int head_base, uint64_t* __restrict__ keys, int tsel) {
+  const int th = tensor_head(blockIdx.y, tsel), bh = th >> 1, tensor = th & 1;
   const int pos = blockIdx.x * 256 + threadIdx.x;
   if (pos >= n) return;
   const int row = idx ? idx[(size_t)th * n + pos] : pos;
@@ -1031,12 +1037,12 @@ template <int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__ nodes, int lb,
                                                     int nodes_in_level, int n,
                                                     const uint64_t* __restrict__ keys,
-                                                    SelectResult* __restrict__ sel) {
+                                                    SelectResult* __restrict__ sel, int tsel) {
   __shared__ unsigned int hist[256];
   __shared__ int s_digit, s_rank, s_cnt, s_ncand;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem_raw);   // kSelCap keys
-  const int th = blockIdx.y;
+  const int th = tensor_head(blockIdx.y, tsel);
   const TreeNode nd = nodes[lb + blockIdx.x];
   const uint64_t* base = keys + (size_t)th * n + nd.off;
   const int size = nd.size;
@@ -1161,8 +1167,8 @@ constexpr int kPartPer = kPartChunk / kPartThreads;   // 8 positions per thread
 
 __global__ void __launch_bounds__(kPartThreads) part_count_kernel(
     const TreeNode* __restrict__ nodes, int lb, int nodes_in_level, int n, int pch,
-    const uint64_t* __restrict__ keys, const SelectResult* __restrict__ sel, int2* __restrict__ cnt) {
-  const int th = blockIdx.z, nl = blockIdx.y, ch = blockIdx.x;
+    const uint64_t* __restrict__ keys, const SelectResult* __restrict__ sel, int2* __restrict__ cnt, int tsel) {
+  const int th = tensor_head(blockIdx.z, tsel), nl = blockIdx.y, ch = blockIdx.x;
   const TreeNode nd = nodes[lb + nl];
   const SelectResult sr = sel[(size_t)th * nodes_in_level + nl];
   const int p0 = ch * kPartChunk, p1 = min(nd.size, p0 + kPartChunk);
@@ -1213,10 +1219,10 @@ __global__ void __launch_bounds__(kPartThreads) part_scatter_kernel(
     const TreeNode* __restrict__ nodes, int lb, int nodes_in_level, int n, int c, int pch,
     const uint64_t* __restrict__ keys, const SelectResult* __restrict__ sel,
     const int2* __restrict__ cnt, const int* __restrict__ idx_in, int* __restrict__ idx_out,
-    int32_t* __restrict__ perm_q, int32_t* __restrict__ perm_k, int Cc) {
+    int32_t* __restrict__ perm_q, int32_t* __restrict__ perm_k, int Cc, int tsel) {
   __shared__ int warp_tot[kPartThreads / 32];
   __shared__ int total;
-  const int th = blockIdx.z, nl = blockIdx.y, ch = blockIdx.x;
+  const int th = tensor_head(blockIdx.z, tsel), nl = blockIdx.y, ch = blockIdx.x;
   const int bh = th >> 1, tensor = th & 1;
   const TreeNode nd = nodes[lb + nl];
   const int p0 = ch * kPartChunk;
@@ -1282,9 +1288,10 @@ __global__ void __launch_bounds__(256) centroid_kernel(const T* __restrict__ Q, 
                                                        int N_alloc, int n, int c, int C, int levels,
                                                        int32_t* __restrict__ perm_q, int32_t* __restrict__ perm_k,
                                                        int32_t* __restrict__ count_q, int32_t* __restrict__ count_k,
-                                                       double* __restrict__ qbar, double* __restrict__ kbar) {
+                                                       double* __restrict__ qbar, double* __restrict__ kbar,
+                                                       int tsel) {
   constexpr int RG = 256 / D;
-  const int a = blockIdx.x, th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int a = blockIdx.x, th = tensor_head(blockIdx.y, tsel), bh = th >> 1, tensor = th & 1;
   const int cnt = (a < C - 1) ? c : n - (C - 1) * c;
   int32_t* perm = (tensor == 0 ? perm_q : perm_k) + (size_t)bh * C * c + (size_t)a * c;
   if (levels == 0) {
@@ -1312,13 +1319,16 @@ __global__ void __launch_bounds__(256) centroid_kernel(const T* __restrict__ Q, 
 
 template <typename T, int D>
 cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_cluster_params* p,
-                        const ca_clusters* out, const TreePlan& plan, const ClusterWs& L, char* ws,
-                        cudaStream_t st) {
-  const int n = s->n_valid, N_alloc = s->N_alloc, c = s->c, C = plan.C;
-  const int BH = L.BH, TH = L.TH, NI = plan.internal;
+                        const ca_clusters* out, const TreePlan& plan, const TreePlan& plan_k, const ClusterWs& L,
+                        char* ws, cudaStream_t st) {
+  const int n = s->n_valid, N_alloc = s->N_alloc;
+  const int BH = L.BH, TH = L.TH, NI = L.NI;
   const int nch = L.nch;
-  TreeNode* nodes = reinterpret_cast<TreeNode*>(ws + L.nodes);
-  int* level_begin = reinterpret_cast<int*>(ws + L.level_begin);
+  // Queries and keys share one tree when their cluster sizes are equal; with
+  // unequal sizes each tensor walks its own (its nodes in their own table).
+  const bool same_tree = key_c(s) == s->c;
+  TreeNode* nodes_t[2] = {reinterpret_cast<TreeNode*>(ws + L.nodes), reinterpret_cast<TreeNode*>(ws + L.nodes_k)};
+  int* level_begin_t[2] = {reinterpret_cast<int*>(ws + L.level_begin), reinterpret_cast<int*>(ws + L.level_begin_k)};
   double* M = reinterpret_cast<double*>(ws + L.M);
   double* colpart = reinterpret_cast<double*>(ws + L.colsum_part);
   double* metpart = reinterpret_cast<double*>(ws + L.met_part);
@@ -1339,8 +1349,10 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
   const bool random_clusters = p->method == 1;
   const bool diagonal = p->method == 2;
   double* basis = reinterpret_cast<double*>(ws + L.basis);
-  if (plan.levels > 0) {
-    plan_kernel<<<1, 1024, 0, st>>>(n, c, nodes, level_begin);
+  const bool any_split = plan.levels > 0 || plan_k.levels > 0;
+  if (any_split) {
+    plan_kernel<<<1, 1024, 0, st>>>(n, s->c, nodes_t[0], level_begin_t[0]);
+    if (!same_tree) plan_kernel<<<1, 1024, 0, st>>>(n, key_c(s), nodes_t[1], level_begin_t[1]);
     if (!random_clusters) {
       colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
       const size_t syrk_smem = SyrkCfg<D>::template smem<T>();
@@ -1370,53 +1382,69 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
         if (e != cudaSuccess) return e;
       }
     }
-    const int m_cap = sample_factor * D;
-    const int dir_warps = DirCfg<T, D>::warps(m_cap);
-    const size_t dir_smem = (size_t)D * D * 8 + (size_t)dir_warps * DirCfg<T, D>::warp_bytes(m_cap);
-    cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
-    cudaFuncSetAttribute(dirc_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DirCCfg<T, D>::kSmem);
-    cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
-    cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
-    for (int l = 0; l < plan.levels; ++l) {
-      const int lb = plan.level_begin[l], le = plan.level_begin[l + 1], nl = le - lb;
+  }
+  const int m_cap = sample_factor * D;
+  const int dir_warps = DirCfg<T, D>::warps(m_cap);
+  const size_t dir_smem = (size_t)D * D * 8 + (size_t)dir_warps * DirCfg<T, D>::warp_bytes(m_cap);
+  cudaFuncSetAttribute(dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dir_smem);
+  cudaFuncSetAttribute(dirc_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DirCCfg<T, D>::kSmem);
+  cudaFuncSetAttribute(select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
+  cudaFuncSetAttribute(select_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSelCap * 8);
+  // The levels of one tree, for both tensors (tsel < 0) or one (tsel = 0, 1);
+  // then the centroids of the clusters that tree makes.
+  auto run_tree = [&](const TreePlan& pl, int tsel) -> cudaError_t {
+    const int c = tsel == 1 ? key_c(s) : s->c, C = pl.C;
+    const int rows = tsel < 0 ? TH : BH;   // grid rows: tensor-heads
+    TreeNode* nodes = nodes_t[tsel == 1 ? 1 : 0];
+    for (int l = 0; l < pl.levels; ++l) {
+      const int lb = pl.level_begin[l], le = pl.level_begin[l + 1], nl = le - lb;
       const int* idx_in = (l == 0) ? nullptr : idxbuf[l & 1];
       int* idx_out = idxbuf[(l + 1) & 1];
       if (random_clusters) {
-        hash_keys_kernel<<<dim3((n + 255) / 256, TH), 256, 0, st>>>(n, idx_in, p->seed, p->head_base, keys);
+        hash_keys_kernel<<<dim3((n + 255) / 256, rows), 256, 0, st>>>(n, idx_in, p->seed, p->head_base, keys, tsel);
       } else if (diagonal) {
-        const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, TH, basis, inv_s, idx_in,
-                                                    NI, wvec, p->seed, p->head_base, st);
+        const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, rows, basis, inv_s, idx_in,
+                                                    NI, wvec, p->seed, p->head_base, tsel, st);
         if (e != cudaSuccess) return e;
-      } else if (sample_factor == 1 && (D == 128 || (long long)nl * TH <= kDirCMaxNodes64)) {
+      } else if (sample_factor == 1 && (D == 128 || (long long)nl * rows <= kDirCMaxNodes64)) {
         // a block per node: d = 128, or d = 64 levels with few nodes (about
         // four blocks per SM over the whole level)
-        const int npc = (int)(((long long)nl * TH + 4 * 148 - 1) / (4 * 148));
-        dirc_kernel<T, D><<<dim3((nl + npc - 1) / npc, TH), DirCCfg<T, D>::kThreads, DirCCfg<T, D>::kSmem, st>>>(
+        const int npc = (int)(((long long)nl * rows + 4 * 148 - 1) / (4 * 148));
+        dirc_kernel<T, D><<<dim3((nl + npc - 1) / npc, rows), DirCCfg<T, D>::kThreads, DirCCfg<T, D>::kSmem, st>>>(
             Q, K, N_alloc, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base,
-            power_iters);
+            power_iters, tsel);
       } else {
-        dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, TH), dir_warps * 32, dir_smem, st>>>(
+        dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, rows), dir_warps * 32, dir_smem, st>>>(
             Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base, power_iters,
-            sample_factor);
+            sample_factor, tsel);
       }
       if (!random_clusters)
-        project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, TH), 256, 0, st>>>(
-            Q, K, N_alloc, n, nodes, lb, le, inv_s, idx_in, NI, wvec, keys);
-      if (plan.level_max_size[l] <= kSelCap)   // candidates buffer sized to the level's largest node
-        select_kernel<256><<<dim3(nl, TH), 256, (size_t)plan.level_max_size[l] * 8, st>>>(nodes, lb, nl, n, keys,
-                                                                                        sel);
+        project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, rows), 256, 0, st>>>(
+            Q, K, N_alloc, n, nodes, lb, le, inv_s, idx_in, NI, wvec, keys, tsel);
+      if (pl.level_max_size[l] <= kSelCap)   // candidates buffer sized to the level's largest node
+        select_kernel<256><<<dim3(nl, rows), 256, (size_t)pl.level_max_size[l] * 8, st>>>(nodes, lb, nl, n, keys,
+                                                                                        sel, tsel);
       else
-        select_kernel<1024><<<dim3(nl, TH), 1024, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel);
-      const int pch = (plan.level_max_size[l] + kPartChunk - 1) / kPartChunk;
-      part_count_kernel<<<dim3(pch, nl, TH), kPartThreads, 0, st>>>(nodes, lb, nl, n, pch, keys, sel, ccnt);
-      part_scatter_kernel<<<dim3(pch, nl, TH), kPartThreads, 0, st>>>(nodes, lb, nl, n, c, pch, keys, sel,
+        select_kernel<1024><<<dim3(nl, rows), 1024, kSelCap * 8, st>>>(nodes, lb, nl, n, keys, sel, tsel);
+      const int pch = (pl.level_max_size[l] + kPartChunk - 1) / kPartChunk;
+      part_count_kernel<<<dim3(pch, nl, rows), kPartThreads, 0, st>>>(nodes, lb, nl, n, pch, keys, sel, ccnt, tsel);
+      part_scatter_kernel<<<dim3(pch, nl, rows), kPartThreads, 0, st>>>(nodes, lb, nl, n, c, pch, keys, sel,
                                                                       ccnt, idx_in, idx_out, out->perm_q,
-                                                                      out->perm_k, C * c);
+                                                                      out->perm_k, C * c, tsel);
     }
+    centroid_kernel<T, D><<<dim3(C, rows), 256, 0, st>>>(Q, K, N_alloc, n, c, C, pl.levels, out->perm_q,
+                                                         out->perm_k, out->count_q, out->count_k, out->qbar,
+                                                         out->kbar, tsel);
+    return cudaGetLastError();
+  };
+  cudaError_t e;
+  if (same_tree) {
+    e = run_tree(plan, -1);
+  } else {
+    e = run_tree(plan, 0);
+    if (e == cudaSuccess) e = run_tree(plan_k, 1);
   }
-  centroid_kernel<T, D><<<dim3(C, TH), 256, 0, st>>>(Q, K, N_alloc, n, c, C, plan.levels, out->perm_q,
-                                                     out->perm_k, out->count_q, out->count_k, out->qbar,
-                                                     out->kbar);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1442,26 +1470,33 @@ bool host_plan(int n, int c, TreePlan* plan) {
   return ok;
 }
 
-bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, ClusterWs* w) {
+bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, const TreePlan& plan_k, ClusterWs* w) {
   const size_t n = s->n_valid, d = s->d;
   const size_t BH = (size_t)s->B * s->H, TH = 2 * BH;
-  const size_t NI = plan.internal > 0 ? plan.internal : 1;
-  w->BH = (int)BH; w->TH = (int)TH;
+  const int ni = plan.internal > plan_k.internal ? plan.internal : plan_k.internal;
+  const size_t NI = ni > 0 ? (size_t)ni : 1;
+  w->BH = (int)BH; w->TH = (int)TH; w->NI = (int)NI;
   w->nch = (int)((n + kMetricChunk - 1) / kMetricChunk);
   int pmax = 1;
   size_t chunk_cnt = 1;
-  for (int l = 0; l < plan.levels; ++l) {
-    const int pch = (plan.level_max_size[l] + kPartChunk - 1) / kPartChunk;
-    const int nl = plan.level_begin[l + 1] - plan.level_begin[l];
-    pmax = pch > pmax ? pch : pmax;
-    const size_t need = (size_t)nl * pch;
-    chunk_cnt = need > chunk_cnt ? need : chunk_cnt;
+  for (const TreePlan* pl : {&plan, &plan_k}) {
+    for (int l = 0; l < pl->levels; ++l) {
+      const int pch = (pl->level_max_size[l] + kPartChunk - 1) / kPartChunk;
+      const int nl = pl->level_begin[l + 1] - pl->level_begin[l];
+      pmax = pch > pmax ? pch : pmax;
+      const size_t need = (size_t)nl * pch;
+      chunk_cnt = need > chunk_cnt ? need : chunk_cnt;
+    }
   }
   w->pch_max = pmax;
+  const size_t NIq = plan.internal > 0 ? (size_t)plan.internal : 1;
+  const size_t NIk = plan_k.internal > 0 ? (size_t)plan_k.internal : 1;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
-  w->nodes = take(NI * sizeof(TreeNode));
+  w->nodes = take(NIq * sizeof(TreeNode));
   w->level_begin = take((kMaxLevels + 1) * sizeof(int));
+  w->nodes_k = take(NIk * sizeof(TreeNode));
+  w->level_begin_k = take((kMaxLevels + 1) * sizeof(int));
   w->M = take(TH * d * d * 8);
   w->kmean = take(BH * d * 8);
   w->colsum_part = take(BH * w->nch * d * 8);
@@ -1482,16 +1517,16 @@ bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, ClusterWs* w) {
 }
 
 cudaError_t launch_cluster(const void* Q, const void* K, const ca_shape* s, const ca_cluster_params* p,
-                           const ca_clusters* out, const TreePlan& plan, const ClusterWs& L, char* ws,
-                           cudaStream_t st) {
+                           const ca_clusters* out, const TreePlan& plan, const TreePlan& plan_k, const ClusterWs& L,
+                           char* ws, cudaStream_t st) {
   if (s->dtype == CA_BF16) {
     using T = __nv_bfloat16;
-    if (s->d == 64) return run_cluster<T, 64>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
-    return run_cluster<T, 128>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
+    if (s->d == 64) return run_cluster<T, 64>((const T*)Q, (const T*)K, s, p, out, plan, plan_k, L, ws, st);
+    return run_cluster<T, 128>((const T*)Q, (const T*)K, s, p, out, plan, plan_k, L, ws, st);
   }
   using T = float;
-  if (s->d == 64) return run_cluster<T, 64>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
-  return run_cluster<T, 128>((const T*)Q, (const T*)K, s, p, out, plan, L, ws, st);
+  if (s->d == 64) return run_cluster<T, 64>((const T*)Q, (const T*)K, s, p, out, plan, plan_k, L, ws, st);
+  return run_cluster<T, 128>((const T*)Q, (const T*)K, s, p, out, plan, plan_k, L, ws, st);
 }
 
 }  // namespace ca

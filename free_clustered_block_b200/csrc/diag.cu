@@ -332,7 +332,8 @@ __global__ void __launch_bounds__(256) diag_dir_kernel(const T* __restrict__ Q, 
                                                        const double* __restrict__ W,
                                                        const double* __restrict__ inv_s,
                                                        const int* __restrict__ idx, int NI,
-                                                       double* __restrict__ wvec, uint64_t seed, int head_base) {
+                                                       double* __restrict__ wvec, uint64_t seed, int head_base,
+                                                       int tsel) {
   using Cfg = DiagDirCfg<T, D>;
   constexpr int TI = Cfg::TI, TJ = Cfg::TJ, KC = Cfg::KC, XS = Cfg::XS;
   constexpr int VEC = Cfg::VEC, CPR = Cfg::CPR, NCH = Cfg::NCH;
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(256) diag_dir_kernel(const T* __restrict__ Q, 
   __shared__ double mean_s[D], ssc[D];
   __shared__ int srow[D];
   __shared__ int jbest_s;
-  const int th = blockIdx.y, bh = th >> 1, tensor = th & 1;
+  const int th = tsel < 0 ? (int)blockIdx.y : 2 * (int)blockIdx.y + tsel, bh = th >> 1, tensor = th & 1;
   const int t = threadIdx.x, ty = t / 16, tx = t % 16;
   const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
   {
@@ -506,29 +507,30 @@ cudaError_t launch_diag_basis(int D, int TH, int BH, int nch, int n, const doubl
 template <typename T, int D>
 cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const TreeNode* nodes, int lvl_begin,
                             int nodes_in_level, int TH, const double* W, const double* inv_s, const int* idx,
-                            int NI, double* wvec, uint64_t seed, int head_base, cudaStream_t st) {
+                            int NI, double* wvec, uint64_t seed, int head_base, int tsel, cudaStream_t st) {
   using Cfg = DiagDirCfg<T, D>;
   const int per_sm = D == 64 ? 3 : 1;   // CTAs resident per SM (shared memory)
   const int npc = (int)(((long long)nodes_in_level * TH + 148 * per_sm - 1) / (148 * per_sm));
   cudaFuncSetAttribute(diag_dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem);
+  // TH: the grid rows (every tensor-head, or one tensor's heads when tsel >= 0)
   diag_dir_kernel<T, D><<<dim3((nodes_in_level + npc - 1) / npc, TH), Cfg::kThreads, Cfg::kSmem, st>>>(
-      Q, K, N_alloc, n, nodes, lvl_begin, nodes_in_level, npc, W, inv_s, idx, NI, wvec, seed, head_base);
+      Q, K, N_alloc, n, nodes, lvl_begin, nodes_in_level, npc, W, inv_s, idx, NI, wvec, seed, head_base, tsel);
   return cudaGetLastError();
 }
 
 template cudaError_t launch_diag_dir<__nv_bfloat16, 64>(const __nv_bfloat16*, const __nv_bfloat16*, int, int,
                                                          const TreeNode*, int, int, int, const double*,
-                                                         const double*, const int*, int, double*, uint64_t, int,
+                                                         const double*, const int*, int, double*, uint64_t, int, int,
                                                          cudaStream_t);
 template cudaError_t launch_diag_dir<__nv_bfloat16, 128>(const __nv_bfloat16*, const __nv_bfloat16*, int, int,
                                                           const TreeNode*, int, int, int, const double*,
-                                                          const double*, const int*, int, double*, uint64_t, int,
+                                                          const double*, const int*, int, double*, uint64_t, int, int,
                                                           cudaStream_t);
 template cudaError_t launch_diag_dir<float, 64>(const float*, const float*, int, int, const TreeNode*, int, int,
                                                 int, const double*, const double*, const int*, int, double*,
-                                                uint64_t, int, cudaStream_t);
+                                                uint64_t, int, int, cudaStream_t);
 template cudaError_t launch_diag_dir<float, 128>(const float*, const float*, int, int, const TreeNode*, int, int,
                                                  int, const double*, const double*, const int*, int, double*,
-                                                 uint64_t, int, cudaStream_t);
+                                                 uint64_t, int, int, cudaStream_t);
 
 }  // namespace ca

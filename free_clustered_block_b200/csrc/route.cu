@@ -29,15 +29,16 @@ constexpr int kRouteWarps = kRouteThreads / 32;
 // one block per SM either way (its registers), so the score rows may use most of shared memory
 constexpr size_t kRouteSmemBudget = 200 * 1024;
 
+// C query clusters (rows), Ck key clusters (columns).
 template <int D, int QA>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* __restrict__ qbar,
-                                                                 const double* __restrict__ kbar, int C, int k,
+                                                                 const double* __restrict__ kbar, int C, int Ck, int k,
                                                                  int32_t* __restrict__ kept_idx,
                                                                  uint32_t* __restrict__ kept_bits,
                                                                  int32_t* __restrict__ kept_count) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* qs = reinterpret_cast<double*>(smem_raw);   // QA x D
-  double* sc = qs + QA * D;                           // QA x C scores
+  double* sc = qs + QA * D;                           // QA x Ck scores
   __shared__ uint32_t hist[kRouteWarps][256];
 
   const int a0 = blockIdx.x * QA, bh = blockIdx.y;
@@ -49,8 +50,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* _
   __syncthreads();
 
   // ---- scores ----
-  const double* kb = kbar + (size_t)bh * C * D;
-  for (int b = threadIdx.x; b < C; b += kRouteThreads) {
+  const double* kb = kbar + (size_t)bh * Ck * D;
+  for (int b = threadIdx.x; b < Ck; b += kRouteThreads) {
     double s[QA];
 #pragma unroll
     for (int r = 0; r < QA; ++r) s[r] = 0.0;
@@ -74,20 +75,20 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* _
       }
     }
 #pragma unroll
-    for (int r = 0; r < QA; ++r) sc[(size_t)r * C + b] = s[r];
+    for (int r = 0; r < QA; ++r) sc[(size_t)r * Ck + b] = s[r];
   }
   __syncthreads();
 
   // ---- selection, one warp per query cluster ----
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  const int W = (C + 31) / 32;
+  const int W = (Ck + 31) / 32;
   uint32_t* h = hist[warp];
   for (int r = warp; r < nq; r += kRouteWarps) {
-    const double* row = sc + (size_t)r * C;
+    const double* row = sc + (size_t)r * Ck;
     // common prefix of all keys
     uint64_t kand = ~0ull, kor = 0ull;
-    for (int b = lane; b < C; b += 32) {
+    for (int b = lane; b < Ck; b += 32) {
       const uint64_t key = ordered_key(row[b]);
       kand &= key; kor |= key;
     }
@@ -100,15 +101,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* _
     int L = diff ? (__clzll((long long)diff) & ~7) : 64;   // decided prefix length (bits)
     uint64_t P = L == 0 ? 0ull : (L == 64 ? kand : kand >> (64 - L));
     int krem = k;                     // still to take among keys whose prefix equals P
-    bool all = (k >= C);              // every key matching P is kept
+    bool all = (k >= Ck);             // every key matching P is kept
     while (!all && L < 64) {
       for (int i = lane; i < 256; i += 32) h[i] = 0u;
       __syncwarp();
       const int shift = 56 - L;
-      for (int b0 = 0; b0 < C; b0 += 32) {
+      for (int b0 = 0; b0 < Ck; b0 += 32) {
         const int b = b0 + lane;
         int dig = 256 + lane;          // no bin
-        if (b < C) {
+        if (b < Ck) {
           const uint64_t key = ordered_key(row[b]);
           if (L == 0 || (key >> (64 - L)) == P) dig = (int)((key >> shift) & 255u);
         }
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* _
     for (int i = 0; i < W; ++i) {
       const int b = i * 32 + lane;
       bool take = false, eq = false;
-      if (b < C) {
+      if (b < Ck) {
         const uint64_t key = ordered_key(row[b]);
         const uint64_t top = L == 0 ? 0ull : (L == 64 ? key : key >> (64 - L));
         take = top > P;
@@ -174,47 +175,51 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(const double* _
 }
 
 template <int D, int QA>
-size_t route_smem(int C) {
-  return (size_t)QA * D * 8 + (size_t)QA * C * 8;
+size_t route_smem(int Ck) {
+  return (size_t)QA * D * 8 + (size_t)QA * Ck * 8;
 }
 
 template <int D, int QA>
-cudaError_t launch_qa(const ca_shape* s, int C, const double* qbar, const double* kbar, int k, int32_t* kept_idx,
-                      uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
-  const size_t smem = route_smem<D, QA>(C);
+cudaError_t launch_qa(const ca_shape* s, int C, int Ck, const double* qbar, const double* kbar, int k,
+                      int32_t* kept_idx, uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
+  const size_t smem = route_smem<D, QA>(Ck);
   cudaError_t e = cudaFuncSetAttribute(route_kernel<D, QA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((C + QA - 1) / QA, s->B * s->H);
-  route_kernel<D, QA><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, k, kept_idx, kept_bits, kept_count);
+  route_kernel<D, QA><<<grid, kRouteThreads, smem, st>>>(qbar, kbar, C, Ck, k, kept_idx, kept_bits, kept_count);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_d(const ca_shape* s, int C, const double* qbar, const double* kbar, int k, int32_t* kept_idx,
-                     uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
+cudaError_t launch_d(const ca_shape* s, int C, int Ck, const double* qbar, const double* kbar, int k,
+                     int32_t* kept_idx, uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
   // as many query clusters per block as the score rows allow in the budget
-  if (route_smem<D, 16>(C) <= kRouteSmemBudget) return launch_qa<D, 16>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
-  if (route_smem<D, 8>(C) <= kRouteSmemBudget) return launch_qa<D, 8>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
-  if (route_smem<D, 4>(C) <= kRouteSmemBudget) return launch_qa<D, 4>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
-  if (route_smem<D, 2>(C) <= kRouteSmemBudget) return launch_qa<D, 2>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
-  return launch_qa<D, 1>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 16>(Ck) <= kRouteSmemBudget)
+    return launch_qa<D, 16>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 8>(Ck) <= kRouteSmemBudget)
+    return launch_qa<D, 8>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 4>(Ck) <= kRouteSmemBudget)
+    return launch_qa<D, 4>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (route_smem<D, 2>(Ck) <= kRouteSmemBudget)
+    return launch_qa<D, 2>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  return launch_qa<D, 1>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
 }
 
 }  // namespace
 
-size_t route_smem_bytes(int C, int D) {
-  return D == 64 ? route_smem<64, 1>(C) : route_smem<128, 1>(C);
+size_t route_smem_bytes(int Ck, int D) {
+  return D == 64 ? route_smem<64, 1>(Ck) : route_smem<128, 1>(Ck);
 }
 
-cudaError_t launch_route(const ca_shape* s, int C, const double* qbar, const double* kbar, int k,
+cudaError_t launch_route(const ca_shape* s, int C, int Ck, const double* qbar, const double* kbar, int k,
                          int32_t* kept_idx, uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
-  if (s->d == 64) return launch_d<64>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
-  return launch_d<128>(s, C, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  if (s->d == 64) return launch_d<64>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
+  return launch_d<128>(s, C, Ck, qbar, kbar, k, kept_idx, kept_bits, kept_count, st);
 }
 
 // ---------------------------------------------------------------------------
 // Adaptive selection (Section 3.3.2, second method): one block per query
-// cluster. w_b = s_ab / sqrt(d) + ln|b| is the log of the estimated attention
+// cluster (C below is the number of key clusters). w_b = s_ab / sqrt(d) + ln|b| is the log of the estimated attention
 // mass |b| e^{s_ab / sqrt(d)}; the key clusters are sorted by decreasing w
 // (ties to the lower index, bitonic network in shared memory), their masses
 // e^{w - w_max} summed in that order by one thread, and the shortest prefix
@@ -234,8 +239,8 @@ int adaptive_cpad(int C) {
 
 template <int D>
 __global__ void __launch_bounds__(kAdaptThreads) route_adaptive_kernel(
-    const double* __restrict__ qbar, const double* __restrict__ kbar, const int32_t* __restrict__ count_k, int C,
-    int Cpad, double recall, int min_count, int k, int32_t* __restrict__ kept_idx,
+    const double* __restrict__ qbar, const double* __restrict__ kbar, const int32_t* __restrict__ count_k, int Cq,
+    int C, int Cpad, double recall, int min_count, int k, int32_t* __restrict__ kept_idx,
     uint32_t* __restrict__ kept_bits, int32_t* __restrict__ kept_count) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* w = reinterpret_cast<double*>(smem_raw);             // Cpad: log masses, then masses
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(kAdaptThreads) route_adaptive_kernel(
   __shared__ int kcount;
   const int a = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const double* kb = kbar + (size_t)bh * C * D;
-  for (int e = t; e < D; e += kAdaptThreads) qa[e] = qbar[((size_t)bh * C + a) * D + e];
+  for (int e = t; e < D; e += kAdaptThreads) qa[e] = qbar[((size_t)bh * Cq + a) * D + e];
   for (int e = t; e < Cpad / 32; e += kAdaptThreads) bits[e] = 0u;
   __syncthreads();
   const double scale = 1.0 / sqrt((double)D);
@@ -307,11 +312,11 @@ __global__ void __launch_bounds__(kAdaptThreads) route_adaptive_kernel(
   for (int i = t; i < kk; i += kAdaptThreads) atomicOr(&bits[id[i] >> 5], 1u << (id[i] & 31));
   __syncthreads();
   const int W = (C + 31) / 32;
-  for (int e = t; e < W; e += kAdaptThreads) kept_bits[((size_t)bh * C + a) * W + e] = bits[e];
-  if (t == 0) kept_count[(size_t)bh * C + a] = kk;
+  for (int e = t; e < W; e += kAdaptThreads) kept_bits[((size_t)bh * Cq + a) * W + e] = bits[e];
+  if (t == 0) kept_count[(size_t)bh * Cq + a] = kk;
   // ascending kept list: one warp scans the words' popcounts, 32 at a time
   if (t < 32) {
-    int32_t* krow = kept_idx + ((size_t)bh * C + a) * k;
+    int32_t* krow = kept_idx + ((size_t)bh * Cq + a) * k;
     int base = 0;
     for (int w0 = 0; w0 < W; w0 += 32) {
       const int e = w0 + t;
@@ -336,27 +341,28 @@ __global__ void __launch_bounds__(kAdaptThreads) route_adaptive_kernel(
 
 }  // namespace
 
-size_t route_adaptive_smem(int C) {
-  const int Cpad = adaptive_cpad(C);
+size_t route_adaptive_smem(int Ck) {
+  const int Cpad = adaptive_cpad(Ck);
   return (size_t)Cpad * 12 + (size_t)(Cpad / 32) * 4;
 }
 
-cudaError_t launch_route_adaptive(const ca_shape* s, int C, const double* qbar, const double* kbar,
+// Cq query clusters (one block each), C key clusters.
+cudaError_t launch_route_adaptive(const ca_shape* s, int Cq, int C, const double* qbar, const double* kbar,
                                   const int32_t* count_k, double recall, int min_count, int k, int32_t* kept_idx,
                                   uint32_t* kept_bits, int32_t* kept_count, cudaStream_t st) {
   const int Cpad = adaptive_cpad(C);
   const size_t smem = route_adaptive_smem(C);
-  const dim3 grid(C, s->B * s->H);
+  const dim3 grid(Cq, s->B * s->H);
   cudaError_t e;
   if (s->d == 64) {
     e = cudaFuncSetAttribute(route_adaptive_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_adaptive_kernel<64><<<grid, kAdaptThreads, smem, st>>>(qbar, kbar, count_k, C, Cpad, recall, min_count, k,
+    route_adaptive_kernel<64><<<grid, kAdaptThreads, smem, st>>>(qbar, kbar, count_k, Cq, C, Cpad, recall, min_count, k,
                                                                  kept_idx, kept_bits, kept_count);
   } else {
     e = cudaFuncSetAttribute(route_adaptive_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    route_adaptive_kernel<128><<<grid, kAdaptThreads, smem, st>>>(qbar, kbar, count_k, C, Cpad, recall, min_count,
+    route_adaptive_kernel<128><<<grid, kAdaptThreads, smem, st>>>(qbar, kbar, count_k, Cq, C, Cpad, recall, min_count,
                                                                   k, kept_idx, kept_bits, kept_count);
   }
   return cudaGetLastError();

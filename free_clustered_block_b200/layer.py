@@ -8,7 +8,7 @@ from __future__ import annotations
 from dataclasses import dataclass
 from typing import Optional
 
-from . import (CA_BF16, CA_FP32, ca_attend, ca_attend_prepare, ca_attend_prepared, ca_cluster, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
+from . import (CA_BF16, CA_FP32, ca_attend, ca_attend_prepare, ca_attend_prepared, ca_cluster, num_key_clusters, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
                attend_workspace_bytes, cluster_workspace_bytes, clusters_struct, forward_workspace_bytes,
                make_params, make_shape, num_clusters, routes_struct)
 
@@ -38,6 +38,9 @@ class ClusterAttention:
 
     Q, K, V, O: torch CUDA tensors [B, H, N_alloc, d], bf16 or fp32, contiguous.
 
+    c_k: key cluster size (0: the same as c, the query cluster size); the
+    paper's evaluated blocks are c = 64 queries against c_k = 128 keys.
+
     head_base: global index of the first (b, h) pair these tensors hold, when
     they are a slice of a larger layer's heads (one GPU's share of a layer
     split across GPUs); the clusters are then those the whole layer would get.
@@ -47,11 +50,11 @@ class ClusterAttention:
                  dtype: str = "bf16", compensate: bool = True, power_iters: int = 8,
                  sample_factor: int = 1, transform: bool = True, seed: int = 0, device="cuda",
                  selection: str = "topk", recall: float = 0.9, min_count: int = 16,
-                 clustering: str = "split", head_base: int = 0):
+                 clustering: str = "split", head_base: int = 0, c_k: int = 0):
         import torch
         self.torch = torch
         self.dtype_code = CA_BF16 if dtype == "bf16" else CA_FP32
-        self.shape = make_shape(B, H, N_alloc, n_valid, d, c, self.dtype_code)
+        self.shape = make_shape(B, H, N_alloc, n_valid, d, c, self.dtype_code, c_k)
         # adaptive selection pairs with the eq. 15 query representation
         self.selection = selection
         self.recall, self.min_count = recall, min_count
@@ -63,17 +66,19 @@ class ClusterAttention:
         C = num_clusters(self.shape)
         if C < 0:
             raise ValueError("invalid shape")
-        self.C = C
+        Ck = num_key_clusters(self.shape)
+        self.C, self.Ck = C, Ck
+        self.c_k = c_k or c
         BH = B * H
         i32, f64 = torch.int32, torch.float64
-        W = (C + 31) // 32
+        W = (Ck + 31) // 32
         self.buf = Buffers(
             perm_q=torch.empty(BH * C * c, dtype=i32, device=device),
-            perm_k=torch.empty(BH * C * c, dtype=i32, device=device),
+            perm_k=torch.empty(BH * Ck * self.c_k, dtype=i32, device=device),
             count_q=torch.empty(BH * C, dtype=i32, device=device),
-            count_k=torch.empty(BH * C, dtype=i32, device=device),
+            count_k=torch.empty(BH * Ck, dtype=i32, device=device),
             qbar=torch.empty(BH * C * d, dtype=f64, device=device),
-            kbar=torch.empty(BH * C * d, dtype=f64, device=device),
+            kbar=torch.empty(BH * Ck * d, dtype=f64, device=device),
             kept_idx=torch.empty(BH * C * k, dtype=i32, device=device),
             kept_bits=torch.empty(BH * C * W, dtype=torch.int32, device=device),
             kept_count=torch.empty(BH * C, dtype=i32, device=device),

@@ -46,16 +46,20 @@ typedef enum {
 
 typedef enum { CA_BF16 = 0, CA_FP32 = 1 } ca_dtype;
 
-/* Problem shape. C = ceil(n_valid / c) clusters for queries and for keys.
- * Supported: d in {64, 128}; c in {64, 128, 256}; 1 <= n_valid <= N_alloc;
- * dtype CA_BF16 or CA_FP32. */
+/* Problem shape. C = ceil(n_valid / c) query clusters and
+ * C_k = ceil(n_valid / c_k) key clusters (c_k = 0 means c_k = c, so C_k = C).
+ * Unequal sizes are the paper's evaluated block shape (Section 3.1,
+ * "Overview": 64 queries against 128 keys per block).
+ * Supported: d in {64, 128}; c and c_k in {64, 128, 256}; 1 <= n_valid <=
+ * N_alloc; dtype CA_BF16 or CA_FP32. */
 typedef struct {
   int B, H;          /* batch, heads */
   int N_alloc;       /* rows allocated per head */
   int n_valid;       /* tokens per head (rows 0..n_valid-1) */
   int d;             /* head dimension */
-  int c;             /* cluster size (queries and keys) */
+  int c;             /* query cluster size (and key cluster size when c_k is 0) */
   int dtype;         /* ca_dtype of Q, K, V and O */
+  int c_k;           /* key cluster size, or 0 for c */
 } ca_shape;
 
 /* Clustering knobs (paper Section 3.2.1, "Basic recursive splitting" and
@@ -101,14 +105,17 @@ typedef struct {
   int head_base;
 } ca_cluster_params;
 
-/* Clustering result, one entry per (b, h), C = ca_num_clusters(shape):
- *  perm_q, perm_k  int32 [B][H][C*c]: slot a*c+j holds the original row of the
- *                  j-th member of cluster a (ascending rows); -1 in pad slots.
- *                  Every cluster holds c members except possibly the last,
- *                  which holds n_valid - (C-1)*c (Section 3.1).
- *  count_q, count_k int32 [B][H][C]: members per cluster.
- *  qbar, kbar      fp64 [B][H][C][d]: centroids in the original, untransformed
- *                  space (Section 3.3.1, eq. 18). */
+/* Clustering result, one entry per (b, h), C = ca_num_clusters(shape) query
+ * clusters of c slots and C_k = ca_num_key_clusters(shape) key clusters of
+ * c_k slots:
+ *  perm_q          int32 [B][H][C*c], perm_k int32 [B][H][C_k*c_k]: slot a*c+j
+ *                  holds the original row of the j-th member of cluster a
+ *                  (ascending rows); -1 in pad slots. Every cluster is full
+ *                  except possibly the last, which holds the remainder
+ *                  (Section 3.1).
+ *  count_q         int32 [B][H][C], count_k int32 [B][H][C_k]: members per cluster.
+ *  qbar            fp64 [B][H][C][d], kbar fp64 [B][H][C_k][d]: centroids in
+ *                  the original, untransformed space (Section 3.3.1, eq. 18). */
 typedef struct {
   int32_t* perm_q;
   int32_t* perm_k;
@@ -118,10 +125,10 @@ typedef struct {
   double* kbar;
 } ca_clusters;
 
-/* Routing result:
+/* Routing result (C query clusters, C_k key clusters):
  *  kept_idx   int32 [B][H][C][k]: the key clusters kept by each query
- *             cluster, ascending (row stride k);
- *  kept_bits  uint32 [B][H][C][ceil(C/32)]: the same set as a bitmask
+ *             cluster, ascending (row stride k), 1 <= k <= C_k;
+ *  kept_bits  uint32 [B][H][C][ceil(C_k/32)]: the same set as a bitmask
  *             (bit b%32 of word b/32);
  *  kept_count int32 [B][H][C] or NULL: how many entries of each kept_idx row
  *             are used. NULL means every query cluster keeps exactly k (top-k
@@ -135,8 +142,12 @@ typedef struct {
   int32_t* kept_count;
 } ca_routes;
 
-/* Number of clusters C = ceil(n_valid / c); -1 if the shape is invalid. Host only. */
+/* Number of query clusters C = ceil(n_valid / c); -1 if the shape is invalid. Host only. */
 int ca_num_clusters(const ca_shape* shape);
+
+/* Number of key clusters C_k = ceil(n_valid / c_k) (C when c_k is 0); -1 if
+ * the shape is invalid. Host only. */
+int ca_num_key_clusters(const ca_shape* shape);
 
 /* Validate a shape without launching anything. Host only. */
 ca_status ca_check_shape(const ca_shape* shape);
@@ -200,7 +211,7 @@ ca_status ca_cluster_noalloc(const void* Q, const void* K, const ca_shape* shape
  * centroids: device qbar/kbar (fp64) as produced by ca_cluster or supplied by
  * the caller; only qbar and kbar are read, and both must be 16-byte aligned
  * (CA_ERR_INVALID_ARG otherwise). out: device kept_idx and kept_bits;
- * out->k is k. 1 <= k <= C, C <= 8192.
+ * out->k is k. 1 <= k <= C_k; C, C_k <= 8192.
  */
 ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
                    const ca_routes* out, void* stream);
@@ -214,9 +225,9 @@ ca_status ca_route(const ca_shape* shape, const ca_clusters* centroids,
  * at least min(min_count, C) of them (the paper uses 16). Exact greedy
  * selection in fp64 (masses e^{w - w_max}, summed in that order), not the
  * paper's two-pass histogram. Reads centroids->qbar, kbar (16-byte aligned)
- * and count_k. out->k is the capacity of a kept_idx row (k = C always
+ * and count_k. out->k is the capacity of a kept_idx row (k = C_k always
  * suffices; a longer selection is cut at k); out->kept_count is required.
- * recall in [0, 1]; min_count >= 1; C <= 8192.
+ * recall in [0, 1]; min_count >= 1; C, C_k <= 8192.
  */
 ca_status ca_route_adaptive(const ca_shape* shape, const ca_clusters* centroids, double recall,
                             int min_count, const ca_routes* out, void* stream);

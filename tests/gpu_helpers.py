@@ -36,7 +36,7 @@ class Run:
     """Device buffers for one workload and the C-ABI calls on them."""
 
     def __init__(self, w, k=None, compensate=None, seed=0, power_iters=8, transform=True, selection="topk",
-                 recall=0.9, min_count=16, clustering="split"):
+                 recall=0.9, min_count=16, clustering="split", c_k=0):
         t = torch()
         self.w = w
         self.k = w.k if k is None else k
@@ -48,8 +48,10 @@ class Run:
         self.layer = ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, self.k, dtype=w.dtype,
                                          compensate=self.compensate, power_iters=power_iters,
                                          transform=transform, seed=seed, selection=selection, recall=recall,
-                                         min_count=min_count, clustering=clustering)
+                                         min_count=min_count, clustering=clustering, c_k=c_k)
         self.C = self.layer.C
+        self.Ck = self.layer.Ck
+        self.ck = self.layer.c_k
 
     def cluster(self):
         self.layer.cluster(self.Q, self.K)
@@ -57,12 +59,13 @@ class Run:
         check_device_error()
         b = self.layer.buf
         BH, C, c, d = self.w.B * self.w.H, self.C, self.w.c, self.w.d
+        Ck, ck = self.Ck, self.ck
         return dict(perm_q=b.perm_q.cpu().numpy().reshape(BH, C * c),
-                    perm_k=b.perm_k.cpu().numpy().reshape(BH, C * c),
+                    perm_k=b.perm_k.cpu().numpy().reshape(BH, Ck * ck),
                     count_q=b.count_q.cpu().numpy().reshape(BH, C),
-                    count_k=b.count_k.cpu().numpy().reshape(BH, C),
+                    count_k=b.count_k.cpu().numpy().reshape(BH, Ck),
                     qbar=b.qbar.cpu().numpy().reshape(BH, C, d),
-                    kbar=b.kbar.cpu().numpy().reshape(BH, C, d))
+                    kbar=b.kbar.cpu().numpy().reshape(BH, Ck, d))
 
     def set_clusters(self, heads):
         """Overwrite the device cluster buffers with oracle results (list over bh)."""
@@ -81,7 +84,7 @@ class Run:
         check_device_error()
         b = self.layer.buf
         BH, C = self.w.B * self.w.H, self.C
-        W = (C + 31) // 32
+        W = (self.Ck + 31) // 32
         return (b.kept_idx.cpu().numpy().reshape(BH, C, self.k),
                 b.kept_bits.cpu().numpy().view(np.uint32).reshape(BH, C, W))
 
@@ -95,7 +98,7 @@ class Run:
         t = torch()
         b = self.layer.buf
         b.kept_idx.copy_(t.from_numpy(np.concatenate([k.ravel() for k in kept_list]).astype(np.int32)))
-        bits = np.concatenate([orc.route_bits(k, self.C).ravel() for k in kept_list])
+        bits = np.concatenate([orc.route_bits(k, self.Ck).ravel() for k in kept_list])
         b.kept_bits.copy_(t.from_numpy(bits.view(np.int32)))
 
     def attend(self):
