@@ -330,6 +330,8 @@ struct TcParams {
   int tiles_per_cluster;      // c / 128 (1 when c = 64)
   int rows_per_tile;          // min(c, 128): query rows of a tile that belong to its cluster
   int n_tiles;                // sparse: query tiles over all heads
+  int pair;                   // 1: a tile holds two query clusters of 64 (rows 0-63 and 64-127)
+                              // and runs over the union of their kept key clusters
   int compensate;
   int J_cent;                 // compensation blocks per tile: ceil(C / 64) with compensation, else 0
   int dense;                  // 1: identity order, every key block kept
@@ -347,20 +349,25 @@ struct TcParams {
 };
 
 struct Tile {
+  int exists;    // the CTA has this tile (the last CTA may have one only)
   int bh, a, sub;
+  int two;       // pair mode: the tile holds query clusters a and a + 1
   int kq;        // kept key clusters
   int J_kept;    // kept key blocks
   int J;         // all blocks (kept, then compensation); 0 for a missing tile
   int qrow;      // first Q row of the tile (permuted rows; head rows in dense mode)
 };
 
-__device__ __forceinline__ Tile make_tile(const TcParams& p, int t) {
+// kq_union: in pair mode, the size of the tile's union of kept clusters
+// (computed by the kernel's prologue), ignored otherwise.
+__device__ __forceinline__ Tile make_tile(const TcParams& p, int t, int kq_union = 0) {
   Tile T;
-  T.bh = 0; T.a = 0; T.sub = 0; T.kq = 0; T.J_kept = 0; T.J = 0; T.qrow = 0;
+  T.exists = 0; T.bh = 0; T.a = 0; T.sub = 0; T.two = 0; T.kq = 0; T.J_kept = 0; T.J = 0; T.qrow = 0;
   if (p.dense) {
     const int ti = blockIdx.x * 2 + t;
     T.bh = blockIdx.y;
     if (ti < p.dense_tiles) {
+      T.exists = 1;
       T.qrow = ti * 128;
       T.J_kept = p.dense_key_blocks;
       T.J = T.J_kept;
@@ -369,6 +376,18 @@ __device__ __forceinline__ Tile make_tile(const TcParams& p, int t) {
   }
   const int ti = blockIdx.x * 2 + t;
   if (ti >= p.n_tiles) return T;
+  T.exists = 1;
+  if (p.pair) {
+    const int pairs = (p.C + 1) / 2;
+    T.bh = ti / pairs;
+    T.a = 2 * (ti % pairs);
+    T.two = T.a + 1 < p.C;
+    T.kq = kq_union;
+    T.J_kept = p.ck >= 128 ? T.kq * (p.ck / 128) : (T.kq + 1) / 2;
+    T.J = T.J_kept + p.J_cent;
+    T.qrow = (T.bh * p.C + T.a) * p.c;
+    return T;
+  }
   const int per_head = p.C * p.tiles_per_cluster;
   T.bh = ti / per_head;
   const int rem = ti % per_head;
@@ -522,23 +541,84 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   int32_t* kcnt_s = kept_s + 2 * Cfg::kMaxKept;                         // [2][kMaxKept]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Tile T0 = make_tile(p, 0), T1 = make_tile(p, 1);
+  __shared__ int kq_union[2];
+  if (p.pair) {
+    // Pair mode: each tile runs over the union of its two query clusters'
+    // kept key clusters, listed in ascending order from the OR of their
+    // bitmasks; an entry's count carries which of the two keep it (bit 16:
+    // the first cluster, bit 17: the second).
+    int* wcnt = reinterpret_cast<int*>(bias_w);   // [2][256] word counts, free until the softmax stages biases
+    const int W = (p.Ck + 31) / 32;
+    for (int t = 0; t < 2; ++t) {
+      const Tile B = make_tile(p, t);
+      const uint32_t* r0 = p.kept_bits + ((size_t)B.bh * p.C + B.a) * W;
+      const uint32_t* r1 = B.two ? r0 + W : nullptr;
+      for (int w = threadIdx.x; w < W; w += Cfg::kThreads)
+        wcnt[t * 256 + w] = B.exists ? __popc(r0[w] | (r1 ? r1[w] : 0u)) : 0;
+    }
+    __syncthreads();
+    if (warp < 2) {
+      // exclusive scan of the W word counts of tile `warp` (W <= 256: 8 per lane)
+      const int t = warp;
+      int v[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) { const int w = lane * 8 + q; v[q] = w < W ? wcnt[t * 256 + w] : 0; tot += v[q]; }
+      int inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      int run = inc - tot;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int w = lane * 8 + q;
+        if (w < W) wcnt[t * 256 + w] = run;
+        run += v[q];
+      }
+      if (lane == 31) kq_union[t] = inc;
+    }
+    __syncthreads();
+    for (int t = 0; t < 2; ++t) {
+      const Tile B = make_tile(p, t);
+      if (!B.exists) continue;
+      const uint32_t* r0 = p.kept_bits + ((size_t)B.bh * p.C + B.a) * W;
+      const uint32_t* r1 = B.two ? r0 + W : nullptr;
+      for (int w = threadIdx.x; w < W; w += Cfg::kThreads) {
+        const uint32_t m0 = r0[w], m1 = r1 ? r1[w] : 0u;
+        uint32_t u = m0 | m1;
+        int o = wcnt[t * 256 + w];
+        while (u) {
+          const int bit = __ffs(u) - 1;
+          const int b = w * 32 + bit;
+          kept_s[t * Cfg::kMaxKept + o] = b;
+          kcnt_s[t * Cfg::kMaxKept + o] = p.count_k[(size_t)B.bh * p.Ck + b] | (int)(((m0 >> bit) & 1u) << 16) |
+                                          (int)(((m1 >> bit) & 1u) << 17);
+          ++o;
+          u &= u - 1;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const Tile T0 = make_tile(p, 0, p.pair ? kq_union[0] : 0), T1 = make_tile(p, 1, p.pair ? kq_union[1] : 0);
   // both tiles attend the same key blocks: dense attention, or the two
   // halves of one 256-query cluster
   const bool shared_kv = T1.J > 0 && (p.dense || (p.c == 256 && T0.bh == T1.bh && T0.a == T1.a));
   // kept lists (and the kept clusters' sizes) in shared memory when they fit
-  const bool kept_sm0 = !p.dense && T0.kq <= Cfg::kMaxKept;
-  const bool kept_sm1 = !p.dense && T1.kq <= Cfg::kMaxKept;
+  // (pair mode: already there, the unions)
+  const bool kept_sm0 = !p.dense && (p.pair || T0.kq <= Cfg::kMaxKept);
+  const bool kept_sm1 = !p.dense && (p.pair || T1.kq <= Cfg::kMaxKept);
   const int32_t* kept_g0 = p.dense ? nullptr : p.kept_idx + ((size_t)T0.bh * p.C + T0.a) * p.k;
   const int32_t* kept_g1 = p.dense ? nullptr : p.kept_idx + ((size_t)T1.bh * p.C + T1.a) * p.k;
-  if (kept_sm0 && T0.J > 0) {
+  if (!p.pair && kept_sm0 && T0.J > 0) {
     for (int i = threadIdx.x; i < T0.kq; i += Cfg::kThreads) {
       const int b = kept_g0[i];
       kept_s[i] = b;
       kcnt_s[i] = p.count_k[(size_t)T0.bh * p.Ck + b];
     }
   }
-  if (kept_sm1 && T1.J > 0) {
+  if (!p.pair && kept_sm1 && T1.J > 0) {
     for (int i = threadIdx.x; i < T1.kq; i += Cfg::kThreads) {
       const int b = kept_g1[i];
       kept_s[Cfg::kMaxKept + i] = b;
@@ -778,8 +858,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Cfg::kRegSoftmax));
     constexpr unsigned kPoly = D == 64 ? (unsigned)CA_TC_POLY64 : (unsigned)CA_TC_POLY128;
     const int t = warp >> 2;
-    const Tile Tt = make_tile(p, t);
+    const Tile Tt = make_tile(p, t, p.pair ? kq_union[t] : 0);
     const int q4 = warp & 3;                  // TMEM lane quarter of this warp
+    const int grp = p.pair ? (q4 >> 1) : 0;   // pair mode: rows 64-127 belong to the second query cluster
     const int row = q4 * 32 + lane;           // row of the query tile
     const uint32_t lane_addr = tmem + ((uint32_t)(q4 * 32) << 16);
     const uint32_t s_addr = lane_addr + (uint32_t)(t * 128);
@@ -787,14 +868,22 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t o_addr = lane_addr + Cfg::kOCol + (uint32_t)(t * D);
     const float sc = p.scale_log2;
     float* bias = bias_w + warp * 64;
+    // (a tile holding one cluster only: its second half's rows are discarded,
+    // and read the first cluster's row)
     const uint32_t* kb_row =
-        p.dense ? nullptr : p.kept_bits + ((size_t)Tt.bh * p.C + Tt.a) * ((p.Ck + 31) / 32);
+        p.dense ? nullptr : p.kept_bits + ((size_t)Tt.bh * p.C + Tt.a + (Tt.two ? grp : 0)) * ((p.Ck + 31) / 32);
     // the tile's kept clusters' sizes: staged in shared memory, or read through the kept list
-    const bool ksm = !p.dense && Tt.kq <= Cfg::kMaxKept;
+    const bool ksm = !p.dense && (p.pair || Tt.kq <= Cfg::kMaxKept);
     const int32_t* kcnt_t = kcnt_s + t * Cfg::kMaxKept;
     const int32_t* kept_t = p.dense ? nullptr : p.kept_idx + ((size_t)Tt.bh * p.C + Tt.a) * p.k;
     const int32_t* cnt_h = p.count_k + (size_t)Tt.bh * p.Ck;
-    auto cnt_of = [&](int i) -> int { return ksm ? kcnt_t[i] : cnt_h[kept_t[i]]; };
+    // members of the kept cluster i for this thread's rows (in pair mode only
+    // the clusters its own query cluster keeps; the others are masked)
+    auto cnt_of = [&](int i) -> int {
+      if (!ksm) return cnt_h[kept_t[i]];
+      const int e = kcnt_t[i];
+      return (!p.pair || ((e >> (16 + grp)) & 1)) ? (e & 0xFFFF) : 0;
+    };
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     // P_t and O_t of the previous block are free once its PV completed
@@ -880,21 +969,28 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
-    // epilogue: O / l to the query's original row
-    if (ok && Tt.J > 0) {
-      ok = __all_sync(0xffffffffu, wait_bar(&pv_done[t], (Tt.J - 1) & 1, limit, abort_flag));
+    // epilogue: O / l to the query's original row (zero when the tile had no
+    // block at all: nothing kept and no compensation)
+    if (ok && Tt.exists) {
+      if (Tt.J > 0) ok = __all_sync(0xffffffffu, wait_bar(&pv_done[t], (Tt.J - 1) & 1, limit, abort_flag));
       if (ok) {
-        tc_fence_after();
+        if (Tt.J > 0) tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         int orow;
         if (p.dense) orow = Tt.qrow + row < p.n_valid ? Tt.qrow + row : -1;
+        else if (p.pair) orow = row < (Tt.two ? 128 : 64) ? p.perm_q[(size_t)Tt.qrow + row] : -1;
         else orow = (Tt.sub * 128 + row < p.c && row < p.rows_per_tile) ? p.perm_q[(size_t)Tt.qrow + row] : -1;
         __nv_bfloat16* dst = p.O + ((size_t)Tt.bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
-          CA_TMEM_LD32(o_addr + (uint32_t)c0, o);
-          tmem_wait_ld();
+          if (Tt.J > 0) {
+            CA_TMEM_LD32(o_addr + (uint32_t)c0, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) o[q] = 0u;
+          }
           if (orow >= 0) {
             uint4 w[4];
             uint32_t* wp = reinterpret_cast<uint32_t*>(w);
@@ -1010,7 +1106,10 @@ cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_
   p.k = rt->k; p.Cpad = L.Cpad; p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
   p.tiles_per_cluster = c >= 128 ? c / 128 : 1;
   p.rows_per_tile = c >= 128 ? 128 : c;
-  p.n_tiles = BH * C * p.tiles_per_cluster;
+  // 64-query clusters go two to a 128-row tile while their union of kept key
+  // clusters (at most 2 k) fits the kernel's staged list
+  p.pair = (c == 64 && 2 * rt->k <= 512) ? 1 : 0;
+  p.n_tiles = p.pair ? BH * ((C + 1) / 2) : BH * C * p.tiles_per_cluster;
   p.compensate = compensate;
   p.J_cent = compensate ? (Ck + 63) / 64 : 0;
   p.dense = 0;
