@@ -18,14 +18,18 @@
 //               query's original row;
 //   warps 4-7   the same for tile 1;
 //   warp 8      TMA producer (one thread): both Q tiles once, then a ring of
-//               K slots and a ring of V slots, each slot one 128-row tile;
-//   warp 9      MMA issuer (the warp polls, one leader lane issues each
-//               group of products from precomputed descriptors):
-//               S_t = Q_t K_j^T and O_t += P_t V_j, each tile advancing on
-//               its own as soon as the operands are ready. At d = 128, S_t of
-//               block j+1 overwrites P_t of block j, so it waits for
-//               O_t += P_t V_j; at d = 64, P_t has its own TMEM columns.
-//   warps 10-11 idle.
+//               K slots and a ring of V slots, each slot one 128-row tile,
+//               filled in a fixed order (V two entries behind K);
+//   warps 9, 10 MMA issuers, one per tile (one leader lane issues each group
+//               of products from precomputed descriptors): S_t = Q_t K_j^T
+//               and O_t += P_t V_j in the tile's own order. At d = 128, S_t
+//               of block j+1 overwrites P_t of block j, so it waits for
+//               O_t += P_t V_j; at d = 64, P_t has its own TMEM columns and
+//               S_t of block j+1 is computed while block j's softmax runs;
+//   warp 11     idle.
+// Every wait is an mbarrier try_wait, which suspends the warp until the
+// phase completes: the producer and the issuers take no issue slots from the
+// softmax warps that share their SM sub-partitions.
 // A key block is 128 key slots: one or half of a kept key cluster (c = 128,
 // 256), two kept clusters of 64 (c = 64), or 128 consecutive keys (dense).
 // A compensation block is 64 key-cluster centroids: bf16 hi parts in rows
@@ -92,17 +96,6 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(su32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Non-blocking probe, for loops that poll several barriers (try_wait may
-// suspend the thread until the one barrier it names completes).
-__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(su32(b)), "r"(parity)
       : "memory");
@@ -303,22 +296,6 @@ __device__ __forceinline__ void drain_bar(uint64_t* b, uint32_t parity) {
     if ((i & 31) == 31 && now_ns() - t0 > kDrainLimitNs) return;
   }
 }
-// Progress watchdog of a polling loop: call on every turn without progress;
-// returns false (after raising the timeout) once no progress was made for
-// limit_ns, or when another role aborted.
-struct Watchdog {
-  uint64_t t0 = 0;
-  uint32_t idle = 0;
-  __device__ __forceinline__ void progressed() { idle = 0; }
-  __device__ __forceinline__ bool ok(uint64_t limit_ns, volatile int* abort_flag) {
-    if (idle == 0) t0 = now_ns();
-    __nanosleep(32);   // leave the issue slots to the softmax warps meanwhile
-    if ((++idle & 31) != 0) return true;
-    if (*abort_flag) return false;
-    if (now_ns() - t0 > limit_ns) { raise_timeout(abort_flag); return false; }
-    return true;
-  }
-};
 
 // ---------------------------------------------------------------------------
 // Kernel parameters and per-tile bookkeeping
@@ -533,8 +510,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* s_free = s_full + 2;           // [2] S_t read into registers (128 arrivals; separate P only)
   uint64_t* p_full = s_free + 2;           // [2] P_t written (128 arrivals)
   uint64_t* pv_done = p_full + 2;          // [2] O_t += P_t V completed
-  uint64_t* drain = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = pv_done + 2;           // [2] one per MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* bias_w = reinterpret_cast<float*>(smem + Cfg::kBiasOff);   // [8 warps][64]
   int32_t* kept_s = reinterpret_cast<int32_t*>(smem + Cfg::kKeptOff);   // [2][kMaxKept]
@@ -642,7 +619,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       mbar_init(&p_full[t], 128);
       mbar_init(&pv_done[t], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -658,7 +636,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint64_t limit = p.wait_limit;
   const int NI = T0.J + T1.J;                   // (tile, block) items
   const int NR = shared_kv ? T0.J : NI;         // ring items (one per item, or one per block when shared)
-  const int nsb = p.ck >= 128 ? p.ck / 128 : 1;   // key blocks per kept cluster (c_k >= 128)
   // Ring index of block j of tile t: the producer fills the rings in the
   // interleaved order (0,0), (1,0), (0,1), (1,1), ... (or one entry per block
   // when the tiles share K/V); each tile consumes its own entries in order.
@@ -699,7 +676,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tma_3d(d, mk, bar, sb * 64, j * 128, Tt.bh);
           } else if (j < Tt.J_kept) {
             if (p.ck >= 128) {
-              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.Ck + kept_at(t, j / nsb)) * p.ck + (j % nsb) * 128);
+              // c_k is 128 or 256: one or two key blocks per kept cluster (a
+              // shift, not a division: this thread shares its SM sub-partition's
+              // MUFU unit with a softmax warp's exponentials)
+              const int sh = p.ck >> 8;
+              tma_2d(d, mk, bar, sb * 64, (Tt.bh * p.Ck + kept_at(t, j >> sh)) * p.ck + (j & sh) * 128);
             } else {
               // two key clusters of 64; an odd count repeats the first (its
               // columns are masked, and its values stay finite)
@@ -714,22 +695,25 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           }
         }
       };
-      int kn = 0, vn = 0;
-      Watchdog wd;
-      while (vn < NR) {
-        bool prog = false;
-        if (kn < NR && mbar_test(&kempty[kn % KS], ((kn / KS) & 1) ^ 1)) {
+      // Fixed order: K of ring entry i, then V of entry i - kVLag (V is
+      // consumed a softmax later than K). Each slot is refilled once the
+      // products that read it have completed; the waits are bounded
+      // try_waits, so the warp sleeps in hardware meanwhile.
+      constexpr int kVLag = 2;
+      int kn = 0, vn = 0;   // entries whose K / V copies were issued
+      while (ok && vn < NR) {
+        if (kn < NR) {
+          if (!(ok = wait_bar(&kempty[kn % KS], ((kn / KS) & 1) ^ 1, limit, abort_flag))) break;
           load_item(kn, false, sK + (kn % KS) * Cfg::kTileBytes, &kfull[kn % KS]);
           ++kn;
-          prog = true;
         }
-        if (vn < kn && mbar_test(&vempty[vn % VS], ((vn / VS) & 1) ^ 1)) {
+        // V of the entries up to kn - kVLag, or of all the rest once every K is issued
+        const int vlim = kn < NR ? kn - kVLag : NR;
+        while (vn < vlim) {
+          if (!(ok = wait_bar(&vempty[vn % VS], ((vn / VS) & 1) ^ 1, limit, abort_flag))) break;
           load_item(vn, true, sV + (vn % VS) * Cfg::kTileBytes, &vfull[vn % VS]);
           ++vn;
-          prog = true;
         }
-        if (prog) wd.progressed();
-        else if (!wd.ok(limit, abort_flag)) { ok = false; break; }
       }
       if (!ok) {
         // Let every copy already issued land before the CTA leaves.
@@ -739,38 +723,43 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int i = (vn > VS ? vn - VS : 0); i < vn; ++i) drain_bar(&vfull[i % VS], (i / VS) & 1);
       }
     }
-   } else if (warp == 9) {
-    // ------------------------------------------------------------- MMA issuer
-    // The whole warp runs this loop (so decisions are warp-uniform); the
-    // leader lane issues the products. Each tile advances on its own: its next PV_t as soon as P_t and the V tile
-    // are there, its next S_t as soon as the K tile is there and S_t (or, at
-    // d = 128, P_t under it) has been consumed.
-    constexpr uint32_t id_qk128 = idesc_bf16(128, 128, 0);
-    constexpr uint32_t id_qk64 = idesc_bf16(128, 64, 0);
-    constexpr uint32_t id_pv = idesc_bf16(128, D, 1);
-    bool ok = true;
-    if (T0.J > 0) ok = __all_sync(0xffffffffu, wait_bar(&q_full[0], 0, limit, abort_flag));
-    if (ok && T1.J > 0) ok = __all_sync(0xffffffffu, wait_bar(&q_full[1], 0, limit, abort_flag));
-    int qn0 = 0, qn1 = 0, pn0 = 0, pn1 = 0;
-    Watchdog wd;
+   } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------- MMA issuers
+    // Warp 9 issues tile 0's products, warp 10 tile 1's, each in its tile's
+    // own order: S_t of block j+1 as soon as S_t of block j has been read
+    // (separate P) or O_t += P_t V_j has completed (P under S), O_t += P_t V_j
+    // as soon as P_t is written. Every wait is a (bounded) mbarrier try_wait,
+    // which suspends the warp in hardware instead of spending issue slots;
+    // the leader lane issues from precomputed descriptors.
+    const int t = warp - 9;
+    const int J = t ? T1.J : T0.J, J_kept = t ? T1.J_kept : T0.J_kept;
+    const uint32_t id_qk = idesc_bf16(128, 128, 0);
+    const uint32_t id_qk64 = idesc_bf16(128, 64, 0);
+    const uint32_t id_pv = idesc_bf16(128, D, 1);
     // Descriptor templates: the start address sits in the low 14 bits (in
     // 16-byte units), so a tile or a K step is a small constant added to the
     // low word; every product's descriptors cost one add each.
-    const uint64_t qd0 = sdesc(su32(sQ), 16, 1024);
+    const uint64_t qd = sdesc(su32(sQ), 16, 1024) + (uint64_t)((t * Cfg::kTileBytes) >> 4);
     const uint64_t kd0 = sdesc(su32(sK), 16, 1024);
     const uint64_t vd0 = sdesc(su32(sV), Cfg::kSubBytes, 1024);
+    const uint32_t s_tmem = tmem + (uint32_t)(t * 128);
+    const uint32_t p_tmem = tmem + Cfg::kPCol + (uint32_t)(t * Cfg::kPStride);
+    const uint32_t o_tmem = tmem + Cfg::kOCol + (uint32_t)(t * D);
     const bool leader = elect_one();
-    // S_t = Q_t K_j^T into TMEM (leader lane), then the commits
-    auto issue_qk = [&](int t, int j, int r) {
+    auto wait_all = [&](uint64_t* b, uint32_t parity) -> bool {
+      const bool r = __all_sync(0xffffffffu, wait_bar(b, parity, limit, abort_flag));
+      if (r) tc_fence_after();
+      return r;
+    };
+    // S_t = Q_t K_j^T (block j in ring entry r), then the commits
+    auto issue_qk = [&](int j, int r) {
       if (leader) {
-        const uint64_t qd = qd0 + (uint64_t)((t * Cfg::kTileBytes) >> 4);
         const uint64_t kd = kd0 + (uint64_t)(((r % KS) * Cfg::kTileBytes) >> 4);
-        const uint32_t s_tmem = tmem + (uint32_t)(t * 128);
-        if (j < (t ? T1.J_kept : T0.J_kept)) {
+        if (j < J_kept) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = (uint64_t)(((kk >> 2) * Cfg::kSubBytes + (kk & 3) * 32) >> 4);
-            mma_ss(s_tmem, qd + off, kd + off, id_qk128, kk > 0 ? 1u : 0u);
+            mma_ss(s_tmem, qd + off, kd + off, id_qk, kk > 0 ? 1u : 0u);
           }
         } else {
           // centroid hi parts (rows 0-63), then lo parts (rows 64-127)
@@ -789,13 +778,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       __syncwarp();
     };
-    // O_t += P_t V_j (leader lane), then the commits
-    auto issue_pv = [&](int t, int j, int r) {
+    // O_t += P_t V_j (block j in ring entry r), then the commits
+    auto issue_pv = [&](int j, int r) {
       if (leader) {
         const uint64_t vd = vd0 + (uint64_t)(((r % VS) * Cfg::kTileBytes) >> 4);
-        const uint32_t p_tmem = tmem + Cfg::kPCol + (uint32_t)(t * Cfg::kPStride);
-        const uint32_t o_tmem = tmem + Cfg::kOCol + (uint32_t)(t * D);
-        if (j < (t ? T1.J_kept : T0.J_kept)) {
+        if (j < J_kept) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(o_tmem, p_tmem + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
@@ -813,44 +800,33 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       __syncwarp();
     };
-    while (ok && (pn0 < T0.J || pn1 < T1.J)) {
-      bool prog = false;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int J = t ? T1.J : T0.J;
-        int& qn = t ? qn1 : qn0;
-        int& pn = t ? pn1 : pn0;
-        if (pn < qn) {
-          const int r = ring_of(t, pn);
-          const bool rdy = mbar_test(&p_full[t], pn & 1) && mbar_test(&vfull[r % VS], (r / VS) & 1);
-          if (__all_sync(0xffffffffu, rdy)) {
-            tc_fence_after();
-            issue_pv(t, pn, r);
-            ++pn;
-            prog = true;
-          }
-        }
-        if (qn < J) {
-          const int r = ring_of(t, qn);
-          // S_t of block qn overwrites what block qn - 1 left there: its S
-          // must have been read (separate P), or its PV completed (P under S)
-          uint64_t* freed = Cfg::kAliasP ? &pv_done[t] : &s_free[t];
-          const bool rdy = (qn == 0 || (Cfg::kAliasP ? pn >= qn : true)) &&
-                           (qn == 0 || mbar_test(freed, (qn - 1) & 1)) && mbar_test(&kfull[r % KS], (r / KS) & 1);
-          if (__all_sync(0xffffffffu, rdy)) {
-            tc_fence_after();
-            issue_qk(t, qn, r);
-            ++qn;
-            prog = true;
-          }
-        }
+    auto qk_step = [&](int j) -> bool {
+      const int r = ring_of(t, j);
+      if (!wait_all(&kfull[r % KS], (r / KS) & 1)) return false;
+      issue_qk(j, r);
+      return true;
+    };
+    bool ok = J == 0 || wait_all(&q_full[t], 0);
+    if (ok && J > 0) ok = qk_step(0);
+    for (int j = 0; ok && j < J; ++j) {
+      // separate P: S_t of block j+1 may overwrite S_t of block j once it was read
+      if (!Cfg::kAliasP && j + 1 < J) {
+        if (!(ok = wait_all(&s_free[t], j & 1))) break;
+        if (!(ok = qk_step(j + 1))) break;
       }
-      if (prog) wd.progressed();
-      else if (!wd.ok(limit, abort_flag)) ok = false;
+      const int r = ring_of(t, j);
+      if (!(ok = wait_all(&p_full[t], j & 1))) break;
+      if (!(ok = wait_all(&vfull[r % VS], (r / VS) & 1))) break;
+      issue_pv(j, r);
+      // P under S: S_t of block j+1 waits for O_t += P_t V_j to complete
+      if (Cfg::kAliasP && j + 1 < J) {
+        if (!(ok = wait_all(&pv_done[t], j & 1))) break;
+        if (!(ok = qk_step(j + 1))) break;
+      }
     }
-    // Drain: every MMA issued so far has completed once `drain` flips.
-    tc_commit_elect(drain);
-    if (lane == 0) drain_bar(drain, 0);
+    // Drain: every MMA this warp issued has completed once its barrier flips.
+    tc_commit_elect(&drain[t]);
+    if (lane == 0) drain_bar(&drain[t], 0);
     __syncwarp();
    }
   } else {
@@ -930,7 +906,10 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         v0 = min(max(rem, 0), 64);
         v1 = min(max(rem - 64, 0), 64);
       } else if (p.ck >= 128) {
-        const int rem = cnt_of(j / nsb) - (j % nsb) * 128;
+        // c_k is 128 or 256: one or two key blocks per kept cluster (shifts,
+        // not a division, on the softmax warps' path)
+        const int sh = p.ck >> 8;
+        const int rem = cnt_of(j >> sh) - (j & sh) * 128;
         v0 = min(max(rem, 0), 64);
         v1 = min(max(rem - 64, 0), 64);
       } else {

@@ -8,9 +8,9 @@ import pytest
 import workloads as wl
 from oracle import ca_oracle as orc
 
-pytestmark = pytest.mark.gpu
+from tests import parity
 
-TOL = {"bf16": 1e-2, "fp32": 1e-5}
+pytestmark = pytest.mark.gpu
 
 CASES = {
     "lowrank-bf16-d64-n3900pad-c128": lambda: wl.make_workload("lowrank", H=2, N=4096, n_valid=3900, d=64, c=128,
@@ -56,8 +56,7 @@ def test_random_clusters_end_to_end(name, compensate):
         kept = orc.topk_route(orc.centroid_scores(ref.qbar, ref.kbar), w.k)
         want = orc.compensated_attention(Qf, Kf, Vf, ref.perm_q, ref.count_q, ref.perm_k, ref.count_k, kept, w.c,
                                          compensate=compensate)
-        err = np.abs(O[b, h, :w.n_valid] - want).max()
-        assert err <= TOL[w.dtype], f"{name} bh={bh}: max abs {err:.3g}"
+        parity.check(f"random clusters {name} smc={int(compensate)} bh={bh}", O[b, h, :w.n_valid], want, w.dtype)
 
 
 @pytest.mark.parametrize("name", list(CASES))

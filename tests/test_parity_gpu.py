@@ -5,7 +5,8 @@ Bar:
  * routing masks: bit-exact given the oracle's centroids;
  * attention output given the oracle's permutation, mask and centroids:
    max-abs error <= 1e-2 for bf16 inputs (bf16 products, fp32 accumulation),
-   <= 1e-5 for fp32 inputs.
+   <= 1e-5 for fp32 inputs, and relative-L2 error within the bounds derived
+   in tests/parity.py (observed values printed at the end of the session).
 """
 import math
 
@@ -15,42 +16,12 @@ import pytest
 import workloads as wl
 from oracle import ca_oracle as orc
 
+from tests import parity
+from tests.cases import CASES
+
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": 1e-2, "fp32": 1e-5}
-
-
-def _cases():
-    return {
-        "cfg1": lambda: wl.config_workload(1),
-        "mix-fp32-d64-n1000-c64": lambda: wl.make_workload("mixture", H=2, N=1000, d=64, c=64, k=5,
-                                                           dtype="fp32", seed=5),
-        "lowrank-bf16-d64-n3900pad-c128": lambda: wl.make_workload("lowrank", H=3, N=4096, n_valid=3900, d=64,
-                                                                   c=128, k=6, dtype="bf16", seed=6),
-        "lowrank-bf16-d128-n2048-c128": lambda: wl.make_workload("lowrank", H=2, N=2048, d=128, c=128, k=4,
-                                                                 dtype="bf16", seed=7),
-        "mix-bf16-d64-n768-c256-tie": lambda: wl.make_workload("mixture", H=2, N=768, d=64, c=256, k=2,
-                                                               dtype="bf16", seed=8),
-        "single-cluster-n100-c128": lambda: wl.make_workload("mixture", H=1, N=128, n_valid=100, d=64, c=128,
-                                                             k=1, dtype="bf16", seed=9),
-        "n-equals-c": lambda: wl.make_workload("mixture", H=1, N=64, d=64, c=64, k=1, dtype="fp32", seed=10),
-        "n-2c-plus-1": lambda: wl.make_workload("lowrank", H=2, N=320, n_valid=257, d=64, c=128, k=2,
-                                                dtype="bf16", seed=11),
-        "fp32-d128-n640-c64": lambda: wl.make_workload("lowrank", H=1, N=640, d=128, c=64, k=3, dtype="fp32",
-                                                       seed=12),
-        "grid-bf16-d128-c128": lambda: wl.make_workload("grid", H=2, N=6144, d=128, c=128, k=7, dtype="bf16",
-                                                        seed=13, grid=(8, 9, 80)),
-        "heavytail-bf16-d64-c256": lambda: wl.make_workload("heavytail", H=1, N=8192, d=64, c=256, k=4,
-                                                            dtype="bf16", seed=14),
-        # 64-key blocks on the tensor cores, with compensation blocks
-        "heavytail-bf16-d64-c64": lambda: wl.make_workload("heavytail", H=1, N=8192, d=64, c=64, k=8,
-                                                           dtype="bf16", seed=15),
-        "lowrank-bf16-d128-c64": lambda: wl.make_workload("lowrank", H=1, N=2048, n_valid=2000, d=128, c=64,
-                                                          k=5, dtype="bf16", seed=16),
-    }
-
-
-CASES = _cases()
+TOL = parity.MAX_ABS
 
 
 def oracle_clusters(w, seed=0):
@@ -108,8 +79,7 @@ def test_attend_given_oracle_clusters_and_mask(helpers, name, compensate):
         Qf, Kf, Vf = (x[b, hh, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         want = orc.compensated_attention(Qf, Kf, Vf, h.perm_q, h.count_q, h.perm_k, h.count_k, kept[bh], w.c,
                                          compensate=compensate)
-        err = np.abs(O[b, hh, :w.n_valid] - want).max()
-        assert err <= TOL[w.dtype], f"{name} bh={bh}: max abs {err:.3g}"
+        parity.check(f"attend {name} smc={int(compensate)} bh={bh}", O[b, hh, :w.n_valid], want, w.dtype)
         assert np.all(O[b, hh, w.n_valid:] == 0)
 
 
@@ -124,8 +94,7 @@ def test_dense_attention(helpers, name):
             Qf, Kf, Vf = (x[b, hh, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
             rows = np.arange(0, w.n_valid, max(1, w.n_valid // 300))
             want = orc.dense_attention(Qf, Kf, Vf, rows=rows)
-            err = np.abs(O[b, hh, rows] - want).max()
-            assert err <= TOL[w.dtype], f"{name}: max abs {err:.3g}"
+            parity.check(f"dense {name} bh={b * w.H + hh}", O[b, hh, rows], want, w.dtype)
             assert np.all(O[b, hh, w.n_valid:] == 0)
 
 
@@ -138,8 +107,7 @@ def test_forward_end_to_end_matches_oracle_forward(helpers, name):
         b, hh = divmod(bh, w.H)
         Qf, Kf, Vf = (x[b, hh, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         fr = orc.forward_head(Qf, Kf, Vf, w.c, w.k, seed=0, bh=bh)
-        err = np.abs(O[b, hh, :w.n_valid] - fr.O).max()
-        assert err <= TOL[w.dtype], f"{name} bh={bh}: max abs {err:.3g}"
+        parity.check(f"forward {name} bh={bh}", O[b, hh, :w.n_valid], fr.O, w.dtype)
         # error against dense attention, GPU and oracle side by side
         rows = np.arange(0, w.n_valid, max(1, w.n_valid // 200))
         dense = orc.dense_attention(Qf, Kf, Vf, rows=rows)
@@ -183,5 +151,4 @@ def test_full_size_config(helpers, cfg):
         want = orc.compensated_attention(Qf, Kf, Vf, h.perm_q, h.count_q, h.perm_k, h.count_k, kept, w.c,
                                          clusters=sample)
         rows = np.concatenate([h.perm_q[a * w.c: a * w.c + h.count_q[a]] for a in sample])
-        err = np.abs(O[b, hh, rows] - want[rows]).max()
-        assert err <= TOL[w.dtype], f"cfg{cfg} bh={bh}: max abs {err:.3g}"
+        parity.check(f"full-size cfg{cfg} bh={bh} ({len(sample)} clusters)", O[b, hh, rows], want[rows], w.dtype)

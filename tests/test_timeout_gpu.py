@@ -12,6 +12,7 @@ import pytest
 import free_clustered_block_b200 as ca
 import workloads as wl
 from oracle import ca_oracle as orc
+from tests import parity
 
 pytestmark = pytest.mark.gpu
 
@@ -51,4 +52,4 @@ def test_wait_nothing_completes_times_out_and_the_context_recovers():
         b, hh = divmod(bh, w.H)
         Qf, Kf, Vf = (x[b, hh, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         want = orc.compensated_attention(Qf, Kf, Vf, h.perm_q, h.count_q, h.perm_k, h.count_k, kept[bh], w.c)
-        assert np.abs(O[b, hh, :w.n_valid] - want).max() <= 1e-2
+        parity.check(f"after a timeout bh={bh}", O[b, hh, :w.n_valid], want, w.dtype)

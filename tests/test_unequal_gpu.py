@@ -13,9 +13,9 @@ import pytest
 import workloads as wl
 from oracle import ca_oracle as orc
 
-pytestmark = pytest.mark.gpu
+from tests import parity
 
-TOL = {"bf16": 1e-2, "fp32": 1e-5}
+pytestmark = pytest.mark.gpu
 
 CASES = {
     "q64-k128-bf16-d64": (lambda: wl.make_workload("lowrank", H=2, N=4096, n_valid=4000, d=64, c=64, k=5,
@@ -89,8 +89,7 @@ def test_attention_given_oracle_clusters_and_mask(helpers, name, compensate):
         Qf, Kf, Vf = (x[b, hh, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         want = orc.compensated_attention(Qf, Kf, Vf, h.perm_q, h.count_q, h.perm_k, h.count_k, kept[bh], w.c,
                                          compensate=compensate, c_k=ck)
-        err = np.abs(O[b, hh, :w.n_valid] - want).max()
-        assert err <= TOL[w.dtype], f"{name} bh={bh}: max abs {err:.3g}"
+        parity.check(f"unequal attend {name} smc={int(compensate)} bh={bh}", O[b, hh, :w.n_valid], want, w.dtype)
         assert np.all(O[b, hh, w.n_valid:] == 0)
 
 
@@ -104,8 +103,7 @@ def test_forward_end_to_end(helpers, name):
         b, hh = divmod(bh, w.H)
         Qf, Kf, Vf = (x[b, hh, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
         fr = orc.forward_head(Qf, Kf, Vf, w.c, w.k, seed=0, bh=bh, c_k=ck)
-        err = np.abs(O[b, hh, :w.n_valid] - fr.O).max()
-        assert err <= TOL[w.dtype], f"{name} bh={bh}: max abs {err:.3g}"
+        parity.check(f"unequal forward {name} bh={bh}", O[b, hh, :w.n_valid], fr.O, w.dtype)
 
 
 def test_adaptive_selection_with_unequal_sizes(helpers):
