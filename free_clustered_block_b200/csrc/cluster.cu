@@ -672,7 +672,7 @@ struct DirCCfg {
 };
 
 template <typename T, int D_>
-__global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
+__global__ void __launch_bounds__(2 * D_, D_ == 64 ? 3 : 1) dirc_kernel(
     const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, int npc, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
@@ -777,14 +777,34 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
       }
     }
     __syncthreads();
+    // d = 64: this thread's half row (for X w) and half column (for X^T v) of
+    // the sample, converted to fp64 once per node instead of at every use (an
+    // f32 -> f64 conversion issues at a quarter of the fp64 FMA rate); the
+    // products below keep the same operands in the same order either way
+    constexpr bool kRegX = D == 64;
+    double xr_reg[kRegX ? HD : 1], xc_reg[kRegX ? HD : 1];
+    if constexpr (kRegX) {
+#pragma unroll
+      for (int c = 0; c < HD; ++c) xr_reg[c] = (double)to_f(Xs[rj * RS + rh * HD + c]);
+#pragma unroll
+      for (int j = 0; j < HD; ++j) xc_reg[j] = (double)to_f(Xs[(ch * HD + j) * RS + ca]);
+    }
+    auto xcol = [&](int j) -> double {   // X[ch * HD + j][ca]
+      if constexpr (kRegX) return xc_reg[j];
+      else return (double)to_f(Xs[(ch * HD + j) * RS + ca]);
+    };
+    auto xrow = [&](int c) -> double {   // X[rj][rh * HD + c]
+      if constexpr (kRegX) return xr_reg[c];
+      else return (double)to_f(Xs[rj * RS + rh * HD + c]);
+    };
     // sample mean
     {
       double a0 = 0.0, a1 = 0.0;
       const int j0 = ch * HD;
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < HD; j += 2) {
-        a0 = fma(vs[j0 + j], (double)to_f(Xs[(j0 + j) * RS + ca]), a0);
-        a1 = fma(vs[j0 + j + 1], (double)to_f(Xs[(j0 + j + 1) * RS + ca]), a1);
+        a0 = fma(vs[j0 + j], xcol(j), a0);
+        a1 = fma(vs[j0 + j + 1], xcol(j + 1), a1);
       }
       red[ch][ca] = a0 + a1;
       __syncthreads();
@@ -816,14 +836,13 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
       double v = 0.0;
       {
         double d0 = 0.0, d1 = 0.0, d2 = 0.0, d3 = 0.0;
-        const T* xr = Xs + rj * RS + rh * HD;
         const double* wr = ws + rh * HD;
-#pragma unroll 4
+#pragma unroll
         for (int c = 0; c < HD; c += 4) {
-          d0 = fma((double)to_f(xr[c]), wr[c], d0);
-          d1 = fma((double)to_f(xr[c + 1]), wr[c + 1], d1);
-          d2 = fma((double)to_f(xr[c + 2]), wr[c + 2], d2);
-          d3 = fma((double)to_f(xr[c + 3]), wr[c + 3], d3);
+          d0 = fma(xrow(c), wr[c], d0);
+          d1 = fma(xrow(c + 1), wr[c + 1], d1);
+          d2 = fma(xrow(c + 2), wr[c + 2], d2);
+          d3 = fma(xrow(c + 3), wr[c + 3], d3);
         }
         double d = (d0 + d1) + (d2 + d3);
         d += __shfl_xor_sync(0xffffffffu, d, 1);
@@ -842,10 +861,10 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
       {
         double a0 = 0.0, a1 = 0.0;
         const int j0 = ch * HD;
-#pragma unroll 4
+#pragma unroll
         for (int j = 0; j < HD; j += 2) {
-          a0 = fma(fj[j0 + j], (double)to_f(Xs[(j0 + j) * RS + ca]), a0);
-          a1 = fma(fj[j0 + j + 1], (double)to_f(Xs[(j0 + j + 1) * RS + ca]), a1);
+          a0 = fma(fj[j0 + j], xcol(j), a0);
+          a1 = fma(fj[j0 + j + 1], xcol(j + 1), a1);
         }
         red[ch][ca] = a0 + a1;
       }
@@ -875,6 +894,9 @@ __global__ void __launch_bounds__(2 * D_, 1) dirc_kernel(
 // d = 64 levels with at most this many nodes (over all tensor-heads) use the
 // block-per-node power iteration
 constexpr long long kDirCMaxNodes64 = 148 * 4;
+#ifndef CA_DIRC_ALL64
+#define CA_DIRC_ALL64 0
+#endif
 
 constexpr int kProjSpan = 1024;
 constexpr int kProjNodes = 20;   // > kProjSpan / 65 + 2
@@ -1406,7 +1428,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
         const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, rows, basis, inv_s, idx_in,
                                                     NI, wvec, p->seed, p->head_base, tsel, st);
         if (e != cudaSuccess) return e;
-      } else if (sample_factor == 1 && (D == 128 || (long long)nl * rows <= kDirCMaxNodes64)) {
+      } else if (sample_factor == 1 && (D == 128 || CA_DIRC_ALL64 || (long long)nl * rows <= kDirCMaxNodes64)) {
         // a block per node: d = 128, or d = 64 levels with few nodes (about
         // four blocks per SM over the whole level)
         const int npc = (int)(((long long)nl * rows + 4 * 148 - 1) / (4 * 148));
