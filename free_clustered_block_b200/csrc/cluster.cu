@@ -894,9 +894,6 @@ __global__ void __launch_bounds__(2 * D_, D_ == 64 ? 3 : 1) dirc_kernel(
 // d = 64 levels with at most this many nodes (over all tensor-heads) use the
 // block-per-node power iteration
 constexpr long long kDirCMaxNodes64 = 148 * 4;
-#ifndef CA_DIRC_ALL64
-#define CA_DIRC_ALL64 0
-#endif
 
 constexpr int kProjSpan = 1024;
 constexpr int kProjNodes = 20;   // > kProjSpan / 65 + 2
@@ -1428,7 +1425,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
         const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, rows, basis, inv_s, idx_in,
                                                     NI, wvec, p->seed, p->head_base, tsel, st);
         if (e != cudaSuccess) return e;
-      } else if (sample_factor == 1 && (D == 128 || CA_DIRC_ALL64 || (long long)nl * rows <= kDirCMaxNodes64)) {
+      } else if (sample_factor == 1 && (D == 128 || (long long)nl * rows <= kDirCMaxNodes64)) {
         // a block per node: d = 128, or d = 64 levels with few nodes (about
         // four blocks per SM over the whole level)
         const int npc = (int)(((long long)nl * rows + 4 * 148 - 1) / (4 * 148));
