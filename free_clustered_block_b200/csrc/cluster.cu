@@ -140,7 +140,9 @@ __global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, in
 }
 
 // ---------------------------------------------------------------------------
-// S1: partial second-moment matrices over a row chunk.
+// S1: partial second-moment matrices over a row chunk, on the fp64 CUDA
+// cores (the weighted query covariance of the diagonalized splitting; the
+// metrics themselves use syrk_mma_kernel below).
 // z = 0: Q^T Q (uncentred); z = 1: (K - kmean)^T (K - kmean).
 // Only the upper triangle of 8 x 8 tiles is accumulated (the matrix is
 // symmetric): thread t of row group g owns tile t over the staged rows
@@ -280,6 +282,138 @@ __global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* _
             const int r = 8 * I + i, c = 4 * J + j;
             if (c >= r) red[r * D + c] = (gg == 0 ? 0.0 : red[r * D + c]) + acc[i][j];
           }
+      }
+      __syncthreads();
+    }
+    for (int e = threadIdx.x; e < D * D; e += NTH) {
+      const int i = e / D, j = e % D;
+      out[e] = j >= i ? red[e] : red[j * D + i];
+    }
+  }
+}
+
+// The same partial second-moment matrices on the fp64 tensor-core path
+// (mma.sync m8n8k4 f64): the upper triangle of 32 x 32 blocks, one warp per
+// (block, row group); per step of four rows a warp loads four A and four B
+// fragments (one double per lane each) and issues sixteen 8 x 8 x 4 products,
+// so shared memory delivers half a byte per FMA instead of three for the
+// 8 x 4 register tiles of syrk_kernel. Rows are staged as in syrk_kernel
+// (cp.async of the raw rows while the previous tile is multiplied, then one
+// conversion to fp64 minus the mean); the row groups are summed in a fixed
+// order through shared memory.
+template <int D>
+struct SyrkMmaCfg {
+  static constexpr int NB = D / 32;                   // 32-wide blocks per dimension
+  static constexpr int NBT = NB * (NB + 1) / 2;       // blocks on or above the diagonal: 3 / 10
+  static constexpr int RG = D == 64 ? 4 : 1;          // row groups
+  static constexpr int kWarps = NBT * RG;             // 12 / 10
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kRows = 64;                    // rows staged per step (a multiple of 4 RG)
+  static constexpr int kP = D + 4;                    // fp64 row stride: fragment loads hit distinct banks
+  static constexpr size_t kXsBytes = (size_t)kRows * kP * 8 > (RG > 1 ? (size_t)D * D * 8 : 0)
+                                         ? (size_t)kRows * kP * 8
+                                         : (size_t)D * D * 8;
+  template <typename T>
+  static constexpr size_t smem() { return kXsBytes + (size_t)kRows * D * sizeof(T); }
+};
+
+__device__ __forceinline__ void dmma_884(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(SyrkMmaCfg<D>::kThreads, 1) syrk_mma_kernel(
+    const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, int nch,
+    const double* __restrict__ colpart, double* __restrict__ part) {
+  using Cfg = SyrkMmaCfg<D>;
+  constexpr int RG = Cfg::RG, NTH = Cfg::kThreads, ROWS = Cfg::kRows, P = Cfg::kP;
+  constexpr int VEC = 16 / sizeof(T);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* xs = reinterpret_cast<double*>(smem_raw);            // ROWS x P, later D x D for the group sum
+  T* raw = reinterpret_cast<T*>(smem_raw + Cfg::kXsBytes);     // ROWS x D as loaded
+  __shared__ double mean[D];
+  const int bh = blockIdx.y, z = blockIdx.z, ch = blockIdx.x;
+  const T* X = (z == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, tg = lane & 3;                      // fragment row / column in group
+  const int rg = warp / Cfg::NBT, blk = warp % Cfg::NBT;
+  int bi = 0, rem = blk;                                       // block (bi, bj), bj >= bi
+  while (rem >= Cfg::NB - bi) { rem -= Cfg::NB - bi; ++bi; }
+  const int bj = bi + rem;
+
+  auto issue = [&](int rt) {
+    const int rows = min(ROWS, r1 - rt);
+    for (int e = threadIdx.x; e < rows * (D / VEC); e += NTH)
+      cp_async16(raw + e * VEC, X + (size_t)rt * D + (size_t)e * VEC);
+    cp_async_commit();
+  };
+  if (r0 < r1) issue(r0);
+  for (int c = threadIdx.x; c < D; c += NTH) {
+    double m = 0.0;
+    if (z == 1) {
+      for (int i = 0; i < nch; ++i) m += colpart[((size_t)bh * nch + i) * D + c];
+      m /= (double)n;
+    }
+    mean[c] = m;
+  }
+  double acc[4][4][2];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
+  for (int rt = r0; rt < r1; rt += ROWS) {
+    cp_async_wait_all();
+    __syncthreads();   // raw tile complete, mean written, previous tile's products done
+    const int rows = min(ROWS, r1 - rt);
+    for (int e = threadIdx.x; e < ROWS * D; e += NTH) {
+      const int rr = e / D, cc = e % D;
+      xs[rr * P + cc] = rr < rows ? (double)to_f(raw[e]) - mean[cc] : 0.0;
+    }
+    __syncthreads();
+    if (rt + ROWS < r1) issue(rt + ROWS);
+#pragma unroll 2
+    for (int k0 = 4 * rg; k0 < ROWS; k0 += 4 * RG) {
+      const double* xr = xs + (k0 + tg) * P;
+      double fa[4], fb[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) fa[a] = xr[32 * bi + 8 * a + g];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) fb[b] = xr[32 * bj + 8 * b + g];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) dmma_884(acc[a][b], fa[a], fb[b]);
+    }
+  }
+  double* out = part + (((size_t)bh * 2 + z) * nch + ch) * D * D;
+  // this lane's entries: row 32 bi + 8 a + g, columns 32 bj + 8 b + 2 tg + {0, 1}
+  if constexpr (RG == 1) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = 32 * bi + 8 * a + g, c = 32 * bj + 8 * b + 2 * tg + i;
+          if (c >= r) { out[r * D + c] = acc[a][b][i]; out[c * D + r] = acc[a][b][i]; }
+        }
+  } else {
+    __syncthreads();    // last tile's products done before xs becomes the group sum
+    double* red = xs;   // D x D, entries (r, c >= r)
+    for (int gg = 0; gg < RG; ++gg) {
+      if (rg == gg) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = 32 * bi + 8 * a + g, c = 32 * bj + 8 * b + 2 * tg + i;
+              if (c >= r) red[r * D + c] = (gg == 0 ? 0.0 : red[r * D + c]) + acc[a][b][i];
+            }
       }
       __syncthreads();
     }
@@ -1375,9 +1509,10 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     if (!random_clusters) {
       colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
       const size_t syrk_smem = SyrkCfg<D>::template smem<T>();
-      cudaFuncSetAttribute(syrk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
-      syrk_kernel<T, D><<<dim3(nch, BH, 2), SyrkCfg<D>::kThreads, syrk_smem, st>>>(Q, K, N_alloc, n, nch, colpart,
-                                                                                  metpart);
+      const size_t mma_smem = SyrkMmaCfg<D>::template smem<T>();
+      cudaFuncSetAttribute(syrk_mma_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mma_smem);
+      syrk_mma_kernel<T, D><<<dim3(nch, BH, 2), SyrkMmaCfg<D>::kThreads, mma_smem, st>>>(Q, K, N_alloc, n, nch,
+                                                                                        colpart, metpart);
       metric_reduce_kernel<D><<<dim3(D * D / 256, TH), 256, 0, st>>>(metpart, nch, n, transform, M);
       if (D == 64 && normalize) {
         qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
