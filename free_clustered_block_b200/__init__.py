@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(HERE, "libca.so")
 
 CA_OK, CA_ERR_INVALID_ARG, CA_ERR_UNSUPPORTED, CA_ERR_WORKSPACE, CA_ERR_CUDA, CA_ERR_TIMEOUT = range(6)
 CA_BF16, CA_FP32 = 0, 1
+CA_LAYOUT_BHND, CA_LAYOUT_BNHD = 0, 1
 
 EXPORTED = [
     "ca_num_clusters", "ca_check_shape", "ca_cluster_workspace_bytes", "ca_attend_workspace_bytes",
@@ -45,7 +46,8 @@ class CAError(RuntimeError):
 class ca_shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N_alloc", ctypes.c_int),
                 ("n_valid", ctypes.c_int), ("d", ctypes.c_int), ("c", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("c_k", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("c_k", ctypes.c_int), ("layout", ctypes.c_int),
+                ("H_total", ctypes.c_int)]
 
 
 class ca_cluster_params(ctypes.Structure):
@@ -135,9 +137,12 @@ def _stream(stream) -> Optional[int]:
     return getattr(stream, "cuda_stream", stream)
 
 
-def make_shape(B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, dtype: int, c_k: int = 0) -> ca_shape:
-    """c: query cluster size; c_k: key cluster size (0: the same as c)."""
-    return ca_shape(B, H, N_alloc, n_valid, d, c, dtype, c_k)
+def make_shape(B: int, H: int, N_alloc: int, n_valid: int, d: int, c: int, dtype: int, c_k: int = 0,
+               layout: int = 0, H_total: int = 0) -> ca_shape:
+    """c: query cluster size; c_k: key cluster size (0: the same as c).
+    layout: CA_LAYOUT_BHND ([B, H, N, d]) or CA_LAYOUT_BNHD ([B, N, H_total, d],
+    the call's heads first; H_total 0 means H)."""
+    return ca_shape(B, H, N_alloc, n_valid, d, c, dtype, c_k, layout, H_total)
 
 
 def make_params(power_iters: int = 8, sample_factor: int = 1, transform: int = 1,

@@ -34,6 +34,11 @@ ca_status check_shape(const ca_shape* s) {
   if ((long long)s->N_alloc > (1ll << 30) || C * s->c > (1ll << 30) || Ck * ck > (1ll << 30))
     return CA_ERR_UNSUPPORTED;
   if ((long long)s->B * s->H > 65535) return CA_ERR_UNSUPPORTED;   // grid.y
+  if (s->layout != CA_LAYOUT_BHND && s->layout != CA_LAYOUT_BNHD) return CA_ERR_INVALID_ARG;
+  if (s->layout == CA_LAYOUT_BHND && s->H_total != 0 && s->H_total != s->H) return CA_ERR_INVALID_ARG;
+  if (s->layout == CA_LAYOUT_BNHD && s->H_total != 0 && s->H_total < s->H) return CA_ERR_INVALID_ARG;
+  if (s->layout == CA_LAYOUT_BNHD && (long long)(s->H_total ? s->H_total : s->H) * s->d * 4 > (1ll << 31))
+    return CA_ERR_UNSUPPORTED;
   return CA_OK;
 }
 
@@ -317,12 +322,16 @@ namespace {
 constexpr int kHostGroups = 4;
 
 int host_groups(const ca_shape* s) {
+  // a group of heads is a contiguous byte range only in the [B][H][N][d] layout
+  if (s->layout != CA_LAYOUT_BHND) return 1;
   const int BH = s->B * s->H;
   return BH < kHostGroups ? BH : kHostGroups;
 }
 
-// Shape of group g: B = 1, H = the group's head count; first flattened head in *first.
+// Shape of group g: B = 1, H = the group's head count; first flattened head in
+// *first. A single group is the whole shape.
 ca_shape group_shape(const ca_shape* s, int g, int G, int* first) {
+  if (G == 1) { *first = 0; return *s; }
   const int BH = s->B * s->H, base = BH / G, extra = BH % G;
   *first = g * base + (g < extra ? g : extra);
   ca_shape gs = *s;
@@ -337,6 +346,7 @@ extern "C" {
 
 size_t ca_forward_host_workspace_bytes(const ca_shape* s, int k) {
   if (check_shape(s) != CA_OK) return 0;
+  if (!layout_contiguous(s)) return 0;   // host buffers hold exactly the call's heads
   int first = 0;
   const ca_shape g0 = group_shape(s, 0, host_groups(s), &first);   // the largest group
   const size_t base = ca_forward_workspace_bytes(&g0, k);
@@ -351,6 +361,7 @@ ca_status ca_forward_host(const void* Qh, const void* Kh, const void* Vh, const 
                           size_t workspace_bytes, void* stream) {
   ca_status st = check_shape(s);
   if (st != CA_OK) return st;
+  if (!layout_contiguous(s)) return CA_ERR_UNSUPPORTED;
   if (!Qh || !Kh || !Vh || !Oh) return CA_ERR_INVALID_ARG;
   if ((st = check_params(s, params)) != CA_OK) return st;
   const size_t need = ca_forward_host_workspace_bytes(s, k);
@@ -389,7 +400,7 @@ ca_status ca_forward_host(const void* Qh, const void* Kh, const void* Vh, const 
   for (int g = 0; g < G && e == cudaSuccess; ++g) {
     int b0 = 0;
     const ca_shape gs = group_shape(s, g, G, &b0);
-    const size_t off = (size_t)b0 * head_bytes, bytes = (size_t)gs.H * head_bytes;
+    const size_t off = (size_t)b0 * head_bytes, bytes = G == 1 ? t : (size_t)gs.H * head_bytes;
     e = cudaMemcpyAsync(dQ + off, static_cast<const char*>(Qh) + off, bytes, cudaMemcpyHostToDevice, s_in);
     if (e == cudaSuccess)
       e = cudaMemcpyAsync(dK + off, static_cast<const char*>(Kh) + off, bytes, cudaMemcpyHostToDevice, s_in);
@@ -400,7 +411,7 @@ ca_status ca_forward_host(const void* Qh, const void* Kh, const void* Vh, const 
   for (int g = 0; g < G && e == cudaSuccess && st == CA_OK; ++g) {
     int b0 = 0;
     const ca_shape gs = group_shape(s, g, G, &b0);
-    const size_t off = (size_t)b0 * head_bytes, bytes = (size_t)gs.H * head_bytes;
+    const size_t off = (size_t)b0 * head_bytes, bytes = G == 1 ? t : (size_t)gs.H * head_bytes;
     e = cudaStreamWaitEvent(cs, ev_in[g], 0);
     if (e != cudaSuccess) break;
     ca_cluster_params pg = p;

@@ -26,7 +26,7 @@ template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v
 // and their lo parts in rows 64-127 ([BH][Cpad / 64][128][D]).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) centroid_prep_kernel(
-    const T* __restrict__ V, int N_alloc, int c, int C, int Cpad, const int32_t* __restrict__ perm_k,
+    const T* __restrict__ V, TensorLayout TL, int c, int C, int Cpad, const int32_t* __restrict__ perm_k,
     const int32_t* __restrict__ count_k, const double* __restrict__ kbar, float* __restrict__ kbar32,
     float* __restrict__ vbar32, __nv_bfloat16* __restrict__ kbar_hl, __nv_bfloat16* __restrict__ vbar_hl,
     float* __restrict__ logcnt) {
@@ -45,9 +45,9 @@ __global__ void __launch_bounds__(256) centroid_prep_kernel(
   }
   const int cnt = count_k[(size_t)bh * C + b];
   const int32_t* mem = perm_k + (size_t)bh * C * c + (size_t)b * c;
-  const T* Vh = V + (size_t)bh * N_alloc * D;
+  const T* Vh = V + TL.head(bh);
   double s = 0.0;
-  for (int j = rg; j < cnt; j += RG) s += (double)to_f(Vh[(size_t)mem[j] * D + col]);
+  for (int j = rg; j < cnt; j += RG) s += (double)to_f(Vh[(size_t)mem[j] * TL.sn + col]);
   __shared__ double red[256];
   red[threadIdx.x] = s;
   __syncthreads();
@@ -74,13 +74,13 @@ __global__ void __launch_bounds__(256) centroid_prep_kernel(
 template <int D>
 __global__ void __launch_bounds__(256) permute_rows_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-    const __nv_bfloat16* __restrict__ V, int N_alloc, int slots_q, int slots_k, const int32_t* __restrict__ perm_q,
+    const __nv_bfloat16* __restrict__ V, TensorLayout TL, int slots_q, int slots_k, const int32_t* __restrict__ perm_q,
     const int32_t* __restrict__ perm_k, __nv_bfloat16* __restrict__ Qp, __nv_bfloat16* __restrict__ Kp,
     __nv_bfloat16* __restrict__ Vp) {
   constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
   const int bh = blockIdx.y, z = blockIdx.z;
   const int slots = z == 0 ? slots_q : slots_k;
-  const __nv_bfloat16* src = (z == 0 ? Q : (z == 1 ? K : V)) + (size_t)bh * N_alloc * D;
+  const __nv_bfloat16* src = (z == 0 ? Q : (z == 1 ? K : V)) + TL.head(bh);
   __nv_bfloat16* dst = (z == 0 ? Qp : (z == 1 ? Kp : Vp)) + (size_t)bh * slots * D;
   const int32_t* perm = (z == 0 ? perm_q : perm_k) + (size_t)bh * slots;
   const size_t e = (size_t)blockIdx.x * 256 + threadIdx.x;
@@ -88,18 +88,16 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(
   if (slot >= slots) return;
   const int row = perm[slot];
   uint4 val = make_uint4(0, 0, 0, 0);
-  if (row >= 0) val = *reinterpret_cast<const uint4*>(src + (size_t)row * D + v * 8);
+  if (row >= 0) val = *reinterpret_cast<const uint4*>(src + (size_t)row * TL.sn + v * 8);
   *reinterpret_cast<uint4*>(dst + (size_t)slot * D + v * 8) = val;
 }
 
-__global__ void zero_rows_kernel(uint4* __restrict__ O, size_t row_vecs, size_t rows_per_head,
-                                 size_t first_row, size_t pad_rows, size_t BH) {
-  const size_t per_head = pad_rows * row_vecs;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < per_head * BH;
-       e += (size_t)gridDim.x * blockDim.x) {
-    const size_t bh = e / per_head, r = e % per_head;
-    O[(bh * rows_per_head + first_row) * row_vecs + r] = make_uint4(0, 0, 0, 0);
-  }
+// O rows first_row .. first_row + pad_rows - 1 of head blockIdx.y (TL in
+// 16-byte vectors): thread (x, y) zeroes vector x of one row.
+__global__ void zero_rows_kernel(uint4* __restrict__ O, TensorLayout TL, int first_row, int pad_rows) {
+  const int r = blockIdx.x * blockDim.y + threadIdx.y;
+  if (r >= pad_rows) return;
+  O[TL.head(blockIdx.y) + (long long)(first_row + r) * TL.sn + threadIdx.x] = make_uint4(0, 0, 0, 0);
 }
 
 }  // namespace
@@ -135,13 +133,14 @@ cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, cons
   __nv_bfloat16* vhl = reinterpret_cast<__nv_bfloat16*>(ws + L.vbar_hl);
   float* logcnt = reinterpret_cast<float*>(ws + L.logcnt);
   const dim3 g(Cpad, BH);
+  const TensorLayout TL = tensor_layout(s);
   if (s->dtype == CA_BF16) {
     using T = __nv_bfloat16;
     if (s->d == 64)
-      centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+      centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, TL, c, C, Cpad, cl->perm_k,
                                                      cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
     else
-      centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+      centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, TL, c, C, Cpad, cl->perm_k,
                                                       cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
     const int slots_q = L.C * s->c, slots_k = C * c;
     const int slots = slots_q > slots_k ? slots_q : slots_k;
@@ -151,18 +150,18 @@ cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, cons
     T* Kp = reinterpret_cast<T*>(ws + L.kp);
     T* Vp = reinterpret_cast<T*>(ws + L.vp);
     if (s->d == 64)
-      permute_rows_kernel<64><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc, slots_q,
+      permute_rows_kernel<64><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, TL, slots_q,
                                                   slots_k, cl->perm_q, cl->perm_k, Qp, Kp, Vp);
     else
-      permute_rows_kernel<128><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, s->N_alloc,
+      permute_rows_kernel<128><<<gp, 256, 0, st>>>((const T*)Q, (const T*)K, (const T*)V, TL,
                                                    slots_q, slots_k, cl->perm_q, cl->perm_k, Qp, Kp, Vp);
   } else {
     using T = float;
     if (s->d == 64)
-      centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+      centroid_prep_kernel<T, 64><<<g, 256, 0, st>>>((const T*)V, TL, c, C, Cpad, cl->perm_k,
                                                      cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
     else
-      centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, s->N_alloc, c, C, Cpad, cl->perm_k,
+      centroid_prep_kernel<T, 128><<<g, 256, 0, st>>>((const T*)V, TL, c, C, Cpad, cl->perm_k,
                                                       cl->count_k, cl->kbar, kbar32, vbar32, khl, vhl, logcnt);
   }
   return cudaGetLastError();
@@ -170,14 +169,17 @@ cudaError_t launch_attend_prep(const void* Q, const void* K, const void* V, cons
 
 cudaError_t launch_zero_pad_rows(void* O, const ca_shape* s, cudaStream_t st) {
   if (s->N_alloc <= s->n_valid) return cudaSuccess;
-  const size_t esz = (s->dtype == CA_BF16) ? 2 : 4;
-  const size_t row_vecs = (size_t)s->d * esz / 16;
-  const size_t BH = (size_t)s->B * s->H;
-  const size_t pad = (size_t)(s->N_alloc - s->n_valid);
-  const size_t total = pad * row_vecs * BH;
-  const unsigned blocks = (unsigned)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-  zero_rows_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<uint4*>(O), row_vecs, (size_t)s->N_alloc,
-                                           (size_t)s->n_valid, pad, BH);
+  const int esz = (s->dtype == CA_BF16) ? 2 : 4;
+  const int row_vecs = s->d * esz / 16;   // 8, 16 or 32
+  const int BH = s->B * s->H;
+  const int pad = s->N_alloc - s->n_valid;
+  // the layout in 16-byte vectors (every stride is a whole number of rows of d elements)
+  TensorLayout TV = tensor_layout(s);
+  const long long vec = 16 / esz;
+  TV.sb /= vec; TV.sh /= vec; TV.sn /= vec;
+  const dim3 block(row_vecs, 256 / row_vecs);
+  const dim3 grid((pad + block.y - 1) / block.y, BH);
+  zero_rows_kernel<<<grid, block, 0, st>>>(reinterpret_cast<uint4*>(O), TV, s->n_valid, pad);
   return cudaGetLastError();
 }
 

@@ -71,7 +71,7 @@ __device__ __forceinline__ void simt_tile(SimtState<D>& st, const float* Ks, con
 // mode 0: clustered (kept blocks + optional compensation); mode 1: dense.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
-    const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, int N_alloc, int n_valid,
+    const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, TensorLayout TL, int n_valid,
     int c, int C, int ck, int Ck, int k, const int32_t* __restrict__ perm_q, const int32_t* __restrict__ perm_k,
     const int32_t* __restrict__ kept_idx, const uint32_t* __restrict__ kept_bits,
     const int32_t* __restrict__ kept_count, const float* __restrict__ kbar32, const float* __restrict__ vbar32, const float* __restrict__ logcnt,
@@ -84,9 +84,9 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
   __shared__ int krow[kTile];
   const int bh = blockIdx.y;
   const int r = threadIdx.x / TPR, p = threadIdx.x % TPR;
-  const T* Qh = Q + (size_t)bh * N_alloc * D;
-  const T* Kh = K + (size_t)bh * N_alloc * D;
-  const T* Vh = V + (size_t)bh * N_alloc * D;
+  const T* Qh = Q + TL.head(bh);
+  const T* Kh = K + TL.head(bh);
+  const T* Vh = V + TL.head(bh);
   int a = 0, row = -1;
   if (mode == 0) {
     const int per = c / kRows;
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
   st.m = -INFINITY; st.l = 0.f;
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    st.q[e] = row >= 0 ? to_f(Qh[(size_t)row * D + e * TPR + p]) : 0.f;
+    st.q[e] = row >= 0 ? to_f(Qh[(size_t)row * TL.sn + e * TPR + p]) : 0.f;
     st.o[e] = 0.f;
   }
   auto load_rows = [&](int count_keys) {
@@ -109,8 +109,8 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
     for (int e = threadIdx.x; e < kTile * D; e += NT) {
       const int j = e / D, col = e % D;
       const int kr = krow[j];
-      Ks[e] = kr >= 0 ? to_f(Kh[(size_t)kr * D + col]) : 0.f;
-      Vs[e] = kr >= 0 ? to_f(Vh[(size_t)kr * D + col]) : 0.f;
+      Ks[e] = kr >= 0 ? to_f(Kh[(size_t)kr * TL.sn + col]) : 0.f;
+      Vs[e] = kr >= 0 ? to_f(Vh[(size_t)kr * TL.sn + col]) : 0.f;
     }
     (void)count_keys;
   };
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kRows * (D / 16)) simt_attend_kernel(
   }
   if (row >= 0) {
     const float inv = st.l > 0.f ? 1.f / st.l : 0.f;
-    T* Oh = O + (size_t)bh * N_alloc * D + (size_t)row * D;
+    T* Oh = O + TL.head(bh) + (size_t)row * TL.sn;
 #pragma unroll
     for (int e = 0; e < 16; ++e) Oh[e * TPR + p] = from_f<T>(st.o[e] * inv);
   }
@@ -189,7 +189,7 @@ cudaError_t run_simt(const void* Q, const void* K, const void* V, const ca_shape
   const float* vbar32 = L ? reinterpret_cast<const float*>(ws + L->vbar32) : nullptr;
   const float* logcnt = L ? reinterpret_cast<const float*>(ws + L->logcnt) : nullptr;
   simt_attend_kernel<T, D><<<grid, kRows * (D / 16), 0, st>>>(
-      (const T*)Q, (const T*)K, (const T*)V, s->N_alloc, s->n_valid, c, C, ck, Ck, rt ? rt->k : 0,
+      (const T*)Q, (const T*)K, (const T*)V, tensor_layout(s), s->n_valid, c, C, ck, Ck, rt ? rt->k : 0,
       cl ? cl->perm_q : nullptr, cl ? cl->perm_k : nullptr, rt ? rt->kept_idx : nullptr,
       rt ? rt->kept_bits : nullptr, rt ? rt->kept_count : nullptr, kbar32, vbar32, logcnt, L ? L->Cpad : 0, compensate, mode, scale,
       (T*)O);

@@ -108,11 +108,12 @@ __device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, uint64
       "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-__device__ __forceinline__ void tma_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+__device__ __forceinline__ void tma_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                       int w) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
       "[%2];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
       : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -321,7 +322,9 @@ struct TcParams {
   const int32_t* kept_count;  // [BH][C] kept per query cluster, or null (k each)
   const uint32_t* kept_bits;  // [BH][C][W]
   const float* logcnt;        // [BH][Cpad] natural log of counts (-inf past C)
-  __nv_bfloat16* O;           // [BH][N_alloc][D]
+  __nv_bfloat16* O;           // the caller's layout (TL)
+  TensorLayout TL;            // of Q, K, V and O
+  int dense_tok_inner;        // dense maps: 1 when the token dimension precedes the head dimension
   uint64_t wait_limit;
 };
 
@@ -602,6 +605,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       kcnt_s[Cfg::kMaxKept + i] = p.count_k[(size_t)T1.bh * p.Ck + b];
     }
   }
+  // dense mode: tile of 128 tokens of head bh from a 4-D map over (d, tokens,
+  // heads, batch) or (d, heads, tokens, batch), whichever orders the strides
+  // (head and batch of each tile computed once: no division per load)
+  auto tma_dense = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int x, int row, int hd, int bt) {
+    if (p.dense_tok_inner) tma_4d(dst, map, bar, x, row, hd, bt);
+    else tma_4d(dst, map, bar, x, hd, row, bt);
+  };
   auto kept_at = [&](int t, int i) -> int {
     const bool sm = t ? kept_sm1 : kept_sm0;
     return sm ? kept_s[t * Cfg::kMaxKept + i] : (t ? kept_g1 : kept_g0)[i];
@@ -652,13 +662,15 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // ------------------------------------------------------------- producer
     if (lane == 0) {
       bool ok = true;
+      // dense mode: both tiles are of head T0.bh (head and batch computed once)
+      const int dh = T0.bh % p.TL.H, db = T0.bh / p.TL.H;
       for (int t = 0; t < 2; ++t) {
         const Tile& Tt = t ? T1 : T0;
         if (Tt.J == 0) continue;
         mbar_expect_tx(&q_full[t], Cfg::kTileBytes);
         for (int sb = 0; sb < Cfg::kSub; ++sb) {
           unsigned char* dst = sQ + t * Cfg::kTileBytes + sb * Cfg::kSubBytes;
-          if (p.dense) tma_3d(dst, &tm_q, &q_full[t], sb * 64, Tt.qrow, Tt.bh);
+          if (p.dense) tma_dense(dst, &tm_q, &q_full[t], sb * 64, Tt.qrow, dh, db);
           else tma_2d(dst, &tm_q, &q_full[t], sb * 64, Tt.qrow);
         }
       }
@@ -673,7 +685,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int sb = 0; sb < Cfg::kSub; ++sb) {
           unsigned char* d = dst + sb * Cfg::kSubBytes;
           if (p.dense) {
-            tma_3d(d, mk, bar, sb * 64, j * 128, Tt.bh);
+            tma_dense(d, mk, bar, sb * 64, j * 128, dh, db);
           } else if (j < Tt.J_kept) {
             if (p.ck >= 128) {
               // c_k is 128 or 256: one or two key blocks per kept cluster (a
@@ -959,7 +971,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (p.dense) orow = Tt.qrow + row < p.n_valid ? Tt.qrow + row : -1;
         else if (p.pair) orow = row < (Tt.two ? 128 : 64) ? p.perm_q[(size_t)Tt.qrow + row] : -1;
         else orow = (Tt.sub * 128 + row < p.c && row < p.rows_per_tile) ? p.perm_q[(size_t)Tt.qrow + row] : -1;
-        __nv_bfloat16* dst = p.O + ((size_t)Tt.bh * p.N_alloc + (orow < 0 ? 0 : orow)) * D;
+        __nv_bfloat16* dst = p.O + p.TL.head(Tt.bh) + (size_t)(orow < 0 ? 0 : orow) * p.TL.sn;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -1034,15 +1046,24 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, int D, int box
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-// 3-D bf16 map over [BH][N_alloc][D] exposing only rows < n_valid of each head.
-bool make_map_3d(CUtensorMap* m, const void* base, int BH, int N_alloc, int n_valid, int D, int box_rows) {
+// 4-D bf16 map over the caller's tensor exposing only tokens < n_valid of
+// each head: dimensions (d, tokens, heads, batch) when consecutive tokens of
+// a head are closer than consecutive heads (CA_LAYOUT_BHND), else (d, heads,
+// tokens, batch) (CA_LAYOUT_BNHD), so the strides increase; a box is 64
+// columns of 128 tokens of one head either way.
+bool make_map_dense(CUtensorMap* m, const void* base, const ca_shape* s, bool* tok_inner) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n_valid, (cuuint64_t)BH};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N_alloc * D * 2};
-  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
-  const cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  const TensorLayout L = tensor_layout(s);
+  const bool ti = L.sn <= L.sh;
+  *tok_inner = ti;
+  const cuuint64_t D = (cuuint64_t)s->d, n = (cuuint64_t)s->n_valid, H = (cuuint64_t)s->H, B = (cuuint64_t)s->B;
+  const cuuint64_t dims[4] = {D, ti ? n : H, ti ? H : n, B};
+  const cuuint64_t strides[3] = {(cuuint64_t)(ti ? L.sn : L.sh) * 2, (cuuint64_t)(ti ? L.sh : L.sn) * 2,
+                                 (cuuint64_t)L.sb * 2};
+  const cuuint32_t box[4] = {64, ti ? 128u : 1u, ti ? 1u : 128u, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1083,6 +1104,7 @@ cudaError_t launch_attend_tc(const ca_shape* s, const ca_clusters* cl, const ca_
   TcParams p{};
   p.C = C; p.c = c; p.Ck = Ck; p.ck = ck;
   p.k = rt->k; p.Cpad = L.Cpad; p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
+  p.TL = tensor_layout(s);
   p.tiles_per_cluster = c >= 128 ? c / 128 : 1;
   p.rows_per_tile = c >= 128 ? 128 : c;
   // 64-query clusters go two to a 128-row tile while their union of kept key
@@ -1136,12 +1158,14 @@ cudaError_t launch_dense_tc(const void* Q, const void* K, const void* V, const c
                             cudaStream_t st) {
   const int BH = s->B * s->H, D = s->d;
   CUtensorMap maps[5];
-  bool ok = make_map_3d(&maps[0], Q, BH, s->N_alloc, s->n_valid, D, 128) &&
-            make_map_3d(&maps[1], K, BH, s->N_alloc, s->n_valid, D, 128) &&
-            make_map_3d(&maps[2], V, BH, s->N_alloc, s->n_valid, D, 128);
+  bool ti = true;
+  bool ok = make_map_dense(&maps[0], Q, s, &ti) && make_map_dense(&maps[1], K, s, &ti) &&
+            make_map_dense(&maps[2], V, s, &ti);
   if (!ok) return cudaErrorInvalidValue;
   maps[3] = maps[1]; maps[4] = maps[2];
   TcParams p{};
+  p.TL = tensor_layout(s);
+  p.dense_tok_inner = ti ? 1 : 0;
   p.n_valid = s->n_valid; p.N_alloc = s->N_alloc;
   p.tiles_per_cluster = 1; p.rows_per_tile = 128;
   p.compensate = 0; p.J_cent = 0; p.dense = 1;

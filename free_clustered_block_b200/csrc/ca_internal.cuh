@@ -107,6 +107,34 @@ __device__ __forceinline__ uint64_t ordered_key(double v) {
 
 // Key cluster size and the cluster counts of a (validated) shape.
 inline int key_c(const ca_shape* s) { return s->c_k ? s->c_k : s->c; }
+
+// Where the caller's Q, K, V and O keep element j of token r of head bh = b H + h:
+// b sb + h sh + r sn + j (elements).
+struct TensorLayout {
+  long long sb, sh, sn;
+  int H;
+  __host__ __device__ __forceinline__ long long head(int bh) const {
+    // head-major: every head one stride apart (no integer division, which
+    // would use the MUFU unit that the attention's exponentials keep busy)
+    if (sb == (long long)H * sh) return (long long)bh * sh;
+    return (long long)(bh / H) * sb + (long long)(bh % H) * sh;
+  }
+};
+inline TensorLayout tensor_layout(const ca_shape* s) {
+  TensorLayout L;
+  const long long d = s->d, N = s->N_alloc;
+  L.H = s->H;
+  if (s->layout == CA_LAYOUT_BNHD) {
+    const long long Ht = s->H_total > 0 ? s->H_total : s->H;
+    L.sn = Ht * d; L.sh = d; L.sb = N * Ht * d;
+  } else {
+    L.sn = d; L.sh = N * d; L.sb = (long long)s->H * N * d;
+  }
+  return L;
+}
+inline bool layout_contiguous(const ca_shape* s) {
+  return s->layout == CA_LAYOUT_BHND || s->H_total == 0 || s->H_total == s->H;
+}
 inline int num_q_clusters(const ca_shape* s) { return (s->n_valid + s->c - 1) / s->c; }
 inline int num_k_clusters(const ca_shape* s) { return (s->n_valid + key_c(s) - 1) / key_c(s); }
 
@@ -134,7 +162,7 @@ bool cluster_ws_layout(const ca_shape* s, const TreePlan& plan, const TreePlan& 
 cudaError_t launch_diag_basis(int D, int TH, int BH, int nch, int n, const double* part, const double* M,
                               double* C, double* scratch, double* W, cudaStream_t st);
 template <typename T, int D>
-cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const TreeNode* nodes, int lvl_begin,
+cudaError_t launch_diag_dir(const T* Q, const T* K, TensorLayout TL, int n, const TreeNode* nodes, int lvl_begin,
                             int nodes_in_level, int TH, const double* W, const double* inv_s, const int* idx,
                             int NI, double* wvec, uint64_t seed, int head_base, int tsel, cudaStream_t st);
 

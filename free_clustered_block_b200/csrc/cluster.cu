@@ -114,20 +114,37 @@ __global__ void __launch_bounds__(1024) plan_kernel(int n, int c, TreeNode* node
 // With kW the rows are scaled by w[bh n + row] first (the queries' 1 / |R_k q|
 // for the covariance of their representations).
 template <typename T, int D, bool kW = false>
-__global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, int N_alloc, int n,
+__global__ void __launch_bounds__(256) colsum_kernel(const T* __restrict__ K, TensorLayout TL, int n,
                                                      double* __restrict__ part,
                                                      const double* __restrict__ w = nullptr) {
   constexpr int RG = 256 / D;
   const int bh = blockIdx.y, ch = blockIdx.x, nch = gridDim.x;
   const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
   const int col = threadIdx.x % D, rg = threadIdx.x / D;
-  const T* base = K + (size_t)bh * N_alloc * D;
+  const T* base = K + TL.head(bh);
   double acc = 0.0;
-  if constexpr (kW) {
-    for (int r = r0 + rg; r < r1; r += RG)
-      acc = fma((double)to_f(base[(size_t)r * D + col]), w[(size_t)bh * n + r], acc);
-  } else {
-    for (int r = r0 + rg; r < r1; r += RG) acc += (double)to_f(base[(size_t)r * D + col]);
+  // rows r0 + rg, r0 + rg + RG, ... summed in that order, four loads in flight
+  const size_t step = (size_t)RG * TL.sn;
+  const T* src = base + (size_t)(r0 + rg) * TL.sn + col;
+  int r = r0 + rg;
+  for (; r + 3 * RG < r1; r += 4 * RG, src += 4 * step) {
+    const T x0 = src[0], x1 = src[step], x2 = src[2 * step], x3 = src[3 * step];
+    if constexpr (kW) {
+      const double* wr = w + (size_t)bh * n + r;
+      acc = fma((double)to_f(x0), wr[0], acc);
+      acc = fma((double)to_f(x1), wr[RG], acc);
+      acc = fma((double)to_f(x2), wr[2 * RG], acc);
+      acc = fma((double)to_f(x3), wr[3 * RG], acc);
+    } else {
+      acc += (double)to_f(x0);
+      acc += (double)to_f(x1);
+      acc += (double)to_f(x2);
+      acc += (double)to_f(x3);
+    }
+  }
+  for (; r < r1; r += RG, src += step) {
+    if constexpr (kW) acc = fma((double)to_f(src[0]), w[(size_t)bh * n + r], acc);
+    else acc += (double)to_f(src[0]);
   }
   __shared__ double red[256];
   red[threadIdx.x] = acc;
@@ -186,7 +203,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // result goes to the queries' slot (z = 0) of part. This is the covariance of
 // the query representations before the transform (diagonalized splitting).
 template <typename T, int D, bool kW = false>
-__global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* __restrict__ K, int N_alloc,
+__global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* __restrict__ K, TensorLayout TL,
                                              int n, int nch, const double* __restrict__ colpart,
                                              double* __restrict__ part, const double* __restrict__ w = nullptr) {
   using Cfg = SyrkCfg<D>;
@@ -197,13 +214,13 @@ __global__ void __maxnreg__(128) syrk_kernel(const T* __restrict__ Q, const T* _
   T* raw = reinterpret_cast<T*>(smem_raw + Cfg::kXsBytes);   // ROWS x D as loaded
   __shared__ double mean[D];
   const int bh = blockIdx.y, z = blockIdx.z, ch = blockIdx.x;
-  const T* X = (z == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (z == 0 ? Q : K) + TL.head(bh);
   const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
 
   auto issue = [&](int rt) {
     const int rows = min(ROWS, r1 - rt);
     for (int e = threadIdx.x; e < rows * (D / VEC); e += NTH)
-      cp_async16(raw + e * VEC, X + (size_t)rt * D + (size_t)e * VEC);
+      cp_async16(raw + e * VEC, X + (size_t)(rt + e / (D / VEC)) * TL.sn + (size_t)(e % (D / VEC)) * VEC);
     cp_async_commit();
   };
   if (r0 < r1) issue(r0);
@@ -325,7 +342,7 @@ __device__ __forceinline__ void dmma_884(double (&c)[2], double a, double b) {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(SyrkMmaCfg<D>::kThreads, 1) syrk_mma_kernel(
-    const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, int nch,
+    const T* __restrict__ Q, const T* __restrict__ K, TensorLayout TL, int n, int nch,
     const double* __restrict__ colpart, double* __restrict__ part) {
   using Cfg = SyrkMmaCfg<D>;
   constexpr int RG = Cfg::RG, NTH = Cfg::kThreads, ROWS = Cfg::kRows, P = Cfg::kP;
@@ -335,7 +352,7 @@ __global__ void __launch_bounds__(SyrkMmaCfg<D>::kThreads, 1) syrk_mma_kernel(
   T* raw = reinterpret_cast<T*>(smem_raw + Cfg::kXsBytes);     // ROWS x D as loaded
   __shared__ double mean[D];
   const int bh = blockIdx.y, z = blockIdx.z, ch = blockIdx.x;
-  const T* X = (z == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (z == 0 ? Q : K) + TL.head(bh);
   const int r0 = ch * kMetricChunk, r1 = min(n, r0 + kMetricChunk);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, tg = lane & 3;                      // fragment row / column in group
@@ -347,7 +364,7 @@ __global__ void __launch_bounds__(SyrkMmaCfg<D>::kThreads, 1) syrk_mma_kernel(
   auto issue = [&](int rt) {
     const int rows = min(ROWS, r1 - rt);
     for (int e = threadIdx.x; e < rows * (D / VEC); e += NTH)
-      cp_async16(raw + e * VEC, X + (size_t)rt * D + (size_t)e * VEC);
+      cp_async16(raw + e * VEC, X + (size_t)(rt + e / (D / VEC)) * TL.sn + (size_t)(e % (D / VEC)) * VEC);
     cp_async_commit();
   };
   if (r0 < r1) issue(r0);
@@ -460,7 +477,7 @@ __global__ void __launch_bounds__(256) metric_reduce_kernel(const double* __rest
 // tx+16j, then the row dot with X.
 // ---------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int N_alloc, int n,
+__global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, TensorLayout TL, int n,
                                                     const double* __restrict__ M, int transform,
                                                     double* __restrict__ inv_s) {
   constexpr int R = 128, B = D / 16, RS = D + 1;
@@ -475,10 +492,10 @@ __global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int
     return;
   }
   for (int e = threadIdx.x; e < D * D; e += 256) Ms[e] = M[(size_t)th * D * D + e];
-  const T* X = Q + (size_t)bh * N_alloc * D;
+  const T* X = Q + TL.head(bh);
   for (int e = threadIdx.x; e < R * D; e += 256) {
     const int rr = e / D, cc = e % D, r = r0 + rr;
-    xs[rr * RS + cc] = (r < n) ? to_f(X[(size_t)r * D + cc]) : 0.f;
+    xs[rr * RS + cc] = (r < n) ? to_f(X[(size_t)r * TL.sn + cc]) : 0.f;
   }
   __syncthreads();
   const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
@@ -518,7 +535,7 @@ __global__ void __launch_bounds__(256) qnorm_kernel(const T* __restrict__ Q, int
 // upper triangle of the symmetric M (2080 fma per row instead of 4160); every
 // lane reads the same M entries, so the shared-memory loads are broadcasts.
 template <typename T>
-__global__ void __launch_bounds__(128, 3) qnorm64_kernel(const T* __restrict__ Q, int N_alloc, int n,
+__global__ void __launch_bounds__(128, 3) qnorm64_kernel(const T* __restrict__ Q, TensorLayout TL, int n,
                                                       const double* __restrict__ M,
                                                       double* __restrict__ inv_s) {
   constexpr int D = 64;
@@ -530,7 +547,7 @@ __global__ void __launch_bounds__(128, 3) qnorm64_kernel(const T* __restrict__ Q
   double x[D];
   {
     constexpr int VEC = 16 / sizeof(T);
-    const uint4* src = reinterpret_cast<const uint4*>(Q + ((size_t)bh * N_alloc + (r < n ? r : 0)) * D);
+    const uint4* src = reinterpret_cast<const uint4*>(Q + TL.head(bh) + (size_t)(r < n ? r : 0) * TL.sn);
     uint4 raw[D / VEC];
 #pragma unroll
     for (int v = 0; v < D / VEC; ++v) raw[v] = __ldg(src + v);
@@ -598,7 +615,7 @@ struct DirCfg {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(512) dir_kernel(
-    const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
+    const T* __restrict__ Q, const T* __restrict__ K, TensorLayout TL, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
     int head_base, int power_iters, int sample_factor, int tsel) {
@@ -627,7 +644,7 @@ __global__ void __launch_bounds__(512) dir_kernel(
   const int m = min(m_cap, nd.size);
   const uint64_t key = node_stream(seed, (uint64_t)(head_base + bh), (uint64_t)tensor, nd.heap);
   const uint64_t r = (nd.size > m) ? (splitmix64(key ^ kSampleTag) % (uint64_t)nd.size) : 0ull;
-  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (tensor == 0 ? Q : K) + TL.head(bh);
   const int* idx_th = idx ? idx + (size_t)th * n : nullptr;
   for (int j = lane; j < m; j += 32) {
     const int pos = (nd.size > m) ? (int)(((uint64_t)j * (uint64_t)nd.size + r) / (uint64_t)m) : j;
@@ -650,7 +667,7 @@ __global__ void __launch_bounds__(512) dir_kernel(
       for (int u = 0; u < 4; ++u) {
         const int j = j0 + u * RPI + sub;
         v4[u] = make_uint4(0, 0, 0, 0);
-        if (j < m) v4[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * D + part * (16 / sizeof(T)));
+        if (j < m) v4[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * TL.sn + part * (16 / sizeof(T)));
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -807,7 +824,7 @@ struct DirCCfg {
 
 template <typename T, int D_>
 __global__ void __launch_bounds__(2 * D_, D_ == 64 ? 3 : 1) dirc_kernel(
-    const T* __restrict__ Q, const T* __restrict__ K, int N_alloc, int n, const TreeNode* __restrict__ nodes,
+    const T* __restrict__ Q, const T* __restrict__ K, TensorLayout TL, int n, const TreeNode* __restrict__ nodes,
     int lvl_begin, int nodes_in_level, int npc, const double* __restrict__ M, const double* __restrict__ inv_s,
     const int* __restrict__ idx, int NI, double* __restrict__ zvec, double* __restrict__ wvec, uint64_t seed,
     int head_base, int power_iters, int tsel) {
@@ -827,7 +844,7 @@ __global__ void __launch_bounds__(2 * D_, D_ == 64 ? 3 : 1) dirc_kernel(
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int ca = t & (D - 1), ch = t / D;       // column / half split
   const int rj = t >> 1, rh = t & 1;            // row / half split
-  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (tensor == 0 ? Q : K) + TL.head(bh);
   {
     const double2* src = reinterpret_cast<const double2*>(M + (size_t)th * D * D);
     double2* dst = reinterpret_cast<double2*>(Ms);
@@ -897,7 +914,7 @@ __global__ void __launch_bounds__(2 * D_, D_ == 64 ? 3 : 1) dirc_kernel(
           const int j = e / CPR, part = e % CPR;
           v4[u] = make_uint4(0, 0, 0, 0);
           if (e < D * CPR && j < m)
-            v4[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * D + part * VEC);
+            v4[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * TL.sn + part * VEC);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -1035,7 +1052,7 @@ constexpr int kProjU = 4;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                      int N_alloc, int n, const TreeNode* __restrict__ nodes,
+                                                      TensorLayout TL, int n, const TreeNode* __restrict__ nodes,
                                                       int lb, int le, const double* __restrict__ inv_s,
                                                       const int* __restrict__ idx, int NI,
                                                       const double* __restrict__ wvec,
@@ -1050,7 +1067,7 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
   __shared__ int rows_s[kProjSpan];      // source row of each position
   __shared__ int s_cnt;
   const int th = tensor_head(blockIdx.y, tsel), bh = th >> 1, tensor = th & 1;
-  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (tensor == 0 ? Q : K) + TL.head(bh);
   const int base = blockIdx.x * kProjSpan;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp == 0) {
@@ -1132,7 +1149,7 @@ __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, c
       raw[u] = make_uint4(0, 0, 0, 0);
       sc[u] = 1.0;
       if (slot[u] != 255) {
-        raw[u] = *reinterpret_cast<const uint4*>(X + (size_t)row[u] * D + gl * EPL);
+        raw[u] = *reinterpret_cast<const uint4*>(X + (size_t)row[u] * TL.sn + gl * EPL);
         if (tensor == 0) sc[u] = inv_s[(size_t)bh * n + row[u]];
       }
     }
@@ -1438,7 +1455,7 @@ __global__ void __launch_bounds__(kPartThreads) part_scatter_kernel(
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(256) centroid_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                       int N_alloc, int n, int c, int C, int levels,
+                                                       TensorLayout TL, int n, int c, int C, int levels,
                                                        int32_t* __restrict__ perm_q, int32_t* __restrict__ perm_k,
                                                        int32_t* __restrict__ count_q, int32_t* __restrict__ count_k,
                                                        double* __restrict__ qbar, double* __restrict__ kbar,
@@ -1453,12 +1470,12 @@ __global__ void __launch_bounds__(256) centroid_kernel(const T* __restrict__ Q, 
   }
   for (int j = cnt + threadIdx.x; j < c; j += 256) perm[j] = -1;
   if (threadIdx.x == 0) ((tensor == 0) ? count_q : count_k)[(size_t)bh * C + a] = cnt;
-  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (tensor == 0 ? Q : K) + TL.head(bh);
   const int col = threadIdx.x % D, rg = threadIdx.x / D;
   double s = 0.0;
   for (int j = rg; j < cnt; j += RG) {
     const int row = (levels == 0) ? j : perm[j];
-    s += (double)to_f(X[(size_t)row * D + col]);
+    s += (double)to_f(X[(size_t)row * TL.sn + col]);
   }
   __shared__ double red[256];
   red[threadIdx.x] = s;
@@ -1474,7 +1491,8 @@ template <typename T, int D>
 cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_cluster_params* p,
                         const ca_clusters* out, const TreePlan& plan, const TreePlan& plan_k, const ClusterWs& L,
                         char* ws, cudaStream_t st) {
-  const int n = s->n_valid, N_alloc = s->N_alloc;
+  const int n = s->n_valid;
+  const TensorLayout TL = tensor_layout(s);
   const int BH = L.BH, TH = L.TH, NI = L.NI;
   const int nch = L.nch;
   // Queries and keys share one tree when their cluster sizes are equal; with
@@ -1507,29 +1525,29 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
     plan_kernel<<<1, 1024, 0, st>>>(n, s->c, nodes_t[0], level_begin_t[0]);
     if (!same_tree) plan_kernel<<<1, 1024, 0, st>>>(n, key_c(s), nodes_t[1], level_begin_t[1]);
     if (!random_clusters) {
-      colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, N_alloc, n, colpart);
+      colsum_kernel<T, D><<<dim3(nch, BH), 256, 0, st>>>(K, TL, n, colpart);
       const size_t syrk_smem = SyrkCfg<D>::template smem<T>();
       const size_t mma_smem = SyrkMmaCfg<D>::template smem<T>();
       cudaFuncSetAttribute(syrk_mma_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mma_smem);
-      syrk_mma_kernel<T, D><<<dim3(nch, BH, 2), SyrkMmaCfg<D>::kThreads, mma_smem, st>>>(Q, K, N_alloc, n, nch,
+      syrk_mma_kernel<T, D><<<dim3(nch, BH, 2), SyrkMmaCfg<D>::kThreads, mma_smem, st>>>(Q, K, TL, n, nch,
                                                                                         colpart, metpart);
       metric_reduce_kernel<D><<<dim3(D * D / 256, TH), 256, 0, st>>>(metpart, nch, n, transform, M);
       if (D == 64 && normalize) {
-        qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, N_alloc, n, M, inv_s);
+        qnorm64_kernel<T><<<dim3((n + 127) / 128, BH), 128, 0, st>>>(Q, TL, n, M, inv_s);
       } else {
         const size_t qn_smem = (size_t)D * D * 8 + (size_t)128 * (D + 1) * 4;
         cudaFuncSetAttribute(qnorm_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qn_smem);
-        qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, N_alloc, n, M, normalize, inv_s);
+        qnorm_kernel<T, D><<<dim3((n + 127) / 128, BH), 256, qn_smem, st>>>(Q, TL, n, M, normalize, inv_s);
       }
       if (diagonal) {
         // covariance of the scaled query rows (weights 1 / |R_k q| in the
         // top-k form, 1 otherwise): weighted column sums into the key sums'
         // buffer and the centred weighted Gram into the queries' slot of the
         // partials, both free once M and the query scales exist
-        colsum_kernel<T, D, true><<<dim3(nch, BH), 256, 0, st>>>(Q, N_alloc, n, colpart, inv_s);
+        colsum_kernel<T, D, true><<<dim3(nch, BH), 256, 0, st>>>(Q, TL, n, colpart, inv_s);
         cudaFuncSetAttribute(syrk_kernel<T, D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)syrk_smem);
         syrk_kernel<T, D, true><<<dim3(nch, BH, 1), SyrkCfg<D>::kThreads, syrk_smem, st>>>(
-            Q, K, N_alloc, n, nch, colpart, metpart, inv_s);
+            Q, K, TL, n, nch, colpart, metpart, inv_s);
         const cudaError_t e = launch_diag_basis(D, TH, BH, nch, n, metpart, M,
                                                 reinterpret_cast<double*>(ws + L.cov),
                                                 reinterpret_cast<double*>(ws + L.basis_scratch), basis, st);
@@ -1557,7 +1575,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
       if (random_clusters) {
         hash_keys_kernel<<<dim3((n + 255) / 256, rows), 256, 0, st>>>(n, idx_in, p->seed, p->head_base, keys, tsel);
       } else if (diagonal) {
-        const cudaError_t e = launch_diag_dir<T, D>(Q, K, N_alloc, n, nodes, lb, nl, rows, basis, inv_s, idx_in,
+        const cudaError_t e = launch_diag_dir<T, D>(Q, K, TL, n, nodes, lb, nl, rows, basis, inv_s, idx_in,
                                                     NI, wvec, p->seed, p->head_base, tsel, st);
         if (e != cudaSuccess) return e;
       } else if (sample_factor == 1 && (D == 128 || (long long)nl * rows <= kDirCMaxNodes64)) {
@@ -1565,16 +1583,16 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
         // four blocks per SM over the whole level)
         const int npc = (int)(((long long)nl * rows + 4 * 148 - 1) / (4 * 148));
         dirc_kernel<T, D><<<dim3((nl + npc - 1) / npc, rows), DirCCfg<T, D>::kThreads, DirCCfg<T, D>::kSmem, st>>>(
-            Q, K, N_alloc, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base,
+            Q, K, TL, n, nodes, lb, nl, npc, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base,
             power_iters, tsel);
       } else {
         dir_kernel<T, D><<<dim3((nl + dir_warps - 1) / dir_warps, rows), dir_warps * 32, dir_smem, st>>>(
-            Q, K, N_alloc, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base, power_iters,
+            Q, K, TL, n, nodes, lb, nl, M, inv_s, idx_in, NI, zvec, wvec, p->seed, p->head_base, power_iters,
             sample_factor, tsel);
       }
       if (!random_clusters)
         project_kernel<T, D><<<dim3((n + kProjSpan - 1) / kProjSpan, rows), 256, 0, st>>>(
-            Q, K, N_alloc, n, nodes, lb, le, inv_s, idx_in, NI, wvec, keys, tsel);
+            Q, K, TL, n, nodes, lb, le, inv_s, idx_in, NI, wvec, keys, tsel);
       if (pl.level_max_size[l] <= kSelCap)   // candidates buffer sized to the level's largest node
         select_kernel<256><<<dim3(nl, rows), 256, (size_t)pl.level_max_size[l] * 8, st>>>(nodes, lb, nl, n, keys,
                                                                                         sel, tsel);
@@ -1586,7 +1604,7 @@ cudaError_t run_cluster(const T* Q, const T* K, const ca_shape* s, const ca_clus
                                                                       ccnt, idx_in, idx_out, out->perm_q,
                                                                       out->perm_k, C * c, tsel);
     }
-    centroid_kernel<T, D><<<dim3(C, rows), 256, 0, st>>>(Q, K, N_alloc, n, c, C, pl.levels, out->perm_q,
+    centroid_kernel<T, D><<<dim3(C, rows), 256, 0, st>>>(Q, K, TL, n, c, C, pl.levels, out->perm_q,
                                                          out->perm_k, out->count_q, out->count_k, out->qbar,
                                                          out->kbar, tsel);
     return cudaGetLastError();

@@ -327,7 +327,7 @@ struct DiagDirCfg {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) diag_dir_kernel(const T* __restrict__ Q, const T* __restrict__ K,
-                                                       int N_alloc, int n, const TreeNode* __restrict__ nodes,
+                                                       TensorLayout TL, int n, const TreeNode* __restrict__ nodes,
                                                        int lvl_begin, int nodes_in_level, int npc,
                                                        const double* __restrict__ W,
                                                        const double* __restrict__ inv_s,
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(256) diag_dir_kernel(const T* __restrict__ Q, 
   __shared__ int jbest_s;
   const int th = tsel < 0 ? (int)blockIdx.y : 2 * (int)blockIdx.y + tsel, bh = th >> 1, tensor = th & 1;
   const int t = threadIdx.x, ty = t / 16, tx = t % 16;
-  const T* X = (tensor == 0 ? Q : K) + (size_t)bh * N_alloc * D;
+  const T* X = (tensor == 0 ? Q : K) + TL.head(bh);
   {
     // the basis arrives transposed: a straight 16-byte copy, all loads of a thread in flight
     const double2* src = reinterpret_cast<const double2*>(W + (size_t)th * D * D);
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(256) diag_dir_kernel(const T* __restrict__ Q, 
           const int e = (u0 + u) * 256 + t, j = e / CPR, k0 = (e % CPR) * VEC;
           raw[u] = make_uint4(0u, 0u, 0u, 0u);
           if (j < m && k0 >= kc && k0 < kc + KC)
-            raw[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * D + k0);
+            raw[u] = *reinterpret_cast<const uint4*>(X + (size_t)srow[j] * TL.sn + k0);
         }
 #pragma unroll
         for (int u = 0; u < NB8; ++u) {
@@ -505,7 +505,7 @@ cudaError_t launch_diag_basis(int D, int TH, int BH, int nch, int n, const doubl
 }
 
 template <typename T, int D>
-cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const TreeNode* nodes, int lvl_begin,
+cudaError_t launch_diag_dir(const T* Q, const T* K, TensorLayout TL, int n, const TreeNode* nodes, int lvl_begin,
                             int nodes_in_level, int TH, const double* W, const double* inv_s, const int* idx,
                             int NI, double* wvec, uint64_t seed, int head_base, int tsel, cudaStream_t st) {
   using Cfg = DiagDirCfg<T, D>;
@@ -514,22 +514,22 @@ cudaError_t launch_diag_dir(const T* Q, const T* K, int N_alloc, int n, const Tr
   cudaFuncSetAttribute(diag_dir_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::kSmem);
   // TH: the grid rows (every tensor-head, or one tensor's heads when tsel >= 0)
   diag_dir_kernel<T, D><<<dim3((nodes_in_level + npc - 1) / npc, TH), Cfg::kThreads, Cfg::kSmem, st>>>(
-      Q, K, N_alloc, n, nodes, lvl_begin, nodes_in_level, npc, W, inv_s, idx, NI, wvec, seed, head_base, tsel);
+      Q, K, TL, n, nodes, lvl_begin, nodes_in_level, npc, W, inv_s, idx, NI, wvec, seed, head_base, tsel);
   return cudaGetLastError();
 }
 
-template cudaError_t launch_diag_dir<__nv_bfloat16, 64>(const __nv_bfloat16*, const __nv_bfloat16*, int, int,
+template cudaError_t launch_diag_dir<__nv_bfloat16, 64>(const __nv_bfloat16*, const __nv_bfloat16*, TensorLayout, int,
                                                          const TreeNode*, int, int, int, const double*,
                                                          const double*, const int*, int, double*, uint64_t, int, int,
                                                          cudaStream_t);
-template cudaError_t launch_diag_dir<__nv_bfloat16, 128>(const __nv_bfloat16*, const __nv_bfloat16*, int, int,
+template cudaError_t launch_diag_dir<__nv_bfloat16, 128>(const __nv_bfloat16*, const __nv_bfloat16*, TensorLayout, int,
                                                           const TreeNode*, int, int, int, const double*,
                                                           const double*, const int*, int, double*, uint64_t, int, int,
                                                           cudaStream_t);
-template cudaError_t launch_diag_dir<float, 64>(const float*, const float*, int, int, const TreeNode*, int, int,
+template cudaError_t launch_diag_dir<float, 64>(const float*, const float*, TensorLayout, int, const TreeNode*, int, int,
                                                 int, const double*, const double*, const int*, int, double*,
                                                 uint64_t, int, int, cudaStream_t);
-template cudaError_t launch_diag_dir<float, 128>(const float*, const float*, int, int, const TreeNode*, int, int,
+template cudaError_t launch_diag_dir<float, 128>(const float*, const float*, TensorLayout, int, const TreeNode*, int, int,
                                                  int, const double*, const double*, const int*, int, double*,
                                                  uint64_t, int, int, cudaStream_t);
 

@@ -8,7 +8,7 @@ from __future__ import annotations
 from dataclasses import dataclass
 from typing import Optional
 
-from . import (CA_BF16, CA_FP32, ca_attend, ca_attend_prepare, ca_attend_prepared, ca_cluster, num_key_clusters, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
+from . import (CA_BF16, CA_FP32, CA_LAYOUT_BHND, CA_LAYOUT_BNHD, ca_attend, ca_attend_prepare, ca_attend_prepared, ca_cluster, num_key_clusters, ca_dense_attend, ca_forward, ca_route, ca_route_adaptive,
                attend_workspace_bytes, cluster_workspace_bytes, clusters_struct, forward_workspace_bytes,
                make_params, make_shape, num_clusters, routes_struct)
 
@@ -50,11 +50,16 @@ class ClusterAttention:
                  dtype: str = "bf16", compensate: bool = True, power_iters: int = 8,
                  sample_factor: int = 1, transform: bool = True, seed: int = 0, device="cuda",
                  selection: str = "topk", recall: float = 0.9, min_count: int = 16,
-                 clustering: str = "split", head_base: int = 0, c_k: int = 0):
+                 clustering: str = "split", head_base: int = 0, c_k: int = 0, layout: str = "bhnd",
+                 H_total: int = 0):
         import torch
         self.torch = torch
         self.dtype_code = CA_BF16 if dtype == "bf16" else CA_FP32
-        self.shape = make_shape(B, H, N_alloc, n_valid, d, c, self.dtype_code, c_k)
+        if layout not in ("bhnd", "bnhd"):
+            raise ValueError("layout is 'bhnd' ([B, H, N, d]) or 'bnhd' ([B, N, H_total, d])")
+        self.layout = layout
+        self.shape = make_shape(B, H, N_alloc, n_valid, d, c, self.dtype_code, c_k,
+                                CA_LAYOUT_BNHD if layout == "bnhd" else CA_LAYOUT_BHND, H_total)
         # adaptive selection pairs with the eq. 15 query representation
         self.selection = selection
         self.recall, self.min_count = recall, min_count

@@ -13,9 +13,10 @@
  *    name ends in _host. Nothing here allocates or frees device memory; work
  *    that needs scratch takes a caller-provided workspace whose size is given
  *    by the matching *_workspace_bytes() query.
- *  - Q, K, V and O are head-major [B][H][N_alloc][d], rows contiguous, and
- *    16-byte aligned. Rows n_valid..N_alloc-1 are padding: never read as
- *    tokens; O's padding rows are written as 0.
+ *  - Q, K, V and O share the shape's layout (ca_layout: head-major
+ *    [B][H][N_alloc][d] or token-major [B][N_alloc][H_total][d]), each row of
+ *    d elements contiguous, 16-byte aligned. Rows (tokens) n_valid..N_alloc-1
+ *    are padding: never read as tokens; O's padding rows are written as 0.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream). Calls are asynchronous on it and never synchronise the host,
  *    except ca_get_device_error() and the _host variant.
@@ -46,12 +47,20 @@ typedef enum {
 
 typedef enum { CA_BF16 = 0, CA_FP32 = 1 } ca_dtype;
 
+/* Memory layout of Q, K, V and O (the same for all four):
+ *  CA_LAYOUT_BHND  [B][H][N_alloc][d], each head's rows contiguous;
+ *  CA_LAYOUT_BNHD  [B][N_alloc][H_total][d], the heads of one token
+ *                  contiguous (the layout a fused QKV projection produces);
+ *                  the call's H heads are heads 0..H-1 of the pointers, so a
+ *                  slice of heads h0..h0+H-1 passes pointers offset by h0*d. */
+typedef enum { CA_LAYOUT_BHND = 0, CA_LAYOUT_BNHD = 1 } ca_layout;
+
 /* Problem shape. C = ceil(n_valid / c) query clusters and
  * C_k = ceil(n_valid / c_k) key clusters (c_k = 0 means c_k = c, so C_k = C).
  * Unequal sizes are the paper's evaluated block shape (Section 3.1,
  * "Overview": 64 queries against 128 keys per block).
  * Supported: d in {64, 128}; c and c_k in {64, 128, 256}; 1 <= n_valid <=
- * N_alloc; dtype CA_BF16 or CA_FP32. */
+ * N_alloc; dtype CA_BF16 or CA_FP32; layout CA_LAYOUT_BHND or CA_LAYOUT_BNHD. */
 typedef struct {
   int B, H;          /* batch, heads */
   int N_alloc;       /* rows allocated per head */
@@ -60,6 +69,9 @@ typedef struct {
   int c;             /* query cluster size (and key cluster size when c_k is 0) */
   int dtype;         /* ca_dtype of Q, K, V and O */
   int c_k;           /* key cluster size, or 0 for c */
+  int layout;        /* ca_layout of Q, K, V and O */
+  int H_total;       /* CA_LAYOUT_BNHD: heads per token in memory (>= H), or 0 for H;
+                        CA_LAYOUT_BHND: 0 or H */
 } ca_shape;
 
 /* Clustering knobs (paper Section 3.2.1, "Basic recursive splitting" and
@@ -170,7 +182,7 @@ size_t ca_forward_workspace_bytes(const ca_shape* shape, int k);
  * below the split, recurse until every set but at most one holds c vectors.
  * The metric is injected into the power iteration (Section 6.1), so no
  * eigendecomposition is run. Ties between equal projections go by row index.
- * Q, K: device [B][H][N_alloc][d] of shape->dtype. out: device buffers, see
+ * Q, K: device, shape->dtype, in shape->layout. out: device buffers, see
  * ca_clusters. workspace: device, >= ca_cluster_workspace_bytes(shape).
  * Errors: CA_ERR_INVALID_ARG / CA_ERR_UNSUPPORTED / CA_ERR_WORKSPACE before
  * any launch; CA_ERR_CUDA if a launch fails.
@@ -244,7 +256,7 @@ ca_status ca_route_adaptive(const ca_shape* shape, const ca_clusters* centroids,
  * Reads clusters->perm_q/perm_k/count_k/kbar and routes->kept_idx/kept_bits
  * (and routes->kept_count when it is not NULL: per-query-cluster counts, as
  * written by ca_route_adaptive);
- * vbar is computed here. O: device [B][H][N_alloc][d], written in original
+ * vbar is computed here. O: device, in shape->layout, written in original
  * row order (padding rows 0). workspace >= ca_attend_workspace_bytes(shape).
  */
 ca_status ca_attend(const void* Q, const void* K, const void* V, const ca_shape* shape,
@@ -300,7 +312,11 @@ ca_status ca_forward(const void* Q, const void* K, const void* V, const ca_shape
  * group's inputs overlaps the forward of the previous group, and the copy of
  * a group's output the forward of the next. The forward runs on `stream`;
  * the copies on two short-lived helper streams that start after the work
- * already queued on `stream`. workspace >= ca_forward_host_workspace_bytes(shape, k).
+ * already queued on `stream`. In CA_LAYOUT_BNHD a group of heads is not a
+ * contiguous byte range, so the heads form one group (no overlap); the host
+ * buffers must hold exactly the call's heads (H_total 0 or H, else
+ * CA_ERR_UNSUPPORTED, and the workspace query returns 0).
+ * workspace >= ca_forward_host_workspace_bytes(shape, k).
  */
 size_t ca_forward_host_workspace_bytes(const ca_shape* shape, int k);
 ca_status ca_forward_host(const void* Q_host, const void* K_host, const void* V_host,

@@ -57,10 +57,22 @@ def test_shape_validation(lib):
         (ca.make_shape(0, 1, 1024, 1024, 64, 64, ca.CA_FP32), ca.CA_ERR_INVALID_ARG),   # B
         (ca.make_shape(1, 1, 1024, 0, 64, 64, ca.CA_FP32), ca.CA_ERR_INVALID_ARG),      # empty
         (ca.make_shape(1, 1, 1024, 1024, 64, 64, 7), ca.CA_ERR_INVALID_ARG),            # dtype
+        (ca.make_shape(1, 2, 1024, 1024, 64, 64, ca.CA_FP32, layout=2), ca.CA_ERR_INVALID_ARG),       # layout
+        (ca.make_shape(1, 2, 1024, 1024, 64, 64, ca.CA_FP32, layout=ca.CA_LAYOUT_BHND, H_total=3),
+         ca.CA_ERR_INVALID_ARG),                                                                      # BHND H_total
+        (ca.make_shape(1, 2, 1024, 1024, 64, 64, ca.CA_FP32, layout=ca.CA_LAYOUT_BNHD, H_total=1),
+         ca.CA_ERR_INVALID_ARG),                                                                      # H_total < H
     ]
     for s, want in bad:
         assert lib.ca_check_shape(ctypes.byref(s)) == want
         assert lib.ca_num_clusters(ctypes.byref(s)) == -1
+    # token-major: a slice of heads (H_total > H) is a valid shape, but the
+    # host-buffer forward needs the buffers to hold exactly the call's heads
+    sl = ca.make_shape(1, 2, 1024, 1024, 64, 64, ca.CA_BF16, layout=ca.CA_LAYOUT_BNHD, H_total=4)
+    assert lib.ca_check_shape(ctypes.byref(sl)) == ca.CA_OK
+    assert ca.forward_host_workspace_bytes(sl, 4) == 0
+    full = ca.make_shape(1, 4, 1024, 1024, 64, 64, ca.CA_BF16, layout=ca.CA_LAYOUT_BNHD)
+    assert ca.forward_host_workspace_bytes(full, 4) > 0
 
 
 def _fake(addr):
