@@ -390,12 +390,13 @@ def affinity_cores():
         return os.cpu_count() or 1
 
 
-def make_layer(ca, w, args, head_base=0):
+def make_layer(ca, w, args, head_base=0, layout=None):
     adaptive = args.selection == "adaptive"
     return ca.ClusterAttention(w.B, w.H, w.N_alloc, w.n_valid, w.d, w.c, key_clusters(w) if adaptive else w.k,
                                dtype=w.dtype, compensate=w.compensate, selection=args.selection,
                                recall=args.recall, min_count=16, clustering=args.clustering,
-                               head_base=head_base, c_k=getattr(w, "c_k", 0))
+                               head_base=head_base, c_k=getattr(w, "c_k", 0),
+                               layout=layout or args.layout)
 
 
 def head_share(w, world, rank):
@@ -549,7 +550,7 @@ def run_sweep(args):
                     Q, K, V = (torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
                                .cuda().contiguous() for x in (w.Q, w.K, w.V))
                     O = torch.empty_like(Q)
-                    layer = make_layer(ca, w, args)
+                    layer = make_layer(ca, w, args, layout="bhnd")
                     total_ms, stage, _ = time_layer(ca, torch, w, layer, Q, K, V, O, args.steps, args.warmup,
                                                     no_barrier, 0, sample_clocks=False)
                     ms = total_ms / args.steps
@@ -608,7 +609,13 @@ def run_ours(args):
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(x):
-        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(tdt).cuda().contiguous()
+        # [B, H, N, d], or token-major [B, N, H, d] with --layout bnhd
+        a = x if args.layout == "bhnd" else x.transpose(0, 2, 1, 3)
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).cuda().contiguous()
+
+    def head_rows(O, h):
+        """Rows [N, d] of head h of batch 0 of a layer output."""
+        return O[0, h] if args.layout == "bhnd" else O[0, :, h]
 
     Q, K, V = dev(w.Q), dev(w.K), dev(w.V)
     O = torch.empty_like(Q)
@@ -704,6 +711,7 @@ def run_ours(args):
                          if w.dtype == "bf16" else "clustering and routing f64; attention f32"),
         "data": "synthetic",
         "config": dict(workload_config(w_layer), selection=args.selection, clustering=args.clustering,
+                       layout="[B, H, N, d]" if args.layout == "bhnd" else "[B, N, H, d] (token-major)",
                        parallelism=(f"heads split over {world} GPUs ({w.H} per GPU, head_base {head_base} on "
                                     f"rank {rank})" if shard_heads else
                                     (f"an independent layer per GPU ({world} GPUs)" if world > 1 else "one GPU")),
@@ -726,7 +734,7 @@ def run_ours(args):
         kept = {}
         t_cpu, smp = oracle_sample(w, keep=kept, selection=args.selection, recall=args.recall,
                                    clustering=args.clustering)
-        line["error_vs_dense_fp64"] = error_vs_dense(w, O[0, kept["head"]].float().cpu().numpy(), kept)
+        line["error_vs_dense_fp64"] = error_vs_dense(w, head_rows(O, kept["head"]).float().cpu().numpy(), kept)
         line["cpu_baseline"] = {"value": 1.0 / t_cpu, "unit": UNIT, "cores": affinity_cores(),
                                 "blas_threads": blas_threads(), "kind": "oracle",
                                 "sample": f"head 0 clustered and routed in full, attention of 48 of {w.C} query "
@@ -764,6 +772,8 @@ def main():
     ap.add_argument("--shard", choices=["heads", "layers"], default="heads",
                     help="with N > 1 GPUs: split one layer's heads over the GPUs (default) or run an independent "
                          "layer per GPU")
+    ap.add_argument("--layout", choices=["bhnd", "bnhd"], default="bhnd",
+                    help="memory layout of Q, K, V and O: head-major [B, H, N, d] or token-major [B, N, H, d]")
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=CONFIG_ID,
                     help="workload (default 2: the metric's N = 64k configuration); 5: the sweep over cluster "
                          "size, keep fraction and compensation at N = 32,768, one JSON line per point")
