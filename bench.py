@@ -48,10 +48,10 @@ CONFIG_ID = 2
 # SHA-256 starts with `sha` and the workload it names; for any other source
 # or workload the bench reports null.
 ATTN_CAPTURES = [
-    {"sha": "2ffdbbe8fdc42cdd", "workload": "cfg2-lowrank-N65536-d64-bf16",
-     "traffic": 205566720 + 52314112, "tensor_pipe_pct": 31.10},
-    {"sha": "2ffdbbe8fdc42cdd", "workload": "cfg3-grid-21x45x80-d128-bf16",
-     "traffic": 2460196096 + 779414784, "tensor_pipe_pct": 47.77},
+    {"sha": "ff025bea226f0ade", "workload": "cfg2-lowrank-N65536-d64-bf16",
+     "traffic": 205868288 + 52257536, "tensor_pipe_pct": 31.01},
+    {"sha": "ff025bea226f0ade", "workload": "cfg3-grid-21x45x80-d128-bf16",
+     "traffic": 2505658880 + 781805568, "tensor_pipe_pct": 46.43},
 ]
 
 

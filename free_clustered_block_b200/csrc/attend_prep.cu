@@ -46,8 +46,19 @@ __global__ void __launch_bounds__(256) centroid_prep_kernel(
   const int cnt = count_k[(size_t)bh * C + b];
   const int32_t* mem = perm_k + (size_t)bh * C * c + (size_t)b * c;
   const T* Vh = V + TL.head(bh);
+  // members rg, rg + RG, ... summed in that order, four row loads in flight
   double s = 0.0;
-  for (int j = rg; j < cnt; j += RG) s += (double)to_f(Vh[(size_t)mem[j] * TL.sn + col]);
+  int j = rg;
+  for (; j + 3 * RG < cnt; j += 4 * RG) {
+    const int r0 = mem[j], r1 = mem[j + RG], r2 = mem[j + 2 * RG], r3 = mem[j + 3 * RG];
+    const T x0 = Vh[(size_t)r0 * TL.sn + col], x1 = Vh[(size_t)r1 * TL.sn + col];
+    const T x2 = Vh[(size_t)r2 * TL.sn + col], x3 = Vh[(size_t)r3 * TL.sn + col];
+    s += (double)to_f(x0);
+    s += (double)to_f(x1);
+    s += (double)to_f(x2);
+    s += (double)to_f(x3);
+  }
+  for (; j < cnt; j += RG) s += (double)to_f(Vh[(size_t)mem[j] * TL.sn + col]);
   __shared__ double red[256];
   red[threadIdx.x] = s;
   __syncthreads();

@@ -1047,8 +1047,8 @@ __global__ void __launch_bounds__(2 * D_, D_ == 64 ? 3 : 1) dirc_kernel(
 constexpr long long kDirCMaxNodes64 = 148 * 4;
 
 constexpr int kProjSpan = 1024;
-constexpr int kProjNodes = 20;   // > kProjSpan / 65 + 2
-constexpr int kProjU = 4;
+constexpr int kProjNodes = 20;   // > kProjSpan / 65 + 2, and at most 32 (one lane each)
+constexpr int kProjU = 4;        // 8 measured slower (fewer blocks per SM)
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) project_kernel(const T* __restrict__ Q, const T* __restrict__ K,
@@ -1202,6 +1202,7 @@ __global__ void __launch_bounds__(256) hash_keys_kernel(int n, const int* __rest
 // ---------------------------------------------------------------------------
 struct SelectResult { uint64_t T; int eq_left; int pad; };
 constexpr int kSelCap = 8192;
+constexpr int kSelU = 4;   // keys per thread in flight in the global passes (16 measured the same)
 
 template <int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__ nodes, int lb,
@@ -1238,16 +1239,16 @@ __global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__
       }
     };
     if (global_mode) {
-      // four keys per thread per step, their loads in flight together
-      for (int i0 = 0; i0 < cnt_total; i0 += NT * 4) {
-        uint64_t kk[4];
+      // kSelU keys per thread per step, their loads in flight together
+      for (int i0 = 0; i0 < cnt_total; i0 += NT * kSelU) {
+        uint64_t kk[kSelU];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kSelU; ++u) {
           const int i = i0 + u * NT + threadIdx.x;
           kk[u] = i < cnt_total ? base[i] : 0ull;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < kSelU; ++u)
           count(i0 + u * NT + (int)threadIdx.x < cnt_total && (kk[u] & mask) == prefix, kk[u]);
       }
     } else {
@@ -1291,15 +1292,15 @@ __global__ void __launch_bounds__(NT) select_kernel(const TreeNode* __restrict__
       if (threadIdx.x == 0) s_ncand = 0;
       __syncthreads();
       if (global_mode) {
-        for (int i0 = 0; i0 < size; i0 += NT * 4) {
-          uint64_t kk[4];
+        for (int i0 = 0; i0 < size; i0 += NT * kSelU) {
+          uint64_t kk[kSelU];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int u = 0; u < kSelU; ++u) {
             const int i = i0 + u * NT + threadIdx.x;
             kk[u] = i < size ? base[i] : ~prefix;   // ~prefix never matches (the mask is not empty)
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
+          for (int u = 0; u < kSelU; ++u)
             if ((kk[u] & mask) == prefix) cand[atomicAdd(&s_ncand, 1)] = kk[u];
         }
       } else {
@@ -1472,8 +1473,20 @@ __global__ void __launch_bounds__(256) centroid_kernel(const T* __restrict__ Q, 
   if (threadIdx.x == 0) ((tensor == 0) ? count_q : count_k)[(size_t)bh * C + a] = cnt;
   const T* X = (tensor == 0 ? Q : K) + TL.head(bh);
   const int col = threadIdx.x % D, rg = threadIdx.x / D;
+  // members rg, rg + RG, ... summed in that order, four row loads in flight
   double s = 0.0;
-  for (int j = rg; j < cnt; j += RG) {
+  int j = rg;
+  for (; j + 3 * RG < cnt; j += 4 * RG) {
+    int r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) r[u] = (levels == 0) ? j + u * RG : perm[j + u * RG];
+    T x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = X[(size_t)r[u] * TL.sn + col];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) s += (double)to_f(x[u]);
+  }
+  for (; j < cnt; j += RG) {
     const int row = (levels == 0) ? j : perm[j];
     s += (double)to_f(X[(size_t)row * TL.sn + col]);
   }
