@@ -73,3 +73,45 @@ def test_rounding_model_error_is_inside_the_bound(name):
     assert 1.0e-3 <= rel <= 3.3e-3, f"{name}: model rel-L2 {rel:.3g}"
     assert rel <= parity.REL_L2["bf16"] / 3
     assert max_abs <= parity.MAX_ABS["bf16"]
+
+
+def _model_fp32(Q, K, V, h, kept, c):
+    """Compensated attention with every operation in fp32 (the SIMT kernel's precision)."""
+    f = np.float32
+    d = Q.shape[1]
+    Q32, K32, V32 = Q.astype(f), K.astype(f), V.astype(f)
+    Ck = h.count_k.shape[0]
+    kmem = [h.perm_k[b * c: b * c + h.count_k[b]] for b in range(Ck)]
+    kbar = np.stack([K[m].mean(axis=0) for m in kmem]).astype(f)   # centroids arrive from fp64
+    vbar = np.stack([V[m].mean(axis=0) for m in kmem]).astype(f)
+    logcnt = np.log(h.count_k.astype(f))
+    sc = f(1.0 / np.sqrt(d))
+    O = np.zeros(Q.shape, f)
+    for a in range(h.count_q.shape[0]):
+        qm = h.perm_q[a * c: a * c + h.count_q[a]]
+        kept_a = np.asarray(kept[a], np.int64)
+        J = np.concatenate([kmem[b] for b in kept_a])
+        logits = (Q32[qm] @ K32[J].T) * sc
+        vals = V32[J]
+        excl = np.setdiff1d(np.arange(Ck), kept_a)
+        if excl.size:
+            logits = np.concatenate([logits, (Q32[qm] @ kbar[excl].T) * sc + logcnt[excl]], axis=1)
+            vals = np.concatenate([vals, vbar[excl]], axis=0)
+        w = np.exp(logits - logits.max(axis=1, keepdims=True))
+        O[qm] = (w @ vals) / w.sum(axis=1, keepdims=True)
+    return O.astype(np.float64)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fp32_model_error_is_inside_the_bound(name):
+    w = CASES[name]()
+    if w.dtype != "fp32":
+        pytest.skip("bf16 case")
+    Qf, Kf, Vf = (x[0, 0, :w.n_valid].astype(np.float64) for x in (w.Q, w.K, w.V))
+    h = orc.cluster_head(Qf, Kf, w.c, seed=0, bh=0)
+    kept = orc.topk_route(orc.centroid_scores(h.qbar, h.kbar), w.k)
+    exact = orc.compensated_attention(Qf, Kf, Vf, h.perm_q, h.count_q, h.perm_k, h.count_k, kept, w.c)
+    max_abs, rel = parity.errors(_model_fp32(Qf, Kf, Vf, h, kept, w.c), exact)
+    # the derivation's estimate is ~5e-6; the bound leaves a factor of four
+    assert rel <= parity.REL_L2["fp32"] / 4, f"{name}: model rel-L2 {rel:.3g}"
+    assert max_abs <= parity.MAX_ABS["fp32"]
